@@ -1,0 +1,392 @@
+"""Benchmark of the chunked TTT / linear-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llm_d64|momentum_d128|long_d128] [--chunk C] [--segments P]
+
+A step is one chunked forward of the whole layer (all heads, all tokens, final
+state) over one batch of synthetic inputs already resident in HBM.  Default
+workload: the LLM-shaped layer (B=4, H=16, T=4096, d=64, bf16, per-token
+learning rate, chunk 64).  Prints ONE JSON line on rank 0.
+
+Multi-GPU (torchrun): every rank runs its own batch (independent sequences,
+no collective on the data path: weak scaling); value = tokens of all ranks /
+max-over-ranks device time.  `--impl reference` times the float64 CPU oracle
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import CONFIGS, make_case  # noqa: E402
+
+METRIC = "TTT-layer tokens/sec (chunked fwd, 1 B200) and % tensor peak; decode HBM GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def algorithmic_bytes(c, B, H, T):
+    """Minimum HBM bytes of one forward: read q, k, v (and eta), write o and
+    the final state once."""
+    el = 2 if c.dtype == "bf16" else 4
+    qkvo = B * H * T * (2 * c.d_k + 2 * c.d_v) * el
+    eta = B * H * T * 4 if c.eta_mode == "token" else 0
+    state = B * H * c.d_v * c.d_k * 4 * (2 if c.beta else 1)
+    return qkvo + eta + state
+
+
+def executed_flops(c, B, H, T, chunk):
+    """Tensor-core flops the chunked kernel executes (full C x C score tiles):
+    per token-head 2*C*d (Q K^T) + 2*C*d (P V) + 2*d*d (Q W^T) + 2*d*d (V^T K)."""
+    d = c.d_k
+    per = 4 * chunk * d + 4 * d * d
+    return B * H * T * per
+
+
+def src_hash():
+    h = hashlib.sha1()
+    cdir = os.path.join(ROOT, "test_layers_causal_b200", "csrc")
+    for f in sorted(os.listdir(cdir)):
+        with open(os.path.join(cdir, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def read_traffic(workload, chunk):
+    """DRAM bytes per forward from a committed ncu summary, if it was taken on
+    the current kernel sources (profiles/<workload>_c<chunk>.traffic.txt holds
+    lines `src_hash=...` and `dram_bytes_per_call=...`)."""
+    p = os.path.join(ROOT, "profiles", f"{workload}_c{chunk}.traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if "=" in line:
+                a, b = line.strip().split("=", 1)
+                kv[a.strip()] = b.strip()
+    if kv.get("src_hash") != src_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_call"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [l.strip().split(", ") for l in self.tmp.read().splitlines() if l.strip()]
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            if len(r) >= 9:
+                for n, val in zip(names, r[5:9]):
+                    if val.strip().lower() == "active":
+                        reasons.add(n)
+        busy = [s for s in sm if mx and s > 0.3 * max(mx)]
+        return {"sm_mhz": statistics.median(busy or sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- oracle ----
+def oracle_sample(c, heads, rank_seed=0):
+    """Runs the float64 oracle on `heads` (b, h) sequences of the workload at
+    full length; returns (seconds, head-tokens)."""
+    import numpy as np
+
+    import oracle
+    x = make_case(c, B=1, H=heads)
+    f = lambda t: t.float().double().numpy()  # noqa: E731
+    eta = f(x["eta"]) if x["eta"] is not None else x["eta_const"]
+    t0 = time.perf_counter()
+    oracle.ttt_recurrence_f64(f(x["q"]), f(x["k"]), f(x["v"]), eta, beta=c.beta)
+    dt = time.perf_counter() - t0
+    del np
+    return dt, heads * c.T
+
+
+def cpu_baseline(c, heads):
+    dt, head_tokens = oracle_sample(c, heads)
+    total_head_tokens = c.B * c.H * c.T
+    t_full = dt * total_head_tokens / head_tokens
+    return {"value": c.B * c.T / t_full, "unit": "tokens/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{heads} of {c.B * c.H} (b,h) sequences at full length T={c.T} "
+                      f"({dt:.1f} s of float64 numpy), scaled to the whole layer"}
+
+
+def run_reference(args, c, ws, rank):
+    if rank != 0:
+        return
+    heads = max(1, min(c.B * c.H, args.ref_heads))
+    for _ in range(args.warmup):
+        oracle_sample(c, heads)
+    times = []
+    for _ in range(args.steps):
+        dt, _ = oracle_sample(c, heads)
+        times.append(dt * (c.B * c.H) / heads)
+    t = sum(times) / len(times)
+    val = c.B * c.T / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(c, args),
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": f"each step: {heads} of {c.B * c.H} (b,h) sequences at full length, "
+                                   "scaled to the whole layer"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(c, args):
+    return {"workload": c.name, "B": c.B, "H": c.H, "T": c.T, "d_k": c.d_k, "d_v": c.d_v,
+            "chunk": args.chunk or c.chunk, "eta": "per-token" if c.eta_mode == "token" else "constant",
+            "beta": c.beta, "global_batch": c.B, "seq_len": c.T, "parallelism": f"dp{args.gpus}",
+            "l2": f"{args.sets} rotating input sets (inputs larger than L2)"}
+
+
+# ----------------------------------------------------------------- ours ----
+def run_ours(args, c, ws, rank, local):
+    import test_layers_causal_b200 as ttt
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    chunk = args.chunk or c.chunk
+    x = make_case(c)
+    qh, kh, vh = x["q"], x["k"], x["v"]
+    etah = x["eta"]
+    # rotating device copies so that consecutive steps do not hit in L2
+    sets = []
+    for _ in range(args.sets):
+        q, k, v = qh.to(dev), kh.to(dev), vh.to(dev)
+        eta = etah.to(dev) if etah is not None else None
+        o = torch.empty_like(v)
+        S = torch.empty(c.B, c.H, c.d_v, c.d_k, device=dev, dtype=torch.float32)
+        M = torch.empty_like(S) if c.beta else None
+        sets.append((q, k, v, eta, o, S, M))
+    wsb = ttt.workspace_bytes(sets[0][0], sets[0][2], chunk=chunk, beta=c.beta, segments=args.segments)
+    work = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        q, k, v, eta, o, S, M = sets[i % len(sets)]
+        ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=chunk,
+                            segments=args.segments, out=o, state_out=S, mom_out=M, workspace=work)
+
+    # CUDA graph per input set: one replay = one step, no host launch overhead
+    for i in range(len(sets)):
+        step(i)
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(len(sets)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(i)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    status = ttt.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        graphs[i % len(graphs)].replay()
+    # keep the GPU busy ~1 s right before the timed region so the clock
+    # samples describe the loaded state
+    t_end = time.time() + 1.0
+    i = 0
+    while time.time() < t_end:
+        graphs[i % len(graphs)].replay()
+        i += 1
+        if i % 200 == 0:
+            torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
+    ev0.record(stream)
+    for i in range(args.steps):
+        graphs[i % len(graphs)].replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    barrier(ws)
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, ws)
+    ms_per_step = ms_max / args.steps
+    tokens_per_step = c.B * c.T
+    value = tokens_per_step * ws / (ms_per_step * 1e-3)
+    if ttt.device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+
+    # ---- end to end: pinned host buffers in, o (and final state) back out
+    qp, kp, vp = (t.pin_memory() for t in (qh, kh, vh))
+    ep = etah.pin_memory() if etah is not None else None
+    oh = torch.empty(vh.shape, dtype=vh.dtype, pin_memory=True)
+    Sh = torch.empty(c.B, c.H, c.d_v, c.d_k, dtype=torch.float32, pin_memory=True)
+    bufs = ttt.host.DeviceBuffers(qp, kp, vp, ep, device=dev)
+    kw = dict(eta_const=x["eta_const"], beta=c.beta, chunk=chunk, segments=args.segments, workspace=work)
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(3):
+        ttt.forward_chunked_host(qp, kp, vp, ep, o_host=oh, bufs=bufs, state_host=Sh, **kw)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        _, h2d, d2h = ttt.forward_chunked_host(qp, kp, vp, ep, o_host=oh, bufs=bufs, state_host=Sh, **kw)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws) / e2e_steps
+    e2e_val = tokens_per_step * ws / (e2e_ms * 1e-3)
+
+    # ---- roofline of the forward call
+    peaks, src = load_peaks()
+    nbytes = algorithmic_bytes(c, c.B, c.H, c.T)
+    achieved = nbytes / (ms_per_step * 1e-3) / 1e9
+    flops = executed_flops(c, c.B, c.H, c.T, chunk)
+    tflops = flops / (ms_per_step * 1e-3) / 1e12
+    traffic = read_traffic(c.name, chunk)
+    nseg_launch = 3 if wsb > 0 else 1
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if c.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": workload_config(c, args),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": "ttt_la_forward_chunked (segment-state pass, scan, chunk pass)"
+                               if nseg_launch == 3 else "ttt_la_forward_chunked (chunk pass)",
+                     "algorithmic_bytes": nbytes, "peak_source": f"{src} (copy bandwidth)"},
+        "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                   "frac": tflops / peaks["bf16_tflops"], "executed_flops": flops},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * nseg_launch,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(c, args.ref_heads)
+    for g in graphs:
+        del g
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llm_d64", choices=sorted(CONFIGS))
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--segments", type=int, default=0)
+    ap.add_argument("--sets", type=int, default=4)
+    ap.add_argument("--ref-heads", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    c = CONFIGS[args.workload]
+    if c.dtype != "bf16":
+        raise SystemExit("bench workloads are the bf16 layers")
+    ws, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, c, ws, rank)
+        else:
+            run_ours(args, c, ws, rank, local)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

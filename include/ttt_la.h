@@ -1,0 +1,158 @@
+/*
+ * ttt_la.h -- C ABI of the causal TTT / linear-attention layer for B200 (sm_100a).
+ *
+ * The layer (from "Test-Time Training with KV Binding Is Secretly Linear
+ * Attention", Liu et al.; Table 2 of the thelatestinai.com listing, Variants
+ * 3-5, and the kualia.ai explainer, section "The Linear Attention
+ * Equivalence"): per sequence and head, a fast weight W (d_v x d_k, fp32)
+ * takes one gradient step per token on the key-value binding loss
+ * L_t(W) = -sigma v_t^T W k_t, then reads out o_t = W_t q_t:
+ *
+ *   no momentum (beta == 0):  W_t = W_{t-1} + sigma * eta_t * v_t k_t^T
+ *   SGD momentum (beta != 0): M_t = beta M_{t-1} - sigma * v_t k_t^T
+ *                             W_t = W_{t-1} - eta_t * M_t
+ *   o_t = W_t q_t                      (update first, then read)
+ *
+ * sigma = +1 (descent) or -1 (gradient ascent, Table 1 of the same listing).
+ * M is the momentum buffer of gradients.  The fast weights reset for every
+ * sequence (explainer "Test Time Training", wpnews.pro): state_in == NULL
+ * means W_0 = 0 (and M_0 = 0).
+ *
+ * Three computations of the same layer:
+ *   ttt_la_forward_chunked   chunk-parallel form ("fully parallel
+ *                            formulations", abstract): intra-chunk causal
+ *                            (Q K^T * coefficients) V plus the carried state,
+ *                            on the tensor cores (bf16 inputs) or in fp32 FMA
+ *                            (fp32 inputs).
+ *   ttt_la_forward_recurrent token-by-token recurrence ("Recurrent Impl.",
+ *                            Table 2).
+ *   ttt_la_decode_step       one token for N sequences, state updated in place.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers, row-major and contiguous, 16-byte
+ *    aligned.  q, k: [B,H,T,d_k]; v, o: [B,H,T,d_v]; eta: [B,H,T] fp32;
+ *    state / momentum: [B,H,d_v,d_k] fp32 (row n of W holds the weights that
+ *    produce output feature n).  dtype applies to q, k, v and o together.
+ *  - The caller owns every buffer; the library allocates no device memory.
+ *    Scratch for the chunked path is the caller's `workspace`
+ *    (ttt_la_workspace_size bytes).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Argument errors are detected on the host before any
+ *    launch and return TTT_LA_ERR_INVALID_ARG / TTT_LA_ERR_UNSUPPORTED with
+ *    nothing launched.  A failed launch returns TTT_LA_ERR_CUDA.
+ *  - Every in-kernel wait is bounded in time.  A wait that runs out records
+ *    TTT_LA_ERR_TIMEOUT in the library's device status word, the kernel
+ *    drains its own copies, frees its tensor memory and returns;
+ *    ttt_la_get_last_device_status reads (and clears) that word.
+ *  - o must not alias q, k, v, eta or the states.  state_out may equal
+ *    state_in (in place), and mom_out may equal mom_in.
+ */
+#ifndef TTT_LA_H
+#define TTT_LA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TTT_LA_API __attribute__((visibility("default")))
+#else
+#define TTT_LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_LA_OK = 0,
+  TTT_LA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, short workspace */
+  TTT_LA_ERR_UNSUPPORTED = 2,  /* valid but not built: (d_k, d_v, chunk, dtype) combination */
+  TTT_LA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  TTT_LA_ERR_TIMEOUT = 4       /* a bounded in-kernel wait ran out (device status word) */
+} ttt_la_status;
+
+typedef enum { TTT_LA_F32 = 0, TTT_LA_BF16 = 1 } ttt_la_dtype;
+
+/* Arguments of a whole-sequence forward (chunked or recurrent). */
+typedef struct ttt_la_args {
+  int32_t B, H, T;          /* batch, heads, tokens (T >= 1, any value) */
+  int32_t d_k, d_v;         /* head dims */
+  int32_t dtype;            /* ttt_la_dtype of q, k, v, o */
+  const void *q, *k, *v;    /* [B,H,T,d_k], [B,H,T,d_k], [B,H,T,d_v] */
+  const float *eta;         /* [B,H,T] per-token learning rate, or NULL -> eta_const */
+  float eta_const;          /* learning rate when eta == NULL */
+  float beta;               /* SGD momentum; 0 -> plain SGD (momentum buffers unused) */
+  int32_t ascent;           /* 0: gradient descent (sigma=+1); 1: ascent (sigma=-1) */
+  int32_t chunk;            /* chunked path: tokens per chunk (64 or 128); ignored otherwise */
+  int32_t segments;         /* chunked path: sequence segments per (b,h) run in parallel;
+                               0 = automatic (fill the SMs); ignored otherwise */
+  const float *state_in;    /* [B,H,d_v,d_k] W_0, or NULL -> zeros */
+  float *state_out;         /* [B,H,d_v,d_k] W_T, or NULL -> not returned */
+  const float *mom_in;      /* [B,H,d_v,d_k] M_0 (momentum only), or NULL -> zeros */
+  float *mom_out;           /* [B,H,d_v,d_k] M_T (momentum only), or NULL -> not returned */
+  void *o;                  /* [B,H,T,d_v] output, dtype */
+  void *workspace;          /* device scratch, >= ttt_la_workspace_size(args) bytes */
+  size_t workspace_bytes;
+} ttt_la_args;
+
+/* Bytes of caller-provided scratch that ttt_la_forward_chunked needs for
+ * these arguments (0 when the call needs none; pointers are not read). */
+TTT_LA_API size_t ttt_la_workspace_size(const ttt_la_args *args);
+
+/* Chunk-parallel forward.  Within each chunk of `chunk` tokens the outputs are
+ * the causal, coefficient-weighted attention of the chunk's queries on its
+ * keys and values plus the read-out of the state carried in from earlier
+ * chunks; the state after each chunk is the carried state plus the chunk's
+ * weighted V^T K (with momentum, the pair (W, M) follows the affine chunk map
+ * W' = W - g M + dW, M' = beta^C M + dM).  bf16 inputs run on the tcgen05
+ * tensor cores with fp32 accumulation: d_k == d_v in {64, 128},
+ * chunk in {64, 128}.  fp32 inputs run in fp32 FMA: d_k, d_v multiples of 4
+ * up to 128, chunk in {16, 32, 64}.  Other combinations: UNSUPPORTED. */
+TTT_LA_API ttt_la_status ttt_la_forward_chunked(const ttt_la_args *args, void *stream);
+
+/* Token-by-token forward (the recurrence itself): fp32 or bf16 inputs,
+ * d_k in {32, 64, 128}, d_v <= 1024; chunk and workspace are ignored. */
+TTT_LA_API ttt_la_status ttt_la_forward_recurrent(const ttt_la_args *args, void *stream);
+
+/* One decode step for N independent sequences: for every (n, h)
+ * applies the single-token update to state (and mom when beta != 0) IN PLACE
+ * and writes o = W q.  q, k: [N,H,d_k]; v, o: [N,H,d_v]; eta: [N,H] or NULL;
+ * state, mom: [N,H,d_v,d_k] fp32.  d_k in {32, 64, 128}; memory-bound. */
+typedef struct ttt_la_decode_args {
+  int32_t N, H, d_k, d_v;
+  int32_t dtype;            /* of q, k, v, o */
+  const void *q, *k, *v;
+  const float *eta;         /* [N,H] or NULL -> eta_const */
+  float eta_const, beta;
+  int32_t ascent;
+  float *state;             /* [N,H,d_v,d_k] fp32, read and written in place */
+  float *mom;               /* [N,H,d_v,d_k] fp32 in place; required iff beta != 0 */
+  void *o;                  /* [N,H,d_v] */
+} ttt_la_decode_args;
+
+TTT_LA_API ttt_la_status ttt_la_decode_step(const ttt_la_decode_args *args, void *stream);
+
+/* Synchronises `stream`, returns the device status word (TTT_LA_OK or
+ * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
+TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);
+
+/* Sets the time limit of every in-kernel wait (nanoseconds, >= 1000);
+ * default 1e9 (one second).  Affects launches made after the call. */
+TTT_LA_API ttt_la_status ttt_la_set_wait_limit_ns(int64_t limit_ns);
+
+/* Self-test of the bounded-wait machinery: launches one block that waits on
+ * an mbarrier that nothing completes, with the given limit.  The wait runs out,
+ * the block records TTT_LA_ERR_TIMEOUT and returns; read it with
+ * ttt_la_get_last_device_status.  Never hangs. */
+TTT_LA_API ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void *stream);
+
+/* Human-readable name of a status code (static string). */
+TTT_LA_API const char *ttt_la_status_string(ttt_la_status s);
+
+/* Library version string (static). */
+TTT_LA_API const char *ttt_la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_LA_H */

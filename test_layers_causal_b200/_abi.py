@@ -1,0 +1,238 @@
+"""ctypes binding of libttt_la.so (include/ttt_la.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module only
+fills the C structs with tensor pointers and sizes, allocates outputs and
+scratch through PyTorch, and turns status codes into exceptions.  There is no
+CPU path: if the shared library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libttt_la.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+F32, BF16 = 0, 1
+
+_c_i32, _c_f32, _c_vp, _c_sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class TttArgs(ctypes.Structure):
+    """Mirror of ``ttt_la_args``."""
+    _fields_ = [
+        ("B", _c_i32), ("H", _c_i32), ("T", _c_i32), ("d_k", _c_i32), ("d_v", _c_i32), ("dtype", _c_i32),
+        ("q", _c_vp), ("k", _c_vp), ("v", _c_vp), ("eta", _c_vp),
+        ("eta_const", _c_f32), ("beta", _c_f32), ("ascent", _c_i32), ("chunk", _c_i32), ("segments", _c_i32),
+        ("state_in", _c_vp), ("state_out", _c_vp), ("mom_in", _c_vp), ("mom_out", _c_vp),
+        ("o", _c_vp), ("workspace", _c_vp), ("workspace_bytes", _c_sz),
+    ]
+
+
+class TttDecodeArgs(ctypes.Structure):
+    """Mirror of ``ttt_la_decode_args``."""
+    _fields_ = [
+        ("N", _c_i32), ("H", _c_i32), ("d_k", _c_i32), ("d_v", _c_i32), ("dtype", _c_i32),
+        ("q", _c_vp), ("k", _c_vp), ("v", _c_vp), ("eta", _c_vp),
+        ("eta_const", _c_f32), ("beta", _c_f32), ("ascent", _c_i32),
+        ("state", _c_vp), ("mom", _c_vp), ("o", _c_vp),
+    ]
+
+
+# (name, restype, argtypes) for every symbol of include/ttt_la.h
+SIGNATURES = [
+    ("ttt_la_workspace_size", _c_sz, [ctypes.POINTER(TttArgs)]),
+    ("ttt_la_forward_chunked", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
+    ("ttt_la_forward_recurrent", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
+    ("ttt_la_decode_step", ctypes.c_int, [ctypes.POINTER(TttDecodeArgs), _c_vp]),
+    ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
+    ("ttt_la_set_wait_limit_ns", ctypes.c_int, [ctypes.c_int64]),
+    ("ttt_la_selftest_wait_timeout", ctypes.c_int, [ctypes.c_int64, _c_vp]),
+    ("ttt_la_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("ttt_la_version", ctypes.c_char_p, []),
+]
+
+_lib = None
+
+
+class TttError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        msg = status_string(code) if _lib is not None else str(code)
+        super().__init__(f"{fn} failed: {msg} (status {code})")
+
+
+def lib():
+    """Loads the shared library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m test_layers_causal_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().ttt_la_status_string(int(code)).decode()
+
+
+def version() -> str:
+    return lib().ttt_la_version().decode()
+
+
+def _check(fn, code):
+    if code != OK:
+        raise TttError(fn, code)
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("inputs must be contiguous CUDA tensors")
+
+
+def _seq_args(q, k, v, eta, eta_const, beta, ascent, chunk, segments, state_in, mom_in, o, S_out, M_out):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    a = TttArgs()
+    a.B, a.H, a.T, a.d_k, a.d_v, a.dtype = B, H, T, dk, dv, _dtype_code(q)
+    a.q, a.k, a.v, a.eta = q.data_ptr(), k.data_ptr(), v.data_ptr(), (eta.data_ptr() if eta is not None else None)
+    a.eta_const = float(1.0 / math.sqrt(dk) if eta_const is None else eta_const)
+    a.beta, a.ascent, a.chunk, a.segments = float(beta), int(bool(ascent)), int(chunk), int(segments)
+    a.state_in = state_in.data_ptr() if state_in is not None else None
+    a.mom_in = mom_in.data_ptr() if mom_in is not None else None
+    a.state_out = S_out.data_ptr() if S_out is not None else None
+    a.mom_out = M_out.data_ptr() if M_out is not None else None
+    a.o = o.data_ptr()
+    return a
+
+
+def _check_shapes(q, k, v, eta, state_in, mom_in):
+    if q.dim() != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k: [B,H,T,d_k]; v: [B,H,T,d_v]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share a dtype")
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if eta is not None and (eta.shape != (B, H, T) or eta.dtype != torch.float32):
+        raise ValueError("eta must be fp32 [B,H,T]")
+    for s in (state_in, mom_in):
+        if s is not None and (s.shape != (B, H, dv, dk) or s.dtype != torch.float32):
+            raise ValueError("state_in / mom_in must be fp32 [B,H,d_v,d_k]")
+    _need_cuda(q, k, v, eta, state_in, mom_in)
+
+
+def _alloc_outputs(q, v, beta, return_state, out, state_out=None, mom_out=None):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if out is None else out
+    S = M = None
+    if return_state:
+        S = torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32) if state_out is None else state_out
+        if beta != 0:
+            M = torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32) if mom_out is None else mom_out
+    return o, S, M
+
+
+def forward_chunked(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, chunk=64, segments=0,
+                    state_in=None, mom_in=None, return_state=True, out=None, workspace=None, stream=None,
+                    state_out=None, mom_out=None):
+    """Chunk-parallel forward (ttt_la_forward_chunked).  Returns (o, W_T, M_T);
+    W_T / M_T are None when not requested / without momentum.  `out`,
+    `state_out`, `mom_out` and `workspace` may be preallocated buffers."""
+    _check_shapes(q, k, v, eta, state_in, mom_in)
+    o, S, M = _alloc_outputs(q, v, beta, return_state, out, state_out, mom_out)
+    a = _seq_args(q, k, v, eta, eta_const, beta, ascent, chunk, segments, state_in, mom_in, o, S, M)
+    L = lib()
+    need = L.ttt_la_workspace_size(ctypes.byref(a))
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check("ttt_la_forward_chunked", L.ttt_la_forward_chunked(ctypes.byref(a), _stream_handle(stream)))
+    return o, S, M
+
+
+def workspace_bytes(q, v, chunk=64, beta=0.0, segments=0):
+    """Scratch bytes ttt_la_forward_chunked needs for these shapes."""
+    B, H, T, dk = q.shape
+    a = TttArgs()
+    a.B, a.H, a.T, a.d_k, a.d_v, a.dtype = B, H, T, dk, v.shape[-1], _dtype_code(q)
+    a.q, a.k, a.v, a.o = 16, 32, 48, 64  # never dereferenced by the size query
+    a.beta, a.chunk, a.segments = float(beta), int(chunk), int(segments)
+    return int(lib().ttt_la_workspace_size(ctypes.byref(a)))
+
+
+def forward_recurrent(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, state_in=None, mom_in=None,
+                      return_state=True, out=None, stream=None):
+    """Token-by-token forward (ttt_la_forward_recurrent).  Returns (o, W_T, M_T)."""
+    _check_shapes(q, k, v, eta, state_in, mom_in)
+    o, S, M = _alloc_outputs(q, v, beta, return_state, out)
+    a = _seq_args(q, k, v, eta, eta_const, beta, ascent, 0, 0, state_in, mom_in, o, S, M)
+    _check("ttt_la_forward_recurrent", lib().ttt_la_forward_recurrent(ctypes.byref(a), _stream_handle(stream)))
+    return o, S, M
+
+
+def decode_step(q, k, v, state, mom=None, eta=None, eta_const=None, beta=0.0, ascent=False, out=None,
+                stream=None):
+    """One decode step (ttt_la_decode_step): q, k [N,H,d_k], v [N,H,d_v];
+    state (and mom with momentum) [N,H,d_v,d_k] fp32 updated in place.
+    Returns o [N,H,d_v]."""
+    if q.dim() != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k: [N,H,d_k]; v: [N,H,d_v]")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if state.shape != (N, H, dv, dk) or state.dtype != torch.float32:
+        raise ValueError("state must be fp32 [N,H,d_v,d_k]")
+    if eta is not None and (eta.shape != (N, H) or eta.dtype != torch.float32):
+        raise ValueError("eta must be fp32 [N,H]")
+    _need_cuda(q, k, v, state, mom, eta)
+    o = torch.empty_like(v) if out is None else out
+    a = TttDecodeArgs()
+    a.N, a.H, a.d_k, a.d_v, a.dtype = N, H, dk, dv, _dtype_code(q)
+    a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    a.eta = eta.data_ptr() if eta is not None else None
+    a.eta_const = float(1.0 / math.sqrt(dk) if eta_const is None else eta_const)
+    a.beta, a.ascent = float(beta), int(bool(ascent))
+    a.state, a.mom, a.o = state.data_ptr(), (mom.data_ptr() if mom is not None else None), o.data_ptr()
+    _check("ttt_la_decode_step", lib().ttt_la_decode_step(ctypes.byref(a), _stream_handle(stream)))
+    return o
+
+
+def device_status(stream=None) -> int:
+    """Synchronises and returns (then clears) the device status word."""
+    return int(lib().ttt_la_get_last_device_status(_stream_handle(stream)))
+
+
+def set_wait_limit_ns(ns: int):
+    _check("ttt_la_set_wait_limit_ns", lib().ttt_la_set_wait_limit_ns(int(ns)))
+
+
+def selftest_wait_timeout(ns: int, stream=None):
+    _check("ttt_la_selftest_wait_timeout", lib().ttt_la_selftest_wait_timeout(int(ns), _stream_handle(stream)))

@@ -1,0 +1,372 @@
+// ttt_la.cu -- C ABI of libttt_la: argument checks, kernel selection and
+// launches for the causal TTT / linear-attention layer (see include/ttt_la.h).
+//
+// One translation unit holds every kernel so that the device status word is a
+// single symbol.  Host code never computes any part of the layer: it checks
+// arguments, builds TMA descriptors and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/ttt_la.h"
+#include "chunked_simt.cuh"
+#include "chunked_tc.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "recurrent.cuh"
+
+namespace {
+
+uint64_t g_limit_ns = 1000000000ull;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// ------------------------------------------------------------ TMA maps ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [BH][T][d] bf16 tensor, boxes of 64 elements x `rows` tokens, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int BH, int T, int d, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(T) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------ argument checks ----
+ttt_la_status check_seq(const ttt_la_args* a) {
+  if (!a) return TTT_LA_ERR_INVALID_ARG;
+  if (a->B < 1 || a->H < 1 || a->T < 1 || a->d_k < 1 || a->d_v < 1) return TTT_LA_ERR_INVALID_ARG;
+  if (a->dtype != TTT_LA_F32 && a->dtype != TTT_LA_BF16) return TTT_LA_ERR_INVALID_ARG;
+  if (!a->q || !a->k || !a->v || !a->o) return TTT_LA_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o)) return TTT_LA_ERR_INVALID_ARG;
+  if ((a->eta && !aligned16(a->eta)) || (a->state_in && !aligned16(a->state_in)) ||
+      (a->state_out && !aligned16(a->state_out)) || (a->mom_in && !aligned16(a->mom_in)) ||
+      (a->mom_out && !aligned16(a->mom_out)))
+    return TTT_LA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(a->B) * a->H;
+  if (bh > (1 << 30) || static_cast<long long>(a->T) * std::max(a->d_k, a->d_v) * bh > (1ll << 40))
+    return TTT_LA_ERR_INVALID_ARG;
+  if (!(a->beta >= 0.f && a->beta < 1.f) && a->beta != 0.f) return TTT_LA_ERR_INVALID_ARG;
+  if (a->o == a->q || a->o == a->k || a->o == a->v) return TTT_LA_ERR_INVALID_ARG;
+  return TTT_LA_OK;
+}
+
+ttt::SeqParams seq_params(const ttt_la_args* a) {
+  ttt::SeqParams p;
+  p.B = a->B;
+  p.H = a->H;
+  p.T = a->T;
+  p.dk = a->d_k;
+  p.dv = a->d_v;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.eta = a->eta;
+  p.eta_const = a->eta_const;
+  p.beta = a->beta;
+  p.sigma = a->ascent ? -1.f : 1.f;
+  p.S_in = a->state_in;
+  p.S_out = a->state_out;
+  p.M_in = a->mom_in;
+  p.M_out = a->mom_out;
+  p.o = a->o;
+  return p;
+}
+
+ttt_la_status launched() { return cudaGetLastError() == cudaSuccess ? TTT_LA_OK : TTT_LA_ERR_CUDA; }
+
+// ------------------------------------------------------------ recurrent ----
+template <int DK, typename T, bool MOM>
+ttt_la_status launch_recurrent(const ttt_la_args* a, cudaStream_t st) {
+  using Sh = ttt::RecurrentShape<DK>;
+  dim3 grid(a->B * a->H, (a->d_v + Sh::ROWS - 1) / Sh::ROWS);
+  ttt::recurrent_kernel<DK, T, MOM><<<grid, 128, 0, st>>>(seq_params(a));
+  return launched();
+}
+template <typename T, bool MOM>
+ttt_la_status recurrent_dk(const ttt_la_args* a, cudaStream_t st) {
+  switch (a->d_k) {
+    case 32: return launch_recurrent<32, T, MOM>(a, st);
+    case 64: return launch_recurrent<64, T, MOM>(a, st);
+    case 128: return launch_recurrent<128, T, MOM>(a, st);
+    default: return TTT_LA_ERR_UNSUPPORTED;
+  }
+}
+
+// --------------------------------------------------------------- chunked ----
+struct SegPlan {
+  int nchunks, cps, nseg;
+};
+
+int tc_ctas_per_sm(int C, int D) { return (C == 64 && D == 64) ? 2 : 1; }
+
+SegPlan plan_segments(const ttt_la_args* a) {
+  SegPlan s;
+  const int C = a->chunk;
+  s.nchunks = (a->T + C - 1) / C;
+  const int bh = a->B * a->H;
+  int nseg;
+  if (a->segments > 0) {
+    nseg = a->segments;
+  } else {
+    const int target = sm_count() * tc_ctas_per_sm(C, a->d_k);
+    nseg = (target + bh - 1) / bh;
+  }
+  nseg = std::max(1, std::min(nseg, s.nchunks));
+  s.cps = (s.nchunks + nseg - 1) / nseg;
+  s.nseg = (s.nchunks + s.cps - 1) / s.cps;
+  return s;
+}
+
+bool tc_supported(const ttt_la_args* a) {
+  return a->dtype == TTT_LA_BF16 && a->d_k == a->d_v && (a->d_k == 64 || a->d_k == 128) &&
+         (a->chunk == 64 || a->chunk == 128) && a->beta == 0.f;
+}
+
+bool simt_supported(const ttt_la_args* a, ttt::SimtShape* sh) {
+  if (a->dtype != TTT_LA_F32) return false;
+  if (!(a->chunk == 16 || a->chunk == 32 || a->chunk == 64)) return false;
+  if (a->d_k > 128 || a->d_v > 128) return false;
+  const bool mom = a->beta != 0.f;
+  if (mom && (a->d_k > 64 || a->d_v > 64)) return false;
+  sh->C = a->chunk;
+  sh->dk = a->d_k;
+  sh->dv = a->d_v;
+  sh->mom = mom;
+  return sh->bytes() <= 227 * 1024;
+}
+
+template <int C, int D>
+ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
+  using C1 = ttt::TcCfg<C, D, false>;
+  using C3 = ttt::TcCfg<C, D, true>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C1::SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C3::SMEM) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
+  const int bh = a->B * a->H;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
+      !make_map(&mv, a->v, bh, a->T, D, C) || !make_map(&mo, a->o, bh, a->T, D, C))
+    return TTT_LA_ERR_CUDA;
+  ttt::TcParams p;
+  p.BH = bh;
+  p.T = a->T;
+  p.nchunks = sp.nchunks;
+  p.cps = sp.cps;
+  p.nseg = sp.nseg;
+  p.eta = a->eta;
+  p.eta_const = a->eta_const;
+  p.sigma = a->ascent ? -1.f : 1.f;
+  p.S_in = a->state_in;
+  p.ws = static_cast<float*>(a->workspace);
+  p.S_out = a->state_out;
+  p.limit_ns = g_limit_ns;
+  if (sp.nseg > 1) {
+    ttt::chunked_tc_kernel<C, D, false><<<bh * (sp.nseg - 1), 192, C1::SMEM, st>>>(mq, mk, mv, mo, p);
+    if (cudaGetLastError() != cudaSuccess) return TTT_LA_ERR_CUDA;
+    dim3 g((D * D + 255) / 256, bh);
+    ttt::segment_scan_kernel<<<g, 256, 0, st>>>(p.ws, a->state_in, sp.nseg, D * D);
+    if (cudaGetLastError() != cudaSuccess) return TTT_LA_ERR_CUDA;
+  }
+  ttt::chunked_tc_kernel<C, D, true><<<bh * sp.nseg, 192, C3::SMEM, st>>>(mq, mk, mv, mo, p);
+  return launched();
+}
+
+template <bool MOM>
+ttt_la_status launch_simt(const ttt_la_args* a, const ttt::SimtShape& sh, cudaStream_t st) {
+  static size_t attr_bytes = 0;
+  const size_t bytes = sh.bytes();
+  if (bytes > 48 * 1024 && bytes > attr_bytes) {
+    if (cudaFuncSetAttribute(ttt::chunked_simt_f32_kernel<MOM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes)) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_bytes = bytes;
+  }
+  ttt::chunked_simt_f32_kernel<MOM><<<a->B * a->H, 256, bytes, st>>>(seq_params(a), sh);
+  return launched();
+}
+
+size_t workspace_for(const ttt_la_args* a) {
+  if (!tc_supported(a)) return 0;
+  const SegPlan sp = plan_segments(a);
+  if (sp.nseg <= 1) return 0;
+  return static_cast<size_t>(a->B) * a->H * sp.nseg * a->d_v * a->d_k * sizeof(float);
+}
+
+// ---------------------------------------------------------------- decode ----
+template <int DK, typename T, bool MOM>
+ttt_la_status launch_decode(const ttt_la_decode_args* a, cudaStream_t st) {
+  constexpr int U = 4;
+  constexpr int RPW = 32 / (DK / 4);
+  ttt::DecodeParams p;
+  p.N = a->N;
+  p.H = a->H;
+  p.dk = a->d_k;
+  p.dv = a->d_v;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.eta = a->eta;
+  p.eta_const = a->eta_const;
+  p.beta = a->beta;
+  p.sigma = a->ascent ? -1.f : 1.f;
+  p.S = a->state;
+  p.M = a->mom;
+  p.o = a->o;
+  const long long rows = static_cast<long long>(a->N) * a->H * a->d_v;
+  const long long warps = (rows + RPW * U - 1) / (RPW * U);
+  const long long blocks_needed = (warps + 7) / 8;
+  const int blocks = static_cast<int>(std::min<long long>(blocks_needed, static_cast<long long>(sm_count()) * 8));
+  ttt::decode_step_kernel<DK, T, MOM, U><<<blocks, 256, 0, st>>>(p);
+  return launched();
+}
+template <typename T, bool MOM>
+ttt_la_status decode_dk(const ttt_la_decode_args* a, cudaStream_t st) {
+  switch (a->d_k) {
+    case 32: return launch_decode<32, T, MOM>(a, st);
+    case 64: return launch_decode<64, T, MOM>(a, st);
+    case 128: return launch_decode<128, T, MOM>(a, st);
+    default: return TTT_LA_ERR_UNSUPPORTED;
+  }
+}
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    ttt::mbar_init(&bar, 1);
+    ttt::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ttt::mbar_wait(&bar, 0, limit_ns);  // nothing ever arrives
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ttt_la_status_string(ttt_la_status s) {
+  switch (s) {
+    case TTT_LA_OK: return "ok";
+    case TTT_LA_ERR_INVALID_ARG: return "invalid argument";
+    case TTT_LA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TTT_LA_ERR_CUDA: return "CUDA error";
+    case TTT_LA_ERR_TIMEOUT: return "in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* ttt_la_version(void) { return "ttt_la 0.1 (sm_100a)"; }
+
+ttt_la_status ttt_la_set_wait_limit_ns(int64_t limit_ns) {
+  if (limit_ns < 1000) return TTT_LA_ERR_INVALID_ARG;
+  g_limit_ns = static_cast<uint64_t>(limit_ns);
+  return TTT_LA_OK;
+}
+
+size_t ttt_la_workspace_size(const ttt_la_args* a) {
+  if (check_seq(a) != TTT_LA_OK) return 0;
+  return workspace_for(a);
+}
+
+ttt_la_status ttt_la_forward_chunked(const ttt_la_args* a, void* stream) {
+  ttt_la_status s = check_seq(a);
+  if (s != TTT_LA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool mom = a->beta != 0.f;
+  ttt::SimtShape sh;
+  if (a->dtype == TTT_LA_F32) {
+    if (!simt_supported(a, &sh)) return TTT_LA_ERR_UNSUPPORTED;
+    return mom ? launch_simt<true>(a, sh, st) : launch_simt<false>(a, sh, st);
+  }
+  if (!tc_supported(a)) return TTT_LA_ERR_UNSUPPORTED;
+  if (a->eta == nullptr && !(a->eta_const == a->eta_const)) return TTT_LA_ERR_INVALID_ARG;
+  const SegPlan sp = plan_segments(a);
+  if (sp.nseg > 1) {
+    const size_t need = static_cast<size_t>(a->B) * a->H * sp.nseg * a->d_v * a->d_k * sizeof(float);
+    if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace)) return TTT_LA_ERR_INVALID_ARG;
+  }
+  if (a->d_k == 64) return a->chunk == 64 ? launch_tc<64, 64>(a, sp, st) : launch_tc<128, 64>(a, sp, st);
+  return a->chunk == 64 ? launch_tc<64, 128>(a, sp, st) : launch_tc<128, 128>(a, sp, st);
+}
+
+ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {
+  ttt_la_status s = check_seq(a);
+  if (s != TTT_LA_OK) return s;
+  if (a->d_v > 1024) return TTT_LA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool mom = a->beta != 0.f;
+  if (a->dtype == TTT_LA_F32)
+    return mom ? recurrent_dk<float, true>(a, st) : recurrent_dk<float, false>(a, st);
+  return mom ? recurrent_dk<__nv_bfloat16, true>(a, st) : recurrent_dk<__nv_bfloat16, false>(a, st);
+}
+
+ttt_la_status ttt_la_decode_step(const ttt_la_decode_args* a, void* stream) {
+  if (!a) return TTT_LA_ERR_INVALID_ARG;
+  if (a->N < 1 || a->H < 1 || a->d_k < 1 || a->d_v < 1) return TTT_LA_ERR_INVALID_ARG;
+  if (a->dtype != TTT_LA_F32 && a->dtype != TTT_LA_BF16) return TTT_LA_ERR_INVALID_ARG;
+  if (!a->q || !a->k || !a->v || !a->o || !a->state) return TTT_LA_ERR_INVALID_ARG;
+  const bool mom = a->beta != 0.f;
+  if (mom && !a->mom) return TTT_LA_ERR_INVALID_ARG;
+  if (!(a->beta >= 0.f && a->beta < 1.f)) return TTT_LA_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o) || !aligned16(a->state) ||
+      (a->mom && !aligned16(a->mom)) || (a->eta && !aligned16(a->eta)))
+    return TTT_LA_ERR_INVALID_ARG;
+  if (static_cast<long long>(a->N) * a->H * a->d_v >= (1ll << 31)) return TTT_LA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a->dtype == TTT_LA_F32) return mom ? decode_dk<float, true>(a, st) : decode_dk<float, false>(a, st);
+  return mom ? decode_dk<__nv_bfloat16, true>(a, st) : decode_dk<__nv_bfloat16, false>(a, st);
+}
+
+ttt_la_status ttt_la_get_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TTT_LA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ttt::g_status, sizeof(int)) != cudaSuccess) return TTT_LA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(ttt::g_status, &zero, sizeof(int)) != cudaSuccess) return TTT_LA_ERR_CUDA;
+  return v == 0 ? TTT_LA_OK : TTT_LA_ERR_TIMEOUT;
+}
+
+ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return TTT_LA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns));
+  return launched();
+}
+
+}  // extern "C"

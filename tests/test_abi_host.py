@@ -1,0 +1,161 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched):
+the library loads, exports every symbol include/ttt_la.h declares, the ctypes
+structs match the C layout, and bad arguments are rejected before launch."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "ttt_la.h")
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from test_layers_causal_b200 import _abi
+    from test_layers_causal_b200.build import build
+    build()
+    _abi.lib()
+    return _abi
+
+
+def declared_functions():
+    src = open(HDR).read()
+    return re.findall(r"TTT_LA_API\s+[\w\s\*]+?\b(ttt_la_\w+)\s*\(", src)
+
+
+def test_header_declares_entry_points():
+    names = set(declared_functions())
+    for n in ("ttt_la_forward_chunked", "ttt_la_forward_recurrent", "ttt_la_decode_step",
+              "ttt_la_workspace_size", "ttt_la_get_last_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(abi):
+    L = abi.lib()
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (ttt_la_\w+)", out))
+    assert set(declared_functions()) <= exported
+    assert {name for name, _, _ in abi.SIGNATURES} == set(declared_functions())
+
+
+def test_struct_layout_matches_c(abi):
+    """Compile a probe against the header with gcc and compare sizeof/offsetof."""
+    probe = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "ttt_la.h"
+#define P(T, f) printf(#T "." #f " %zu\n", offsetof(T, f))
+int main(void) {
+  printf("ttt_la_args %zu\n", sizeof(ttt_la_args));
+  printf("ttt_la_decode_args %zu\n", sizeof(ttt_la_decode_args));
+  P(ttt_la_args, q); P(ttt_la_args, eta); P(ttt_la_args, eta_const); P(ttt_la_args, segments);
+  P(ttt_la_args, state_in); P(ttt_la_args, o); P(ttt_la_args, workspace_bytes);
+  P(ttt_la_decode_args, q); P(ttt_la_decode_args, eta_const); P(ttt_la_decode_args, state);
+  P(ttt_la_decode_args, o);
+  return 0;
+}
+"""
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "probe.c")
+        exe = os.path.join(d, "probe")
+        open(c, "w").write(probe)
+        subprocess.run(["gcc", "-I" + os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        lines = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    vals = dict(l.split() for l in lines if l.strip())
+    assert int(vals["ttt_la_args"]) == ctypes.sizeof(abi.TttArgs)
+    assert int(vals["ttt_la_decode_args"]) == ctypes.sizeof(abi.TttDecodeArgs)
+    for key, v in vals.items():
+        if "." in key:
+            struct, field = key.split(".")
+            cls = abi.TttArgs if struct == "ttt_la_args" else abi.TttDecodeArgs
+            assert getattr(cls, field).offset == int(v), key
+
+
+def test_status_strings(abi):
+    L = abi.lib()
+    assert L.ttt_la_status_string(0) == b"ok"
+    assert b"timed out" in L.ttt_la_status_string(4)
+    assert b"sm_100a" in L.ttt_la_version()
+
+
+def _args(abi, **kw):
+    a = abi.TttArgs()
+    a.B, a.H, a.T, a.d_k, a.d_v, a.dtype = 1, 2, 100, 64, 64, abi.BF16
+    a.q, a.k, a.v, a.o = 0x10000, 0x20000, 0x30000, 0x40000  # never dereferenced on these paths
+    a.chunk, a.eta_const = 64, 0.125
+    for n, x in kw.items():
+        setattr(a, n, x)
+    return a
+
+
+@pytest.mark.parametrize("bad", [
+    dict(B=0), dict(T=0), dict(d_k=0), dict(dtype=7), dict(q=None), dict(o=None),
+    dict(q=0x10004), dict(eta=0x1008), dict(state_in=0x2004), dict(o=0x10000),
+    dict(beta=1.5), dict(beta=-0.5),
+])
+def test_invalid_arguments_rejected_before_launch(abi, bad):
+    L = abi.lib()
+    a = _args(abi, **bad)
+    assert L.ttt_la_forward_chunked(ctypes.byref(a), None) == abi.ERR_INVALID_ARG
+    assert L.ttt_la_forward_recurrent(ctypes.byref(a), None) == abi.ERR_INVALID_ARG
+    assert L.ttt_la_workspace_size(ctypes.byref(a)) == 0
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(d_k=96, d_v=96), dict(d_k=64, d_v=128), dict(chunk=32), dict(chunk=256),
+    dict(dtype=0, chunk=128), dict(dtype=0, d_k=256, d_v=256, chunk=64),
+    dict(dtype=0, d_k=128, d_v=128, beta=0.9, chunk=64),
+])
+def test_unsupported_combinations(abi, cfg):
+    L = abi.lib()
+    a = _args(abi, **cfg)
+    assert L.ttt_la_forward_chunked(ctypes.byref(a), None) == abi.ERR_UNSUPPORTED
+
+
+def test_recurrent_unsupported_head_dim(abi):
+    a = _args(abi, d_k=48, d_v=48)
+    assert abi.lib().ttt_la_forward_recurrent(ctypes.byref(a), None) == abi.ERR_UNSUPPORTED
+
+
+def test_decode_validation(abi):
+    L = abi.lib()
+    d = abi.TttDecodeArgs()
+    d.N, d.H, d.d_k, d.d_v, d.dtype = 4, 2, 128, 128, abi.BF16
+    d.q, d.k, d.v, d.o, d.state = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    d.beta = 0.9  # momentum without a buffer
+    assert L.ttt_la_decode_step(ctypes.byref(d), None) == abi.ERR_INVALID_ARG
+    d.beta, d.state = 0.0, 0x50008  # misaligned state
+    assert L.ttt_la_decode_step(ctypes.byref(d), None) == abi.ERR_INVALID_ARG
+    d.state, d.N = 0x50000, 0
+    assert L.ttt_la_decode_step(ctypes.byref(d), None) == abi.ERR_INVALID_ARG
+    assert L.ttt_la_decode_step(None, None) == abi.ERR_INVALID_ARG
+
+
+def test_workspace_query(abi):
+    L = abi.lib()
+    one_seq_long = _args(abi, B=1, H=1, T=65536, chunk=128)
+    ws = L.ttt_la_workspace_size(ctypes.byref(one_seq_long))
+    assert ws > 0 and ws % (64 * 64 * 4) == 0
+    many = _args(abi, B=64, H=16, T=256, chunk=64)  # enough sequences: no split
+    assert L.ttt_la_workspace_size(ctypes.byref(many)) == 0
+    fixed = _args(abi, B=1, H=1, T=64 * 10, chunk=64, segments=3)
+    assert L.ttt_la_workspace_size(ctypes.byref(fixed)) == 3 * 64 * 64 * 4
+    # short workspace is refused on the host
+    fixed.workspace, fixed.workspace_bytes = 0x60000, 100
+    assert L.ttt_la_forward_chunked(ctypes.byref(fixed), None) == abi.ERR_INVALID_ARG
+    assert L.ttt_la_set_wait_limit_ns(10) == abi.ERR_INVALID_ARG
+    assert L.ttt_la_selftest_wait_timeout(10, None) == abi.ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from test_layers_causal_b200 import _abi
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _abi.lib()

@@ -1,0 +1,214 @@
+"""GPU parity: every CUDA entry point against the float64 oracle on the same
+seeded inputs, through the C ABI.  Sizes span several chunks and a ragged
+last chunk; the full workloads are checked on sampled heads."""
+import math
+
+import pytest
+import torch
+
+from synth import CONFIGS, make_case, make_qkv
+from tests.gpu_util import assert_bf16, assert_f32, oracle_forward
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import test_layers_causal_b200 as ttt
+
+
+def _case(B, H, T, dk, dv, dtype, seed, token_eta=True, device="cuda"):
+    q, k, v, z = make_qkv((B, H), T, dk, dv, seed)
+    eta = (torch.sigmoid(z) / math.sqrt(dk)).float() if token_eta else None
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    q, k, v = (x.to(dt).contiguous() for x in (q, k, v))
+    return (q.to(device), k.to(device), v.to(device), None if eta is None else eta.to(device),
+            1.0 / math.sqrt(dk))
+
+
+def _state(B, H, dv, dk, seed, scale=0.3):
+    g = torch.Generator().manual_seed(seed)
+    return (scale * torch.randn(B, H, dv, dk, generator=g)).cuda()
+
+
+# ------------------------------------------------------------- decode ----
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("beta,ascent", [(0.0, False), (0.9, False), (0.0, True), (0.5, True)])
+def test_decode_step_parity(dtype, d, beta, ascent):
+    N, H = 5, 3
+    q, k, v, eta, ec = _case(N, H, 1, d, d, dtype, 20 + d)
+    q, k, v, eta = q[:, :, 0].contiguous(), k[:, :, 0].contiguous(), v[:, :, 0].contiguous(), eta[:, :, 0].contiguous()
+    S0 = _state(N, H, d, d, 1)
+    M0 = _state(N, H, d, d, 2) if beta else None
+    S, M = S0.clone(), (M0.clone() if M0 is not None else None)
+    o = ttt.decode_step(q, k, v, S, M, eta=eta, beta=beta, ascent=ascent)
+    o_ref, S_ref, M_ref = oracle_forward(q[:, :, None], k[:, :, None], v[:, :, None], eta[:, :, None], ec,
+                                         beta, ascent, S0, M0)
+    assert_f32(o.float(), o_ref[:, :, 0], "o") if dtype == "f32" else assert_bf16(o, o_ref[:, :, 0], "o", lead=1)
+    assert_f32(S, S_ref, "state")
+    if beta:
+        assert_f32(M, M_ref, "momentum")
+
+
+# ---------------------------------------------------------- recurrent ----
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("beta", [0.0, 0.9])
+def test_recurrent_parity(dtype, d, beta):
+    B, H, T = 2, 2, 203
+    q, k, v, eta, ec = _case(B, H, T, d, d, dtype, 30 + d)
+    S0 = _state(B, H, d, d, 3)
+    M0 = _state(B, H, d, d, 4) if beta else None
+    o, S, M = ttt.forward_recurrent(q, k, v, eta, beta=beta, state_in=S0, mom_in=M0)
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, ec, beta, False, S0, M0)
+    if dtype == "f32":
+        assert_f32(o, o_ref, "o")
+    else:
+        assert_bf16(o, o_ref, "o")
+    assert_f32(S, S_ref, "state") if dtype == "f32" else assert_bf16(S, S_ref, "state")
+    if beta:
+        assert_f32(M, M_ref, "momentum") if dtype == "f32" else assert_bf16(M, M_ref, "momentum")
+
+
+def test_recurrent_ascent_and_const_eta():
+    q, k, v, _, ec = _case(1, 3, 77, 64, 64, "f32", 5, token_eta=False)
+    o, S, _ = ttt.forward_recurrent(q, k, v, None, eta_const=ec, ascent=True)
+    o_ref, S_ref, _ = oracle_forward(q, k, v, None, ec, 0.0, True)
+    assert_f32(o, o_ref, "o")
+    assert_f32(S, S_ref, "state")
+
+
+# ------------------------------------------------------ chunked, fp32 ----
+def test_chunked_f32_tiny_config():
+    c = CONFIGS["tiny_f32"]
+    x = make_case(c)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, S, _ = ttt.forward_chunked(q, k, v, None, eta_const=x["eta_const"], chunk=c.chunk)
+    o_ref, S_ref, _ = oracle_forward(q, k, v, None, x["eta_const"])
+    assert_f32(o, o_ref, "o")
+    assert_f32(S, S_ref, "state")
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("beta", [0.0, 0.9])
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 48), (16, 64)])
+def test_chunked_f32_parity(chunk, beta, dk, dv):
+    B, H, T = 2, 2, 150
+    q, k, v, eta, ec = _case(B, H, T, dk, dv, "f32", 40 + chunk)
+    S0 = _state(B, H, dv, dk, 5)
+    M0 = _state(B, H, dv, dk, 6) if beta else None
+    o, S, M = ttt.forward_chunked(q, k, v, eta, beta=beta, chunk=chunk, state_in=S0, mom_in=M0, ascent=True)
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, ec, beta, True, S0, M0)
+    assert_f32(o, o_ref, "o")
+    assert_f32(S, S_ref, "state")
+    if beta:
+        assert_f32(M, M_ref, "momentum")
+
+
+def test_chunked_f32_d128_no_momentum():
+    q, k, v, eta, ec = _case(1, 2, 130, 128, 128, "f32", 9)
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=64)
+    o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec)
+    assert_f32(o, o_ref, "o")
+    assert_f32(S, S_ref, "state")
+
+
+# ------------------------------------------- chunked, bf16 tensor cores ----
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("chunk", [64, 128])
+@pytest.mark.parametrize("segments", [1, 3])
+@pytest.mark.parametrize("token_eta", [True, False])
+def test_chunked_tc_parity(d, chunk, segments, token_eta):
+    B, H, T = 2, 3, 5 * chunk + 37  # several chunks and a ragged tail
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 50 + d + chunk, token_eta)
+    S0 = _state(B, H, d, d, 7, scale=0.1)
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, eta_const=ec, chunk=chunk, segments=segments, state_in=S0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec, 0.0, False, S0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+
+
+@pytest.mark.parametrize("d,chunk", [(64, 64), (128, 128)])
+def test_chunked_tc_ascent_zero_state_and_exact_multiple(d, chunk):
+    B, H, T = 1, 2, 4 * chunk
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 60 + d, True)
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=chunk, ascent=True, segments=2)
+    o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec, 0.0, True)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+
+
+def test_chunked_tc_short_sequences():
+    """T shorter than a chunk, T = 1, and T one past a chunk boundary."""
+    for T in (1, 17, 65):
+        q, k, v, eta, ec = _case(2, 2, T, 64, 64, "bf16", 70 + T)
+        o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=64)
+        o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec)
+        assert_bf16(o, o_ref, f"o T={T}")
+        assert_bf16(S, S_ref, f"state T={T}")
+
+
+def test_chunked_tc_query_is_key():
+    q, k, v, eta, ec = _case(1, 2, 300, 128, 128, "bf16", 80)
+    o, _, _ = ttt.forward_chunked(k, k, v, eta, chunk=128, segments=2)
+    o_ref, _, _ = oracle_forward(k, k, v, eta, ec)
+    assert_bf16(o, o_ref, "o")
+
+
+def test_chunked_segments_and_recurrent_agree():
+    """Invariants on the GPU: the result does not depend on the segment split,
+    and the chunked and recurrent paths compute the same layer."""
+    q, k, v, eta, ec = _case(2, 2, 1000, 64, 64, "bf16", 90)
+    o1, S1, _ = ttt.forward_chunked(q, k, v, eta, chunk=64, segments=1)
+    o5, S5, _ = ttt.forward_chunked(q, k, v, eta, chunk=64, segments=5)
+    orr, Sr, _ = ttt.forward_recurrent(q, k, v, eta)
+    o1, o5, orr = o1.float(), o5.float(), orr.float()
+    assert (o1 - o5).norm() / o1.norm() < 1e-2
+    assert (S1 - S5).norm() / S1.norm() < 1e-2
+    assert (o1 - orr).norm() / orr.norm() < 2e-2
+
+
+# ------------------------------------------------ full-size workloads ----
+def _full_case(name, heads):
+    c = CONFIGS[name]
+    x = make_case(c)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    eta = x["eta"].cuda() if x["eta"] is not None else None
+    return c, x, q, k, v, eta, heads
+
+
+@pytest.mark.parametrize("name,heads", [("llm_d64", [(0, 0), (3, 15), (1, 7)]), ("long_d128", [(0, 0), (0, 5)])])
+def test_full_size_sampled_heads(name, heads):
+    c, x, q, k, v, eta, heads = _full_case(name, heads)
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=c.chunk)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    for b, h in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        o_ref, S_ref, _ = oracle_forward(q[sl], k[sl], v[sl], None if eta is None else eta[sl], x["eta_const"],
+                                         c.beta)
+        assert_bf16(o[sl], o_ref, f"o {name} head {b},{h}")
+        assert_bf16(S[sl], S_ref, f"state {name} head {b},{h}")
+
+
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_long_context_chunk_sweep_consistent(chunk):
+    """The long-context workload at every swept chunk size gives the same layer."""
+    c, x, q, k, v, eta, _ = _full_case("long_d128", [])
+    o, S, _ = ttt.forward_chunked(q, k, v, None, eta_const=x["eta_const"], chunk=chunk)
+    o_ref, S_ref, _ = ttt.forward_chunked(q, k, v, None, eta_const=x["eta_const"], chunk=128, segments=1)
+    assert (o.float() - o_ref.float()).norm() / o_ref.float().norm() < 1e-2
+    assert (S - S_ref).norm() / S_ref.norm() < 1e-2
+
+
+# ---------------------------------------------------- bounded waits ----
+def test_wait_timeout_is_reported_not_hung():
+    assert ttt.device_status() == 0
+    ttt.selftest_wait_timeout(20_000_000)  # 20 ms on a barrier nothing completes
+    assert ttt.device_status() == 4        # TTT_LA_ERR_TIMEOUT, read and cleared
+    assert ttt.device_status() == 0
+    # the context is still usable
+    q, k, v, eta, ec = _case(1, 1, 64, 64, 64, "bf16", 3)
+    o, _, _ = ttt.forward_chunked(q, k, v, eta, chunk=64)
+    assert torch.isfinite(o.float()).all()
