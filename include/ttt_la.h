@@ -68,7 +68,8 @@ typedef enum {
   TTT_LA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, short workspace */
   TTT_LA_ERR_UNSUPPORTED = 2,  /* valid but not built: (d_k, d_v, chunk, dtype) combination */
   TTT_LA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
-  TTT_LA_ERR_TIMEOUT = 4       /* a bounded in-kernel wait ran out (device status word) */
+  TTT_LA_ERR_TIMEOUT = 4,      /* a bounded in-kernel wait ran out (device status word) */
+  TTT_LA_ERR_SCRATCH_LIMIT = 5 /* ttt_la_forward_chunked_noalloc: scratch need exceeds its fixed array */
 } ttt_la_status;
 
 typedef enum { TTT_LA_F32 = 0, TTT_LA_BF16 = 1 } ttt_la_dtype;
@@ -131,6 +132,30 @@ typedef struct ttt_la_decode_args {
 } ttt_la_decode_args;
 
 TTT_LA_API ttt_la_status ttt_la_decode_step(const ttt_la_decode_args *args, void *stream);
+
+/* Chunked forward for callers that cannot allocate device memory.  Some
+ * callers only ever receive their input and output buffers: a plugin running
+ * inside another engine's memory plan, or code whose device memory is owned
+ * entirely by someone else's pool, has no way to call cudaMalloc (and
+ * latency-critical callers avoid it because it can synchronise the device).
+ * This variant computes exactly what ttt_la_forward_chunked computes, but its
+ * scratch is a fixed array inside the library instead of args->workspace
+ * (which is ignored):
+ *  - the array holds TTT_LA_STATIC_SCRATCH_BYTES (8 MiB) and lives on every
+ *    GPU that loads the library until the process exits;
+ *  - a call whose ttt_la_workspace_size(args) exceeds it returns
+ *    TTT_LA_ERR_SCRATCH_LIMIT with nothing launched (use the allocating entry
+ *    point, or fewer segments, for such shapes);
+ *  - the first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture;
+ *  - every call on a device shares the one array, and the array keeps the last
+ *    call's contents: calls whose executions overlap on the GPU (different
+ *    streams, no ordering between them) race on it.  Whatever must start at
+ *    zero is cleared by the call itself.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * The paper has no counterpart of this entry point; it exists for callers. */
+#define TTT_LA_STATIC_SCRATCH_BYTES (8u << 20)
+TTT_LA_API ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args *args, void *stream);
 
 /* Synchronises `stream`, returns the device status word (TTT_LA_OK or
  * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */

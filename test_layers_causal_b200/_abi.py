@@ -16,7 +16,8 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libttt_la.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = 0, 1, 2, 3, 4, 5
+STATIC_SCRATCH_BYTES = 8 << 20  # TTT_LA_STATIC_SCRATCH_BYTES
 F32, BF16 = 0, 1
 
 _c_i32, _c_f32, _c_vp, _c_sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -47,6 +48,7 @@ class TttDecodeArgs(ctypes.Structure):
 SIGNATURES = [
     ("ttt_la_workspace_size", _c_sz, [ctypes.POINTER(TttArgs)]),
     ("ttt_la_forward_chunked", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
+    ("ttt_la_forward_chunked_noalloc", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
     ("ttt_la_forward_recurrent", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
     ("ttt_la_decode_step", ctypes.c_int, [ctypes.POINTER(TttDecodeArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),

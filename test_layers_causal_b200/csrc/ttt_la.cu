@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/ttt_la.h"
 #include "chunked_simt.cuh"
@@ -266,6 +267,29 @@ ttt_la_status decode_dk(const ttt_la_decode_args* a, cudaStream_t st) {
   }
 }
 
+// Scratch of ttt_la_forward_chunked_noalloc: one fixed array per device,
+// shared by every call on that device (see include/ttt_la.h).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TTT_LA_STATIC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// symbol names a host-side stand-in, never the device array, so the address is
+// looked up with cudaGetSymbolAddress once per device (that device current)
+// and cached.  Returns nullptr when the lookup fails.
+void* noalloc_scratch_ptr() {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* ptrs[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -288,6 +312,7 @@ const char* ttt_la_status_string(ttt_la_status s) {
     case TTT_LA_ERR_UNSUPPORTED: return "unsupported configuration";
     case TTT_LA_ERR_CUDA: return "CUDA error";
     case TTT_LA_ERR_TIMEOUT: return "in-kernel wait timed out";
+    case TTT_LA_ERR_SCRATCH_LIMIT: return "scratch need exceeds the fixed no-alloc array";
   }
   return "unknown status";
 }
@@ -324,6 +349,23 @@ ttt_la_status ttt_la_forward_chunked(const ttt_la_args* a, void* stream) {
   }
   if (a->d_k == 64) return a->chunk == 64 ? launch_tc<64, 64>(a, sp, st) : launch_tc<128, 64>(a, sp, st);
   return a->chunk == 64 ? launch_tc<64, 128>(a, sp, st) : launch_tc<128, 128>(a, sp, st);
+}
+
+ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args* a, void* stream) {
+  ttt_la_status s = check_seq(a);
+  if (s != TTT_LA_OK) return s;
+  const size_t need = workspace_for(a);
+  if (need > TTT_LA_STATIC_SCRATCH_BYTES) return TTT_LA_ERR_SCRATCH_LIMIT;
+  ttt_la_args b = *a;
+  b.workspace = nullptr;
+  b.workspace_bytes = 0;
+  if (need > 0) {
+    void* p = noalloc_scratch_ptr();
+    if (!p) return TTT_LA_ERR_CUDA;
+    b.workspace = p;
+    b.workspace_bytes = TTT_LA_STATIC_SCRATCH_BYTES;
+  }
+  return ttt_la_forward_chunked(&b, stream);
 }
 
 ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {
