@@ -167,16 +167,22 @@ bool simt_supported(const ttt_la_args* a, ttt::SimtShape* sh) {
   return sh->bytes() <= 227 * 1024;
 }
 
+// Scratch layout of the chunked tensor-core path: fp32 [BH][nseg][2][d_v][d_k]
+// (segment totals, inclusive states), then nseg*BH publication flags and one
+// tile counter (uint32), which every call clears before its launch.
+size_t tc_ws_floats(int bh, int nseg, int D) { return static_cast<size_t>(bh) * nseg * 2 * D * D; }
+size_t tc_ws_bytes(int bh, int nseg, int D) {
+  const size_t b = tc_ws_floats(bh, nseg, D) * sizeof(float) + (static_cast<size_t>(bh) * nseg + 1) * sizeof(unsigned);
+  return (b + 15) & ~static_cast<size_t>(15);
+}
+
 template <int C, int D>
 ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
-  using C1 = ttt::TcCfg<C, D, false>;
-  using C3 = ttt::TcCfg<C, D, true>;
+  using Cfg = ttt::TcCfg<C, D>;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C1::SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C3::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+        cudaSuccess)
       return TTT_LA_ERR_CUDA;
     attr_done = true;
   }
@@ -195,17 +201,17 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
   p.eta_const = a->eta_const;
   p.sigma = a->ascent ? -1.f : 1.f;
   p.S_in = a->state_in;
-  p.ws = static_cast<float*>(a->workspace);
+  p.ws = nullptr;
+  p.flags = nullptr;
   p.S_out = a->state_out;
   p.limit_ns = g_limit_ns;
   if (sp.nseg > 1) {
-    ttt::chunked_tc_kernel<C, D, false><<<bh * (sp.nseg - 1), 192, C1::SMEM, st>>>(mq, mk, mv, mo, p);
-    if (cudaGetLastError() != cudaSuccess) return TTT_LA_ERR_CUDA;
-    dim3 g((D * D + 255) / 256, bh);
-    ttt::segment_scan_kernel<<<g, 256, 0, st>>>(p.ws, a->state_in, sp.nseg, D * D);
-    if (cudaGetLastError() != cudaSuccess) return TTT_LA_ERR_CUDA;
+    p.ws = static_cast<float*>(a->workspace);
+    p.flags = reinterpret_cast<unsigned*>(p.ws + tc_ws_floats(bh, sp.nseg, D));
+    if (cudaMemsetAsync(p.flags, 0, (static_cast<size_t>(bh) * sp.nseg + 1) * sizeof(unsigned), st) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
   }
-  ttt::chunked_tc_kernel<C, D, true><<<bh * sp.nseg, 192, C3::SMEM, st>>>(mq, mk, mv, mo, p);
+  ttt::chunked_tc_kernel<C, D><<<bh * sp.nseg, 224, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
   return launched();
 }
 
@@ -227,7 +233,7 @@ size_t workspace_for(const ttt_la_args* a) {
   if (!tc_supported(a)) return 0;
   const SegPlan sp = plan_segments(a);
   if (sp.nseg <= 1) return 0;
-  return static_cast<size_t>(a->B) * a->H * sp.nseg * a->d_v * a->d_k * sizeof(float);
+  return tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k);
 }
 
 // ---------------------------------------------------------------- decode ----
@@ -344,7 +350,7 @@ ttt_la_status ttt_la_forward_chunked(const ttt_la_args* a, void* stream) {
   if (a->eta == nullptr && !(a->eta_const == a->eta_const)) return TTT_LA_ERR_INVALID_ARG;
   const SegPlan sp = plan_segments(a);
   if (sp.nseg > 1) {
-    const size_t need = static_cast<size_t>(a->B) * a->H * sp.nseg * a->d_v * a->d_k * sizeof(float);
+    const size_t need = tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k);
     if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace)) return TTT_LA_ERR_INVALID_ARG;
   }
   if (a->d_k == 64) return a->chunk == 64 ? launch_tc<64, 64>(a, sp, st) : launch_tc<128, 64>(a, sp, st);

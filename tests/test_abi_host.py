@@ -139,13 +139,19 @@ def test_decode_validation(abi):
 
 def test_workspace_query(abi):
     L = abi.lib()
+    def expected(bh, nseg, d):  # fp32 [bh][nseg][2][d][d], then bh*nseg flags + 1 counter
+        b = bh * nseg * 2 * d * d * 4 + (bh * nseg + 1) * 4
+        return (b + 15) // 16 * 16
+
     one_seq_long = _args(abi, B=1, H=1, T=65536, chunk=128)
     ws = L.ttt_la_workspace_size(ctypes.byref(one_seq_long))
-    assert ws > 0 and ws % (64 * 64 * 4) == 0
+    assert ws > 0 and ws % 16 == 0
     many = _args(abi, B=64, H=16, T=256, chunk=64)  # enough sequences: no split
     assert L.ttt_la_workspace_size(ctypes.byref(many)) == 0
-    fixed = _args(abi, B=1, H=1, T=64 * 10, chunk=64, segments=3)
-    assert L.ttt_la_workspace_size(ctypes.byref(fixed)) == 3 * 64 * 64 * 4
+    fixed = _args(abi, B=1, H=1, T=64 * 10, chunk=64, segments=3)  # 10 chunks -> 4+4+2
+    assert L.ttt_la_workspace_size(ctypes.byref(fixed)) == expected(1, 3, 64)
+    fixed4 = _args(abi, B=2, H=3, T=64 * 10, chunk=64, segments=4)  # 10 chunks -> 3+3+3+1
+    assert L.ttt_la_workspace_size(ctypes.byref(fixed4)) == expected(6, 4, 64)
     # short workspace is refused on the host
     fixed.workspace, fixed.workspace_bytes = 0x60000, 100
     assert L.ttt_la_forward_chunked(ctypes.byref(fixed), None) == abi.ERR_INVALID_ARG
