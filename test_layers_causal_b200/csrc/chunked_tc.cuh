@@ -23,11 +23,12 @@
 //   phase B: the chunk loop above from W_start(p); K and V come back from L2
 //           (phase A just read them), Q from HBM.
 //
-// Block = 7 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the
-// MMAs (one thread), warps 2-5 (128 threads, one TMEM lane each) scale K by
-// the learning rate, mask scores, convert fp32 accumulators into bf16
-// operands and stage O, warp 6 stores O with TMA.  Per phase-B chunk the MMA
-// thread issues
+// Block = 8 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the
+// MMAs (one thread, descriptors precomputed), warps 2-5 (128 threads, one
+// TMEM lane each) mask scores, convert fp32 accumulators into bf16 operands
+// and stage O, warp 6 stores O with TMA, warp 7 scales every K tile by the
+// learning rate as it lands (fetching eta two chunks ahead).  Per phase-B
+// chunk the MMA thread issues
 //   (1) Sc    = Q K~^T              [TMEM, M=C,   N=C]
 //   (2) O[b]  = Q Wbf^T             [TMEM, M=C,   N=d_v]   Wbf = bf16(W) in smem
 //   (3) W    += V^T K~              [TMEM, M=d_v, N=d_k]   (after Wbf was taken)
@@ -85,6 +86,12 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int C, int kk) {
   return sdesc_sw128(base + static_cast<uint32_t>(kk * 2048), static_cast<uint32_t>(C * 128), 1024);
 }
 
+// Offsets (in the descriptor's 16-byte address units) of k-step kk.
+__host__ __device__ constexpr uint64_t k_step(int rows, int kk) {
+  return static_cast<uint64_t>(((kk >> 2) * rows * 128 + (kk & 3) * 32) >> 4);
+}
+__host__ __device__ constexpr uint64_t mn_step(int kk) { return static_cast<uint64_t>(kk * 2048 >> 4); }
+
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -126,7 +133,7 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int blk, int row
 }
 
 template <int C, int D>
-__global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
+__global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
     chunked_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                       const TcParams p) {
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BIG);
   uint64_t* full = bars;                // [NST] TMA landed
-  uint64_t* kready = bars + NST;        // [NST] K scaled by the epilogue
+  uint64_t* kready = bars + NST;        // [NST] K scaled by the scaler warp
   uint64_t* empty = bars + 2 * NST;     // [NST] stage free
   uint64_t* staged = bars + 3 * NST;    // [NST] O of phase-B chunk it staged (index it % NST)
   uint64_t* sc_full = bars + 4 * NST;   // scores in TMEM
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&kready[s], 128);
+      mbar_init(&kready[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&staged[s], 128);
     }
@@ -235,43 +242,47 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
       constexpr uint32_t ID_O_QW = idesc_bf16_f32(C, D, false, false);
       constexpr uint32_t ID_W = idesc_bf16_f32(D, D, true, true);
       constexpr uint32_t ID_O_PV = idesc_bf16_f32(C, D, false, true);
+      // Descriptors are built once per tile and advanced by constant offsets
+      // (the start address is the low field; no carry leaves it below 256 KB).
+      const uint64_t d_wbf = sdesc_sw128(sbase + NST * STAGE, 16, 1024);
       // phase A: segment total of V^T K~
       for (int g = 0; g < nA; ++g) {
         const int s = g % NST;
         const uint32_t stk = sbase + s * STAGE + TILE, stv = stk + TILE;
+        const uint64_t dkm = sdesc_sw128(stk, C * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
         if (!dead) dead = !mbar_wait(&kready[s], (g / NST) & 1, lim);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          mma_bf16_ss(t_w, desc_mn(stv, C, kk), desc_mn(stk, C, kk), ID_W, (g > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ss(t_w, dvm + mn_step(kk), dkm + mn_step(kk), ID_W, (g > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&empty[s]);
       }
       if (nA > 0) tc_commit(sdone);
       // phase B
-      const uint32_t sbf_a = sbase + NST * STAGE;
       for (int it = 0; it < nB; ++it) {
         const int g = nA + it, s = g % NST, b = it & 1;
         const uint32_t stq = sbase + s * STAGE, stk = stq + TILE, stv = stq + 2 * TILE;
+        const uint64_t dq = sdesc_sw128(stq, 16, 1024), dkk = sdesc_sw128(stk, 16, 1024);
+        const uint64_t dkm = sdesc_sw128(stk, C * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
         const uint32_t t_o = t_o0 + b * D;
         if (!dead) dead = !mbar_wait(&kready[s], (g / NST) & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(t_sc, desc_k(stq, C, kk), desc_k(stk, C, kk), ID_SC, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_sc, dq + k_step(C, kk), dkk + k_step(C, kk), ID_SC, kk > 0);
         tc_commit(sc_full);
         if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
         if (it >= 2 && !dead) dead = !mbar_wait(&o_free[b], ((it - 2) >> 1) & 1, lim);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(t_o, desc_k(stq, C, kk), desc_k(sbf_a, D, kk), ID_O_QW, kk > 0);
+          mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_QW, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_w, desc_mn(stv, C, kk), desc_mn(stk, C, kk), ID_W, 1);
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_w, dvm + mn_step(kk), dkm + mn_step(kk), ID_W, 1);
         tc_commit(sdone);
         if (!dead) dead = !mbar_wait(p_ready, it & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, desc_k(stq, C, kk), desc_mn(stv, C, kk), ID_O_PV, 1);
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, dq + k_step(C, kk), dvm + mn_step(kk), ID_O_PV, 1);
         tc_commit(&o_full[b]);
       }
       tc_commit(drain);
@@ -294,6 +305,64 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
       }
       bulk_wait0();
     }
+  } else if (warp == 7) {
+    // ------------------------------------------------------- K scaler --
+    // K~ = diag(sigma * eta) K for every tile as it lands (phase A and B),
+    // in place, swizzle-aware; eta is fetched two chunks ahead.
+    bool dead = false;
+    constexpr int RPL = C / 32;  // rows of a chunk whose eta this lane fetches
+    const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
+    auto fetch = [&](int g, float (&dst)[RPL]) {
+      const int c0 = (chunk0 + (g >= nA ? g - nA : g)) * C;
+#pragma unroll
+      for (int j = 0; j < RPL; ++j) {
+        const int t = c0 + lane + 32 * j;
+        dst[j] = (g < NI && t < p.T) ? (eg ? __ldg(eg + t) : p.eta_const) : 0.f;
+      }
+    };
+    float er[RPL], en[RPL];
+    fetch(0, er);
+    fetch(1, en);
+    constexpr int PER_LANE = C * (D / 8) / 32;  // 16-byte units of the K tile per lane
+    constexpr int BATCH = 8;
+    for (int g = 0; g < NI; ++g) {
+      const int s = g % NST;
+      float* ess = es + s * C;
+#pragma unroll
+      for (int j = 0; j < RPL; ++j) ess[lane + 32 * j] = p.sigma * er[j];
+#pragma unroll
+      for (int j = 0; j < RPL; ++j) er[j] = en[j];
+      fetch(g + 2, en);
+      __syncwarp();
+      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
+      uint8_t* sk = smem + s * STAGE + TILE;
+#pragma unroll 1
+      for (int b0 = 0; b0 < PER_LANE; b0 += BATCH) {
+        uint4 u[BATCH];
+        uint32_t off[BATCH];
+        float e[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int idx = lane + 32 * (b0 + i);
+          const int r = idx / (D / 8), cc = idx % (D / 8);
+          off[i] = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
+          e[i] = ess[r];
+          u[i] = *reinterpret_cast<const uint4*>(sk + off[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          float2 a;
+          a = unpack_bf16x2(u[i].x); u[i].x = pack_bf16x2(a.x * e[i], a.y * e[i]);
+          a = unpack_bf16x2(u[i].y); u[i].y = pack_bf16x2(a.x * e[i], a.y * e[i]);
+          a = unpack_bf16x2(u[i].z); u[i].z = pack_bf16x2(a.x * e[i], a.y * e[i]);
+          a = unpack_bf16x2(u[i].w); u[i].w = pack_bf16x2(a.x * e[i], a.y * e[i]);
+          *reinterpret_cast<uint4*>(sk + off[i]) = u[i];
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&kready[s]);
+    }
   } else {
     // --------------------------------------------------------- epilogue --
     const int et = threadIdx.x - 64;               // 0..127
@@ -306,47 +375,7 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
     const bool wrow_ok = (D == 128) || ok64;
     const int qrow = (C == 128) ? row128 : row64;  // query row of scores / O
     const bool qrow_ok = (C == 128) || ok64;
-    const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
     bool dead = false;
-
-    auto chunk_of = [&](int g) { return chunk0 + (g >= nA ? g - nA : g); };
-    auto eta_at = [&](int g) {
-      const int t = chunk_of(g) * C + et;
-      return (et < C && g < NI && t < p.T) ? p.sigma * (eg ? __ldg(eg + t) : p.eta_const) : 0.f;
-    };
-    float e_pref = eta_at(0);
-
-    // K~ = diag(sigma * eta) K for iteration g, in place, then kready
-    auto scale_k = [&](int g) {
-      const int s = g % NST;
-      uint8_t* sk = smem + s * STAGE + TILE;
-      float* ess = es + s * C;
-      if (et < C) ess[et] = e_pref;
-      e_pref = eta_at(g + 1);
-      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int idx = et; idx < C * (D / 8); idx += 128) {
-        const int r = idx / (D / 8), cc = idx % (D / 8);
-        uint4* ptr = reinterpret_cast<uint4*>(sk + (cc >> 3) * C * 128 + sw128_off(r, cc & 7));
-        uint4 u = *ptr;
-        const float e = ess[r];
-        float2 a;
-        a = unpack_bf16x2(u.x); u.x = pack_bf16x2(a.x * e, a.y * e);
-        a = unpack_bf16x2(u.y); u.y = pack_bf16x2(a.x * e, a.y * e);
-        a = unpack_bf16x2(u.z); u.z = pack_bf16x2(a.x * e, a.y * e);
-        a = unpack_bf16x2(u.w); u.w = pack_bf16x2(a.x * e, a.y * e);
-        *ptr = u;
-      }
-      fence_async_smem();
-      mbar_arrive(&kready[s]);
-    };
-
-    // ---------------------------------------------------------- phase A
-    for (int g = 0; g < nA; ++g) scale_k(g);
-
-    // Phase B's first stage is scaled before the look-back so the MMA can
-    // start the first score tile while the state is being assembled.
-    scale_k(nA);
 
     // --------------------------------------------- look-back, W_start
     {
@@ -373,22 +402,18 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) st_release(flag_me, 1u);
       }
-      if (et == 0) {
-        int first = 0, incl = -1;
-        for (int j = seg - 1; j >= 0; --j) {
-          const unsigned f = dead ? 2u : wait_flag(p.flags + bh * p.nseg + j, lim);
-          if (f == 0) dead = true;
-          if (f >= 2) {
-            incl = j;
-            first = j + 1;
-            break;
-          }
-        }
-        sh_lb[0] = first;
-        sh_lb[1] = incl;
+      // Every predecessor has published at least its total; the nearest one
+      // that has already published its inclusive state cuts the sum short.
+      // One thread per predecessor, so the flags are read in one round trip.
+      if (et == 0) sh_lb[1] = -1;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int j = et; j < seg; j += 128) {
+        const unsigned f = dead ? 1u : wait_flag(p.flags + bh * p.nseg + j, lim);
+        if (f == 0) dead = true;
+        if (f >= 2) atomicMax(&sh_lb[1], j);
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int first = sh_lb[0], incl = sh_lb[1];
+      const int incl = sh_lb[1], first = incl + 1;
       const float* base = nullptr;
       if (incl >= 0) base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
       else if (p.S_in) base = p.S_in + static_cast<size_t>(bh) * DD;
@@ -401,17 +426,40 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
           const size_t off = static_cast<size_t>(wrow) * D + cb * 32;
           if (base) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 x = __ldcg(reinterpret_cast<const float4*>(base + off) + j);
-              acc[4 * j] = x.x; acc[4 * j + 1] = x.y; acc[4 * j + 2] = x.z; acc[4 * j + 3] = x.w;
+            for (int j = 0; j < 4; ++j) {
+              const float8 x = ld_cg_v8(base + off + 8 * j);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[8 * j + e] = x.v[e];
             }
           }
-          for (int jj = first; jj < seg; ++jj) {
-            const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off;
+          // four totals per round: 16 independent 32-byte (full-sector) loads in flight
+          int jj = first;
+          for (; jj + 4 <= seg; jj += 4) {
+            float8 x[4][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 x = __ldcg(reinterpret_cast<const float4*>(ag) + j);
-              acc[4 * j] += x.x; acc[4 * j + 1] += x.y; acc[4 * j + 2] += x.z; acc[4 * j + 3] += x.w;
+            for (int u = 0; u < 4; ++u) {
+              const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD + off;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) x[u][j] = ld_cg_v8(ag + 8 * j);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[u][j].v[e];
+              }
+            }
+          }
+          for (; jj < seg; ++jj) {
+            const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off;
+            float8 x[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[j] = ld_cg_v8(ag + 8 * j);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[j].v[e];
             }
           }
         }
@@ -455,16 +503,20 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
         if (!dead) dead = !mbar_wait(sc_full, it & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < C / 32; ++cb) {
-          uint32_t r[32];
-          tmem_ld32(t_sc + lane_off + cb * 32, r);
+        for (int cb = 0; cb < C / 32; cb += 2) {
+          uint32_t r[2][32];
+          tmem_ld32(t_sc + lane_off + cb * 32, r[0]);
+          tmem_ld32(t_sc + lane_off + cb * 32 + 32, r[1]);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int col = cb * 32 + j;
-            const float a0 = (col <= qrow) ? __uint_as_float(r[j]) : 0.f;
-            const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[j + 1]) : 0.f;
-            pk[(cb * 32 + j) >> 1] = pack_bf16x2(a0, a1);
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const int col = (cb + h) * 32 + j;
+              const float a0 = (col <= qrow) ? __uint_as_float(r[h][j]) : 0.f;
+              const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[h][j + 1]) : 0.f;
+              pk[col >> 1] = pack_bf16x2(a0, a1);
+            }
           }
         }
         if (!dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);  // Q, K slots and Wbf no longer read
@@ -479,16 +531,19 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
         tc_fence_before();
         mbar_arrive(p_ready);
       }
-      // next chunk: scale its K and take its Wbf while (4) runs
+      // next chunk's Wbf (W after this chunk's (3)) while (4) runs
       if (it + 1 < nB) {
-        scale_k(g + 1);
         tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t r[32];
-          tmem_ld32(t_w + lane_off + cb * 32, r);
+        for (int cb = 0; cb < D / 32; cb += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_w + lane_off + cb * 32, r0);
+          tmem_ld32(t_w + lane_off + cb * 32 + 32, r1);
           tmem_ld_wait();
-          if (wrow_ok) store_row32_bf16(sbf, D * 128, wrow, cb * 32, r);
+          if (wrow_ok) {
+            store_row32_bf16(sbf, D * 128, wrow, cb * 32, r0);
+            store_row32_bf16(sbf, D * 128, wrow, cb * 32 + 32, r1);
+          }
         }
         fence_async_smem();
         tc_fence_before();
@@ -501,11 +556,15 @@ __global__ void __launch_bounds__(224, TcCfg<C, D>::MINB)
         tc_fence_after();
         const uint32_t t_o = t_o0 + b * D;
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t r[32];
-          tmem_ld32(t_o + lane_off + cb * 32, r);
+        for (int cb = 0; cb < D / 32; cb += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_o + lane_off + cb * 32, r0);
+          tmem_ld32(t_o + lane_off + cb * 32 + 32, r1);
           tmem_ld_wait();
-          if (qrow_ok) store_row32_bf16(sv, C * 128, qrow, cb * 32, r);
+          if (qrow_ok) {
+            store_row32_bf16(sv, C * 128, qrow, cb * 32, r0);
+            store_row32_bf16(sv, C * 128, qrow, cb * 32 + 32, r1);
+          }
         }
         tc_fence_before();
         mbar_arrive(&o_free[b]);

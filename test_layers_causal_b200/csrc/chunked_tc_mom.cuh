@@ -1,0 +1,640 @@
+// chunked_tc_mom.cuh -- chunk-parallel forward with SGD momentum on the sm_100a
+// tensor cores (Variant 3 of Table 2 in the thelatestinai.com listing of
+// "Test-Time Training with KV Binding Is Secretly Linear Attention": a single
+// linear fast weight, per-token learning rate, momentum in SGD).
+//
+// The recurrence M_t = beta M_{t-1} - sigma v_t k_t^T, W_t = W_{t-1} - eta_t M_t,
+// o_t = W_t q_t regroups exactly over a tile of C tokens (local i, j; n valid):
+//   c_ij = sum_{r=j..i} eta_r beta^(r-j)                        (j <= i)
+//   o_i  = W q_i - g_i M q_i + sigma sum_{j<=i} c_ij (q_i . k_j) v_j,  g_i = beta c_i0
+//   W'   = W - g_{n-1} M + sigma sum_j c_{n-1,j} v_j k_j^T
+//   M'   = beta^n M - sigma sum_j beta^(n-1-j) v_j k_j^T
+// The coefficients come from the tile's suffix sums cl_j = c_{C-1,j} (a warp
+// scan, no division): c_ij = cl_j - beta^(i+1-j) cl_{i+1}.  Unlike the
+// factorisation beta^-j (P_i - P_{j-1}), whose cancellation grows like
+// beta^-C, this one loses at most a factor ~1/(1-beta) for positive eta.
+//
+// Structure as in chunked_tc.cuh (one launch, segments, look-back), with the
+// pair (W, M) as the carried state: a segment acts on it as the affine map
+//   (W, M) -> (W - G M + dW, B M + dM),
+// G = beta * (segment suffix coefficient at its first token), B = beta^L.
+// Phase A walks the segment's tiles backwards so the suffix coefficients carry
+// from tile to tile; the look-back composes the published maps.  Tiles are 64
+// tokens (a 128-token request runs as two 64-token tiles: the same layer),
+// which keeps Q, K, V stages, bf16 copies of W and M, the two scaled K tiles,
+// Q~ = diag(-g) Q and P within shared memory.
+//
+// Per phase-B tile the MMA thread issues
+//   (1) Sc  = Q K^T                       [unscaled K]
+//   (2) O   = Q Wbf^T + Q~ Mbf^T
+//   (3) W  += V^T K1,  M += V^T K2        K1 = diag(sigma c_{n-1,.}) K, K2 = diag(-sigma beta^(n-1-.)) K
+//   (4) O  += P V                         P = bf16(sigma c * Sc), masked
+// after the epilogue has replaced W by W - g_{n-1} M and M by beta^n M in TMEM.
+#pragma once
+#include "common.cuh"
+#include "chunked_tc.cuh"
+
+namespace ttt {
+
+struct TcMomParams {
+  int BH, T, nchunks, cps, nseg;
+  const float* eta;
+  float eta_const, sigma, beta;
+  const float* S_in;   // [BH, dv, dk] or nullptr
+  const float* M_in;   // [BH, dv, dk] or nullptr
+  float* ws;           // [BH, nseg, 4, dv, dk]: dW, dM, W_incl, M_incl
+  float* wsc;          // [BH, nseg, 2]: G, B of each segment map
+  unsigned* flags;     // [BH * nseg] flags, then a tile counter
+  float* S_out;
+  float* M_out;
+  uint64_t limit_ns;
+};
+
+template <int D>
+struct TcMomCfg {
+  static constexpr int C = 64;
+  static constexpr int TILE = C * D * 2;         // bf16 C x D
+  static constexpr int STAGE = 3 * TILE;         // Q, K, V
+  static constexpr int NST = 2;
+  static constexpr int SQ = D * D * 2;           // bf16 D x D
+  static constexpr int OFF_WBF = NST * STAGE;
+  static constexpr int OFF_MBF = OFF_WBF + SQ;
+  static constexpr int OFF_K1 = OFF_MBF + SQ;
+  static constexpr int OFF_K2 = OFF_K1 + TILE;
+  static constexpr int OFF_QT = OFF_K2 + TILE;
+  static constexpr int OFF_P = OFF_QT + TILE;
+  static constexpr int BIG = OFF_P + C * C * 2;
+  static constexpr int NBAR = 3 * NST + 16;
+  static constexpr int SMALL = NBAR * 8 + (NST * (C + 1) + (C + 1) + 8) * 4 + 32;
+  static constexpr int SMEM = BIG + SMALL + 1024;
+  static constexpr int TCOLS_USED = C + 3 * D;   // scores, O, W, M
+  static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
+  static constexpr int MINB = 1;
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+template <int D>
+__global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
+    chunked_tc_mom_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                          const TcMomParams p) {
+  using Cfg = TcMomCfg<D>;
+  constexpr int C = Cfg::C, NST = Cfg::NST, TILE = Cfg::TILE, STAGE = Cfg::STAGE;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BIG);
+  uint64_t* full = bars;               // [NST]
+  uint64_t* empty = bars + NST;        // [NST]
+  uint64_t* staged = bars + 2 * NST;   // [NST] (indexed by phase-B tile % NST)
+  uint64_t* kt_ready = bars + 3 * NST; // scaled K1/K2 (and the tile's cl) ready
+  uint64_t* kt_free = kt_ready + 1;    // (3) of the previous tile done: K1/K2 buffers free
+  uint64_t* sc_full = kt_ready + 2;
+  uint64_t* sdone = kt_ready + 3;      // (2),(3) done / phase-A totals done
+  uint64_t* wbf_ready = kt_ready + 4;  // Wbf, Mbf, Q~ written; W, M rewritten in TMEM
+  uint64_t* p_ready = kt_ready + 5;
+  uint64_t* o_full = kt_ready + 6;
+  uint64_t* seg_ready = kt_ready + 7; // phase-A segment scalars G, B written
+  uint64_t* drain = kt_ready + 8;
+  float* cls = reinterpret_cast<float*>(smem + Cfg::BIG + Cfg::NBAR * 8);  // [NST][C+1] tile suffix sums
+  float* bp = cls + NST * (C + 1);                                          // beta^k, k = 0..C
+  float* segsc = bp + (C + 1);                                              // [0] G, [1] B of this segment
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(segsc + 8);
+  int* sh_tile = reinterpret_cast<int*>(tmem_holder + 1);
+  int* sh_lb = sh_tile + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&staged[s], 128);
+    }
+    mbar_init(kt_ready, 1);
+    mbar_init(kt_free, 1);
+    mbar_init(sc_full, 1);
+    mbar_init(sdone, 1);
+    mbar_init(wbf_ready, 128);
+    mbar_init(p_ready, 128);
+    mbar_init(o_full, 1);
+    mbar_init(seg_ready, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    float b = 1.f;
+    for (int k = 0; k <= C; ++k) {
+      bp[k] = b;
+      b *= p.beta;
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::TCOLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0)
+    *sh_tile = p.flags ? static_cast<int>(atomicAdd(p.flags + p.BH * p.nseg, 1u)) : static_cast<int>(blockIdx.x);
+  __syncthreads();
+  const uint32_t tmem = *tmem_holder;
+  const int tile = *sh_tile;
+  const int seg = tile / p.BH, bh = tile % p.BH;
+  const int chunk0 = seg * p.cps;
+  const int nch = min(p.cps, p.nchunks - chunk0);
+  const int nA = (p.nseg > 1 && seg < p.nseg - 1) ? nch : 0;
+  const int nB = nch;
+  const int NI = nA + nB;
+  // tile of iteration g: phase A walks the segment backwards, phase B forwards
+  auto tile_of = [&](int g) { return chunk0 + (g < nA ? nA - 1 - g : g - nA); };
+  const uint32_t t_w = tmem;            // W: D columns, M = D
+  const uint32_t t_m = tmem + D;        // M: D columns, M = D
+  const uint32_t t_o = tmem + 2 * D;    // O: D columns, M = C
+  const uint32_t t_sc = tmem + 3 * D;   // scores: C columns, M = C
+  uint8_t* wbf = smem + Cfg::OFF_WBF;
+  uint8_t* mbf = smem + Cfg::OFF_MBF;
+  uint8_t* k1s = smem + Cfg::OFF_K1;
+  uint8_t* k2s = smem + Cfg::OFF_K2;
+  uint8_t* qts = smem + Cfg::OFF_QT;
+  uint8_t* ps = smem + Cfg::OFF_P;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      bool dead = false;
+      for (int g = 0; g < NI; ++g) {
+        const int s = g % NST;
+        if (g >= NST && !dead) dead = !mbar_wait(&empty[s], ((g / NST) - 1) & 1, lim);
+        const bool pb = g >= nA;
+        const int t0 = tile_of(g) * C;
+        mbar_arrive_expect_tx(&full[s], pb ? 3 * TILE : 2 * TILE);
+        uint8_t* st = smem + s * STAGE;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) {
+          if (pb) tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmK, &full[s], st + TILE + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmV, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, t0, bh);
+        }
+      }
+      for (int g = max(0, NI - NST); g < NI; ++g) mbar_wait(&full[g % NST], (g / NST) & 1, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      bool dead = false;
+      constexpr uint32_t ID_SC = idesc_bf16_f32(C, C, false, false);
+      constexpr uint32_t ID_O_K = idesc_bf16_f32(C, D, false, false);
+      constexpr uint32_t ID_W = idesc_bf16_f32(D, D, true, true);
+      constexpr uint32_t ID_O_PV = idesc_bf16_f32(C, D, false, true);
+      const uint64_t d_wbf = sdesc_sw128(sbase + Cfg::OFF_WBF, 16, 1024);
+      const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
+      const uint64_t d_k1 = sdesc_sw128(sbase + Cfg::OFF_K1, C * 128, 1024);
+      const uint64_t d_k2 = sdesc_sw128(sbase + Cfg::OFF_K2, C * 128, 1024);
+      const uint64_t d_qt = sdesc_sw128(sbase + Cfg::OFF_QT, 16, 1024);
+      const uint64_t d_p = sdesc_sw128(sbase + Cfg::OFF_P, 16, 1024);
+      for (int g = 0; g < NI; ++g) {
+        const int s = g % NST;
+        const uint32_t stq = sbase + s * STAGE, stv = stq + 2 * TILE;
+        const uint64_t dvm = sdesc_sw128(stv, C * 128, 1024);
+        if (g < nA) {
+          // segment totals: dW += V^T K1, dM += V^T K2 (fresh at g == 0)
+          if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) {
+            const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
+            mma_bf16_ss(t_w, dvm + mn_step(kk), d_k1 + mn_step(kk), ID_W, acc);
+            mma_bf16_ss(t_m, dvm + mn_step(kk), d_k2 + mn_step(kk), ID_W, acc);
+          }
+          tc_commit(&empty[s]);
+          tc_commit(kt_free);
+          if (g == nA - 1) tc_commit(sdone);
+          continue;
+        }
+        const int it = g - nA;
+        const uint64_t dq = sdesc_sw128(stq, 16, 1024), dkk = sdesc_sw128(stq + TILE, 16, 1024);
+        if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_sc, dq + k_step(C, kk), dkk + k_step(C, kk), ID_SC, kk > 0);
+        tc_commit(sc_full);
+        if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);
+        if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_K, kk > 0);
+          mma_bf16_ss(t_o, d_qt + k_step(C, kk), d_mbf + k_step(D, kk), ID_O_K, 1);
+        }
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16_ss(t_w, dvm + mn_step(kk), d_k1 + mn_step(kk), ID_W, 1);
+          mma_bf16_ss(t_m, dvm + mn_step(kk), d_k2 + mn_step(kk), ID_W, 1);
+        }
+        tc_commit(sdone);
+        tc_commit(kt_free);
+        if (!dead) dead = !mbar_wait(p_ready, it & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, d_p + k_step(C, kk), dvm + mn_step(kk), ID_O_PV, 1);
+        tc_commit(o_full);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, lim);
+    }
+  } else if (warp == 6) {
+    // ----------------------------------------------------- O store warp --
+    if (lane == 0) {
+      bool dead = false;
+      for (int it = 0; it < nB; ++it) {
+        const int g = nA + it, s = g % NST;
+        if (!dead) dead = !mbar_wait(&staged[it % NST], (it / NST) & 1, lim);
+        const uint8_t* sv = smem + s * STAGE + 2 * TILE;
+        const int t0 = (chunk0 + it) * C;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) tma_store_3d(&tmO, sv + kb * C * 128, kb * 64, t0, bh);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait0();
+    }
+  } else if (warp == 7) {
+    // ------------------------------------- coefficients and K scaling --
+    bool dead = false;
+    const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
+    const float beta = p.beta, sigma = p.sigma;
+    float R = 0.f, Bc = 1.f;  // phase A carries: suffix coefficient after this tile, beta^(tokens after it)
+    for (int g = 0; g < NI; ++g) {
+      const int s = g % NST;
+      const int t0 = tile_of(g) * C;
+      // eta of rows 2*lane, 2*lane+1 (0 past the sequence end)
+      float e0 = 0.f, e1 = 0.f;
+      {
+        const int ta = t0 + 2 * lane, tb = ta + 1;
+        if (ta < p.T) e0 = eg ? __ldg(eg + ta) : p.eta_const;
+        if (tb < p.T) e1 = eg ? __ldg(eg + tb) : p.eta_const;
+      }
+      // suffix scan over the tile: value at row 2*lane given zero beyond the tile
+      float a = e0 + beta * e1, m = beta * beta;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float ah = __shfl_down_sync(0xffffffffu, a, off);
+        const float mh = __shfl_down_sync(0xffffffffu, m, off);
+        if (lane + off < 32) {
+          a = fmaf(m, ah, a);
+          m *= mh;
+        }
+      }
+      float an = __shfl_down_sync(0xffffffffu, a, 1);
+      if (lane == 31) an = 0.f;
+      const float cl0 = a, cl1 = fmaf(beta, an, e1);  // cl at rows 2*lane, 2*lane+1
+      float* cl = cls + s * (C + 1);
+      cl[2 * lane] = cl0;
+      cl[2 * lane + 1] = cl1;
+      if (lane == 0) cl[C] = 0.f;
+      __syncwarp();
+      // per-row weights of the two scaled K tiles
+      float w1a, w1b, w2a, w2b;
+      if (g < nA) {
+        w1a = sigma * fmaf(bp[C - 2 * lane], R, cl0);
+        w1b = sigma * fmaf(bp[C - 2 * lane - 1], R, cl1);
+        w2a = -sigma * bp[C - 1 - 2 * lane] * Bc;
+        w2b = -sigma * bp[C - 2 - 2 * lane] * Bc;
+        R = fmaf(bp[C], R, __shfl_sync(0xffffffffu, cl0, 0));
+        Bc *= bp[C];
+        if (g == nA - 1 && lane == 0) {
+          segsc[0] = beta * R;  // G: beta * suffix coefficient at the segment's first token
+          segsc[1] = Bc;        // B = beta^L
+          mbar_arrive(seg_ready);
+        }
+      } else {
+        const int n = min(C, p.T - t0);
+        w1a = sigma * cl0;
+        w1b = sigma * cl1;
+        w2a = (2 * lane < n) ? -sigma * bp[n - 1 - 2 * lane] : 0.f;
+        w2b = (2 * lane + 1 < n) ? -sigma * bp[n - 2 - 2 * lane] : 0.f;
+      }
+      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
+      if (g > 0 && !dead) dead = !mbar_wait(kt_free, (g - 1) & 1, lim);
+      // K1 = diag(w1) K, K2 = diag(w2) K; row r's weights live in lane r/2
+      const uint8_t* sk = smem + s * STAGE + TILE;
+      constexpr int PER_LANE = C * (D / 8) / 32;
+#pragma unroll 4
+      for (int i = 0; i < PER_LANE; ++i) {
+        const int idx = lane + 32 * i;
+        const int r = idx / (D / 8), cc = idx % (D / 8);
+        const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
+        const int src = r >> 1;
+        const float x1a = __shfl_sync(0xffffffffu, w1a, src), x1b = __shfl_sync(0xffffffffu, w1b, src);
+        const float x2a = __shfl_sync(0xffffffffu, w2a, src), x2b = __shfl_sync(0xffffffffu, w2b, src);
+        const float f1 = (r & 1) ? x1b : x1a, f2 = (r & 1) ? x2b : x2a;
+        const uint4 u = *reinterpret_cast<const uint4*>(sk + off);
+        uint4 v1, v2;
+        float2 t;
+        t = unpack_bf16x2(u.x); v1.x = pack_bf16x2(t.x * f1, t.y * f1); v2.x = pack_bf16x2(t.x * f2, t.y * f2);
+        t = unpack_bf16x2(u.y); v1.y = pack_bf16x2(t.x * f1, t.y * f1); v2.y = pack_bf16x2(t.x * f2, t.y * f2);
+        t = unpack_bf16x2(u.z); v1.z = pack_bf16x2(t.x * f1, t.y * f1); v2.z = pack_bf16x2(t.x * f2, t.y * f2);
+        t = unpack_bf16x2(u.w); v1.w = pack_bf16x2(t.x * f1, t.y * f1); v2.w = pack_bf16x2(t.x * f2, t.y * f2);
+        *reinterpret_cast<uint4*>(k1s + off) = v1;
+        *reinterpret_cast<uint4*>(k2s + off) = v2;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(kt_ready);
+    }
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int et = threadIdx.x - 64;
+    const int g4 = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
+    const int row128 = 32 * g4 + lane;
+    const int row64 = 16 * g4 + lane;
+    const bool ok64 = lane < 16;
+    const int wrow = (D == 128) ? row128 : row64;
+    const bool wrow_ok = (D == 128) || ok64;
+    const int qrow = row64;  // C = 64
+    const bool qrow_ok = ok64;
+    const float beta = p.beta, sigma = p.sigma;
+    bool dead = false;
+    const size_t DD = static_cast<size_t>(D) * D;
+
+    // ---- phase A result and look-back
+    {
+      float* me = p.ws ? p.ws + (static_cast<size_t>(bh) * p.nseg + seg) * 4 * DD : nullptr;
+      unsigned* flag_me = p.flags ? p.flags + bh * p.nseg + seg : nullptr;
+      if (nA > 0) {
+        if (!dead) dead = !mbar_wait(sdone, 0, lim);
+        if (!dead) dead = !mbar_wait(seg_ready, 0, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t tq = q ? t_m : t_w;
+#pragma unroll
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t r[32];
+            tmem_ld32(tq + lane_off + cb * 32, r);
+            tmem_ld_wait();
+            if (wrow_ok) {
+              float4* d4 = reinterpret_cast<float4*>(me + q * DD + static_cast<size_t>(wrow) * D + cb * 32);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+            }
+          }
+        }
+        if (et == 0) {
+          p.wsc[(static_cast<size_t>(bh) * p.nseg + seg) * 2 + 0] = segsc[0];
+          p.wsc[(static_cast<size_t>(bh) * p.nseg + seg) * 2 + 1] = segsc[1];
+        }
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) st_release(flag_me, 1u);
+      }
+      if (et == 0) sh_lb[1] = -1;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int j = et; j < seg; j += 128) {
+        const unsigned f = dead ? 1u : wait_flag(p.flags + bh * p.nseg + j, lim);
+        if (f == 0) dead = true;
+        if (f >= 2) atomicMax(&sh_lb[1], j);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int incl = sh_lb[1], first = incl + 1;
+      const float *bw = nullptr, *bm = nullptr;
+      if (incl >= 0) {
+        bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 4 + 2) * DD;
+        bm = bw + DD;
+      } else {
+        if (p.S_in) bw = p.S_in + static_cast<size_t>(bh) * DD;
+        if (p.M_in) bm = p.M_in + static_cast<size_t>(bh) * DD;
+      }
+      const float Gme = (nA > 0) ? segsc[0] : 0.f, Bme = (nA > 0) ? segsc[1] : 1.f;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        float w[32], mm[32];
+        const size_t off = static_cast<size_t>(wrow) * D + cb * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = mm[j] = 0.f;
+        if (wrow_ok) {
+          if (bw) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float8 x = ld_cg_v8(bw + off + 8 * j);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) w[8 * j + e] = x.v[e];
+            }
+          }
+          if (bm) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float8 x = ld_cg_v8(bm + off + 8 * j);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) mm[8 * j + e] = x.v[e];
+            }
+          }
+          // apply the published segment maps in order
+          for (int jj = first; jj < seg; ++jj) {
+            const float* dw = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 4 * DD + off;
+            const float* dm = dw + DD;
+            const float G = __ldcg(p.wsc + (static_cast<size_t>(bh) * p.nseg + jj) * 2);
+            const float B = __ldcg(p.wsc + (static_cast<size_t>(bh) * p.nseg + jj) * 2 + 1);
+            float8 xw[4], xm[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              xw[j] = ld_cg_v8(dw + 8 * j);
+              xm[j] = ld_cg_v8(dm + 8 * j);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int c = 8 * j + e;
+                w[c] = fmaf(-G, mm[c], w[c]) + xw[j].v[e];
+                mm[c] = fmaf(B, mm[c], xm[j].v[e]);
+              }
+            }
+          }
+        }
+        uint32_t r[32], r2[32];
+        if (nA > 0) {  // inclusive state after this segment, from its totals in TMEM
+          tmem_ld32(t_w + lane_off + cb * 32, r);
+          tmem_ld32(t_m + lane_off + cb * 32, r2);
+          tmem_ld_wait();
+          if (wrow_ok) {
+            float* iw = me + 2 * DD + off;
+            float* im = me + 3 * DD + off;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              iw[j] = fmaf(-Gme, mm[j], w[j]) + __uint_as_float(r[j]);
+              im[j] = fmaf(Bme, mm[j], __uint_as_float(r2[j]));
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          r[j] = __float_as_uint(w[j]);
+          r2[j] = __float_as_uint(mm[j]);
+        }
+        tmem_st32(t_w + lane_off + cb * 32, r);
+        tmem_st32(t_m + lane_off + cb * 32, r2);
+      }
+      tmem_st_wait();
+      if (nA > 0) {
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) st_release(flag_me, 2u);
+      }
+    }
+
+    // ---- phase B
+    for (int it = 0; it < nB; ++it) {
+      const int g = nA + it, s = g % NST;
+      const int t0 = (chunk0 + it) * C;
+      const int n = min(C, p.T - t0);
+      uint8_t* st = smem + s * STAGE;
+      const float* cl = cls + s * (C + 1);
+      // Step W: Wbf, Mbf from the state entering this tile; W -= g_end M; M *= beta^n; Q~ = diag(-g) Q
+      if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);  // the tile's cl is in smem
+      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);  // its Q has landed
+      if (it > 0 && !dead) dead = !mbar_wait(sdone, ((nA > 0 ? 1 : 0) + it - 1) & 1, lim);
+      tc_fence_after();
+      const float gend = beta * cl[0];
+      const float bn = bp[n];
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t r[32], r2[32];
+        tmem_ld32(t_w + lane_off + cb * 32, r);
+        tmem_ld32(t_m + lane_off + cb * 32, r2);
+        tmem_ld_wait();
+        if (wrow_ok) {
+          store_row32_bf16(wbf, D * 128, wrow, cb * 32, r);
+          store_row32_bf16(mbf, D * 128, wrow, cb * 32, r2);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float wv = __uint_as_float(r[j]), mv = __uint_as_float(r2[j]);
+          r[j] = __float_as_uint(fmaf(-gend, mv, wv));
+          r2[j] = __float_as_uint(bn * mv);
+        }
+        tmem_st32(t_w + lane_off + cb * 32, r);
+        tmem_st32(t_m + lane_off + cb * 32, r2);
+      }
+      if (qrow_ok) {
+        const float gi = beta * fmaf(-bp[qrow + 1], cl[qrow + 1], cl[0]);
+        const float f = -gi;
+#pragma unroll
+        for (int cc = 0; cc < D / 8; ++cc) {
+          const uint32_t off = (cc >> 3) * C * 128 + sw128_off(qrow, cc & 7);
+          const uint4 u = *reinterpret_cast<const uint4*>(st + off);
+          uint4 v;
+          float2 t;
+          t = unpack_bf16x2(u.x); v.x = pack_bf16x2(t.x * f, t.y * f);
+          t = unpack_bf16x2(u.y); v.y = pack_bf16x2(t.x * f, t.y * f);
+          t = unpack_bf16x2(u.z); v.z = pack_bf16x2(t.x * f, t.y * f);
+          t = unpack_bf16x2(u.w); v.w = pack_bf16x2(t.x * f, t.y * f);
+          *reinterpret_cast<uint4*>(qts + off) = v;
+        }
+      }
+      tmem_st_wait();
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(wbf_ready);
+
+      // Step P: P_ij = sigma * c_ij * Sc_ij for j <= i
+      {
+        if (!dead) dead = !mbar_wait(sc_full, it & 1, lim);
+        tc_fence_after();
+        uint32_t r[2][32];
+        tmem_ld32(t_sc + lane_off, r[0]);
+        tmem_ld32(t_sc + lane_off + 32, r[1]);
+        tmem_ld_wait();
+        if (qrow_ok) {
+          const float cnext = cl[qrow + 1];
+          uint32_t pk[C / 2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const int col = h * 32 + j;
+              float a0 = 0.f, a1 = 0.f;
+              if (col <= qrow) a0 = sigma * fmaf(-bp[qrow + 1 - col], cnext, cl[col]) * __uint_as_float(r[h][j]);
+              if (col + 1 <= qrow)
+                a1 = sigma * fmaf(-bp[qrow - col], cnext, cl[col + 1]) * __uint_as_float(r[h][j + 1]);
+              pk[col >> 1] = pack_bf16x2(a0, a1);
+            }
+          }
+#pragma unroll
+          for (int c16 = 0; c16 < C / 8; ++c16) {
+            const uint4 u = make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
+            *reinterpret_cast<uint4*>(ps + sw128_off(qrow, c16)) = u;
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+      }
+
+      // Step O
+      {
+        uint8_t* sv = st + 2 * TILE;
+        if (!dead) dead = !mbar_wait(o_full, it & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int cb = 0; cb < D / 32; cb += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_o + lane_off + cb * 32, r0);
+          tmem_ld32(t_o + lane_off + cb * 32 + 32, r1);
+          tmem_ld_wait();
+          if (qrow_ok) {
+            store_row32_bf16(sv, C * 128, qrow, cb * 32, r0);
+            store_row32_bf16(sv, C * 128, qrow, cb * 32 + 32, r1);
+          }
+        }
+        fence_async_smem();
+        mbar_arrive(&staged[it % NST]);
+      }
+    }
+
+    // final state (last segment)
+    if (seg == p.nseg - 1 && (p.S_out != nullptr || p.M_out != nullptr)) {
+      if (!dead) dead = !mbar_wait(sdone, ((nA > 0 ? 1 : 0) + nB - 1) & 1, lim);
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float* dst = q ? p.M_out : p.S_out;
+        const uint32_t tq = q ? t_m : t_w;
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t r[32];
+          tmem_ld32(tq + lane_off + cb * 32, r);
+          tmem_ld_wait();
+          if (dst && wrow_ok) {
+            float4* d4 = reinterpret_cast<float4*>(dst + static_cast<size_t>(bh) * DD + static_cast<size_t>(wrow) * D + cb * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::TCOLS);
+}
+
+}  // namespace ttt

@@ -15,6 +15,7 @@
 #include "../../include/ttt_la.h"
 #include "chunked_simt.cuh"
 #include "chunked_tc.cuh"
+#include "chunked_tc_mom.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "recurrent.cuh"
@@ -131,16 +132,21 @@ struct SegPlan {
 
 int tc_ctas_per_sm(int C, int D) { return (C == 64 && D == 64) ? 2 : 1; }
 
+// Tokens per tensor-core tile: the requested chunk, except with momentum, whose
+// kernel always runs 64-token tiles (a 128-token chunk is the same layer).
+int tc_tile(const ttt_la_args* a) { return a->beta != 0.f ? 64 : a->chunk; }
+
 SegPlan plan_segments(const ttt_la_args* a) {
   SegPlan s;
-  const int C = a->chunk;
+  const int C = tc_tile(a);
   s.nchunks = (a->T + C - 1) / C;
   const int bh = a->B * a->H;
   int nseg;
   if (a->segments > 0) {
     nseg = a->segments;
   } else {
-    const int target = sm_count() * tc_ctas_per_sm(C, a->d_k);
+    const int per_sm = a->beta != 0.f ? 1 : tc_ctas_per_sm(C, a->d_k);
+    const int target = sm_count() * per_sm;
     nseg = (target + bh - 1) / bh;
   }
   nseg = std::max(1, std::min(nseg, s.nchunks));
@@ -151,7 +157,7 @@ SegPlan plan_segments(const ttt_la_args* a) {
 
 bool tc_supported(const ttt_la_args* a) {
   return a->dtype == TTT_LA_BF16 && a->d_k == a->d_v && (a->d_k == 64 || a->d_k == 128) &&
-         (a->chunk == 64 || a->chunk == 128) && a->beta == 0.f;
+         (a->chunk == 64 || a->chunk == 128);
 }
 
 bool simt_supported(const ttt_la_args* a, ttt::SimtShape* sh) {
@@ -211,7 +217,7 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
     if (cudaMemsetAsync(p.flags, 0, (static_cast<size_t>(bh) * sp.nseg + 1) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
-  ttt::chunked_tc_kernel<C, D><<<bh * sp.nseg, 224, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
+  ttt::chunked_tc_kernel<C, D><<<bh * sp.nseg, 256, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
   return launched();
 }
 
@@ -229,11 +235,64 @@ ttt_la_status launch_simt(const ttt_la_args* a, const ttt::SimtShape& sh, cudaSt
   return launched();
 }
 
+// Momentum scratch: fp32 [BH][nseg][4][d_v][d_k] (dW, dM, W_incl, M_incl),
+// fp32 [BH][nseg][2] (G, B), then flags and the tile counter.
+size_t tcm_ws_floats(int bh, int nseg, int D) { return static_cast<size_t>(bh) * nseg * (4 * D * D + 2); }
+size_t tcm_ws_bytes(int bh, int nseg, int D) {
+  const size_t b = tcm_ws_floats(bh, nseg, D) * sizeof(float) + (static_cast<size_t>(bh) * nseg + 1) * sizeof(unsigned);
+  return (b + 15) & ~static_cast<size_t>(15);
+}
+
 size_t workspace_for(const ttt_la_args* a) {
   if (!tc_supported(a)) return 0;
   const SegPlan sp = plan_segments(a);
   if (sp.nseg <= 1) return 0;
-  return tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k);
+  return a->beta != 0.f ? tcm_ws_bytes(a->B * a->H, sp.nseg, a->d_k) : tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k);
+}
+
+template <int D>
+ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
+  using Cfg = ttt::TcMomCfg<D>;
+  constexpr int C = Cfg::C;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::chunked_tc_mom_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
+  const int bh = a->B * a->H;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
+      !make_map(&mv, a->v, bh, a->T, D, C) || !make_map(&mo, a->o, bh, a->T, D, C))
+    return TTT_LA_ERR_CUDA;
+  ttt::TcMomParams p;
+  p.BH = bh;
+  p.T = a->T;
+  p.nchunks = sp.nchunks;
+  p.cps = sp.cps;
+  p.nseg = sp.nseg;
+  p.eta = a->eta;
+  p.eta_const = a->eta_const;
+  p.sigma = a->ascent ? -1.f : 1.f;
+  p.beta = a->beta;
+  p.S_in = a->state_in;
+  p.M_in = a->mom_in;
+  p.ws = nullptr;
+  p.wsc = nullptr;
+  p.flags = nullptr;
+  p.S_out = a->state_out;
+  p.M_out = a->mom_out;
+  p.limit_ns = g_limit_ns;
+  if (sp.nseg > 1) {
+    p.ws = static_cast<float*>(a->workspace);
+    p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;
+    p.flags = reinterpret_cast<unsigned*>(p.ws + tcm_ws_floats(bh, sp.nseg, D));
+    if (cudaMemsetAsync(p.flags, 0, (static_cast<size_t>(bh) * sp.nseg + 1) * sizeof(unsigned), st) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+  }
+  ttt::chunked_tc_mom_kernel<D><<<bh * sp.nseg, 256, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
+  return launched();
 }
 
 // ---------------------------------------------------------------- decode ----
@@ -350,9 +409,10 @@ ttt_la_status ttt_la_forward_chunked(const ttt_la_args* a, void* stream) {
   if (a->eta == nullptr && !(a->eta_const == a->eta_const)) return TTT_LA_ERR_INVALID_ARG;
   const SegPlan sp = plan_segments(a);
   if (sp.nseg > 1) {
-    const size_t need = tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k);
+    const size_t need = workspace_for(a);
     if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace)) return TTT_LA_ERR_INVALID_ARG;
   }
+  if (mom) return a->d_k == 64 ? launch_tc_mom<64>(a, sp, st) : launch_tc_mom<128>(a, sp, st);
   if (a->d_k == 64) return a->chunk == 64 ? launch_tc<64, 64>(a, sp, st) : launch_tc<128, 64>(a, sp, st);
   return a->chunk == 64 ? launch_tc<64, 128>(a, sp, st) : launch_tc<128, 128>(a, sp, st);
 }

@@ -110,7 +110,7 @@ def test_invalid_arguments_rejected_before_launch(abi, bad):
 @pytest.mark.parametrize("cfg", [
     dict(d_k=96, d_v=96), dict(d_k=64, d_v=128), dict(chunk=32), dict(chunk=256),
     dict(dtype=0, chunk=128), dict(dtype=0, d_k=256, d_v=256, chunk=64),
-    dict(dtype=0, d_k=128, d_v=128, beta=0.9, chunk=64),
+    dict(dtype=0, d_k=128, d_v=128, beta=0.9, chunk=64), dict(beta=0.9, chunk=32),
 ])
 def test_unsupported_combinations(abi, cfg):
     L = abi.lib()

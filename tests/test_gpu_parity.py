@@ -156,6 +156,34 @@ def test_chunked_tc_query_is_key():
     assert_bf16(o, o_ref, "o")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("chunk", [64, 128])
+@pytest.mark.parametrize("segments", [1, 3])
+@pytest.mark.parametrize("beta,ascent", [(0.9, False), (0.5, True)])
+def test_chunked_tc_momentum_parity(d, chunk, segments, beta, ascent):
+    B, H, T = 2, 2, 6 * 64 + 23
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 100 + d + chunk)
+    S0 = _state(B, H, d, d, 8, scale=0.1)
+    M0 = _state(B, H, d, d, 9, scale=0.1)
+    o, S, M = ttt.forward_chunked(q, k, v, eta, beta=beta, ascent=ascent, chunk=chunk, segments=segments,
+                                  state_in=S0, mom_in=M0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, ec, beta, ascent, S0, M0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+    assert_bf16(M, M_ref, "momentum")
+
+
+def test_chunked_tc_momentum_const_eta_zero_state():
+    q, k, v, _, ec = _case(1, 3, 500, 128, 128, "bf16", 111, token_eta=False)
+    o, S, M = ttt.forward_chunked(q, k, v, None, eta_const=ec, beta=0.9, chunk=128, segments=2)
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, None, ec, 0.9)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+    assert_bf16(M, M_ref, "momentum")
+
+
 def test_chunked_segments_and_recurrent_agree():
     """Invariants on the GPU: the result does not depend on the segment split,
     and the chunked and recurrent paths compute the same layer."""
@@ -178,18 +206,21 @@ def _full_case(name, heads):
     return c, x, q, k, v, eta, heads
 
 
-@pytest.mark.parametrize("name,heads", [("llm_d64", [(0, 0), (3, 15), (1, 7)]), ("long_d128", [(0, 0), (0, 5)])])
+@pytest.mark.parametrize("name,heads", [("llm_d64", [(0, 0), (3, 15), (1, 7)]), ("long_d128", [(0, 0), (0, 5)]),
+                                        ("momentum_d128", [(0, 0), (1, 9)])])
 def test_full_size_sampled_heads(name, heads):
     c, x, q, k, v, eta, heads = _full_case(name, heads)
-    o, S, _ = ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=c.chunk)
+    o, S, M = ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=c.chunk)
     torch.cuda.synchronize()
     assert ttt.device_status() == 0
     for b, h in heads:
         sl = (slice(b, b + 1), slice(h, h + 1))
-        o_ref, S_ref, _ = oracle_forward(q[sl], k[sl], v[sl], None if eta is None else eta[sl], x["eta_const"],
-                                         c.beta)
+        o_ref, S_ref, M_ref = oracle_forward(q[sl], k[sl], v[sl], None if eta is None else eta[sl],
+                                             x["eta_const"], c.beta)
         assert_bf16(o[sl], o_ref, f"o {name} head {b},{h}")
         assert_bf16(S[sl], S_ref, f"state {name} head {b},{h}")
+        if c.beta:
+            assert_bf16(M[sl], M_ref, f"momentum {name} head {b},{h}")
 
 
 @pytest.mark.parametrize("chunk", [64, 128])
