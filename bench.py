@@ -195,10 +195,10 @@ def cpu_baseline(c, heads):
     dt, head_tokens = oracle_sample(c, heads)
     total_head_tokens = c.B * c.H * c.T
     t_full = dt * total_head_tokens / head_tokens
-    return {"value": c.B * c.T / t_full, "unit": "tokens/s", "cores": torch.get_num_threads(),
+    return {"value": c.B * c.T / t_full, "unit": "tokens/s", "cores": 1,
             "kind": "oracle",
             "sample": f"{heads} of {c.B * c.H} (b,h) sequences at full length T={c.T} "
-                      f"({dt:.1f} s of float64 numpy), scaled to the whole layer"}
+                      f"({dt:.1f} s of single-threaded float64 numpy), scaled to the whole layer"}
 
 
 def run_reference(args, c, ws, rank):
@@ -218,12 +218,45 @@ def run_reference(args, c, ws, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(c, args),
-        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"each step: {heads} of {c.B * c.H} (b,h) sequences at full length, "
                                    "scaled to the whole layer"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def decode_measure(ttt, dev, peaks):
+    """The batched decode workload: 256 sequences x 16 heads, d = 128, state
+    carried from a 2048-token chunked prefill, then 512 timed single-token
+    steps.  Every step streams the 256 MiB fp32 state in and out of HBM."""
+    from synth import make_decode_inputs
+    x = make_decode_inputs(dev)
+    pq, pk, pv = x["prefill"]
+    sq, sk, sv = x["steps"]
+    ec = x["eta_const"]
+    _, S, _ = ttt.forward_chunked(pq, pk, pv, None, eta_const=ec, chunk=128)
+    del pq, pk, pv
+    n = sq.shape[0]
+    out = torch.empty_like(sq[0])
+    Sw = S.clone()
+    for t in range(3):
+        ttt.decode_step(sq[t], sk[t], sv[t], Sw, eta_const=ec, out=out)
+    del Sw
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(n):
+        ttt.decode_step(sq[t], sk[t], sv[t], S, eta_const=ec, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / n
+    nbytes = 2 * S.numel() * 4 + 3 * sq[0].numel() * sq.element_size() + out.numel() * out.element_size()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"workload": "decode N256 H16 d128 (2048-token prefill, 512 steps)", "us_per_step": us,
+            "bytes_per_step": nbytes, "hbm_gbs": gbs, "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+            "tokens_per_s": sq.shape[1] / (us * 1e-6), "gpu_launches": n}
 
 
 def workload_config(c, args):
@@ -353,12 +386,41 @@ def run_ours(args, c, ws, rank, local):
         "gpu_launches": args.steps * nseg_launch,
         "clocks": clocks,
     }
+    if not args.no_decode:
+        del sets, graphs
+        torch.cuda.empty_cache()
+        line["decode"] = decode_measure(ttt, dev, peaks)
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(c, args.ref_heads)
-    for g in graphs:
-        del g
+        line["cpu_baseline"] = cpu_baseline(c, c.B * c.H if args.cpu_heads == 0 else args.cpu_heads)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def profile_run(args):
+    """Plain launches (no graphs, no timing) for ncu: --warmup + --steps calls
+    of the workload's forward, or of the decode step on a random 256 MiB state."""
+    import test_layers_causal_b200 as ttt
+    dev = torch.device("cuda", 0)
+    if args.workload == "decode":
+        from synth import DECODE
+        N, H, d = DECODE["N"], DECODE["H"], DECODE["d"]
+        g = torch.Generator(device=dev).manual_seed(DECODE["seed"])
+        S = 0.1 * torch.randn(N, H, d, d, generator=g, device=dev)
+        q, k, v = (torch.randn(N, H, d, generator=g, device=dev).to(torch.bfloat16) for _ in range(3))
+        for _ in range(args.warmup + args.steps):
+            ttt.decode_step(q, k, v, S, eta_const=1.0 / math.sqrt(d))
+    else:
+        c = CONFIGS[args.workload]
+        x = make_case(c)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        eta = x["eta"].to(dev) if x["eta"] is not None else None
+        for _ in range(args.warmup + args.steps):
+            ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=args.chunk or c.chunk,
+                                segments=args.segments)
+    torch.cuda.synchronize()
+    if ttt.device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait")
+    print(f"profile run ok: {args.workload}, {args.warmup + args.steps} calls")
 
 
 def main():
@@ -367,13 +429,22 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llm_d64", choices=sorted(CONFIGS))
+    ap.add_argument("--workload", default="llm_d64", choices=sorted(CONFIGS) + ["decode"])
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--sets", type=int, default=4)
-    ap.add_argument("--ref-heads", type=int, default=8)
+    ap.add_argument("--ref-heads", type=int, default=8, help="(b,h) sequences per reference-arm step")
+    ap.add_argument("--cpu-heads", type=int, default=0, help="cpu_baseline sample; 0 = the whole layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="plain launches for a profiler: no graphs, timing, decode or CPU baseline")
     args = ap.parse_args()
+    if args.profile_run:
+        profile_run(args)
+        return
+    if args.workload == "decode":
+        raise SystemExit("decode is measured inside every chunked run (the 'decode' object)")
     c = CONFIGS[args.workload]
     if c.dtype != "bf16":
         raise SystemExit("bench workloads are the bf16 layers")

@@ -105,3 +105,27 @@ def make_case(case: LayerCase, device="cpu", B=None, H=None, T=None):
         eta=eta, eta_const=case.eta_const, beta=case.beta, chunk=case.chunk,
         ascent=case.ascent,
     )
+
+
+def make_decode_inputs(device="cuda", N=None, H=None, prefill=None, steps=None, d=None, seed=None):
+    """Inputs of the batched decode workload: a bf16 prefill [N,H,T,d] (q, k
+    unit-norm per token, v normal) and per-step bf16 q, k, v [steps,N,H,d],
+    drawn on `device` from one generator in the order prefill q, k, v, then
+    step q, k, v.  Constant learning rate 1/sqrt(d), no momentum."""
+    N = DECODE["N"] if N is None else N
+    H = DECODE["H"] if H is None else H
+    T = DECODE["prefill"] if prefill is None else prefill
+    S = DECODE["steps"] if steps is None else steps
+    d = DECODE["d"] if d is None else d
+    g = torch.Generator(device=device)
+    g.manual_seed(DECODE["seed"] if seed is None else seed)
+
+    def draw(*shape, unit):
+        x = torch.randn(*shape, generator=g, device=device)
+        if unit:
+            x = _unit(x)
+        return x.to(torch.bfloat16)
+
+    pq, pk, pv = draw(N, H, T, d, unit=True), draw(N, H, T, d, unit=True), draw(N, H, T, d, unit=False)
+    sq, sk, sv = draw(S, N, H, d, unit=True), draw(S, N, H, d, unit=True), draw(S, N, H, d, unit=False)
+    return dict(prefill=(pq, pk, pv), steps=(sq, sk, sv), eta_const=1.0 / math.sqrt(d))

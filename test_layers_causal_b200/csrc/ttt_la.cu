@@ -145,9 +145,11 @@ SegPlan plan_segments(const ttt_la_args* a) {
   if (a->segments > 0) {
     nseg = a->segments;
   } else {
+    // as many segments as fit in one wave of resident blocks (never a partial
+    // second wave), at least one per sequence
     const int per_sm = a->beta != 0.f ? 1 : tc_ctas_per_sm(C, a->d_k);
     const int target = sm_count() * per_sm;
-    nseg = (target + bh - 1) / bh;
+    nseg = std::max(1, target / bh);
   }
   nseg = std::max(1, std::min(nseg, s.nchunks));
   s.cps = (s.nchunks + nseg - 1) / nseg;

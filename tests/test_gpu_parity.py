@@ -233,6 +233,42 @@ def test_long_context_chunk_sweep_consistent(chunk):
     assert (S - S_ref).norm() / S_ref.norm() < 1e-2
 
 
+# ------------------------------------------------ decode workload ----
+def test_decode_workload_prefill_then_steps():
+    """256 sequences x 16 heads, d = 128: chunked prefill of 2048 tokens, then
+    512 decode steps.  Sampled sequences against the oracle over all 2560
+    tokens; every head against one chunked pass over the 2560 tokens."""
+    from synth import make_decode_inputs
+    x = make_decode_inputs("cuda")
+    pq, pk, pv = x["prefill"]
+    sq, sk, sv = x["steps"]
+    ec = x["eta_const"]
+    N, H, T, d = pq.shape
+    steps = sq.shape[0]
+    _, S, _ = ttt.forward_chunked(pq, pk, pv, None, eta_const=ec, chunk=128)
+    outs = torch.empty(steps, N, H, d, dtype=torch.bfloat16, device="cuda")
+    for t in range(steps):
+        ttt.decode_step(sq[t], sk[t], sv[t], S, eta_const=ec, out=outs[t])
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    # invariant over all heads: prefill + steps == one pass over the whole sequence
+    fq = torch.cat([pq, sq.permute(1, 2, 0, 3)], dim=2).contiguous()
+    fk = torch.cat([pk, sk.permute(1, 2, 0, 3)], dim=2).contiguous()
+    fv = torch.cat([pv, sv.permute(1, 2, 0, 3)], dim=2).contiguous()
+    del pq, pk, pv
+    o_full, S_full, _ = ttt.forward_chunked(fq, fk, fv, None, eta_const=ec, chunk=128)
+    o_dec = outs.permute(1, 2, 0, 3).float()
+    o_tail = o_full[:, :, T:].float()
+    assert float((o_dec - o_tail).norm() / o_tail.norm()) < 2e-2
+    assert float((S - S_full).norm() / S_full.norm()) < 2e-2
+    # oracle on sampled sequences (all heads), token by token over 2560 tokens
+    for n in (0, N - 1):
+        sl = slice(n, n + 1)
+        o_ref, S_ref, _ = oracle_forward(fq[sl], fk[sl], fv[sl], None, ec)
+        assert_bf16(o_dec[sl], o_ref[:, :, T:], f"decode outputs, sequence {n}")
+        assert_bf16(S[sl], S_ref, f"state after decode, sequence {n}")
+
+
 # ---------------------------------------------------- bounded waits ----
 def test_wait_timeout_is_reported_not_hung():
     assert ttt.device_status() == 0
