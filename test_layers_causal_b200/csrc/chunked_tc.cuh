@@ -58,10 +58,21 @@ struct TcParams {
 template <int C, int D>
 struct TcCfg {
   static constexpr int TILE = C * D * 2;                     // bytes of one bf16 C x D tile
-  static constexpr int STAGE = 3 * TILE;                     // Q, K, V
-  static constexpr int NST = (C == 128 && D == 128) ? 2 : (C == 64 && D == 64 ? 4 : 3);
-  static constexpr int SBF = D * D * 2;                      // bf16 copy of W (B operand)
-  static constexpr int BIG = NST * STAGE + SBF;
+  // 64 x 64 tiles fuse (1) and (2) into one N = C + D MMA, [Sc | O] = Q [K~; Wbf]^T:
+  // the K region of a stage then holds K~ and that chunk's Wbf as adjacent rows
+  // of one operand (order alternating with the chunk's parity, see below).
+  static constexpr bool MRG = (C == 64 && D == 64);
+  static constexpr int KWR = MRG ? C + D : C;                // rows per 64-column block of the K region
+  static constexpr int KREG = KWR * D * 2;
+  static constexpr int OK = TILE, OV = TILE + KREG;          // Q at 0, K region, V
+  static constexpr int STAGE = 2 * TILE + KREG;
+  static constexpr int NST = (C == 128 && D == 128) ? 2 : 3;
+  static constexpr int SBF = MRG ? 0 : D * D * 2;            // bf16 copy of W (B operand)
+  // P gets its own buffer, written as soon as the scores land, except for the
+  // 128 x 128 tile, where it reuses the Q/K slots once (1)-(3) have read them.
+  static constexpr bool PSEP = !(C == 128 && D == 128);
+  static constexpr int PBUF = PSEP ? C * C * 2 : 0;
+  static constexpr int BIG = NST * STAGE + SBF + PBUF;
   static constexpr int NBAR = 4 * NST + 10;
   static constexpr int SMALL = NBAR * 8 + NST * C * 4 + 32;
   static constexpr int SMEM = BIG + SMALL + 1024;            // + alignment slack
@@ -129,6 +140,20 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int blk, int row
     u.z = pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
     u.w = pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
     *reinterpret_cast<uint4*>(tile + (col >> 6) * blk + sw128_off(row, (col & 63) >> 3)) = u;
+  }
+}
+
+// Same for 64 values starting at column `col0` (multiple of 64): one
+// 128-byte row of one 64-column block.
+__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int blk, int row, int col0, const uint32_t (&r)[64]) {
+#pragma unroll
+  for (int q8 = 0; q8 < 8; ++q8) {
+    uint4 u;
+    u.x = pack_bf16x2(__uint_as_float(r[q8 * 8 + 0]), __uint_as_float(r[q8 * 8 + 1]));
+    u.y = pack_bf16x2(__uint_as_float(r[q8 * 8 + 2]), __uint_as_float(r[q8 * 8 + 3]));
+    u.z = pack_bf16x2(__uint_as_float(r[q8 * 8 + 4]), __uint_as_float(r[q8 * 8 + 5]));
+    u.w = pack_bf16x2(__uint_as_float(r[q8 * 8 + 6]), __uint_as_float(r[q8 * 8 + 7]));
+    *reinterpret_cast<uint4*>(tile + (col0 >> 6) * blk + sw128_off(row, q8)) = u;
   }
 }
 
@@ -209,10 +234,18 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
   const int nA = (p.nseg > 1 && seg < p.nseg - 1) ? nch : 0;  // phase-A chunks
   const int nB = nch;
   const int NI = nA + nB;
+  // Row offsets inside the K region (merged tiles): even phase-B chunks hold
+  // [K~ ; Wbf], odd ones [Wbf ; K~], so that the fused MMA writes [Sc | O0] or
+  // [O1 | Sc] and O stays double-buffered around one score region in TMEM.
+  auto krow_of = [&](int g) { return (Cfg::MRG && g >= nA && ((g - nA) & 1)) ? D : 0; };
+  auto wrow_of = [&](int it) { return (it & 1) ? 0 : C; };
   // TMEM column map
-  const uint32_t t_w = tmem;                      // W: D columns, M = D
-  const uint32_t t_sc = tmem + D;                 // scores: C columns, M = C
-  const uint32_t t_o0 = tmem + D + C;             // O[0], O[1]: D columns each, M = C
+  //   separate (1),(2): [W | Sc | O0 | O1]     merged: [W | O1 | Sc | O0]
+  const uint32_t t_w = tmem;                                  // W: D columns, M = D
+  const uint32_t t_sc = Cfg::MRG ? tmem + 2 * D : tmem + D;   // scores: C columns, M = C
+  auto t_o_of = [&](int b) -> uint32_t {                      // O[b]: D columns, M = C
+    return Cfg::MRG ? (b ? tmem + D : tmem + 2 * D + C) : tmem + D + C + b * D;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -228,8 +261,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
           if (pb) tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh);
-          tma_load_3d(&tmK, &full[s], st + TILE + kb * C * 128, kb * 64, t0, bh);
-          tma_load_3d(&tmV, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmK, &full[s], st + Cfg::OK + (kb * Cfg::KWR + krow_of(g)) * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmV, &full[s], st + Cfg::OV + kb * C * 128, kb * 64, t0, bh);
         }
       }
       for (int g = max(0, NI - NST); g < NI; ++g) mbar_wait(&full[g % NST], (g / NST) & 1, lim);
@@ -245,11 +278,12 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       // Descriptors are built once per tile and advanced by constant offsets
       // (the start address is the low field; no carry leaves it below 256 KB).
       const uint64_t d_wbf = sdesc_sw128(sbase + NST * STAGE, 16, 1024);
+      const uint64_t d_pbuf = sdesc_sw128(sbase + NST * STAGE + Cfg::SBF, 16, 1024);
       // phase A: segment total of V^T K~
       for (int g = 0; g < nA; ++g) {
         const int s = g % NST;
-        const uint32_t stk = sbase + s * STAGE + TILE, stv = stk + TILE;
-        const uint64_t dkm = sdesc_sw128(stk, C * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
+        const uint32_t stk = sbase + s * STAGE + Cfg::OK, stv = sbase + s * STAGE + Cfg::OV;
+        const uint64_t dkm = sdesc_sw128(stk, Cfg::KWR * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
         if (!dead) dead = !mbar_wait(&kready[s], (g / NST) & 1, lim);
         tc_fence_after();
 #pragma unroll
@@ -261,28 +295,43 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       // phase B
       for (int it = 0; it < nB; ++it) {
         const int g = nA + it, s = g % NST, b = it & 1;
-        const uint32_t stq = sbase + s * STAGE, stk = stq + TILE, stv = stq + 2 * TILE;
+        const uint32_t stq = sbase + s * STAGE, stk = stq + Cfg::OK, stv = stq + Cfg::OV;
         const uint64_t dq = sdesc_sw128(stq, 16, 1024), dkk = sdesc_sw128(stk, 16, 1024);
-        const uint64_t dkm = sdesc_sw128(stk, C * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
-        const uint32_t t_o = t_o0 + b * D;
+        const uint64_t dkm = sdesc_sw128(stk + krow_of(g) * 128, Cfg::KWR * 128, 1024);
+        const uint64_t dvm = sdesc_sw128(stv, C * 128, 1024);
+        const uint64_t dp = Cfg::PSEP ? d_pbuf : dq;
+        const uint32_t t_o = t_o_of(b);
         if (!dead) dead = !mbar_wait(&kready[s], (g / NST) & 1, lim);
-        tc_fence_after();
+        if (Cfg::MRG) {
+          // [Sc | O] in one N = C + D MMA: needs this chunk's Wbf and a free O[b]
+          if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
+          if (it >= 2 && !dead) dead = !mbar_wait(&o_free[b], ((it - 2) >> 1) & 1, lim);
+          tc_fence_after();
+          constexpr uint32_t ID_SCO = idesc_bf16_f32(C, C + D, false, false);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_sc, dq + k_step(C, kk), dkk + k_step(C, kk), ID_SC, kk > 0);
-        tc_commit(sc_full);
-        if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
-        if (it >= 2 && !dead) dead = !mbar_wait(&o_free[b], ((it - 2) >> 1) & 1, lim);
-        tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(b ? t_o : t_sc, dq + k_step(C, kk), dkk + k_step(Cfg::KWR, kk), ID_SCO, kk > 0);
+          tc_commit(sc_full);
+        } else {
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_QW, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(t_sc, dq + k_step(C, kk), dkk + k_step(C, kk), ID_SC, kk > 0);
+          tc_commit(sc_full);
+          if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
+          if (it >= 2 && !dead) dead = !mbar_wait(&o_free[b], ((it - 2) >> 1) & 1, lim);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_QW, kk > 0);
+        }
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_w, dvm + mn_step(kk), dkm + mn_step(kk), ID_W, 1);
         tc_commit(sdone);
         if (!dead) dead = !mbar_wait(p_ready, it & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, dq + k_step(C, kk), dvm + mn_step(kk), ID_O_PV, 1);
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, dp + k_step(C, kk), dvm + mn_step(kk), ID_O_PV, 1);
         tc_commit(&o_full[b]);
       }
       tc_commit(drain);
@@ -295,7 +344,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       for (int it = 0; it < nB; ++it) {
         const int g = nA + it, s = g % NST;
         if (!dead) dead = !mbar_wait(&staged[it % NST], (it / NST) & 1, lim);
-        const uint8_t* sv = smem + s * STAGE + 2 * TILE;
+        const uint8_t* sv = smem + s * STAGE + Cfg::OV;
         const int t0 = (chunk0 + it) * C;
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) tma_store_3d(&tmO, sv + kb * C * 128, kb * 64, t0, bh);
@@ -335,7 +384,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       fetch(g + 2, en);
       __syncwarp();
       if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
-      uint8_t* sk = smem + s * STAGE + TILE;
+      uint8_t* sk = smem + s * STAGE + Cfg::OK + krow_of(g) * 128;
 #pragma unroll 1
       for (int b0 = 0; b0 < PER_LANE; b0 += BATCH) {
         uint4 u[BATCH];
@@ -345,17 +394,19 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         for (int i = 0; i < BATCH; ++i) {
           const int idx = lane + 32 * (b0 + i);
           const int r = idx / (D / 8), cc = idx % (D / 8);
-          off[i] = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
+          off[i] = (cc >> 3) * Cfg::KWR * 128 + sw128_off(r, cc & 7);
           e[i] = ess[r];
           u[i] = *reinterpret_cast<const uint4*>(sk + off[i]);
         }
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-          float2 a;
-          a = unpack_bf16x2(u[i].x); u[i].x = pack_bf16x2(a.x * e[i], a.y * e[i]);
-          a = unpack_bf16x2(u[i].y); u[i].y = pack_bf16x2(a.x * e[i], a.y * e[i]);
-          a = unpack_bf16x2(u[i].z); u[i].z = pack_bf16x2(a.x * e[i], a.y * e[i]);
-          a = unpack_bf16x2(u[i].w); u[i].w = pack_bf16x2(a.x * e[i], a.y * e[i]);
+          // packed bf16 multiply: eta_r is rounded to bf16 once, then each
+          // product is rounded to bf16 as the operand itself would be
+          const uint32_t e2 = pack_bf16x2(e[i], e[i]);
+          u[i].x = mul_bf16x2(u[i].x, e2);
+          u[i].y = mul_bf16x2(u[i].y, e2);
+          u[i].z = mul_bf16x2(u[i].z, e2);
+          u[i].w = mul_bf16x2(u[i].w, e2);
           *reinterpret_cast<uint4*>(sk + off[i]) = u[i];
         }
       }
@@ -479,7 +530,12 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(acc[j]);
         tmem_st32(t_w + lane_off + cb * 32, r);  // W accumulator := W_start
-        if (wrow_ok) store_row32_bf16(sbf, D * 128, wrow, cb * 32, r);
+        if (wrow_ok) {
+          if (Cfg::MRG)
+            store_row32_bf16(smem + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow, cb * 32, r);
+          else
+            store_row32_bf16(sbf, D * 128, wrow, cb * 32, r);
+        }
       }
       tmem_st_wait();
       if (nA > 0) {
@@ -503,28 +559,28 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         if (!dead) dead = !mbar_wait(sc_full, it & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < C / 32; cb += 2) {
-          uint32_t r[2][32];
-          tmem_ld32(t_sc + lane_off + cb * 32, r[0]);
-          tmem_ld32(t_sc + lane_off + cb * 32 + 32, r[1]);
+        for (int cb = 0; cb < C / 64; ++cb) {
+          uint32_t r[64];
+          tmem_ld64(t_sc + lane_off + cb * 64, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const int col = (cb + h) * 32 + j;
-              const float a0 = (col <= qrow) ? __uint_as_float(r[h][j]) : 0.f;
-              const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[h][j + 1]) : 0.f;
-              pk[col >> 1] = pack_bf16x2(a0, a1);
-            }
+          for (int j = 0; j < 64; j += 2) {
+            const int col = cb * 64 + j;
+            const float a0 = (col <= qrow) ? __uint_as_float(r[j]) : 0.f;
+            const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[j + 1]) : 0.f;
+            pk[col >> 1] = pack_bf16x2(a0, a1);
           }
         }
-        if (!dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);  // Q, K slots and Wbf no longer read
+        // the overlaid P must wait until (1)-(3) have read the Q and K slots;
+        // the separate P buffer only until (4) of the previous tile (o_full, waited
+        // in the previous O step)
+        uint8_t* pdst = Cfg::PSEP ? smem + NST * STAGE + Cfg::SBF : st;
+        if (!Cfg::PSEP && !dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);
         if (qrow_ok) {
 #pragma unroll
           for (int c16 = 0; c16 < C / 8; ++c16) {
             uint4 u = make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
-            *reinterpret_cast<uint4*>(st + (c16 >> 3) * C * 128 + sw128_off(qrow, c16 & 7)) = u;
+            *reinterpret_cast<uint4*>(pdst + (c16 >> 3) * C * 128 + sw128_off(qrow, c16 & 7)) = u;
           }
         }
         fence_async_smem();
@@ -533,16 +589,17 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       }
       // next chunk's Wbf (W after this chunk's (3)) while (4) runs
       if (it + 1 < nB) {
+        if (Cfg::PSEP && !dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < D / 32; cb += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(t_w + lane_off + cb * 32, r0);
-          tmem_ld32(t_w + lane_off + cb * 32 + 32, r1);
+        for (int cb = 0; cb < D / 64; ++cb) {
+          uint32_t r[64];
+          tmem_ld64(t_w + lane_off + cb * 64, r);
           tmem_ld_wait();
           if (wrow_ok) {
-            store_row32_bf16(sbf, D * 128, wrow, cb * 32, r0);
-            store_row32_bf16(sbf, D * 128, wrow, cb * 32 + 32, r1);
+            uint8_t* wdst = Cfg::MRG ? smem + ((g + 1) % NST) * STAGE + Cfg::OK + wrow_of(it + 1) * 128 : sbf;
+            const int wblk = Cfg::MRG ? Cfg::KWR * 128 : D * 128;
+            store_row64_bf16(wdst, wblk, wrow, cb * 64, r);
           }
         }
         fence_async_smem();
@@ -551,20 +608,16 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       }
       // O[b]: TMEM -> bf16 -> V slot, then the store warp takes it
       {
-        uint8_t* sv = st + 2 * TILE;
+        uint8_t* sv = st + Cfg::OV;
         if (!dead) dead = !mbar_wait(&o_full[b], (it >> 1) & 1, lim);
         tc_fence_after();
-        const uint32_t t_o = t_o0 + b * D;
+        const uint32_t t_o = t_o_of(b);
 #pragma unroll
-        for (int cb = 0; cb < D / 32; cb += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(t_o + lane_off + cb * 32, r0);
-          tmem_ld32(t_o + lane_off + cb * 32 + 32, r1);
+        for (int cb = 0; cb < D / 64; ++cb) {
+          uint32_t r[64];
+          tmem_ld64(t_o + lane_off + cb * 64, r);
           tmem_ld_wait();
-          if (qrow_ok) {
-            store_row32_bf16(sv, C * 128, qrow, cb * 32, r0);
-            store_row32_bf16(sv, C * 128, qrow, cb * 32 + 32, r1);
-          }
+          if (qrow_ok) store_row64_bf16(sv, C * 128, qrow, cb * 64, r);
         }
         tc_fence_before();
         mbar_arrive(&o_free[b]);
