@@ -150,28 +150,19 @@ class ClockSampler:
 
 
 def dist_init():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    return ws, rank, local
+    from test_layers_causal_b200 import ranks
+    info = ranks.init()
+    return info.world, info.rank, info.local, info
 
 
-def barrier(ws):
-    if ws > 1:
-        torch.distributed.barrier()
+def barrier(info):
+    from test_layers_causal_b200 import ranks
+    ranks.barrier(info)
 
 
-def max_over_ranks(x, ws):
-    if ws == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+def max_over_ranks(x, info):
+    from test_layers_causal_b200 import ranks
+    return ranks.max_over_ranks(x, info)
 
 
 # --------------------------------------------------------------- oracle ----
@@ -201,7 +192,7 @@ def cpu_baseline(c, heads):
                       f"({dt:.1f} s of single-threaded float64 numpy), scaled to the whole layer"}
 
 
-def run_reference(args, c, ws, rank):
+def run_reference(args, c, ws, rank, info):
     if rank != 0:
         return
     heads = max(1, min(c.B * c.H, args.ref_heads))
@@ -267,7 +258,7 @@ def workload_config(c, args):
 
 
 # ----------------------------------------------------------------- ours ----
-def run_ours(args, c, ws, rank, local):
+def run_ours(args, c, ws, rank, local, info):
     import test_layers_causal_b200 as ttt
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -321,7 +312,7 @@ def run_ours(args, c, ws, rank, local):
         i += 1
         if i % 200 == 0:
             torch.cuda.synchronize()
-    barrier(ws)
+    barrier(info)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler.mark_start()
@@ -331,13 +322,14 @@ def run_ours(args, c, ws, rank, local):
     ev1.record(stream)
     torch.cuda.synchronize()
     sampler.mark_end()
-    barrier(ws)
+    barrier(info)
     clocks = sampler.stop()
     ms = ev0.elapsed_time(ev1)
-    ms_max = max_over_ranks(ms, ws)
+    ms_max = max_over_ranks(ms, info)
     ms_per_step = ms_max / args.steps
     tokens_per_step = c.B * c.T
-    value = tokens_per_step * ws / (ms_per_step * 1e-3)
+    from test_layers_causal_b200 import ranks
+    value = ranks.weak_scaling_tokens_per_s(tokens_per_step, ws, ms_per_step)
     if ttt.device_status() != 0:
         raise RuntimeError("device status reports a timed-out wait")
 
@@ -352,14 +344,14 @@ def run_ours(args, c, ws, rank, local):
     for _ in range(3):
         ttt.forward_chunked_host(qp, kp, vp, ep, o_host=oh, bufs=bufs, state_host=Sh, **kw)
     torch.cuda.synchronize()
-    barrier(ws)
+    barrier(info)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         _, h2d, d2h = ttt.forward_chunked_host(qp, kp, vp, ep, o_host=oh, bufs=bufs, state_host=Sh, **kw)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws) / e2e_steps
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), info) / e2e_steps
     e2e_val = tokens_per_step * ws / (e2e_ms * 1e-3)
 
     # ---- roofline of the forward call
@@ -448,15 +440,15 @@ def main():
     c = CONFIGS[args.workload]
     if c.dtype != "bf16":
         raise SystemExit("bench workloads are the bf16 layers")
-    ws, rank, local = dist_init()
+    ws, rank, local, info = dist_init()
     try:
         if args.impl == "reference":
-            run_reference(args, c, ws, rank)
+            run_reference(args, c, ws, rank, info)
         else:
-            run_ours(args, c, ws, rank, local)
+            run_ours(args, c, ws, rank, local, info)
     finally:
-        if ws > 1:
-            torch.distributed.destroy_process_group()
+        from test_layers_causal_b200 import ranks
+        ranks.finalize(info)
 
 
 if __name__ == "__main__":
