@@ -86,7 +86,7 @@ typedef struct ttt_la_args {
   int32_t ascent;           /* 0: gradient descent (sigma=+1); 1: ascent (sigma=-1) */
   int32_t chunk;            /* chunked path: tokens per chunk (64 or 128); ignored otherwise */
   int32_t segments;         /* chunked path: sequence segments per (b,h) run in parallel;
-                               0 = automatic (fill the SMs); ignored otherwise */
+                               0 = automatic (fill the SMs in one wave); ignored otherwise */
   const float *state_in;    /* [B,H,d_v,d_k] W_0, or NULL -> zeros */
   float *state_out;         /* [B,H,d_v,d_k] W_T, or NULL -> not returned */
   const float *mom_in;      /* [B,H,d_v,d_k] M_0 (momentum only), or NULL -> zeros */

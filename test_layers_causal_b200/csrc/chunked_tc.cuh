@@ -12,16 +12,21 @@
 // where W (d_v x d_k, fp32) is the fast weight carried in from earlier chunks.
 //
 // One launch per forward.  A (b, h) sequence is cut into `nseg` segments of
-// whole chunks so that B*H*nseg blocks fill the SMs.  A block takes its tile
-// (segment, head) from an atomic counter, so every tile it may wait for was
-// taken earlier by a block that is already running; then
+// whole chunks so that B*H*nseg blocks fill the SMs in one wave.  A block
+// takes its tile (segment, head) from an atomic counter; then
 //   phase A (all but the last segment): dW_p = sum over the segment of
-//           V^T K~ in one TMEM accumulator, published as fp32 with a flag;
-//   look-back: W_start(p) = (inclusive state of the nearest predecessor that
-//           has published one, or W_0) + the published totals in between;
-//           W_start(p) + dW_p is published as this segment's inclusive state;
-//   phase B: the chunk loop above from W_start(p); K and V come back from L2
-//           (phase A just read them), Q from HBM.
+//           V^T K~ in one TMEM accumulator (chunks taken last to first),
+//           published as fp32 with a flag;
+//   start:   W_start(p) = W_0 + sum_{p' < p} dW_p', either by a decoupled
+//           look-back (segment p sums the totals after the nearest
+//           predecessor that has published its own start + total; tiles
+//           are taken in segment order, so it never waits for a block that
+//           has not started) or, when that would read many totals and the
+//           grid is one wave, by a cooperative prefix (the head's blocks
+//           each sum one slice of the state over all totals, then meet at a
+//           counter);
+//   phase B: the chunk loop above from W_start(p); its first K and V tiles
+//           come back from L2 (phase A read them last), Q from HBM.
 //
 // Block = 8 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the
 // MMAs (one thread, descriptors precomputed), warps 2-5 (128 threads, one
@@ -49,8 +54,9 @@ struct TcParams {
   const float* eta;               // [BH, T] or nullptr
   float eta_const, sigma;
   const float* S_in;              // [BH, dv, dk] initial state or nullptr
-  float* ws;                      // [BH, nseg, 2, dv, dk]: segment totals, inclusive states
-  unsigned* flags;                // [BH * nseg] publication flags, then 1 tile counter (zeroed per call)
+  float* ws;                      // [BH, nseg, 2, dv, dk]: segment totals, segment start states
+  unsigned* flags;                // [BH * nseg] flags, tile counter, [BH] head counters (zeroed per call)
+  int coop;                       // 1: cooperative prefix (one wave), 0: decoupled look-back
   float* S_out;                   // [BH, dv, dk] final state or nullptr
   uint64_t limit_ns;
 };
@@ -111,15 +117,15 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-// Waits until *p >= 1 (bounded); returns the value seen, 0 on timeout.
-__device__ __forceinline__ unsigned wait_flag(const unsigned* p, uint64_t limit_ns) {
+// Waits until *p >= target (bounded); returns the value seen, 0 on timeout.
+__device__ __forceinline__ unsigned wait_geq(const unsigned* p, unsigned target, uint64_t limit_ns) {
   unsigned v = ld_acquire(p);
-  if (v) return v;
+  if (v >= target) return v;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     __nanosleep(64);
     v = ld_acquire(p);
-    if (v) return v;
+    if (v >= target) return v;
     if (globaltimer_ns() - t0 > limit_ns) {
       record_timeout();
       return 0;
@@ -185,7 +191,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
   float* es = reinterpret_cast<float*>(smem + Cfg::BIG + Cfg::NBAR * 8);  // [NST][C] sigma*eta
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(es + NST * C);
   int* sh_tile = reinterpret_cast<int*>(tmem_holder + 1);
-  int* sh_lb = sh_tile + 1;             // look-back: [0] first aggregate, [1] inclusive index or -1
+  int* sh_lb = sh_tile + 1;             // decoupled look-back: [1] nearest inclusive predecessor or -1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.limit_ns;
@@ -237,6 +243,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
   // Row offsets inside the K region (merged tiles): even phase-B chunks hold
   // [K~ ; Wbf], odd ones [Wbf ; K~], so that the fused MMA writes [Sc | O0] or
   // [O1 | Sc] and O stays double-buffered around one score region in TMEM.
+  // Phase A walks its chunks last to first, so the K/V tiles phase B starts
+  // with are the ones read most recently (still in L2).
+  auto chunk_of = [&](int g) { return g >= nA ? chunk0 + g - nA : chunk0 + nA - 1 - g; };
   auto krow_of = [&](int g) { return (Cfg::MRG && g >= nA && ((g - nA) & 1)) ? D : 0; };
   auto wrow_of = [&](int it) { return (it & 1) ? 0 : C; };
   // TMEM column map
@@ -255,7 +264,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         const int s = g % NST;
         if (g >= NST && !dead) dead = !mbar_wait(&empty[s], ((g / NST) - 1) & 1, lim);
         const bool pb = g >= nA;
-        const int t0 = (chunk0 + (pb ? g - nA : g)) * C;
+        const int t0 = chunk_of(g) * C;
         mbar_arrive_expect_tx(&full[s], pb ? 3 * TILE : 2 * TILE);
         uint8_t* st = smem + s * STAGE;
 #pragma unroll
@@ -362,7 +371,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
     constexpr int RPL = C / 32;  // rows of a chunk whose eta this lane fetches
     const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
     auto fetch = [&](int g, float (&dst)[RPL]) {
-      const int c0 = (chunk0 + (g >= nA ? g - nA : g)) * C;
+      const int c0 = chunk_of(g) * C;
 #pragma unroll
       for (int j = 0; j < RPL; ++j) {
         const int t = c0 + lane + 32 * j;
@@ -453,82 +462,127 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) st_release(flag_me, 1u);
       }
-      // Every predecessor has published at least its total; the nearest one
-      // that has already published its inclusive state cuts the sum short.
-      // One thread per predecessor, so the flags are read in one round trip.
-      if (et == 0) sh_lb[1] = -1;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int j = et; j < seg; j += 128) {
-        const unsigned f = dead ? 1u : wait_flag(p.flags + bh * p.nseg + j, lim);
-        if (f == 0) dead = true;
-        if (f >= 2) atomicMax(&sh_lb[1], j);
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int incl = sh_lb[1], first = incl + 1;
-      const float* base = nullptr;
-      if (incl >= 0) base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
-      else if (p.S_in) base = p.S_in + static_cast<size_t>(bh) * DD;
-#pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-        if (wrow_ok) {
-          const size_t off = static_cast<size_t>(wrow) * D + cb * 32;
-          if (base) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float8 x = ld_cg_v8(base + off + 8 * j);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) acc[8 * j + e] = x.v[e];
-            }
-          }
-          // four totals per round: 16 independent 32-byte (full-sector) loads in flight
-          int jj = first;
-          for (; jj + 4 <= seg; jj += 4) {
-            float8 x[4][4];
+      // W_start = W_0 + the totals of all earlier segments, in one of two ways.
+      const float* base = p.S_in ? p.S_in + static_cast<size_t>(bh) * DD : nullptr;
+      int first = 0, last = 0;  // totals [first, last) still to add to `base`
+      if (p.nseg > 1 && p.coop) {
+        // Cooperative prefix: the grid is a single wave, so the nseg blocks
+        // of a head are resident together.  Once every total is published,
+        // block `seg` prefix-sums element slice `seg` over all segments
+        // (coalesced) into the start-state slots; then the blocks meet at the
+        // head's counter and each reads its own start state.
+        for (int j = et; j < p.nseg - 1; j += 128)
+          if (!dead && wait_geq(p.flags + bh * p.nseg + j, 1u, lim) == 0) dead = true;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int DDi = D * D;
+        const int SL = ((DDi + p.nseg - 1) / p.nseg + 31) / 32 * 32;  // slice, a multiple of 32
+        const int v1 = min(DDi, (seg + 1) * SL) / 4;
+        const int nagg = p.nseg - 1;
+        float4* w4 = reinterpret_cast<float4*>(p.ws + static_cast<size_t>(bh) * p.nseg * 2 * DD);
+        const size_t SEG4 = 2 * DD / 4;  // float4 stride between segments; start states at +DD/4
+        const float4* s4 = reinterpret_cast<const float4*>(base);
+        // two vectors per thread per round, four totals per round
+        for (int v = seg * SL / 4 + et; v < v1; v += 256) {
+          const bool two = v + 128 < v1;
+          float4 run0 = s4 ? __ldcg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 run1 = (s4 && two) ? __ldcg(s4 + v + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int j = 0; j < nagg; j += 4) {
+            float4 a0[4], a1[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD + off;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) x[u][j] = ld_cg_v8(ag + 8 * j);
+              if (j + u < nagg) {
+                a0[u] = __ldcg(w4 + (j + u) * SEG4 + v);
+                if (two) a1[u] = __ldcg(w4 + (j + u) * SEG4 + v + 128);
+              }
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[u][j].v[e];
+              if (j + u < nagg) {
+                __stcg(w4 + (j + u) * SEG4 + DD / 4 + v, run0);
+                run0 = f4_add(run0, a0[u]);
+                if (two) {
+                  __stcg(w4 + (j + u) * SEG4 + DD / 4 + v + 128, run1);
+                  run1 = f4_add(run1, a1[u]);
+                }
               }
             }
           }
-          for (; jj < seg; ++jj) {
-            const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off;
-            float8 x[4];
+          __stcg(w4 + nagg * SEG4 + DD / 4 + v, run0);
+          if (two) __stcg(w4 + nagg * SEG4 + DD / 4 + v + 128, run1);
+        }
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        unsigned* cnt = p.flags + p.BH * p.nseg + 1 + bh;
+        if (et == 0) {
+          atomicAdd(cnt, 1u);
+          if (!dead && wait_geq(cnt, static_cast<unsigned>(p.nseg), lim) == 0) dead = true;
+          __threadfence();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        base = p.ws + (static_cast<size_t>(bh) * p.nseg + seg) * 2 * DD + DD;
+      } else if (seg > 0) {
+        // Decoupled look-back: every predecessor has published at least its
+        // total; the nearest one that has also published its inclusive state
+        // cuts the sum short.  One thread per predecessor reads the flags.
+        if (et == 0) sh_lb[1] = -1;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int j = et; j < seg; j += 128) {
+          const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
+          if (f == 0) dead = true;
+          if (f >= 2) atomicMax(&sh_lb[1], j);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int incl = sh_lb[1];
+        if (incl >= 0) base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
+        first = incl + 1;
+        last = seg;
+      }
+      // This thread's row of W_start, all loads issued before any store.
+      float row[D];
+      {
+        const size_t off = static_cast<size_t>(wrow) * D;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) x[j] = ld_cg_v8(ag + 8 * j);
+        for (int c = 0; c < D / 4; ++c) {
+          const float4 x = (wrow_ok && base) ? __ldcg(reinterpret_cast<const float4*>(base + off) + c)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+          row[4 * c] = x.x, row[4 * c + 1] = x.y, row[4 * c + 2] = x.z, row[4 * c + 3] = x.w;
+        }
+        if (wrow_ok) {
+#pragma unroll 1
+          for (int jj = first; jj < last; ++jj) {
+            const float4* ag = reinterpret_cast<const float4*>(p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int h = 0; h < D / 4; h += 8) {  // half a 64-wide row per round (register budget)
+              float4 x[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[j].v[e];
+              for (int c = 0; c < 8; ++c) x[c] = __ldcg(ag + h + c);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                row[4 * (h + c)] += x[c].x, row[4 * (h + c) + 1] += x[c].y, row[4 * (h + c) + 2] += x[c].z,
+                    row[4 * (h + c) + 3] += x[c].w;
             }
           }
         }
+      }
+      const bool pub_incl = !p.coop && nA > 0;  // decoupled: publish W_start + own total
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t r[32];
-        if (nA > 0) {  // this segment's total is still in t_w: publish the inclusive state
+        if (pub_incl) {
           tmem_ld32(t_w + lane_off + cb * 32, r);
           tmem_ld_wait();
           if (wrow_ok) {
             float4* d4 = reinterpret_cast<float4*>(agg_me + DD + static_cast<size_t>(wrow) * D + cb * 32);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              d4[j] = make_float4(acc[4 * j] + __uint_as_float(r[4 * j]), acc[4 * j + 1] + __uint_as_float(r[4 * j + 1]),
-                                  acc[4 * j + 2] + __uint_as_float(r[4 * j + 2]),
-                                  acc[4 * j + 3] + __uint_as_float(r[4 * j + 3]));
+              __stcg(d4 + j, make_float4(row[cb * 32 + 4 * j] + __uint_as_float(r[4 * j]),
+                                         row[cb * 32 + 4 * j + 1] + __uint_as_float(r[4 * j + 1]),
+                                         row[cb * 32 + 4 * j + 2] + __uint_as_float(r[4 * j + 2]),
+                                         row[cb * 32 + 4 * j + 3] + __uint_as_float(r[4 * j + 3])));
           }
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(acc[j]);
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(row[cb * 32 + j]);
         tmem_st32(t_w + lane_off + cb * 32, r);  // W accumulator := W_start
         if (wrow_ok) {
           if (Cfg::MRG)
@@ -538,7 +592,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         }
       }
       tmem_st_wait();
-      if (nA > 0) {
+      if (pub_incl) {
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) st_release(flag_me, 2u);

@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
       if (et == 0) sh_lb[1] = -1;
       asm volatile("bar.sync 1, 128;" ::: "memory");
       for (int j = et; j < seg; j += 128) {
-        const unsigned f = dead ? 1u : wait_flag(p.flags + bh * p.nseg + j, lim);
+        const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
         if (f == 0) dead = true;
         if (f >= 2) atomicMax(&sh_lb[1], j);
       }
@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
           if (bw) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float8 x = ld_cg_v8(bw + off + 8 * j);
+              const float8 x = ld_cg_f8(bw + off + 8 * j);
 #pragma unroll
               for (int e = 0; e < 8; ++e) w[8 * j + e] = x.v[e];
             }
@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
           if (bm) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float8 x = ld_cg_v8(bm + off + 8 * j);
+              const float8 x = ld_cg_f8(bm + off + 8 * j);
 #pragma unroll
               for (int e = 0; e < 8; ++e) mm[8 * j + e] = x.v[e];
             }
@@ -452,8 +452,8 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
             float8 xw[4], xm[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              xw[j] = ld_cg_v8(dw + 8 * j);
-              xm[j] = ld_cg_v8(dm + 8 * j);
+              xw[j] = ld_cg_f8(dw + 8 * j);
+              xm[j] = ld_cg_f8(dm + 8 * j);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {

@@ -241,17 +241,22 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-// 32-byte L2-coherent load of 8 floats (one full sector per thread).
+// 8 consecutive floats through L2 (two 16-byte loads: the pointers here are
+// only guaranteed 16-byte alignment).
 struct float8 {
   float v[8];
 };
-__device__ __forceinline__ float8 ld_cg_v8(const float* p) {
+__device__ __forceinline__ float8 ld_cg_f8(const float* p) {
+  const float4 a = __ldcg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldcg(reinterpret_cast<const float4*>(p) + 1);
   float8 r;
-  asm volatile("ld.global.cg.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3]), "=f"(r.v[4]), "=f"(r.v[5]), "=f"(r.v[6]),
-                 "=f"(r.v[7])
-               : "l"(p));
+  r.v[0] = a.x, r.v[1] = a.y, r.v[2] = a.z, r.v[3] = a.w;
+  r.v[4] = b.x, r.v[5] = b.y, r.v[6] = b.z, r.v[7] = b.w;
   return r;
+}
+
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
 // Loads 4 consecutive elements as fp32 (16 B for fp32, 8 B for bf16).

@@ -128,6 +128,7 @@ ttt_la_status recurrent_dk(const ttt_la_args* a, cudaStream_t st) {
 // --------------------------------------------------------------- chunked ----
 struct SegPlan {
   int nchunks, cps, nseg;
+  bool coop = false;  // plain kernel: cooperative prefix instead of decoupled look-back
 };
 
 int tc_ctas_per_sm(int C, int D) { return (C == 64 && D == 64) ? 2 : 1; }
@@ -141,19 +142,20 @@ SegPlan plan_segments(const ttt_la_args* a) {
   const int C = tc_tile(a);
   s.nchunks = (a->T + C - 1) / C;
   const int bh = a->B * a->H;
-  int nseg;
-  if (a->segments > 0) {
-    nseg = a->segments;
-  } else {
-    // as many segments as fit in one wave of resident blocks (never a partial
-    // second wave), at least one per sequence
-    const int per_sm = a->beta != 0.f ? 1 : tc_ctas_per_sm(C, a->d_k);
-    const int target = sm_count() * per_sm;
-    nseg = std::max(1, target / bh);
-  }
+  // Automatic: as many segments as fit in one wave of resident blocks (never
+  // a partial second wave), at least one per sequence.
+  const int per_sm = a->beta != 0.f ? 1 : tc_ctas_per_sm(C, a->d_k);
+  const int resident = sm_count() * per_sm;
+  int nseg = a->segments > 0 ? a->segments : std::max(1, resident / bh);
   nseg = std::max(1, std::min(nseg, s.nchunks));
   s.cps = (s.nchunks + nseg - 1) / nseg;
   s.nseg = (s.nchunks + s.cps - 1) / s.cps;
+  // Start states by a cooperative prefix (blocks of a head wait for one
+  // another: only when the whole grid is resident at once) when a decoupled
+  // look-back would have the last segment read more than 192 KB of totals.
+  const size_t lookback_bytes = static_cast<size_t>(s.nseg - 1) * a->d_k * a->d_v * sizeof(float);
+  s.coop = a->beta == 0.f && s.nseg > 1 && static_cast<long long>(bh) * s.nseg <= resident &&
+           lookback_bytes > 192 * 1024;
   return s;
 }
 
@@ -176,11 +178,13 @@ bool simt_supported(const ttt_la_args* a, ttt::SimtShape* sh) {
 }
 
 // Scratch layout of the chunked tensor-core path: fp32 [BH][nseg][2][d_v][d_k]
-// (segment totals, inclusive states), then nseg*BH publication flags and one
-// tile counter (uint32), which every call clears before its launch.
+// (segment totals, segment start states), then nseg*BH publication flags, one
+// tile counter and BH per-head counters (uint32), which every call clears
+// before its launch.
 size_t tc_ws_floats(int bh, int nseg, int D) { return static_cast<size_t>(bh) * nseg * 2 * D * D; }
+size_t tc_flag_words(int bh, int nseg) { return static_cast<size_t>(bh) * nseg + 1 + bh; }
 size_t tc_ws_bytes(int bh, int nseg, int D) {
-  const size_t b = tc_ws_floats(bh, nseg, D) * sizeof(float) + (static_cast<size_t>(bh) * nseg + 1) * sizeof(unsigned);
+  const size_t b = tc_ws_floats(bh, nseg, D) * sizeof(float) + tc_flag_words(bh, nseg) * sizeof(unsigned);
   return (b + 15) & ~static_cast<size_t>(15);
 }
 
@@ -211,12 +215,13 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
   p.S_in = a->state_in;
   p.ws = nullptr;
   p.flags = nullptr;
+  p.coop = sp.coop ? 1 : 0;
   p.S_out = a->state_out;
   p.limit_ns = g_limit_ns;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
     p.flags = reinterpret_cast<unsigned*>(p.ws + tc_ws_floats(bh, sp.nseg, D));
-    if (cudaMemsetAsync(p.flags, 0, (static_cast<size_t>(bh) * sp.nseg + 1) * sizeof(unsigned), st) != cudaSuccess)
+    if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
   ttt::chunked_tc_kernel<C, D><<<bh * sp.nseg, 256, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
@@ -241,7 +246,7 @@ ttt_la_status launch_simt(const ttt_la_args* a, const ttt::SimtShape& sh, cudaSt
 // fp32 [BH][nseg][2] (G, B), then flags and the tile counter.
 size_t tcm_ws_floats(int bh, int nseg, int D) { return static_cast<size_t>(bh) * nseg * (4 * D * D + 2); }
 size_t tcm_ws_bytes(int bh, int nseg, int D) {
-  const size_t b = tcm_ws_floats(bh, nseg, D) * sizeof(float) + (static_cast<size_t>(bh) * nseg + 1) * sizeof(unsigned);
+  const size_t b = tcm_ws_floats(bh, nseg, D) * sizeof(float) + tc_flag_words(bh, nseg) * sizeof(unsigned);
   return (b + 15) & ~static_cast<size_t>(15);
 }
 
@@ -290,7 +295,7 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
     p.ws = static_cast<float*>(a->workspace);
     p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;
     p.flags = reinterpret_cast<unsigned*>(p.ws + tcm_ws_floats(bh, sp.nseg, D));
-    if (cudaMemsetAsync(p.flags, 0, (static_cast<size_t>(bh) * sp.nseg + 1) * sizeof(unsigned), st) != cudaSuccess)
+    if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
   ttt::chunked_tc_mom_kernel<D><<<bh * sp.nseg, 256, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);

@@ -139,8 +139,8 @@ def test_decode_validation(abi):
 
 def test_workspace_query(abi):
     L = abi.lib()
-    def expected(bh, nseg, d):  # fp32 [bh][nseg][2][d][d], then bh*nseg flags + 1 counter
-        b = bh * nseg * 2 * d * d * 4 + (bh * nseg + 1) * 4
+    def expected(bh, nseg, d):  # fp32 [bh][nseg][2][d][d], bh*nseg flags, tile counter, bh head counters
+        b = bh * nseg * 2 * d * d * 4 + (bh * nseg + 1 + bh) * 4
         return (b + 15) // 16 * 16
 
     one_seq_long = _args(abi, B=1, H=1, T=65536, chunk=128)
@@ -152,6 +152,9 @@ def test_workspace_query(abi):
     assert L.ttt_la_workspace_size(ctypes.byref(fixed)) == expected(1, 3, 64)
     fixed4 = _args(abi, B=2, H=3, T=64 * 10, chunk=64, segments=4)  # 10 chunks -> 3+3+3+1
     assert L.ttt_la_workspace_size(ctypes.byref(fixed4)) == expected(6, 4, 64)
+    # a request beyond one wave of resident blocks is honoured (64 chunks / 40 -> 32 segments of 2)
+    wide = _args(abi, B=4, H=16, T=64 * 64, chunk=64, segments=40)
+    assert L.ttt_la_workspace_size(ctypes.byref(wide)) == expected(64, 32, 64)
     # short workspace is refused on the host
     fixed.workspace, fixed.workspace_bytes = 0x60000, 100
     assert L.ttt_la_forward_chunked(ctypes.byref(fixed), None) == abi.ERR_INVALID_ARG

@@ -129,6 +129,22 @@ def test_chunked_tc_parity(d, chunk, segments, token_eta):
     assert_bf16(S, S_ref, "state")
 
 
+@pytest.mark.parametrize("d,chunk,segments", [(128, 64, 8), (128, 128, 6), (64, 64, 16)])
+@pytest.mark.parametrize("with_state", [True, False])
+def test_chunked_tc_many_segments(d, chunk, segments, with_state):
+    """Enough segments that the start states come from the cooperative prefix
+    (the look-back would read more than 192 KB of totals), ragged tail."""
+    B, H, T = 1, 3, segments * 2 * chunk - 29
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 130 + d + segments)
+    S0 = _state(B, H, d, d, 12, scale=0.1) if with_state else None
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=chunk, segments=segments, state_in=S0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec, 0.0, False, S0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+
+
 @pytest.mark.parametrize("d,chunk", [(64, 64), (128, 128)])
 def test_chunked_tc_ascent_zero_state_and_exact_multiple(d, chunk):
     B, H, T = 1, 2, 4 * chunk
@@ -173,6 +189,32 @@ def test_chunked_tc_momentum_parity(d, chunk, segments, beta, ascent):
     assert_bf16(o, o_ref, "o")
     assert_bf16(S, S_ref, "state")
     assert_bf16(M, M_ref, "momentum")
+
+
+def _state_at_16_bytes(S):
+    """The same values at an address that is 16- but not 32-byte aligned
+    (the ABI promises callers only 16)."""
+    flat = torch.empty(S.numel() + 4, device=S.device, dtype=S.dtype)
+    out = flat[4:].view(S.shape)
+    out.copy_(S)
+    assert out.data_ptr() % 32 == 16
+    return out
+
+
+@pytest.mark.parametrize("beta,segments", [(0.0, 1), (0.0, 3), (0.9, 1), (0.9, 3)])
+def test_chunked_tc_states_at_16_byte_alignment(beta, segments):
+    B, H, T, d = 1, 2, 4 * 64 + 9, 128
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 120)
+    S0 = _state_at_16_bytes(_state(B, H, d, d, 10, scale=0.1))
+    M0 = _state_at_16_bytes(_state(B, H, d, d, 11, scale=0.1)) if beta else None
+    o, S, M = ttt.forward_chunked(q, k, v, eta, beta=beta, chunk=64, segments=segments, state_in=S0, mom_in=M0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, ec, beta, False, S0, M0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+    if beta:
+        assert_bf16(M, M_ref, "momentum")
 
 
 def test_chunked_tc_momentum_const_eta_zero_state():
