@@ -361,7 +361,6 @@ def run_ours(args, c, ws, rank, local, info):
     flops = executed_flops(c, c.B, c.H, c.T, chunk)
     tflops = flops / (ms_per_step * 1e-3) / 1e12
     traffic = read_traffic(c.name, chunk)
-    nseg_launch = 3 if wsb > 0 else 1
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -369,13 +368,14 @@ def run_ours(args, c, ws, rank, local, info):
         "config": workload_config(c, args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "kernel": "ttt_la_forward_chunked (segment-state pass, scan, chunk pass)"
-                               if nseg_launch == 3 else "ttt_la_forward_chunked (chunk pass)",
+                     "kernel": ("chunked_tc_mom_kernel" if c.beta else "chunked_tc_kernel")
+                               + (" (phase A, start states, phase B: one launch)" if wsb > 0
+                                  else " (one segment per sequence: phase B only)"),
                      "algorithmic_bytes": nbytes, "peak_source": f"{src} (copy bandwidth)"},
         "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                    "frac": tflops / peaks["bf16_tflops"], "executed_flops": flops},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * nseg_launch,
+        "gpu_launches": args.steps,  # one kernel per step (plus a flag memset when segmented)
         "clocks": clocks,
     }
     if not args.no_decode:

@@ -26,7 +26,7 @@
 //           each sum one slice of the state over all totals, then meet at a
 //           counter);
 //   phase B: the chunk loop above from W_start(p); its first K and V tiles
-//           come back from L2 (phase A read them last), Q from HBM.
+//           are the ones phase A read last (the likeliest to hit in L2).
 //
 // Block = 8 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the
 // MMAs (one thread, descriptors precomputed), warps 2-5 (128 threads, one
@@ -118,7 +118,8 @@ __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 // Waits until *p >= target (bounded); returns the value seen, 0 on timeout.
-__device__ __forceinline__ unsigned wait_geq(const unsigned* p, unsigned target, uint64_t limit_ns) {
+// A slow path, kept out of line so that it costs the callers no registers.
+__device__ __noinline__ unsigned wait_geq(const unsigned* p, unsigned target, uint64_t limit_ns) {
   unsigned v = ld_acquire(p);
   if (v >= target) return v;
   const uint64_t t0 = globaltimer_ns();
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
   // [K~ ; Wbf], odd ones [Wbf ; K~], so that the fused MMA writes [Sc | O0] or
   // [O1 | Sc] and O stays double-buffered around one score region in TMEM.
   // Phase A walks its chunks last to first, so the K/V tiles phase B starts
-  // with are the ones read most recently (still in L2).
+  // with are the ones read most recently.
   auto chunk_of = [&](int g) { return g >= nA ? chunk0 + g - nA : chunk0 + nA - 1 - g; };
   auto krow_of = [&](int g) { return (Cfg::MRG && g >= nA && ((g - nA) & 1)) ? D : 0; };
   auto wrow_of = [&](int it) { return (it & 1) ? 0 : C; };
@@ -260,6 +261,10 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       bool dead = false;
+      // Every tile is loaded as evict-first: the only re-read (K and V of a
+      // segment, phase A then phase B) gains nothing measurable from being
+      // kept, and the streamed tiles then leave L2 to the state totals.
+      const uint64_t pol_once = l2_policy_evict_first();
       for (int g = 0; g < NI; ++g) {
         const int s = g % NST;
         if (g >= NST && !dead) dead = !mbar_wait(&empty[s], ((g / NST) - 1) & 1, lim);
@@ -269,9 +274,10 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         uint8_t* st = smem + s * STAGE;
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
-          if (pb) tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh);
-          tma_load_3d(&tmK, &full[s], st + Cfg::OK + (kb * Cfg::KWR + krow_of(g)) * 128, kb * 64, t0, bh);
-          tma_load_3d(&tmV, &full[s], st + Cfg::OV + kb * C * 128, kb * 64, t0, bh);
+          if (pb) tma_load_3d_hint(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh, pol_once);
+          tma_load_3d_hint(&tmK, &full[s], st + Cfg::OK + (kb * Cfg::KWR + krow_of(g)) * 128, kb * 64, t0, bh,
+                           pol_once);
+          tma_load_3d_hint(&tmV, &full[s], st + Cfg::OV + kb * C * 128, kb * 64, t0, bh, pol_once);
         }
       }
       for (int g = max(0, NI - NST); g < NI; ++g) mbar_wait(&full[g % NST], (g / NST) & 1, lim);
@@ -464,7 +470,6 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       }
       // W_start = W_0 + the totals of all earlier segments, in one of two ways.
       const float* base = p.S_in ? p.S_in + static_cast<size_t>(bh) * DD : nullptr;
-      int first = 0, last = 0;  // totals [first, last) still to add to `base`
       if (p.nseg > 1 && p.coop) {
         // Cooperative prefix: the grid is a single wave, so the nseg blocks
         // of a head are resident together.  Once every total is published,
@@ -520,82 +525,127 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         base = p.ws + (static_cast<size_t>(bh) * p.nseg + seg) * 2 * DD + DD;
-      } else if (seg > 0) {
-        // Decoupled look-back: every predecessor has published at least its
-        // total; the nearest one that has also published its inclusive state
-        // cuts the sum short.  One thread per predecessor reads the flags.
-        if (et == 0) sh_lb[1] = -1;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        for (int j = et; j < seg; j += 128) {
-          const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
-          if (f == 0) dead = true;
-          if (f >= 2) atomicMax(&sh_lb[1], j);
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        const int incl = sh_lb[1];
-        if (incl >= 0) base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
-        first = incl + 1;
-        last = seg;
-      }
-      // This thread's row of W_start, all loads issued before any store.
-      float row[D];
-      {
+        // this thread's row of W_start; with d = 128 all loads are issued
+        // before any store (one round trip), with d = 64 one 32-column block
+        // per round (register budget of two blocks per SM)
+        constexpr int G = (D == 128) ? D / 32 : 1;
         const size_t off = static_cast<size_t>(wrow) * D;
 #pragma unroll
-        for (int c = 0; c < D / 4; ++c) {
-          const float4 x = (wrow_ok && base) ? __ldcg(reinterpret_cast<const float4*>(base + off) + c)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-          row[4 * c] = x.x, row[4 * c + 1] = x.y, row[4 * c + 2] = x.z, row[4 * c + 3] = x.w;
-        }
-        if (wrow_ok) {
-#pragma unroll 1
-          for (int jj = first; jj < last; ++jj) {
-            const float4* ag = reinterpret_cast<const float4*>(p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off);
+        for (int cb0 = 0; cb0 < D / 32; cb0 += G) {
+          float row[G * 32];
 #pragma unroll
-            for (int h = 0; h < D / 4; h += 8) {  // half a 64-wide row per round (register budget)
-              float4 x[8];
+          for (int c = 0; c < G * 8; ++c) {
+            const float4 x = wrow_ok ? __ldcg(reinterpret_cast<const float4*>(base + off + cb0 * 32) + c)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            row[4 * c] = x.x, row[4 * c + 1] = x.y, row[4 * c + 2] = x.z, row[4 * c + 3] = x.w;
+          }
 #pragma unroll
-              for (int c = 0; c < 8; ++c) x[c] = __ldcg(ag + h + c);
+          for (int cb = 0; cb < G; ++cb) {
+            uint32_t r[32];
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                row[4 * (h + c)] += x[c].x, row[4 * (h + c) + 1] += x[c].y, row[4 * (h + c) + 2] += x[c].z,
-                    row[4 * (h + c) + 3] += x[c].w;
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(row[cb * 32 + j]);
+            tmem_st32(t_w + lane_off + (cb0 + cb) * 32, r);  // W accumulator := W_start
+            if (wrow_ok) {
+              if (Cfg::MRG)
+                store_row32_bf16(smem + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow,
+                                 (cb0 + cb) * 32, r);
+              else
+                store_row32_bf16(sbf, D * 128, wrow, (cb0 + cb) * 32, r);
             }
           }
         }
-      }
-      const bool pub_incl = !p.coop && nA > 0;  // decoupled: publish W_start + own total
+        tmem_st_wait();
+      } else {
+        // Decoupled look-back: every predecessor has published at least its
+        // total; the nearest one that has also published its inclusive state
+        // (start + total) cuts the sum short.  One thread per predecessor
+        // reads the flags.
+        int first = 0;
+        if (seg > 0) {
+          if (et == 0) sh_lb[1] = -1;
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          for (int j = et; j < seg; j += 128) {
+            const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
+            if (f == 0) dead = true;
+            if (f >= 2) atomicMax(&sh_lb[1], j);
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          const int incl = sh_lb[1];
+          if (incl >= 0) base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
+          first = incl + 1;
+        }
 #pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        uint32_t r[32];
-        if (pub_incl) {
-          tmem_ld32(t_w + lane_off + cb * 32, r);
-          tmem_ld_wait();
+        for (int cb = 0; cb < D / 32; ++cb) {
+          float acc[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] = 0.f;
           if (wrow_ok) {
-            float4* d4 = reinterpret_cast<float4*>(agg_me + DD + static_cast<size_t>(wrow) * D + cb * 32);
+            const size_t off = static_cast<size_t>(wrow) * D + cb * 32;
+            if (base) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              __stcg(d4 + j, make_float4(row[cb * 32 + 4 * j] + __uint_as_float(r[4 * j]),
-                                         row[cb * 32 + 4 * j + 1] + __uint_as_float(r[4 * j + 1]),
-                                         row[cb * 32 + 4 * j + 2] + __uint_as_float(r[4 * j + 2]),
-                                         row[cb * 32 + 4 * j + 3] + __uint_as_float(r[4 * j + 3])));
+              for (int j = 0; j < 4; ++j) {
+                const float8 x = ld_cg_f8(base + off + 8 * j);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[8 * j + e] = x.v[e];
+              }
+            }
+            // four totals per round: 32 independent 16-byte loads in flight
+            int jj = first;
+            for (; jj + 4 <= seg; jj += 4) {
+              float8 x[4][4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD + off;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[u][j] = ld_cg_f8(ag + 8 * j);
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[u][j].v[e];
+            }
+            for (; jj < seg; ++jj) {
+              const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off;
+              float8 x[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) x[j] = ld_cg_f8(ag + 8 * j);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[j].v[e];
+            }
+          }
+          uint32_t r[32];
+          if (nA > 0) {  // this segment's total is still in t_w: publish the inclusive state
+            tmem_ld32(t_w + lane_off + cb * 32, r);
+            tmem_ld_wait();
+            if (wrow_ok) {
+              float4* d4 = reinterpret_cast<float4*>(agg_me + DD + static_cast<size_t>(wrow) * D + cb * 32);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                d4[j] = make_float4(acc[4 * j] + __uint_as_float(r[4 * j]), acc[4 * j + 1] + __uint_as_float(r[4 * j + 1]),
+                                    acc[4 * j + 2] + __uint_as_float(r[4 * j + 2]),
+                                    acc[4 * j + 3] + __uint_as_float(r[4 * j + 3]));
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(acc[j]);
+          tmem_st32(t_w + lane_off + cb * 32, r);  // W accumulator := W_start
+          if (wrow_ok) {
+            if (Cfg::MRG)
+              store_row32_bf16(smem + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow, cb * 32, r);
+            else
+              store_row32_bf16(sbf, D * 128, wrow, cb * 32, r);
           }
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(row[cb * 32 + j]);
-        tmem_st32(t_w + lane_off + cb * 32, r);  // W accumulator := W_start
-        if (wrow_ok) {
-          if (Cfg::MRG)
-            store_row32_bf16(smem + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow, cb * 32, r);
-          else
-            store_row32_bf16(sbf, D * 128, wrow, cb * 32, r);
+        tmem_st_wait();
+        if (nA > 0) {
+          __threadfence();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (et == 0) st_release(flag_me, 2u);
         }
-      }
-      tmem_st_wait();
-      if (pub_incl) {
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (et == 0) st_release(flag_me, 2u);
       }
       fence_async_smem();
       tc_fence_before();
