@@ -134,34 +134,44 @@ __device__ __noinline__ unsigned wait_geq(const unsigned* p, unsigned target, ui
   }
 }
 
+// 16-byte store to a shared-memory address (32-bit: half the address
+// registers of a generic pointer).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
 // Packs 32 fp32 values (as raw bits) into bf16 and writes them as four
-// 16-byte units of row `row` of a 128B-swizzled K-major tile whose 64-column
-// blocks are `blk` bytes apart, starting at column `col0` (multiple of 32).
-__device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int blk, int row, int col0, const uint32_t (&r)[32]) {
+// 16-byte units of row `row` of a 128B-swizzled K-major tile (shared address
+// `tile`) whose 64-column blocks are `blk` bytes apart, starting at column
+// `col0` (multiple of 32).
+__device__ __forceinline__ void store_row32_bf16(uint32_t tile, int blk, int row, int col0, const uint32_t (&r)[32]) {
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4) {
     const int col = col0 + q4 * 8;
-    uint4 u;
-    u.x = pack_bf16x2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
-    u.y = pack_bf16x2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
-    u.z = pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
-    u.w = pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-    *reinterpret_cast<uint4*>(tile + (col >> 6) * blk + sw128_off(row, (col & 63) >> 3)) = u;
+    st_shared_v4(tile + (col >> 6) * blk + sw128_off(row, (col & 63) >> 3),
+                 pack_bf16x2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1])),
+                 pack_bf16x2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3])),
+                 pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5])),
+                 pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7])));
   }
+}
+__device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int blk, int row, int col0, const uint32_t (&r)[32]) {
+  store_row32_bf16(smem_u32(tile), blk, row, col0, r);
 }
 
 // Same for 64 values starting at column `col0` (multiple of 64): one
 // 128-byte row of one 64-column block.
-__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int blk, int row, int col0, const uint32_t (&r)[64]) {
+__device__ __forceinline__ void store_row64_bf16(uint32_t tile, int blk, int row, int col0, const uint32_t (&r)[64]) {
 #pragma unroll
-  for (int q8 = 0; q8 < 8; ++q8) {
-    uint4 u;
-    u.x = pack_bf16x2(__uint_as_float(r[q8 * 8 + 0]), __uint_as_float(r[q8 * 8 + 1]));
-    u.y = pack_bf16x2(__uint_as_float(r[q8 * 8 + 2]), __uint_as_float(r[q8 * 8 + 3]));
-    u.z = pack_bf16x2(__uint_as_float(r[q8 * 8 + 4]), __uint_as_float(r[q8 * 8 + 5]));
-    u.w = pack_bf16x2(__uint_as_float(r[q8 * 8 + 6]), __uint_as_float(r[q8 * 8 + 7]));
-    *reinterpret_cast<uint4*>(tile + (col0 >> 6) * blk + sw128_off(row, q8)) = u;
-  }
+  for (int q8 = 0; q8 < 8; ++q8)
+    st_shared_v4(tile + (col0 >> 6) * blk + sw128_off(row, q8),
+                 pack_bf16x2(__uint_as_float(r[q8 * 8 + 0]), __uint_as_float(r[q8 * 8 + 1])),
+                 pack_bf16x2(__uint_as_float(r[q8 * 8 + 2]), __uint_as_float(r[q8 * 8 + 3])),
+                 pack_bf16x2(__uint_as_float(r[q8 * 8 + 4]), __uint_as_float(r[q8 * 8 + 5])),
+                 pack_bf16x2(__uint_as_float(r[q8 * 8 + 6]), __uint_as_float(r[q8 * 8 + 7])));
+}
+__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int blk, int row, int col0, const uint32_t (&r)[64]) {
+  store_row64_bf16(smem_u32(tile), blk, row, col0, r);
 }
 
 template <int C, int D>
@@ -175,7 +185,6 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
-  uint8_t* sbf = smem + NST * STAGE;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BIG);
   uint64_t* full = bars;                // [NST] TMA landed
@@ -441,6 +450,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
     const bool wrow_ok = (D == 128) || ok64;
     const int qrow = (C == 128) ? row128 : row64;  // query row of scores / O
     const bool qrow_ok = (C == 128) || ok64;
+    // M = 64 tiles read with the whole warp: row 16*g4 + lane%16, column half lane/16
+    const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
     bool dead = false;
 
     // --------------------------------------------- look-back, W_start
@@ -547,10 +558,10 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
             tmem_st32(t_w + lane_off + (cb0 + cb) * 32, r);  // W accumulator := W_start
             if (wrow_ok) {
               if (Cfg::MRG)
-                store_row32_bf16(smem + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow,
+                store_row32_bf16(sbase + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow,
                                  (cb0 + cb) * 32, r);
               else
-                store_row32_bf16(sbf, D * 128, wrow, (cb0 + cb) * 32, r);
+                store_row32_bf16(sbase + NST * STAGE, D * 128, wrow, (cb0 + cb) * 32, r);
             }
           }
         }
@@ -635,9 +646,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
           tmem_st32(t_w + lane_off + cb * 32, r);  // W accumulator := W_start
           if (wrow_ok) {
             if (Cfg::MRG)
-              store_row32_bf16(smem + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow, cb * 32, r);
+              store_row32_bf16(sbase + (nA % NST) * STAGE + Cfg::OK + wrow_of(0) * 128, Cfg::KWR * 128, wrow, cb * 32, r);
             else
-              store_row32_bf16(sbf, D * 128, wrow, cb * 32, r);
+              store_row32_bf16(sbase + NST * STAGE, D * 128, wrow, cb * 32, r);
           }
         }
         tmem_st_wait();
@@ -659,32 +670,55 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       uint8_t* st = smem + s * STAGE;
       // P = bf16(tril(scores)) into the Q (and K) slots
       {
-        uint32_t pk[C / 2];
         if (!dead) dead = !mbar_wait(sc_full, it & 1, lim);
         tc_fence_after();
-#pragma unroll
-        for (int cb = 0; cb < C / 64; ++cb) {
-          uint32_t r[64];
-          tmem_ld64(t_sc + lane_off + cb * 64, r);
+        if constexpr (C == 64) {
+          // this thread's 32 columns (half) of row row64h, straight into the
+          // separate P buffer (free since the previous tile's (4): o_full,
+          // waited in the previous O step)
+          static_assert(Cfg::PSEP, "64-token tiles keep P in its own buffer");
+          uint32_t r[32];
+          tmem_ld_half32(t_sc + lane_off, r);
           tmem_ld_wait();
+          const uint32_t pdst = sbase + NST * STAGE + Cfg::SBF;
+          const int jmax = row64h - 32 * half;  // last unmasked column of this half
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const int col = cb * 64 + j;
-            const float a0 = (col <= qrow) ? __uint_as_float(r[j]) : 0.f;
-            const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[j + 1]) : 0.f;
-            pk[col >> 1] = pack_bf16x2(a0, a1);
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 8 * i + 2 * e;
+              w[e] = pack_bf16x2((j <= jmax) ? __uint_as_float(r[j]) : 0.f,
+                                 (j + 1 <= jmax) ? __uint_as_float(r[j + 1]) : 0.f);
+            }
+            st_shared_v4(pdst + sw128_off(row64h, 4 * half + i), w[0], w[1], w[2], w[3]);
           }
-        }
-        // the overlaid P must wait until (1)-(3) have read the Q and K slots;
-        // the separate P buffer only until (4) of the previous tile (o_full, waited
-        // in the previous O step)
-        uint8_t* pdst = Cfg::PSEP ? smem + NST * STAGE + Cfg::SBF : st;
-        if (!Cfg::PSEP && !dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);
-        if (qrow_ok) {
+        } else {
+          uint32_t pk[C / 2];
 #pragma unroll
-          for (int c16 = 0; c16 < C / 8; ++c16) {
-            uint4 u = make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
-            *reinterpret_cast<uint4*>(pdst + (c16 >> 3) * C * 128 + sw128_off(qrow, c16 & 7)) = u;
+          for (int cb = 0; cb < C / 64; ++cb) {
+            uint32_t r[64];
+            tmem_ld64(t_sc + lane_off + cb * 64, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const int col = cb * 64 + j;
+              const float a0 = (col <= qrow) ? __uint_as_float(r[j]) : 0.f;
+              const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[j + 1]) : 0.f;
+              pk[col >> 1] = pack_bf16x2(a0, a1);
+            }
+          }
+          // the overlaid P must wait until (1)-(3) have read the Q and K
+          // slots; a separate P buffer only until (4) of the previous tile
+          // (o_full, waited in the previous O step)
+          uint8_t* pdst = Cfg::PSEP ? smem + NST * STAGE + Cfg::SBF : st;
+          if (!Cfg::PSEP && !dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);
+          if (qrow_ok) {
+#pragma unroll
+            for (int c16 = 0; c16 < C / 8; ++c16) {
+              uint4 u = make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
+              *reinterpret_cast<uint4*>(pdst + (c16 >> 3) * C * 128 + sw128_off(qrow, c16 & 7)) = u;
+            }
           }
         }
         fence_async_smem();
@@ -695,14 +729,20 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       if (it + 1 < nB) {
         if (Cfg::PSEP && !dead) dead = !mbar_wait(sdone, (hasA + it) & 1, lim);
         tc_fence_after();
-#pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb) {
-          uint32_t r[64];
-          tmem_ld64(t_w + lane_off + cb * 64, r);
+        const uint32_t wdst =
+            Cfg::MRG ? sbase + ((g + 1) % NST) * STAGE + Cfg::OK + wrow_of(it + 1) * 128 : sbase + NST * STAGE;
+        const int wblk = Cfg::MRG ? Cfg::KWR * 128 : D * 128;
+        if constexpr (D == 64) {
+          uint32_t r[32];
+          tmem_ld_half32(t_w + lane_off, r);
           tmem_ld_wait();
-          if (wrow_ok) {
-            uint8_t* wdst = Cfg::MRG ? smem + ((g + 1) % NST) * STAGE + Cfg::OK + wrow_of(it + 1) * 128 : sbf;
-            const int wblk = Cfg::MRG ? Cfg::KWR * 128 : D * 128;
+          store_row32_bf16(wdst, wblk, row64h, 32 * half, r);
+        } else {
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            uint32_t r[64];
+            tmem_ld64(t_w + lane_off + cb * 64, r);
+            tmem_ld_wait();
             store_row64_bf16(wdst, wblk, wrow, cb * 64, r);
           }
         }
@@ -712,16 +752,28 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
       }
       // O[b]: TMEM -> bf16 -> V slot, then the store warp takes it
       {
-        uint8_t* sv = st + Cfg::OV;
+        const uint32_t sv = sbase + s * STAGE + Cfg::OV;
         if (!dead) dead = !mbar_wait(&o_full[b], (it >> 1) & 1, lim);
         tc_fence_after();
         const uint32_t t_o = t_o_of(b);
-#pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb) {
-          uint32_t r[64];
-          tmem_ld64(t_o + lane_off + cb * 64, r);
+        if constexpr (C == 64 && D == 64) {
+          uint32_t r[32];
+          tmem_ld_half32(t_o + lane_off, r);
           tmem_ld_wait();
-          if (qrow_ok) store_row64_bf16(sv, C * 128, qrow, cb * 64, r);
+          store_row32_bf16(sv, C * 128, row64h, 32 * half, r);
+        } else if constexpr (C == 64) {
+          uint32_t r[64];
+          tmem_ld_half64(t_o + lane_off, r);
+          tmem_ld_wait();
+          store_row64_bf16(sv, C * 128, row64h, 64 * half, r);
+        } else {
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            uint32_t r[64];
+            tmem_ld64(t_o + lane_off + cb * 64, r);
+            tmem_ld_wait();
+            if (qrow_ok) store_row64_bf16(sv, C * 128, qrow, cb * 64, r);
+          }
         }
         tc_fence_before();
         mbar_arrive(&o_free[b]);
