@@ -338,8 +338,8 @@ def run_ours(args, c, ws, rank, local, info):
     ep = etah.pin_memory() if etah is not None else None
     oh = torch.empty(vh.shape, dtype=vh.dtype, pin_memory=True)
     Sh = torch.empty(c.B, c.H, c.d_v, c.d_k, dtype=torch.float32, pin_memory=True)
-    bufs = ttt.host.DeviceBuffers(qp, kp, vp, ep, device=dev)
-    kw = dict(eta_const=x["eta_const"], beta=c.beta, chunk=chunk, segments=args.segments, workspace=work)
+    bufs = ttt.host.HostStaging()
+    kw = dict(eta_const=x["eta_const"], beta=c.beta, chunk=chunk, segments=args.segments)
     e2e_steps = max(3, min(args.steps, 50))
     for _ in range(3):
         ttt.forward_chunked_host(qp, kp, vp, ep, o_host=oh, bufs=bufs, state_host=Sh, **kw)

@@ -157,6 +157,28 @@ TTT_LA_API ttt_la_status ttt_la_decode_step(const ttt_la_decode_args *args, void
 #define TTT_LA_STATIC_SCRATCH_BYTES (8u << 20)
 TTT_LA_API ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args *args, void *stream);
 
+/* Chunked forward with every tensor in host memory: q, k, v, eta, state_in,
+ * mom_in are read from, and o, state_out, mom_out written to, HOST pointers
+ * (page-locked memory lets the copies run asynchronously and overlap;
+ * pageable memory works but serialises them).  args->workspace is ignored.
+ * The B*H sequences are cut into up to 8 pieces of whole sequences; piece j
+ * is copied in on an internal stream while piece j-1 runs on `stream` and
+ * piece j-2 is copied out on a second internal stream, through two sets of
+ * staging buffers in `device_buf` (caller-owned device memory, 16-byte
+ * aligned, at least ttt_la_host_staging_size(args) bytes).  Each piece runs
+ * ttt_la_forward_chunked, so results agree with it up to the rounding of a
+ * different segment split.  Ordering follows `stream`: the copies start after
+ * the work already queued on it, and work queued on it after this call starts
+ * only once every output has reached host memory.  Returns once everything is
+ * queued (the host buffers must stay valid, and the inputs unchanged, until
+ * then).  Calls whose executions overlap must not share `device_buf`.
+ * Errors: as ttt_la_forward_chunked, plus TTT_LA_ERR_INVALID_ARG for a
+ * missing, misaligned or short `device_buf`.  The paper has no counterpart of
+ * this entry point; it is the end-to-end path for callers with host data. */
+TTT_LA_API size_t ttt_la_host_staging_size(const ttt_la_args *args);
+TTT_LA_API ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args *args, void *device_buf,
+                                                     size_t device_bytes, void *stream);
+
 /* Synchronises `stream`, returns the device status word (TTT_LA_OK or
  * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
 TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);

@@ -49,6 +49,8 @@ SIGNATURES = [
     ("ttt_la_workspace_size", _c_sz, [ctypes.POINTER(TttArgs)]),
     ("ttt_la_forward_chunked", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
     ("ttt_la_forward_chunked_noalloc", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
+    ("ttt_la_host_staging_size", _c_sz, [ctypes.POINTER(TttArgs)]),
+    ("ttt_la_forward_chunked_host", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp, _c_sz, _c_vp]),
     ("ttt_la_forward_recurrent", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
     ("ttt_la_decode_step", ctypes.c_int, [ctypes.POINTER(TttDecodeArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
@@ -179,6 +181,34 @@ def forward_chunked(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, c
         a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("ttt_la_forward_chunked", L.ttt_la_forward_chunked(ctypes.byref(a), _stream_handle(stream)))
     return o, S, M
+
+
+def forward_chunked_host(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, chunk=64, segments=0,
+                         state_in=None, mom_in=None, out=None, state_out=None, mom_out=None, staging=None,
+                         stream=None):
+    """Chunked forward on host tensors (ttt_la_forward_chunked_host): q, k, v,
+    eta, state_in, mom_in are read from, and out / state_out / mom_out written
+    to, contiguous CPU tensors (pinned ones let the copies overlap).  `staging`
+    is a uint8 CUDA tensor of at least host_staging_bytes(...) bytes, allocated
+    on the current device when missing or short.  Returns (o, staging); the
+    outputs are complete once `stream` (default: the current one) is."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k: [B,H,T,d_k]; v: [B,H,T,d_v]")
+    for t in (q, k, v, eta, state_in, mom_in, out, state_out, mom_out):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("forward_chunked_host takes contiguous host tensors")
+    o = torch.empty(v.shape, dtype=v.dtype, pin_memory=True) if out is None else out
+    a = _seq_args(q, k, v, eta, eta_const, beta, ascent, chunk, segments, state_in, mom_in, o, state_out, mom_out)
+    L = lib()
+    need = int(L.ttt_la_host_staging_size(ctypes.byref(a)))
+    if need == 0:
+        raise ValueError("invalid arguments for ttt_la_forward_chunked_host")
+    if staging is None or staging.numel() * staging.element_size() < need:
+        staging = torch.empty(need, dtype=torch.uint8, device="cuda")
+    _check("ttt_la_forward_chunked_host",
+           L.ttt_la_forward_chunked_host(ctypes.byref(a), ctypes.c_void_p(staging.data_ptr()),
+                                         staging.numel() * staging.element_size(), _stream_handle(stream)))
+    return o, staging
 
 
 def workspace_bytes(q, v, chunk=64, beta=0.0, segments=0):

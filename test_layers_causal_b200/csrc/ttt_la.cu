@@ -375,6 +375,8 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
 
 }  // namespace
 
+#include "host_pipeline.h"
+
 extern "C" {
 
 const char* ttt_la_status_string(ttt_la_status s) {
@@ -439,6 +441,79 @@ ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args* a, void* stream)
     b.workspace_bytes = TTT_LA_STATIC_SCRATCH_BYTES;
   }
   return ttt_la_forward_chunked(&b, stream);
+}
+
+size_t ttt_la_host_staging_size(const ttt_la_args* a) {
+  if (check_seq(a) != TTT_LA_OK) return 0;
+  return 2 * piece_layout(a).set_bytes;
+}
+
+ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args* a, void* device_buf, size_t device_bytes,
+                                          void* stream) {
+  ttt_la_status s = check_seq(a);
+  if (s != TTT_LA_OK) return s;
+  if (a->dtype == TTT_LA_F32) {
+    ttt::SimtShape sh;
+    if (!simt_supported(a, &sh)) return TTT_LA_ERR_UNSUPPORTED;
+  } else if (!tc_supported(a)) {
+    return TTT_LA_ERR_UNSUPPORTED;
+  }
+  const PieceLayout L = piece_layout(a);
+  if (!device_buf || !aligned16(device_buf) || device_bytes < 2 * L.set_bytes) return TTT_LA_ERR_INVALID_ARG;
+  HostPipe* hp = host_pipe();
+  if (!hp) return TTT_LA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hp->mu);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t es = a->dtype == TTT_LA_BF16 ? 2 : 4;
+  const int bh = a->B * a->H;
+  const size_t qrow = static_cast<size_t>(a->T) * a->d_k * es, vrow = static_cast<size_t>(a->T) * a->d_v * es;
+  const size_t erow = static_cast<size_t>(a->T) * sizeof(float);
+  const size_t srow = static_cast<size_t>(a->d_v) * a->d_k * sizeof(float);
+  auto h2d = [&](size_t dst, const void* src, size_t row, int first, int cnt, uint8_t* base) {
+    if (!src) return true;
+    return cudaMemcpyAsync(base + dst, static_cast<const uint8_t*>(src) + row * first, row * cnt,
+                           cudaMemcpyHostToDevice, hp->s_in) == cudaSuccess;
+  };
+  auto d2h = [&](void* dst, size_t src, size_t row, int first, int cnt, uint8_t* base) {
+    if (!dst) return true;
+    return cudaMemcpyAsync(static_cast<uint8_t*>(dst) + row * first, base + src, row * cnt, cudaMemcpyDeviceToHost,
+                           hp->s_out) == cudaSuccess;
+  };
+  // fork: the copy streams start after the caller's earlier work
+  if (cudaEventRecord(hp->fork, st) != cudaSuccess || cudaStreamWaitEvent(hp->s_in, hp->fork, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->s_out, hp->fork, 0) != cudaSuccess)
+    return TTT_LA_ERR_CUDA;
+  for (int j = 0; j < L.pieces; ++j) {
+    const int b = j & 1, first = j * L.per, cnt = std::min(L.per, bh - first);
+    uint8_t* base = static_cast<uint8_t*>(device_buf) + b * L.set_bytes;
+    // copy in, once the forward of piece j-2 has finished reading this set
+    if (j >= 2 && cudaStreamWaitEvent(hp->s_in, hp->done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    if (!h2d(L.q, a->q, qrow, first, cnt, base) || !h2d(L.k, a->k, qrow, first, cnt, base) ||
+        !h2d(L.v, a->v, vrow, first, cnt, base) || !h2d(L.eta, a->eta, erow, first, cnt, base) ||
+        !h2d(L.s_in, a->state_in, srow, first, cnt, base) || !h2d(L.m_in, a->mom_in, srow, first, cnt, base) ||
+        cudaEventRecord(hp->in_ready[b], hp->s_in) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    // forward on the caller's stream, once the inputs are in and piece j-2's
+    // outputs have left this set
+    if (cudaStreamWaitEvent(st, hp->in_ready[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    if (j >= 2 && cudaStreamWaitEvent(st, hp->out_done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    const ttt_la_args pa = piece_args(a, L, cnt, base);
+    s = ttt_la_forward_chunked(&pa, st);
+    if (s != TTT_LA_OK) return s;
+    if (cudaEventRecord(hp->done[b], st) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    // copy out
+    if (cudaStreamWaitEvent(hp->s_out, hp->done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    if (!d2h(a->o, L.o, vrow, first, cnt, base) || !d2h(a->state_out, L.s_out, srow, first, cnt, base) ||
+        !d2h(a->mom_out, L.m_out, srow, first, cnt, base) ||
+        cudaEventRecord(hp->out_done[b], hp->s_out) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+  }
+  // join: the caller's stream continues once every copy has completed
+  if (cudaEventRecord(hp->join_in, hp->s_in) != cudaSuccess ||
+      cudaEventRecord(hp->join_out, hp->s_out) != cudaSuccess ||
+      cudaStreamWaitEvent(st, hp->join_in, 0) != cudaSuccess || cudaStreamWaitEvent(st, hp->join_out, 0) != cudaSuccess)
+    return TTT_LA_ERR_CUDA;
+  return TTT_LA_OK;
 }
 
 ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {

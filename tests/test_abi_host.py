@@ -105,6 +105,9 @@ def test_invalid_arguments_rejected_before_launch(abi, bad):
     assert L.ttt_la_forward_chunked(ctypes.byref(a), None) == abi.ERR_INVALID_ARG
     assert L.ttt_la_forward_recurrent(ctypes.byref(a), None) == abi.ERR_INVALID_ARG
     assert L.ttt_la_workspace_size(ctypes.byref(a)) == 0
+    assert L.ttt_la_host_staging_size(ctypes.byref(a)) == 0
+    assert L.ttt_la_forward_chunked_host(ctypes.byref(a), ctypes.c_void_p(0x100000), 1 << 30, None) == \
+        abi.ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("cfg", [
@@ -168,3 +171,24 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _abi.lib()
+
+
+def test_host_staging_size_and_checks(abi):
+    """Two staging sets of up to 8 pieces: q, k, v, o (+ eta, states) per
+    piece at 256-byte alignment, plus the piece's scratch; a missing, short or
+    misaligned staging buffer is refused before anything is queued."""
+    L = abi.lib()
+    # 9 sequences -> pieces of 2; bf16 T=100 d=64: 4 tensors of 2*100*64*2 = 25600 B -> 25600 each
+    a = _args(abi, B=3, H=3, T=100, eta=0x50000)
+    per_set = 4 * 25600 + 1024  # + eta 2*100*4 = 800 -> 1024
+    ws = L.ttt_la_workspace_size(ctypes.byref(_args(abi, B=1, H=2, T=100)))
+    assert L.ttt_la_host_staging_size(ctypes.byref(a)) == 2 * (per_set + (ws + 255) // 256 * 256)
+    need = L.ttt_la_host_staging_size(ctypes.byref(a))
+    assert L.ttt_la_forward_chunked_host(ctypes.byref(a), None, need, None) == abi.ERR_INVALID_ARG
+    assert L.ttt_la_forward_chunked_host(ctypes.byref(a), ctypes.c_void_p(0x100000), need - 1, None) == \
+        abi.ERR_INVALID_ARG
+    assert L.ttt_la_forward_chunked_host(ctypes.byref(a), ctypes.c_void_p(0x100008), need, None) == \
+        abi.ERR_INVALID_ARG
+    unsupported = _args(abi, d_k=96, d_v=96)
+    assert L.ttt_la_forward_chunked_host(ctypes.byref(unsupported), ctypes.c_void_p(0x100000), 1 << 30, None) == \
+        abi.ERR_UNSUPPORTED
