@@ -65,17 +65,19 @@ struct TcMomCfg {
   static constexpr int OFF_P = OFF_QT + TILE;
   static constexpr int BIG = OFF_P + C * C * 2;
   static constexpr int NBAR = 3 * NST + 16;
-  static constexpr int SMALL = NBAR * 8 + (NST * (C + 1) + (C + 1) + 8) * 4 + 32;
+  static constexpr int SMALL = NBAR * 8 + (NST * (C + 1) + (C + 1) + 8 + 4 * C) * 4 + 32;
   static constexpr int SMEM = BIG + SMALL + 1024;
   static constexpr int TCOLS_USED = C + 3 * D;   // scores, O, W, M
   static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
   static constexpr int MINB = 1;
+  static constexpr int NSCW = 4;                 // K-scaling warps (7 and 8-10), 16 rows each
+  static constexpr int THREADS = 32 * (7 + NSCW);
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
+__global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
     chunked_tc_mom_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                           const TcMomParams p) {
@@ -99,10 +101,14 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
   uint64_t* o_full = kt_ready + 6;
   uint64_t* seg_ready = kt_ready + 7; // phase-A segment scalars G, B written
   uint64_t* drain = kt_ready + 8;
+  uint64_t* cl_ready = kt_ready + 9;   // [NST] coefficients of phase-B tile `it` in cls[it % NST]
+  uint64_t* cl_free = kt_ready + 11;   // [NST] the epilogue is done with cls[it % NST]
+  uint64_t* o_free = kt_ready + 13;    // O of the previous tile read out of TMEM
   float* cls = reinterpret_cast<float*>(smem + Cfg::BIG + Cfg::NBAR * 8);  // [NST][C+1] tile suffix sums
   float* bp = cls + NST * (C + 1);                                          // beta^k, k = 0..C
   float* segsc = bp + (C + 1);                                              // [0] G, [1] B of this segment
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(segsc + 8);
+  uint32_t* wpk = reinterpret_cast<uint32_t*>(segsc + 8);  // [2 tiles][K1, K2][C] bf16x2 row weights
+  uint32_t* tmem_holder = wpk + 4 * C;
   int* sh_tile = reinterpret_cast<int*>(tmem_holder + 1);
   int* sh_lb = sh_tile + 1;
 
@@ -115,7 +121,7 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
       mbar_init(&empty[s], 1);
       mbar_init(&staged[s], 128);
     }
-    mbar_init(kt_ready, 1);
+    mbar_init(kt_ready, Cfg::NSCW);
     mbar_init(kt_free, 1);
     mbar_init(sc_full, 1);
     mbar_init(sdone, 1);
@@ -124,6 +130,11 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
     mbar_init(o_full, 1);
     mbar_init(seg_ready, 1);
     mbar_init(drain, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&cl_ready[s], 1);
+      mbar_init(&cl_free[s], 128);
+    }
+    mbar_init(o_free, 128);
     fence_mbar_init();
     float b = 1.f;
     for (int k = 0; k <= C; ++k) {
@@ -166,7 +177,6 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
   uint8_t* k1s = smem + Cfg::OFF_K1;
   uint8_t* k2s = smem + Cfg::OFF_K2;
   uint8_t* qts = smem + Cfg::OFF_QT;
-  uint8_t* ps = smem + Cfg::OFF_P;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -231,18 +241,22 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
         if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);
         if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_K, kk > 0);
-          mma_bf16_ss(t_o, d_qt + k_step(C, kk), d_mbf + k_step(D, kk), ID_O_K, 1);
-        }
+        // (3) first: it needs only this tile's K1/K2 and the rewritten W, M
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
           mma_bf16_ss(t_w, dvm + mn_step(kk), d_k1 + mn_step(kk), ID_W, 1);
           mma_bf16_ss(t_m, dvm + mn_step(kk), d_k2 + mn_step(kk), ID_W, 1);
         }
-        tc_commit(sdone);
         tc_commit(kt_free);
+        // (2) overwrites O: the previous tile's O must have been read out
+        if (it > 0 && !dead) dead = !mbar_wait(o_free, (it - 1) & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_K, kk > 0);
+          mma_bf16_ss(t_o, d_qt + k_step(C, kk), d_mbf + k_step(D, kk), ID_O_K, 1);
+        }
+        tc_commit(sdone);
         if (!dead) dead = !mbar_wait(p_ready, it & 1, lim);
         tc_fence_after();
 #pragma unroll
@@ -269,8 +283,11 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
       }
       bulk_wait0();
     }
-  } else if (warp == 7) {
-    // ------------------------------------- coefficients and K scaling --
+  } else if (warp >= 7) {
+    // ------------------- coefficients (warp 7) and K scaling (warps 7-10) --
+    // Warp 7 scans the tile's learning rates and writes the row weights;
+    // the four scaling warps then each scale 16 rows of K into K1 and K2.
+    const int sw = warp - 7;
     bool dead = false;
     const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
     const float beta = p.beta, sigma = p.sigma;
@@ -278,76 +295,89 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
     for (int g = 0; g < NI; ++g) {
       const int s = g % NST;
       const int t0 = tile_of(g) * C;
-      // eta of rows 2*lane, 2*lane+1 (0 past the sequence end)
-      float e0 = 0.f, e1 = 0.f;
-      {
-        const int ta = t0 + 2 * lane, tb = ta + 1;
-        if (ta < p.T) e0 = eg ? __ldg(eg + ta) : p.eta_const;
-        if (tb < p.T) e1 = eg ? __ldg(eg + tb) : p.eta_const;
-      }
-      // suffix scan over the tile: value at row 2*lane given zero beyond the tile
-      float a = e0 + beta * e1, m = beta * beta;
+      uint32_t* wg = wpk + (g & 1) * 2 * C;  // this tile's weights (double-buffered)
+      if (sw == 0) {
+        // eta of rows 2*lane, 2*lane+1 (0 past the sequence end)
+        float e0 = 0.f, e1 = 0.f;
+        {
+          const int ta = t0 + 2 * lane, tb = ta + 1;
+          if (ta < p.T) e0 = eg ? __ldg(eg + ta) : p.eta_const;
+          if (tb < p.T) e1 = eg ? __ldg(eg + tb) : p.eta_const;
+        }
+        // suffix scan over the tile: value at row 2*lane given zero beyond the tile
+        float a = e0 + beta * e1, m = beta * beta;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float ah = __shfl_down_sync(0xffffffffu, a, off);
-        const float mh = __shfl_down_sync(0xffffffffu, m, off);
-        if (lane + off < 32) {
-          a = fmaf(m, ah, a);
-          m *= mh;
+        for (int off = 1; off < 32; off <<= 1) {
+          const float ah = __shfl_down_sync(0xffffffffu, a, off);
+          const float mh = __shfl_down_sync(0xffffffffu, m, off);
+          if (lane + off < 32) {
+            a = fmaf(m, ah, a);
+            m *= mh;
+          }
         }
-      }
-      float an = __shfl_down_sync(0xffffffffu, a, 1);
-      if (lane == 31) an = 0.f;
-      const float cl0 = a, cl1 = fmaf(beta, an, e1);  // cl at rows 2*lane, 2*lane+1
-      float* cl = cls + s * (C + 1);
-      cl[2 * lane] = cl0;
-      cl[2 * lane + 1] = cl1;
-      if (lane == 0) cl[C] = 0.f;
-      __syncwarp();
-      // per-row weights of the two scaled K tiles
-      float w1a, w1b, w2a, w2b;
-      if (g < nA) {
-        w1a = sigma * fmaf(bp[C - 2 * lane], R, cl0);
-        w1b = sigma * fmaf(bp[C - 2 * lane - 1], R, cl1);
-        w2a = -sigma * bp[C - 1 - 2 * lane] * Bc;
-        w2b = -sigma * bp[C - 2 - 2 * lane] * Bc;
-        R = fmaf(bp[C], R, __shfl_sync(0xffffffffu, cl0, 0));
-        Bc *= bp[C];
-        if (g == nA - 1 && lane == 0) {
-          segsc[0] = beta * R;  // G: beta * suffix coefficient at the segment's first token
-          segsc[1] = Bc;        // B = beta^L
-          mbar_arrive(seg_ready);
+        float an = __shfl_down_sync(0xffffffffu, a, 1);
+        if (lane == 31) an = 0.f;
+        const float cl0 = a, cl1 = fmaf(beta, an, e1);  // cl at rows 2*lane, 2*lane+1
+        if (g >= nA) {
+          // phase B: publish the tile's suffix sums for the epilogue, in slot
+          // it % NST once the epilogue is done with that slot's previous tile
+          const int it = g - nA;
+          if (it >= NST && !dead) dead = !mbar_wait(&cl_free[it % NST], ((it / NST) - 1) & 1, lim);
+          float* cl = cls + (it % NST) * (C + 1);
+          cl[2 * lane] = cl0;
+          cl[2 * lane + 1] = cl1;
+          if (lane == 0) cl[C] = 0.f;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&cl_ready[it % NST]);
         }
-      } else {
-        const int n = min(C, p.T - t0);
-        w1a = sigma * cl0;
-        w1b = sigma * cl1;
-        w2a = (2 * lane < n) ? -sigma * bp[n - 1 - 2 * lane] : 0.f;
-        w2b = (2 * lane + 1 < n) ? -sigma * bp[n - 2 - 2 * lane] : 0.f;
+        // per-row weights of the two scaled K tiles
+        float w1a, w1b, w2a, w2b;
+        if (g < nA) {
+          w1a = sigma * fmaf(bp[C - 2 * lane], R, cl0);
+          w1b = sigma * fmaf(bp[C - 2 * lane - 1], R, cl1);
+          w2a = -sigma * bp[C - 1 - 2 * lane] * Bc;
+          w2b = -sigma * bp[C - 2 - 2 * lane] * Bc;
+          R = fmaf(bp[C], R, __shfl_sync(0xffffffffu, cl0, 0));
+          Bc *= bp[C];
+          if (g == nA - 1 && lane == 0) {
+            segsc[0] = beta * R;  // G: beta * suffix coefficient at the segment's first token
+            segsc[1] = Bc;        // B = beta^L
+            mbar_arrive(seg_ready);
+          }
+        } else {
+          const int n = min(C, p.T - t0);
+          w1a = sigma * cl0;
+          w1b = sigma * cl1;
+          w2a = (2 * lane < n) ? -sigma * bp[n - 1 - 2 * lane] : 0.f;
+          w2b = (2 * lane + 1 < n) ? -sigma * bp[n - 2 - 2 * lane] : 0.f;
+        }
+        // row weights as bf16 pairs (each product is then rounded to bf16 as
+        // the operand itself would be)
+        wg[2 * lane] = pack_bf16x2(w1a, w1a);
+        wg[2 * lane + 1] = pack_bf16x2(w1b, w1b);
+        wg[C + 2 * lane] = pack_bf16x2(w2a, w2a);
+        wg[C + 2 * lane + 1] = pack_bf16x2(w2b, w2b);
       }
+      // the weights are visible to the four scaling warps; a warp passes this
+      // barrier for tile g only after finishing tile g-1, so the other
+      // weight buffer is free for warp 7 to fill next
+      asm volatile("bar.sync 2, %0;" ::"n"(32 * Cfg::NSCW) : "memory");
       if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
       if (g > 0 && !dead) dead = !mbar_wait(kt_free, (g - 1) & 1, lim);
-      // K1 = diag(w1) K, K2 = diag(w2) K; row r's weights live in lane r/2
+      // K1 = diag(w1) K, K2 = diag(w2) K for rows [16 sw, 16 sw + 16), packed bf16 multiplies
       const uint8_t* sk = smem + s * STAGE + TILE;
-      constexpr int PER_LANE = C * (D / 8) / 32;
-#pragma unroll 4
+      constexpr int PER_LANE = 16 * (D / 8) / 32;
+#pragma unroll
       for (int i = 0; i < PER_LANE; ++i) {
         const int idx = lane + 32 * i;
-        const int r = idx / (D / 8), cc = idx % (D / 8);
+        const int r = 16 * sw + idx / (D / 8), cc = idx % (D / 8);
         const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
-        const int src = r >> 1;
-        const float x1a = __shfl_sync(0xffffffffu, w1a, src), x1b = __shfl_sync(0xffffffffu, w1b, src);
-        const float x2a = __shfl_sync(0xffffffffu, w2a, src), x2b = __shfl_sync(0xffffffffu, w2b, src);
-        const float f1 = (r & 1) ? x1b : x1a, f2 = (r & 1) ? x2b : x2a;
+        const uint32_t f1 = wg[r], f2 = wg[C + r];
         const uint4 u = *reinterpret_cast<const uint4*>(sk + off);
-        uint4 v1, v2;
-        float2 t;
-        t = unpack_bf16x2(u.x); v1.x = pack_bf16x2(t.x * f1, t.y * f1); v2.x = pack_bf16x2(t.x * f2, t.y * f2);
-        t = unpack_bf16x2(u.y); v1.y = pack_bf16x2(t.x * f1, t.y * f1); v2.y = pack_bf16x2(t.x * f2, t.y * f2);
-        t = unpack_bf16x2(u.z); v1.z = pack_bf16x2(t.x * f1, t.y * f1); v2.z = pack_bf16x2(t.x * f2, t.y * f2);
-        t = unpack_bf16x2(u.w); v1.w = pack_bf16x2(t.x * f1, t.y * f1); v2.w = pack_bf16x2(t.x * f2, t.y * f2);
-        *reinterpret_cast<uint4*>(k1s + off) = v1;
-        *reinterpret_cast<uint4*>(k2s + off) = v2;
+        *reinterpret_cast<uint4*>(k1s + off) =
+            make_uint4(mul_bf16x2(u.x, f1), mul_bf16x2(u.y, f1), mul_bf16x2(u.z, f1), mul_bf16x2(u.w, f1));
+        *reinterpret_cast<uint4*>(k2s + off) =
+            make_uint4(mul_bf16x2(u.x, f2), mul_bf16x2(u.y, f2), mul_bf16x2(u.z, f2), mul_bf16x2(u.w, f2));
       }
       fence_async_smem();
       __syncwarp();
@@ -363,8 +393,8 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
     const bool ok64 = lane < 16;
     const int wrow = (D == 128) ? row128 : row64;
     const bool wrow_ok = (D == 128) || ok64;
-    const int qrow = row64;  // C = 64
-    const bool qrow_ok = ok64;
+    // 64-row tiles read with the whole warp: row 16*g4 + lane%16, column half lane/16
+    const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
     const float beta = p.beta, sigma = p.sigma;
     bool dead = false;
     const size_t DD = static_cast<size_t>(D) * D;
@@ -472,12 +502,18 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
           tmem_ld32(t_m + lane_off + cb * 32, r2);
           tmem_ld_wait();
           if (wrow_ok) {
-            float* iw = me + 2 * DD + off;
-            float* im = me + 3 * DD + off;
+            float4* iw = reinterpret_cast<float4*>(me + 2 * DD + off);
+            float4* im = reinterpret_cast<float4*>(me + 3 * DD + off);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              iw[j] = fmaf(-Gme, mm[j], w[j]) + __uint_as_float(r[j]);
-              im[j] = fmaf(Bme, mm[j], __uint_as_float(r2[j]));
+            for (int j = 0; j < 32; j += 4) {
+              iw[j / 4] = make_float4(fmaf(-Gme, mm[j], w[j]) + __uint_as_float(r[j]),
+                                      fmaf(-Gme, mm[j + 1], w[j + 1]) + __uint_as_float(r[j + 1]),
+                                      fmaf(-Gme, mm[j + 2], w[j + 2]) + __uint_as_float(r[j + 2]),
+                                      fmaf(-Gme, mm[j + 3], w[j + 3]) + __uint_as_float(r[j + 3]));
+              im[j / 4] = make_float4(fmaf(Bme, mm[j], __uint_as_float(r2[j])),
+                                      fmaf(Bme, mm[j + 1], __uint_as_float(r2[j + 1])),
+                                      fmaf(Bme, mm[j + 2], __uint_as_float(r2[j + 2])),
+                                      fmaf(Bme, mm[j + 3], __uint_as_float(r2[j + 3])));
             }
           }
         }
@@ -498,14 +534,16 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
     }
 
     // ---- phase B
-    for (int it = 0; it < nB; ++it) {
+    // Per tile: Step W, Step P, Step O.  (O is staged in the tile's V slot, so
+    // the stage is refilled only after Step O; doing the next Step W first
+    // delays that refill by more than it gains.)
+    auto step_w = [&](int it) {
       const int g = nA + it, s = g % NST;
-      const int t0 = (chunk0 + it) * C;
-      const int n = min(C, p.T - t0);
+      const int n = min(C, p.T - (chunk0 + it) * C);
       uint8_t* st = smem + s * STAGE;
-      const float* cl = cls + s * (C + 1);
+      const float* cl = cls + (it % NST) * (C + 1);
       // Step W: Wbf, Mbf from the state entering this tile; W -= g_end M; M *= beta^n; Q~ = diag(-g) Q
-      if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);  // the tile's cl is in smem
+      if (!dead) dead = !mbar_wait(&cl_ready[it % NST], (it / NST) & 1, lim);  // the tile's cl is in smem
       if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);  // its Q has landed
       if (it > 0 && !dead) dead = !mbar_wait(sdone, ((nA > 0 ? 1 : 0) + it - 1) & 1, lim);
       tc_fence_after();
@@ -530,80 +568,84 @@ __global__ void __launch_bounds__(256, TcMomCfg<D>::MINB)
         tmem_st32(t_w + lane_off + cb * 32, r);
         tmem_st32(t_m + lane_off + cb * 32, r2);
       }
-      if (qrow_ok) {
-        const float gi = beta * fmaf(-bp[qrow + 1], cl[qrow + 1], cl[0]);
-        const float f = -gi;
+      {
+        // this thread's half of row row64h of Q~ = diag(-g) Q
+        const float f = -beta * fmaf(-bp[row64h + 1], cl[row64h + 1], cl[0]);
+        const uint32_t f2 = pack_bf16x2(f, f);
 #pragma unroll
-        for (int cc = 0; cc < D / 8; ++cc) {
-          const uint32_t off = (cc >> 3) * C * 128 + sw128_off(qrow, cc & 7);
+        for (int i = 0; i < D / 16; ++i) {
+          const int cc = half * (D / 16) + i;
+          const uint32_t off = (cc >> 3) * C * 128 + sw128_off(row64h, cc & 7);
           const uint4 u = *reinterpret_cast<const uint4*>(st + off);
-          uint4 v;
-          float2 t;
-          t = unpack_bf16x2(u.x); v.x = pack_bf16x2(t.x * f, t.y * f);
-          t = unpack_bf16x2(u.y); v.y = pack_bf16x2(t.x * f, t.y * f);
-          t = unpack_bf16x2(u.z); v.z = pack_bf16x2(t.x * f, t.y * f);
-          t = unpack_bf16x2(u.w); v.w = pack_bf16x2(t.x * f, t.y * f);
-          *reinterpret_cast<uint4*>(qts + off) = v;
+          *reinterpret_cast<uint4*>(qts + off) =
+              make_uint4(mul_bf16x2(u.x, f2), mul_bf16x2(u.y, f2), mul_bf16x2(u.z, f2), mul_bf16x2(u.w, f2));
         }
       }
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(wbf_ready);
-
-      // Step P: P_ij = sigma * c_ij * Sc_ij for j <= i
+    };
+    auto step_p = [&](int it) {
+      const float* cl = cls + (it % NST) * (C + 1);
+      // Step P: P_ij = sigma * c_ij * Sc_ij for j <= i (this thread: half of row row64h)
       {
         if (!dead) dead = !mbar_wait(sc_full, it & 1, lim);
         tc_fence_after();
-        uint32_t r[2][32];
-        tmem_ld32(t_sc + lane_off, r[0]);
-        tmem_ld32(t_sc + lane_off + 32, r[1]);
+        uint32_t r[32];
+        tmem_ld_half32(t_sc + lane_off, r);
         tmem_ld_wait();
-        if (qrow_ok) {
-          const float cnext = cl[qrow + 1];
-          uint32_t pk[C / 2];
+        const float cnext = cl[row64h + 1];
+        const uint32_t pdst = sbase + Cfg::OFF_P;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+        for (int i = 0; i < 4; ++i) {
+          uint32_t w[4];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const int col = h * 32 + j;
-              float a0 = 0.f, a1 = 0.f;
-              if (col <= qrow) a0 = sigma * fmaf(-bp[qrow + 1 - col], cnext, cl[col]) * __uint_as_float(r[h][j]);
-              if (col + 1 <= qrow)
-                a1 = sigma * fmaf(-bp[qrow - col], cnext, cl[col + 1]) * __uint_as_float(r[h][j + 1]);
-              pk[col >> 1] = pack_bf16x2(a0, a1);
-            }
+          for (int e = 0; e < 4; ++e) {
+            const int j = 8 * i + 2 * e, col = 32 * half + j;
+            float a0 = 0.f, a1 = 0.f;
+            if (col <= row64h) a0 = sigma * fmaf(-bp[row64h + 1 - col], cnext, cl[col]) * __uint_as_float(r[j]);
+            if (col + 1 <= row64h)
+              a1 = sigma * fmaf(-bp[row64h - col], cnext, cl[col + 1]) * __uint_as_float(r[j + 1]);
+            w[e] = pack_bf16x2(a0, a1);
           }
-#pragma unroll
-          for (int c16 = 0; c16 < C / 8; ++c16) {
-            const uint4 u = make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
-            *reinterpret_cast<uint4*>(ps + sw128_off(qrow, c16)) = u;
-          }
+          st_shared_v4(pdst + sw128_off(row64h, 4 * half + i), w[0], w[1], w[2], w[3]);
         }
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(p_ready);
+        mbar_arrive(&cl_free[it % NST]);  // last use of this tile's coefficients
       }
-
-      // Step O
+    };
+    auto step_o = [&](int it) {
+      // Step O (this thread: half of row row64h)
       {
-        uint8_t* sv = st + 2 * TILE;
+        const uint32_t sv = sbase + ((nA + it) % NST) * STAGE + 2 * TILE;
         if (!dead) dead = !mbar_wait(o_full, it & 1, lim);
         tc_fence_after();
-#pragma unroll
-        for (int cb = 0; cb < D / 32; cb += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(t_o + lane_off + cb * 32, r0);
-          tmem_ld32(t_o + lane_off + cb * 32 + 32, r1);
+        if constexpr (D == 64) {
+          uint32_t r[32];
+          tmem_ld_half32(t_o + lane_off, r);
           tmem_ld_wait();
-          if (qrow_ok) {
-            store_row32_bf16(sv, C * 128, qrow, cb * 32, r0);
-            store_row32_bf16(sv, C * 128, qrow, cb * 32 + 32, r1);
-          }
+          tc_fence_before();
+          mbar_arrive(o_free);
+          store_row32_bf16(sv, C * 128, row64h, 32 * half, r);
+        } else {
+          uint32_t r[64];
+          tmem_ld_half64(t_o + lane_off, r);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(o_free);
+          store_row64_bf16(sv, C * 128, row64h, 64 * half, r);
         }
         fence_async_smem();
         mbar_arrive(&staged[it % NST]);
       }
+    };
+    for (int it = 0; it < nB; ++it) {
+      step_w(it);
+      step_p(it);
+      step_o(it);
     }
 
     // final state (last segment)

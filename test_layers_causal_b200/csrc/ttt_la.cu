@@ -298,7 +298,7 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
-  ttt::chunked_tc_mom_kernel<D><<<bh * sp.nseg, 256, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
+  ttt::chunked_tc_mom_kernel<D><<<bh * sp.nseg, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
   return launched();
 }
 
