@@ -450,6 +450,10 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         if (p.M_in) bm = p.M_in + static_cast<size_t>(bh) * DD;
       }
       const float Gme = (nA > 0) ? segsc[0] : 0.f, Bme = (nA > 0) ? segsc[1] : 1.f;
+      // With few segments every block reads all its predecessors' totals (at
+      // most a few maps); publishing inclusive states as well would double
+      // the scratch writes, which cost more than the reads they save.
+      const bool pub_incl = nA > 0 && p.nseg > 8;
 #pragma unroll 1
       for (int cb = 0; cb < D / 32; ++cb) {
         float w[32], mm[32];
@@ -497,7 +501,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           }
         }
         uint32_t r[32], r2[32];
-        if (nA > 0) {  // inclusive state after this segment, from its totals in TMEM
+        if (pub_incl) {  // inclusive state after this segment, from its totals in TMEM
           tmem_ld32(t_w + lane_off + cb * 32, r);
           tmem_ld32(t_m + lane_off + cb * 32, r2);
           tmem_ld_wait();
@@ -526,7 +530,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         tmem_st32(t_m + lane_off + cb * 32, r2);
       }
       tmem_st_wait();
-      if (nA > 0) {
+      if (pub_incl) {
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) st_release(flag_me, 2u);

@@ -217,6 +217,23 @@ def test_chunked_tc_states_at_16_byte_alignment(beta, segments):
         assert_bf16(M, M_ref, "momentum")
 
 
+@pytest.mark.parametrize("d,segments", [(64, 12), (128, 10)])
+def test_chunked_tc_momentum_many_segments(d, segments):
+    """Enough segments that each publishes its inclusive state and later ones
+    start from the nearest published one (few segments read totals only)."""
+    B, H, T = 1, 2, segments * 2 * 64 - 17
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 170 + d)
+    S0 = _state(B, H, d, d, 13, scale=0.1)
+    M0 = _state(B, H, d, d, 14, scale=0.1)
+    o, S, M = ttt.forward_chunked(q, k, v, eta, beta=0.9, chunk=64, segments=segments, state_in=S0, mom_in=M0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, ec, 0.9, False, S0, M0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+    assert_bf16(M, M_ref, "momentum")
+
+
 def test_chunked_tc_momentum_const_eta_zero_state():
     q, k, v, _, ec = _case(1, 3, 500, 128, 128, "bf16", 111, token_eta=False)
     o, S, M = ttt.forward_chunked(q, k, v, None, eta_const=ec, beta=0.9, chunk=128, segments=2)
