@@ -161,7 +161,8 @@ TTT_LA_API ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args *args,
  * mom_in are read from, and o, state_out, mom_out written to, HOST pointers
  * (page-locked memory lets the copies run asynchronously and overlap;
  * pageable memory works but serialises them).  args->workspace is ignored.
- * The B*H sequences are cut into up to 8 pieces of whole sequences; piece j
+ * The B*H sequences are cut into 2 to 8 pieces of whole sequences (about
+ * 24 MB of inputs each, at most one piece per sequence); piece j
  * is copied in on an internal stream while piece j-1 runs on `stream` and
  * piece j-2 is copied out on a second internal stream, through two sets of
  * staging buffers in `device_buf` (caller-owned device memory, 16-byte

@@ -69,10 +69,17 @@ ttt_la_args piece_args(const ttt_la_args* a, const PieceLayout& L, int cnt, uint
 PieceLayout piece_layout(const ttt_la_args* a) {
   PieceLayout L;
   const int bh = a->B * a->H;
-  L.pieces = std::min(bh, 8);
+  const size_t es = a->dtype == TTT_LA_BF16 ? 2 : 4;
+  // about 24 MB of inputs per piece, 2 to 8 pieces: more, smaller pieces hide
+  // more of the copy-out but each costs a launch and a pipeline hand-off
+  const size_t st_all = static_cast<size_t>(a->d_v) * a->d_k * sizeof(float) *
+                        ((a->state_in ? 1 : 0) + (a->mom_in ? 1 : 0));
+  const size_t in_bytes = static_cast<size_t>(bh) *
+                          (static_cast<size_t>(a->T) * ((2 * a->d_k + a->d_v) * es + (a->eta ? 4 : 0)) + st_all);
+  const int want = static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, in_bytes / (24u << 20))));
+  L.pieces = std::min(bh, want);
   L.per = (bh + L.pieces - 1) / L.pieces;
   L.pieces = (bh + L.per - 1) / L.per;
-  const size_t es = a->dtype == TTT_LA_BF16 ? 2 : 4;
   const size_t tok = static_cast<size_t>(L.per) * a->T;
   const size_t st = static_cast<size_t>(L.per) * a->d_v * a->d_k * sizeof(float);
   size_t off = 0;

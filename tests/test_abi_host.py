@@ -178,10 +178,11 @@ def test_host_staging_size_and_checks(abi):
     piece at 256-byte alignment, plus the piece's scratch; a missing, short or
     misaligned staging buffer is refused before anything is queued."""
     L = abi.lib()
-    # 9 sequences -> pieces of 2; bf16 T=100 d=64: 4 tensors of 2*100*64*2 = 25600 B -> 25600 each
+    # 9 small sequences -> the minimum of 2 pieces, of 5 sequences; bf16 T=100 d=64:
+    # 4 tensors of 5*100*64*2 = 64000 B (a multiple of 256) each, eta 5*100*4 = 2000 -> 2048
     a = _args(abi, B=3, H=3, T=100, eta=0x50000)
-    per_set = 4 * 25600 + 1024  # + eta 2*100*4 = 800 -> 1024
-    ws = L.ttt_la_workspace_size(ctypes.byref(_args(abi, B=1, H=2, T=100)))
+    per_set = 4 * 64000 + 2048
+    ws = L.ttt_la_workspace_size(ctypes.byref(_args(abi, B=1, H=5, T=100)))
     assert L.ttt_la_host_staging_size(ctypes.byref(a)) == 2 * (per_set + (ws + 255) // 256 * 256)
     need = L.ttt_la_host_staging_size(ctypes.byref(a))
     assert L.ttt_la_forward_chunked_host(ctypes.byref(a), None, need, None) == abi.ERR_INVALID_ARG
