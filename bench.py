@@ -65,9 +65,12 @@ def executed_flops(c, B, H, T, chunk):
 
 
 def src_hash():
+    """Hash of the kernel sources and their launch planner (the device code in
+    csrc/*.cuh and ttt_la.cu; the host-buffer pipeline does not change what a
+    kernel launch reads or writes)."""
     h = hashlib.sha1()
     cdir = os.path.join(ROOT, "test_layers_causal_b200", "csrc")
-    for f in sorted(os.listdir(cdir)):
+    for f in sorted(x for x in os.listdir(cdir) if x.endswith(".cuh") or x == "ttt_la.cu"):
         with open(os.path.join(cdir, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
