@@ -42,9 +42,10 @@ struct TcMomParams {
   float eta_const, sigma, beta;
   const float* S_in;   // [BH, dv, dk] or nullptr
   const float* M_in;   // [BH, dv, dk] or nullptr
-  float* ws;           // [BH, nseg, 4, dv, dk]: dW, dM, W_incl, M_incl
+  float* ws;           // [BH, nseg, 4, dv, dk]: dW, dM, then W, M inclusive (look-back) or at the start (prefix)
   float* wsc;          // [BH, nseg, 2]: G, B of each segment map
-  unsigned* flags;     // [BH * nseg] flags, then a tile counter
+  unsigned* flags;     // [BH * nseg] flags, a tile counter, [BH] head counters
+  int coop;            // 1: cooperative prefix (grid is one wave), 0: decoupled look-back
   float* S_out;
   float* M_out;
   uint64_t limit_ns;
@@ -432,28 +433,97 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) st_release(flag_me, 1u);
       }
-      if (et == 0) sh_lb[1] = -1;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int j = et; j < seg; j += 128) {
-        const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
-        if (f == 0) dead = true;
-        if (f >= 2) atomicMax(&sh_lb[1], j);
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int incl = sh_lb[1], first = incl + 1;
       const float *bw = nullptr, *bm = nullptr;
-      if (incl >= 0) {
-        bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 4 + 2) * DD;
+      int first = 0;
+      if (p.coop && p.nseg > 1) {
+        // Cooperative prefix (the grid is one wave, so the head's nseg blocks
+        // are resident together): once every segment map is published, block
+        // `seg` runs element slice `seg` of (W, M) through all the maps in
+        // order, coalesced, writing each segment's start state into its
+        // slots 2 and 3; the blocks meet at the head's counter and each then
+        // reads its own start state.
+        for (int j = et; j < p.nseg - 1; j += 128)
+          if (!dead && wait_geq(p.flags + bh * p.nseg + j, 1u, lim) == 0) dead = true;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int DDi = D * D;
+        const int SL = ((DDi + p.nseg - 1) / p.nseg + 31) / 32 * 32;  // slice, a multiple of 32
+        const int v1 = min(DDi, (seg + 1) * SL) / 4;
+        const int nagg = p.nseg - 1;
+        float4* w4 = reinterpret_cast<float4*>(p.ws + static_cast<size_t>(bh) * p.nseg * 4 * DD);
+        const size_t SEG4 = DD, Q4 = DD / 4;  // float4 strides: between segments, between a segment's matrices
+        const float* maps = p.wsc + static_cast<size_t>(bh) * p.nseg * 2;
+        const float4* sw4 = p.S_in ? reinterpret_cast<const float4*>(p.S_in + static_cast<size_t>(bh) * DD) : nullptr;
+        const float4* sm4 = p.M_in ? reinterpret_cast<const float4*>(p.M_in + static_cast<size_t>(bh) * DD) : nullptr;
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = seg * SL / 4 + et; v < v1; v += 128) {
+          float4 w = sw4 ? __ldcg(sw4 + v) : zero, m = sm4 ? __ldcg(sm4 + v) : zero;
+          for (int j = 0; j < nagg; j += 4) {
+            float4 dw[4], dm[4];
+            float G[4], B[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (j + u < nagg) {
+                dw[u] = __ldcg(w4 + (j + u) * SEG4 + v);
+                dm[u] = __ldcg(w4 + (j + u) * SEG4 + Q4 + v);
+                G[u] = __ldcg(maps + 2 * (j + u));
+                B[u] = __ldcg(maps + 2 * (j + u) + 1);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (j + u < nagg) {
+                __stcg(w4 + (j + u) * SEG4 + 2 * Q4 + v, w);
+                __stcg(w4 + (j + u) * SEG4 + 3 * Q4 + v, m);
+                // (W, M) -> (W - G M + dW, B M + dM)
+                w = make_float4(fmaf(-G[u], m.x, w.x) + dw[u].x, fmaf(-G[u], m.y, w.y) + dw[u].y,
+                                fmaf(-G[u], m.z, w.z) + dw[u].z, fmaf(-G[u], m.w, w.w) + dw[u].w);
+                m = make_float4(fmaf(B[u], m.x, dm[u].x), fmaf(B[u], m.y, dm[u].y), fmaf(B[u], m.z, dm[u].z),
+                                fmaf(B[u], m.w, dm[u].w));
+              }
+            }
+          }
+          __stcg(w4 + nagg * SEG4 + 2 * Q4 + v, w);
+          __stcg(w4 + nagg * SEG4 + 3 * Q4 + v, m);
+        }
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        unsigned* cnt = p.flags + p.BH * p.nseg + 1 + bh;
+        if (et == 0) {
+          atomicAdd(cnt, 1u);
+          if (!dead && wait_geq(cnt, static_cast<unsigned>(p.nseg), lim) == 0) dead = true;
+          __threadfence();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + seg) * 4 + 2) * DD;
         bm = bw + DD;
+        first = seg;
       } else {
-        if (p.S_in) bw = p.S_in + static_cast<size_t>(bh) * DD;
-        if (p.M_in) bm = p.M_in + static_cast<size_t>(bh) * DD;
+        // Decoupled look-back: every predecessor has published at least its
+        // map; the nearest one that has also published its inclusive state
+        // cuts the composition short.
+        if (et == 0) sh_lb[1] = -1;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int j = et; j < seg; j += 128) {
+          const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
+          if (f == 0) dead = true;
+          if (f >= 2) atomicMax(&sh_lb[1], j);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int incl = sh_lb[1];
+        first = incl + 1;
+        if (incl >= 0) {
+          bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 4 + 2) * DD;
+          bm = bw + DD;
+        } else {
+          if (p.S_in) bw = p.S_in + static_cast<size_t>(bh) * DD;
+          if (p.M_in) bm = p.M_in + static_cast<size_t>(bh) * DD;
+        }
       }
       const float Gme = (nA > 0) ? segsc[0] : 0.f, Bme = (nA > 0) ? segsc[1] : 1.f;
       // With few segments every block reads all its predecessors' totals (at
       // most a few maps); publishing inclusive states as well would double
       // the scratch writes, which cost more than the reads they save.
-      const bool pub_incl = nA > 0 && p.nseg > 8;
+      const bool pub_incl = !p.coop && nA > 0 && p.nseg > 8;
 #pragma unroll 1
       for (int cb = 0; cb < D / 32; ++cb) {
         float w[32], mm[32];

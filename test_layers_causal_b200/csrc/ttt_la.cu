@@ -291,6 +291,8 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
   p.S_out = a->state_out;
   p.M_out = a->mom_out;
   p.limit_ns = g_limit_ns;
+  // cooperative start states whenever the whole grid is one wave (one block per SM)
+  p.coop = (sp.nseg > 1 && static_cast<long long>(bh) * sp.nseg <= sm_count()) ? 1 : 0;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
     p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;

@@ -217,11 +217,13 @@ def test_chunked_tc_states_at_16_byte_alignment(beta, segments):
         assert_bf16(M, M_ref, "momentum")
 
 
-@pytest.mark.parametrize("d,segments", [(64, 12), (128, 10)])
-def test_chunked_tc_momentum_many_segments(d, segments):
-    """Enough segments that each publishes its inclusive state and later ones
-    start from the nearest published one (few segments read totals only)."""
-    B, H, T = 1, 2, segments * 2 * 64 - 17
+@pytest.mark.parametrize("d,segments,H", [(64, 12, 2), (128, 10, 2), (64, 12, 16), (128, 5, 32)])
+def test_chunked_tc_momentum_many_segments(d, segments, H):
+    """Start states with many segments.  A grid of at most one block per SM
+    takes the cooperative prefix (H = 2); a larger grid the decoupled
+    look-back, with inclusive states published beyond 8 segments (H = 16:
+    192 blocks, 12 segments) and totals only below (H = 32: 160 blocks)."""
+    B, T = 1, segments * 2 * 64 - 17
     q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 170 + d)
     S0 = _state(B, H, d, d, 13, scale=0.1)
     M0 = _state(B, H, d, d, 14, scale=0.1)
