@@ -468,11 +468,12 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
           tmem_ld32(t_w + lane_off + cb * 32, r);
           tmem_ld_wait();
           if (wrow_ok) {
-            float4* d4 = reinterpret_cast<float4*>(agg_me + static_cast<size_t>(wrow) * D + cb * 32);
+            float4* a4 = reinterpret_cast<float4*>(agg_me);  // quad-major
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              __stcg(a4 + qm4<D>(wrow, cb * 8 + j),
+                     make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
           }
         }
         __threadfence();
@@ -500,8 +501,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         // two vectors per thread per round, four totals per round
         for (int v = seg * SL / 4 + et; v < v1; v += 256) {
           const bool two = v + 128 < v1;
-          float4 run0 = s4 ? __ldcg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-          float4 run1 = (s4 && two) ? __ldcg(s4 + v + 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+          // the scratch is quad-major, the caller's W_0 row-major
+          float4 run0 = s4 ? __ldcg(s4 + qm4_to_rm4<D>(v)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 run1 = (s4 && two) ? __ldcg(s4 + qm4_to_rm4<D>(v + 128)) : make_float4(0.f, 0.f, 0.f, 0.f);
           for (int j = 0; j < nagg; j += 4) {
             float4 a0[4], a1[4];
 #pragma unroll
@@ -540,13 +542,12 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         // before any store (one round trip), with d = 64 one 32-column block
         // per round (register budget of two blocks per SM)
         constexpr int G = (D == 128) ? D / 32 : 1;
-        const size_t off = static_cast<size_t>(wrow) * D;
 #pragma unroll
         for (int cb0 = 0; cb0 < D / 32; cb0 += G) {
           float row[G * 32];
 #pragma unroll
           for (int c = 0; c < G * 8; ++c) {
-            const float4 x = wrow_ok ? __ldcg(reinterpret_cast<const float4*>(base + off + cb0 * 32) + c)
+            const float4 x = wrow_ok ? __ldcg(reinterpret_cast<const float4*>(base) + qm4<D>(wrow, cb0 * 8 + c))
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
             row[4 * c] = x.x, row[4 * c + 1] = x.y, row[4 * c + 2] = x.z, row[4 * c + 3] = x.w;
           }
@@ -572,6 +573,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
         // (start + total) cuts the sum short.  One thread per predecessor
         // reads the flags.
         int first = 0;
+        bool base_qm = false;  // base is a published (quad-major) state, not the caller's W_0
         if (seg > 0) {
           if (et == 0) sh_lb[1] = -1;
           asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -582,7 +584,10 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
           const int incl = sh_lb[1];
-          if (incl >= 0) base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
+          if (incl >= 0) {
+            base = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD;
+            base_qm = true;
+          }
           first = incl + 1;
         }
 #pragma unroll
@@ -591,37 +596,39 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
 #pragma unroll
           for (int j = 0; j < 32; ++j) acc[j] = 0.f;
           if (wrow_ok) {
-            const size_t off = static_cast<size_t>(wrow) * D + cb * 32;
             if (base) {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const float8 x = ld_cg_f8(base + off + 8 * j);
+                const float8 x = base_qm ? ld_cg_f8_qm<D>(base, wrow, cb * 8 + 2 * j)
+                                         : ld_cg_f8(base + static_cast<size_t>(wrow) * D + cb * 32 + 8 * j);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) acc[8 * j + e] = x.v[e];
               }
             }
-            // four totals per round: 32 independent 16-byte loads in flight
+            // NR totals per round (4 x NR x 2 independent 16-byte loads in
+            // flight; two for 64-wide rows, within their register budget)
+            constexpr int NR = (D == 128) ? 4 : 2;
             int jj = first;
-            for (; jj + 4 <= seg; jj += 4) {
-              float8 x[4][4];
+            for (; jj + NR <= seg; jj += NR) {
+              float8 x[NR][4];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD + off;
+              for (int u = 0; u < NR; ++u) {
+                const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) x[u][j] = ld_cg_f8(ag + 8 * j);
+                for (int j = 0; j < 4; ++j) x[u][j] = ld_cg_f8_qm<D>(ag, wrow, cb * 8 + 2 * j);
               }
 #pragma unroll
-              for (int u = 0; u < 4; ++u)
+              for (int u = 0; u < NR; ++u)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
                   for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[u][j].v[e];
             }
             for (; jj < seg; ++jj) {
-              const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD + off;
+              const float* ag = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD;
               float8 x[4];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) x[j] = ld_cg_f8(ag + 8 * j);
+              for (int j = 0; j < 4; ++j) x[j] = ld_cg_f8_qm<D>(ag, wrow, cb * 8 + 2 * j);
 #pragma unroll
               for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -633,12 +640,13 @@ __global__ void __launch_bounds__(256, TcCfg<C, D>::MINB)
             tmem_ld32(t_w + lane_off + cb * 32, r);
             tmem_ld_wait();
             if (wrow_ok) {
-              float4* d4 = reinterpret_cast<float4*>(agg_me + DD + static_cast<size_t>(wrow) * D + cb * 32);
+              float4* d4 = reinterpret_cast<float4*>(agg_me + DD);  // quad-major
 #pragma unroll
               for (int j = 0; j < 8; ++j)
-                d4[j] = make_float4(acc[4 * j] + __uint_as_float(r[4 * j]), acc[4 * j + 1] + __uint_as_float(r[4 * j + 1]),
-                                    acc[4 * j + 2] + __uint_as_float(r[4 * j + 2]),
-                                    acc[4 * j + 3] + __uint_as_float(r[4 * j + 3]));
+                __stcg(d4 + qm4<D>(wrow, cb * 8 + j),
+                       make_float4(acc[4 * j] + __uint_as_float(r[4 * j]), acc[4 * j + 1] + __uint_as_float(r[4 * j + 1]),
+                                   acc[4 * j + 2] + __uint_as_float(r[4 * j + 2]),
+                                   acc[4 * j + 3] + __uint_as_float(r[4 * j + 3])));
             }
           }
 #pragma unroll

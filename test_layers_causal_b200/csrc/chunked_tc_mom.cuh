@@ -417,11 +417,12 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
             tmem_ld32(tq + lane_off + cb * 32, r);
             tmem_ld_wait();
             if (wrow_ok) {
-              float4* d4 = reinterpret_cast<float4*>(me + q * DD + static_cast<size_t>(wrow) * D + cb * 32);
+              float4* d4 = reinterpret_cast<float4*>(me + q * DD);  // quad-major
 #pragma unroll
               for (int j = 0; j < 8; ++j)
-                d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                __stcg(d4 + qm4<D>(wrow, cb * 8 + j),
+                       make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                   __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
             }
           }
         }
@@ -435,6 +436,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       }
       const float *bw = nullptr, *bm = nullptr;
       int first = 0;
+      bool base_qm = false;  // bw, bm are published (quad-major) states, not the caller's
       if (p.coop && p.nseg > 1) {
         // Cooperative prefix (the grid is one wave, so the head's nseg blocks
         // are resident together): once every segment map is published, block
@@ -455,35 +457,57 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         const float4* sw4 = p.S_in ? reinterpret_cast<const float4*>(p.S_in + static_cast<size_t>(bh) * DD) : nullptr;
         const float4* sm4 = p.M_in ? reinterpret_cast<const float4*>(p.M_in + static_cast<size_t>(bh) * DD) : nullptr;
         const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int v = seg * SL / 4 + et; v < v1; v += 128) {
-          float4 w = sw4 ? __ldcg(sw4 + v) : zero, m = sm4 ? __ldcg(sm4 + v) : zero;
+        // two positions per thread per round, four maps per round
+        for (int v0 = seg * SL / 4 + et; v0 < v1; v0 += 256) {
+          const int vv[2] = {v0, v0 + 128};
+          const bool ok[2] = {true, v0 + 128 < v1};
+          float4 w[2], m[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {  // the scratch is quad-major, the caller's states row-major
+            w[e] = (sw4 && ok[e]) ? __ldcg(sw4 + qm4_to_rm4<D>(vv[e])) : zero;
+            m[e] = (sm4 && ok[e]) ? __ldcg(sm4 + qm4_to_rm4<D>(vv[e])) : zero;
+          }
           for (int j = 0; j < nagg; j += 4) {
-            float4 dw[4], dm[4];
+            float4 dw[2][4], dm[2][4];
             float G[4], B[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               if (j + u < nagg) {
-                dw[u] = __ldcg(w4 + (j + u) * SEG4 + v);
-                dm[u] = __ldcg(w4 + (j + u) * SEG4 + Q4 + v);
                 G[u] = __ldcg(maps + 2 * (j + u));
                 B[u] = __ldcg(maps + 2 * (j + u) + 1);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  if (ok[e]) {
+                    dw[e][u] = __ldcg(w4 + (j + u) * SEG4 + vv[e]);
+                    dm[e][u] = __ldcg(w4 + (j + u) * SEG4 + Q4 + vv[e]);
+                  }
+                }
               }
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               if (j + u < nagg) {
-                __stcg(w4 + (j + u) * SEG4 + 2 * Q4 + v, w);
-                __stcg(w4 + (j + u) * SEG4 + 3 * Q4 + v, m);
-                // (W, M) -> (W - G M + dW, B M + dM)
-                w = make_float4(fmaf(-G[u], m.x, w.x) + dw[u].x, fmaf(-G[u], m.y, w.y) + dw[u].y,
-                                fmaf(-G[u], m.z, w.z) + dw[u].z, fmaf(-G[u], m.w, w.w) + dw[u].w);
-                m = make_float4(fmaf(B[u], m.x, dm[u].x), fmaf(B[u], m.y, dm[u].y), fmaf(B[u], m.z, dm[u].z),
-                                fmaf(B[u], m.w, dm[u].w));
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  if (!ok[e]) continue;
+                  __stcg(w4 + (j + u) * SEG4 + 2 * Q4 + vv[e], w[e]);
+                  __stcg(w4 + (j + u) * SEG4 + 3 * Q4 + vv[e], m[e]);
+                  // (W, M) -> (W - G M + dW, B M + dM)
+                  const float4 a = w[e], b = m[e], x = dw[e][u], y = dm[e][u];
+                  w[e] = make_float4(fmaf(-G[u], b.x, a.x) + x.x, fmaf(-G[u], b.y, a.y) + x.y,
+                                     fmaf(-G[u], b.z, a.z) + x.z, fmaf(-G[u], b.w, a.w) + x.w);
+                  m[e] = make_float4(fmaf(B[u], b.x, y.x), fmaf(B[u], b.y, y.y), fmaf(B[u], b.z, y.z),
+                                     fmaf(B[u], b.w, y.w));
+                }
               }
             }
           }
-          __stcg(w4 + nagg * SEG4 + 2 * Q4 + v, w);
-          __stcg(w4 + nagg * SEG4 + 3 * Q4 + v, m);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            if (!ok[e]) continue;
+            __stcg(w4 + nagg * SEG4 + 2 * Q4 + vv[e], w[e]);
+            __stcg(w4 + nagg * SEG4 + 3 * Q4 + vv[e], m[e]);
+          }
         }
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -496,6 +520,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + seg) * 4 + 2) * DD;
         bm = bw + DD;
+        base_qm = true;
         first = seg;
       } else {
         // Decoupled look-back: every predecessor has published at least its
@@ -514,6 +539,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         if (incl >= 0) {
           bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 4 + 2) * DD;
           bm = bw + DD;
+          base_qm = true;
         } else {
           if (p.S_in) bw = p.S_in + static_cast<size_t>(bh) * DD;
           if (p.M_in) bm = p.M_in + static_cast<size_t>(bh) * DD;
@@ -534,7 +560,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           if (bw) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float8 x = ld_cg_f8(bw + off + 8 * j);
+              const float8 x = base_qm ? ld_cg_f8_qm<D>(bw, wrow, cb * 8 + 2 * j) : ld_cg_f8(bw + off + 8 * j);
 #pragma unroll
               for (int e = 0; e < 8; ++e) w[8 * j + e] = x.v[e];
             }
@@ -542,22 +568,22 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           if (bm) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float8 x = ld_cg_f8(bm + off + 8 * j);
+              const float8 x = base_qm ? ld_cg_f8_qm<D>(bm, wrow, cb * 8 + 2 * j) : ld_cg_f8(bm + off + 8 * j);
 #pragma unroll
               for (int e = 0; e < 8; ++e) mm[8 * j + e] = x.v[e];
             }
           }
           // apply the published segment maps in order
           for (int jj = first; jj < seg; ++jj) {
-            const float* dw = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 4 * DD + off;
+            const float* dw = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 4 * DD;
             const float* dm = dw + DD;
             const float G = __ldcg(p.wsc + (static_cast<size_t>(bh) * p.nseg + jj) * 2);
             const float B = __ldcg(p.wsc + (static_cast<size_t>(bh) * p.nseg + jj) * 2 + 1);
             float8 xw[4], xm[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              xw[j] = ld_cg_f8(dw + 8 * j);
-              xm[j] = ld_cg_f8(dm + 8 * j);
+              xw[j] = ld_cg_f8_qm<D>(dw, wrow, cb * 8 + 2 * j);
+              xm[j] = ld_cg_f8_qm<D>(dm, wrow, cb * 8 + 2 * j);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -576,15 +602,15 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           tmem_ld32(t_m + lane_off + cb * 32, r2);
           tmem_ld_wait();
           if (wrow_ok) {
-            float4* iw = reinterpret_cast<float4*>(me + 2 * DD + off);
-            float4* im = reinterpret_cast<float4*>(me + 3 * DD + off);
+            float4* iw = reinterpret_cast<float4*>(me + 2 * DD);  // quad-major
+            float4* im = reinterpret_cast<float4*>(me + 3 * DD);
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-              iw[j / 4] = make_float4(fmaf(-Gme, mm[j], w[j]) + __uint_as_float(r[j]),
+              iw[qm4<D>(wrow, cb * 8 + j / 4)] = make_float4(fmaf(-Gme, mm[j], w[j]) + __uint_as_float(r[j]),
                                       fmaf(-Gme, mm[j + 1], w[j + 1]) + __uint_as_float(r[j + 1]),
                                       fmaf(-Gme, mm[j + 2], w[j + 2]) + __uint_as_float(r[j + 2]),
                                       fmaf(-Gme, mm[j + 3], w[j + 3]) + __uint_as_float(r[j + 3]));
-              im[j / 4] = make_float4(fmaf(Bme, mm[j], __uint_as_float(r2[j])),
+              im[qm4<D>(wrow, cb * 8 + j / 4)] = make_float4(fmaf(Bme, mm[j], __uint_as_float(r2[j])),
                                       fmaf(Bme, mm[j + 1], __uint_as_float(r2[j + 1])),
                                       fmaf(Bme, mm[j + 2], __uint_as_float(r2[j + 2])),
                                       fmaf(Bme, mm[j + 3], __uint_as_float(r2[j + 3])));

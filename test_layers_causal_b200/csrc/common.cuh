@@ -304,6 +304,30 @@ __device__ __forceinline__ float8 ld_cg_f8(const float* p) {
   return r;
 }
 
+// Layout of the d x d fp32 state matrices that blocks exchange through global
+// scratch: column-quad-major.  The float4 of row r, columns 4q..4q+3, is at
+// float4 index q * D + r, so the consecutive rows a warp holds (one TMEM lane
+// each) at one column quad are contiguous: 512-byte stores and loads.
+template <int D>
+__device__ __forceinline__ size_t qm4(int r, int q) {
+  return static_cast<size_t>(q) * D + r;
+}
+// Row-major float4 index (D/4 per row) of quad-major float4 index v.
+template <int D>
+__device__ __forceinline__ size_t qm4_to_rm4(int v) {
+  return static_cast<size_t>(v % D) * (D / 4) + v / D;
+}
+// 8 floats of row r from quads q, q + 1 of a quad-major matrix.
+template <int D>
+__device__ __forceinline__ float8 ld_cg_f8_qm(const float* m, int r, int q) {
+  const float4 a = __ldcg(reinterpret_cast<const float4*>(m) + qm4<D>(r, q));
+  const float4 b = __ldcg(reinterpret_cast<const float4*>(m) + qm4<D>(r, q + 1));
+  float8 x;
+  x.v[0] = a.x, x.v[1] = a.y, x.v[2] = a.z, x.v[3] = a.w;
+  x.v[4] = b.x, x.v[5] = b.y, x.v[6] = b.z, x.v[7] = b.w;
+  return x;
+}
+
 __device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
