@@ -65,7 +65,14 @@ struct TcMomCfg {
   static constexpr int OFF_QT = OFF_K2 + TILE;
   static constexpr int OFF_P = OFF_QT + TILE;
   static constexpr int BIG = OFF_P + C * C * 2;
-  static constexpr int NBAR = 3 * NST + 16;
+  // Phase A streams only K and V, through NSA stages: the K/V slots of the
+  // NST Q/K/V stages and two more in buffers that phase B needs only later
+  // (the bf16 copies of W and M; Q~ and P for d = 64).
+  static constexpr int NSA = NST + 2;
+  static constexpr int KA2 = OFF_WBF;                      // K of phase-A stage NST (V at + TILE)
+  static constexpr int KA3 = (D == 128) ? OFF_MBF : OFF_QT;  // K of phase-A stage NST + 1
+  static_assert(KA2 + 2 * TILE <= KA3 && KA3 + 2 * TILE <= (D == 128 ? OFF_K1 : BIG), "phase-A stages");
+  static constexpr int NBAR = 3 * NST + 16 + 2 * NSA + 4;
   static constexpr int SMALL = NBAR * 8 + (NST * (C + 1) + (C + 1) + 8 + 4 * C) * 4 + 32;
   static constexpr int SMEM = BIG + SMALL + 1024;
   static constexpr int TCOLS_USED = C + 3 * D;   // scores, O, W, M
@@ -105,6 +112,12 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
   uint64_t* cl_ready = kt_ready + 9;   // [NST] coefficients of phase-B tile `it` in cls[it % NST]
   uint64_t* cl_free = kt_ready + 11;   // [NST] the epilogue is done with cls[it % NST]
   uint64_t* o_free = kt_ready + 13;    // O of the previous tile read out of TMEM
+  uint64_t* fullA = kt_ready + 14;     // [NSA] phase-A K/V stage loaded
+  uint64_t* emptyA = fullA + Cfg::NSA; // [NSA] phase-A stage consumed
+  // Phase A double-buffers K1/K2: tile g uses set g & 1, set 1 in the Q slots
+  // of stages 0 and 1 (phase A loads no Q).
+  uint64_t* ktA_ready = emptyA + Cfg::NSA;  // [2] set scaled
+  uint64_t* ktA_free = ktA_ready + 2;       // [2] set consumed by its MMAs
   float* cls = reinterpret_cast<float*>(smem + Cfg::BIG + Cfg::NBAR * 8);  // [NST][C+1] tile suffix sums
   float* bp = cls + NST * (C + 1);                                          // beta^k, k = 0..C
   float* segsc = bp + (C + 1);                                              // [0] G, [1] B of this segment
@@ -136,6 +149,14 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       mbar_init(&cl_free[s], 128);
     }
     mbar_init(o_free, 128);
+    for (int k = 0; k < Cfg::NSA; ++k) {
+      mbar_init(&fullA[k], 1);
+      mbar_init(&emptyA[k], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ktA_ready[b], Cfg::NSCW);
+      mbar_init(&ktA_free[b], 1);
+    }
     fence_mbar_init();
     float b = 1.f;
     for (int k = 0; k <= C; ++k) {
@@ -178,26 +199,45 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
   uint8_t* k1s = smem + Cfg::OFF_K1;
   uint8_t* k2s = smem + Cfg::OFF_K2;
   uint8_t* qts = smem + Cfg::OFF_QT;
+  constexpr int NSA = Cfg::NSA;
+  auto ka_off = [&](int k) -> int {  // byte offset of phase-A stage k's K tile; V follows at + TILE
+    return k < NST ? k * STAGE + TILE : (k == NST ? Cfg::KA2 : Cfg::KA3);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       bool dead = false;
       for (int g = 0; g < NI; ++g) {
-        const int s = g % NST;
-        if (g >= NST && !dead) dead = !mbar_wait(&empty[s], ((g / NST) - 1) & 1, lim);
-        const bool pb = g >= nA;
         const int t0 = tile_of(g) * C;
-        mbar_arrive_expect_tx(&full[s], pb ? 3 * TILE : 2 * TILE);
+        if (g < nA) {
+          const int k = g % NSA;
+          if (g >= NSA && !dead) dead = !mbar_wait(&emptyA[k], ((g / NSA) - 1) & 1, lim);
+          mbar_arrive_expect_tx(&fullA[k], 2 * TILE);
+          uint8_t* kd = smem + ka_off(k);
+#pragma unroll
+          for (int kb = 0; kb < D / 64; ++kb) {
+            tma_load_3d(&tmK, &fullA[k], kd + kb * C * 128, kb * 64, t0, bh);
+            tma_load_3d(&tmV, &fullA[k], kd + TILE + kb * C * 128, kb * 64, t0, bh);
+          }
+          continue;
+        }
+        const int it = g - nA, s = it % NST;
+        if (it >= NST) {
+          if (!dead) dead = !mbar_wait(&empty[s], ((it / NST) - 1) & 1, lim);
+        } else if (nA > 0) {
+          if (!dead) dead = !mbar_wait(sdone, 0, lim);  // phase A is done with every stage
+        }
+        mbar_arrive_expect_tx(&full[s], 3 * TILE);
         uint8_t* st = smem + s * STAGE;
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
-          if (pb) tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh);
           tma_load_3d(&tmK, &full[s], st + TILE + kb * C * 128, kb * 64, t0, bh);
           tma_load_3d(&tmV, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, t0, bh);
         }
       }
-      for (int g = max(0, NI - NST); g < NI; ++g) mbar_wait(&full[g % NST], (g / NST) & 1, lim);
+      for (int it = max(0, nB - NST); it < nB; ++it) mbar_wait(&full[it % NST], (it / NST) & 1, lim);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
@@ -211,35 +251,40 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
       const uint64_t d_k1 = sdesc_sw128(sbase + Cfg::OFF_K1, C * 128, 1024);
       const uint64_t d_k2 = sdesc_sw128(sbase + Cfg::OFF_K2, C * 128, 1024);
+      const uint64_t d_k1b = sdesc_sw128(sbase, C * 128, 1024);          // phase A, odd tiles
+      const uint64_t d_k2b = sdesc_sw128(sbase + STAGE, C * 128, 1024);
       const uint64_t d_qt = sdesc_sw128(sbase + Cfg::OFF_QT, 16, 1024);
       const uint64_t d_p = sdesc_sw128(sbase + Cfg::OFF_P, 16, 1024);
       for (int g = 0; g < NI; ++g) {
-        const int s = g % NST;
-        const uint32_t stq = sbase + s * STAGE, stv = stq + 2 * TILE;
+        const int s = g < nA ? g % NSA : (g - nA) % NST;  // phase-A or phase-B stage
+        const uint32_t stq = sbase + s * STAGE;
+        const uint32_t stv = g < nA ? sbase + ka_off(s) + TILE : stq + 2 * TILE;
         const uint64_t dvm = sdesc_sw128(stv, C * 128, 1024);
         if (g < nA) {
           // segment totals: dW += V^T K1, dM += V^T K2 (fresh at g == 0)
-          if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);
+          const int b = g & 1;
+          if (!dead) dead = !mbar_wait(&ktA_ready[b], (g >> 1) & 1, lim);
           tc_fence_after();
+          const uint64_t dk1 = b ? d_k1b : d_k1, dk2 = b ? d_k2b : d_k2;
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
             const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
-            mma_bf16_ss(t_w, dvm + mn_step(kk), d_k1 + mn_step(kk), ID_W, acc);
-            mma_bf16_ss(t_m, dvm + mn_step(kk), d_k2 + mn_step(kk), ID_W, acc);
+            mma_bf16_ss(t_w, dvm + mn_step(kk), dk1 + mn_step(kk), ID_W, acc);
+            mma_bf16_ss(t_m, dvm + mn_step(kk), dk2 + mn_step(kk), ID_W, acc);
           }
-          tc_commit(&empty[s]);
-          tc_commit(kt_free);
+          tc_commit(&emptyA[s]);
+          tc_commit(&ktA_free[b]);
           if (g == nA - 1) tc_commit(sdone);
           continue;
         }
         const int it = g - nA;
         const uint64_t dq = sdesc_sw128(stq, 16, 1024), dkk = sdesc_sw128(stq + TILE, 16, 1024);
-        if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
+        if (!dead) dead = !mbar_wait(&full[s], (it / NST) & 1, lim);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_sc, dq + k_step(C, kk), dkk + k_step(C, kk), ID_SC, kk > 0);
         tc_commit(sc_full);
-        if (!dead) dead = !mbar_wait(kt_ready, g & 1, lim);
+        if (!dead) dead = !mbar_wait(kt_ready, it & 1, lim);
         if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
         tc_fence_after();
         // (3) first: it needs only this tile's K1/K2 and the rewritten W, M
@@ -272,7 +317,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
     if (lane == 0) {
       bool dead = false;
       for (int it = 0; it < nB; ++it) {
-        const int g = nA + it, s = g % NST;
+        const int s = it % NST;
         if (!dead) dead = !mbar_wait(&staged[it % NST], (it / NST) & 1, lim);
         const uint8_t* sv = smem + s * STAGE + 2 * TILE;
         const int t0 = (chunk0 + it) * C;
@@ -293,18 +338,23 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
     const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
     const float beta = p.beta, sigma = p.sigma;
     float R = 0.f, Bc = 1.f;  // phase A carries: suffix coefficient after this tile, beta^(tokens after it)
+    // eta of rows 2*lane, 2*lane+1 of tile g (0 past the sequence end or past the last tile)
+    auto fetch_eta = [&](int g, float& x0, float& x1) {
+      x0 = x1 = 0.f;
+      if (sw != 0 || g >= NI) return;
+      const int ta = tile_of(g) * C + 2 * lane, tb = ta + 1;
+      if (ta < p.T) x0 = eg ? __ldg(eg + ta) : p.eta_const;
+      if (tb < p.T) x1 = eg ? __ldg(eg + tb) : p.eta_const;
+    };
+    float en0, en1;
+    fetch_eta(0, en0, en1);
     for (int g = 0; g < NI; ++g) {
-      const int s = g % NST;
       const int t0 = tile_of(g) * C;
       uint32_t* wg = wpk + (g & 1) * 2 * C;  // this tile's weights (double-buffered)
       if (sw == 0) {
-        // eta of rows 2*lane, 2*lane+1 (0 past the sequence end)
-        float e0 = 0.f, e1 = 0.f;
-        {
-          const int ta = t0 + 2 * lane, tb = ta + 1;
-          if (ta < p.T) e0 = eg ? __ldg(eg + ta) : p.eta_const;
-          if (tb < p.T) e1 = eg ? __ldg(eg + tb) : p.eta_const;
-        }
+        // eta of rows 2*lane, 2*lane+1 of this tile (fetched one tile ahead)
+        const float e0 = en0, e1 = en1;
+        fetch_eta(g + 1, en0, en1);
         // suffix scan over the tile: value at row 2*lane given zero beyond the tile
         float a = e0 + beta * e1, m = beta * beta;
 #pragma unroll
@@ -363,10 +413,29 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       // barrier for tile g only after finishing tile g-1, so the other
       // weight buffer is free for warp 7 to fill next
       asm volatile("bar.sync 2, %0;" ::"n"(32 * Cfg::NSCW) : "memory");
-      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
-      if (g > 0 && !dead) dead = !mbar_wait(kt_free, (g - 1) & 1, lim);
+      const uint8_t* sk;
+      if (g < nA) {
+        const int k = g % NSA;
+        if (!dead) dead = !mbar_wait(&fullA[k], (g / NSA) & 1, lim);
+        sk = smem + ka_off(k);
+      } else {
+        const int it = g - nA;
+        if (!dead) dead = !mbar_wait(&full[it % NST], (it / NST) & 1, lim);
+        sk = smem + (it % NST) * STAGE + TILE;
+      }
+      uint8_t *d1 = k1s, *d2 = k2s;
+      if (g < nA) {
+        if (g & 1) d1 = smem, d2 = smem + STAGE;
+        if (g >= 2 && !dead) dead = !mbar_wait(&ktA_free[g & 1], ((g >> 1) - 1) & 1, lim);
+      } else {
+        const int it = g - nA;
+        if (it > 0) {
+          if (!dead) dead = !mbar_wait(kt_free, (it - 1) & 1, lim);
+        } else if (nA > 0) {
+          if (!dead) dead = !mbar_wait(sdone, 0, lim);  // phase A is done with both sets
+        }
+      }
       // K1 = diag(w1) K, K2 = diag(w2) K for rows [16 sw, 16 sw + 16), packed bf16 multiplies
-      const uint8_t* sk = smem + s * STAGE + TILE;
       constexpr int PER_LANE = 16 * (D / 8) / 32;
 #pragma unroll
       for (int i = 0; i < PER_LANE; ++i) {
@@ -375,14 +444,14 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
         const uint32_t f1 = wg[r], f2 = wg[C + r];
         const uint4 u = *reinterpret_cast<const uint4*>(sk + off);
-        *reinterpret_cast<uint4*>(k1s + off) =
+        *reinterpret_cast<uint4*>(d1 + off) =
             make_uint4(mul_bf16x2(u.x, f1), mul_bf16x2(u.y, f1), mul_bf16x2(u.z, f1), mul_bf16x2(u.w, f1));
-        *reinterpret_cast<uint4*>(k2s + off) =
+        *reinterpret_cast<uint4*>(d2 + off) =
             make_uint4(mul_bf16x2(u.x, f2), mul_bf16x2(u.y, f2), mul_bf16x2(u.z, f2), mul_bf16x2(u.w, f2));
       }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(kt_ready);
+      if (lane == 0) mbar_arrive(g < nA ? &ktA_ready[g & 1] : kt_ready);
     }
   } else {
     // --------------------------------------------------------- epilogue --
@@ -638,13 +707,13 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
     // the stage is refilled only after Step O; doing the next Step W first
     // delays that refill by more than it gains.)
     auto step_w = [&](int it) {
-      const int g = nA + it, s = g % NST;
+      const int s = it % NST;
       const int n = min(C, p.T - (chunk0 + it) * C);
       uint8_t* st = smem + s * STAGE;
       const float* cl = cls + (it % NST) * (C + 1);
       // Step W: Wbf, Mbf from the state entering this tile; W -= g_end M; M *= beta^n; Q~ = diag(-g) Q
       if (!dead) dead = !mbar_wait(&cl_ready[it % NST], (it / NST) & 1, lim);  // the tile's cl is in smem
-      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);  // its Q has landed
+      if (!dead) dead = !mbar_wait(&full[s], (it / NST) & 1, lim);  // its Q has landed
       if (it > 0 && !dead) dead = !mbar_wait(sdone, ((nA > 0 ? 1 : 0) + it - 1) & 1, lim);
       tc_fence_after();
       const float gend = beta * cl[0];
@@ -720,7 +789,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
     auto step_o = [&](int it) {
       // Step O (this thread: half of row row64h)
       {
-        const uint32_t sv = sbase + ((nA + it) % NST) * STAGE + 2 * TILE;
+        const uint32_t sv = sbase + (it % NST) * STAGE + 2 * TILE;
         if (!dead) dead = !mbar_wait(o_full, it & 1, lim);
         tc_fence_after();
         if constexpr (D == 64) {
