@@ -72,7 +72,7 @@ struct TcMomCfg {
   static constexpr int KA2 = OFF_WBF;                      // K of phase-A stage NST (V at + TILE)
   static constexpr int KA3 = (D == 128) ? OFF_MBF : OFF_QT;  // K of phase-A stage NST + 1
   static_assert(KA2 + 2 * TILE <= KA3 && KA3 + 2 * TILE <= (D == 128 ? OFF_K1 : BIG), "phase-A stages");
-  static constexpr int NBAR = 3 * NST + 16 + 2 * NSA + 4;
+  static constexpr int NBAR = 5 * NST + 16 + 2 * NSA + 4;
   static constexpr int SMALL = NBAR * 8 + (NST * (C + 1) + (C + 1) + 8 + 4 * C) * 4 + 32;
   static constexpr int SMEM = BIG + SMALL + 1024;
   static constexpr int TCOLS_USED = C + 3 * D;   // scores, O, W, M
@@ -97,10 +97,16 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
   const uint32_t sbase = smem_u32(smem);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BIG);
-  uint64_t* full = bars;               // [NST]
-  uint64_t* empty = bars + NST;        // [NST]
+  // Phase-B stage s holds Q, K, V of tile it = s mod NST.  Its Q and K slots
+  // are done once the readout (2) has run, its V slot only once O, staged
+  // there, has been stored: two fill/free pairs, so the next tile's Q and K
+  // can load while O is still leaving.
+  uint64_t* full = bars;               // [NST] Q and K loaded
+  uint64_t* empty = bars + NST;        // [NST] Q and K slots free
   uint64_t* staged = bars + 2 * NST;   // [NST] (indexed by phase-B tile % NST)
-  uint64_t* kt_ready = bars + 3 * NST; // scaled K1/K2 (and the tile's cl) ready
+  uint64_t* fullV = bars + 3 * NST;    // [NST] V loaded
+  uint64_t* emptyV = bars + 4 * NST;   // [NST] V slot free (O stored)
+  uint64_t* kt_ready = bars + 5 * NST; // scaled K1/K2 (and the tile's cl) ready
   uint64_t* kt_free = kt_ready + 1;    // (3) of the previous tile done: K1/K2 buffers free
   uint64_t* sc_full = kt_ready + 2;
   uint64_t* sdone = kt_ready + 3;      // (2),(3) done / phase-A totals done
@@ -134,6 +140,8 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&staged[s], 128);
+      mbar_init(&fullV[s], 1);
+      mbar_init(&emptyV[s], 1);
     }
     mbar_init(kt_ready, Cfg::NSCW);
     mbar_init(kt_free, 1);
@@ -223,21 +231,27 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           continue;
         }
         const int it = g - nA, s = it % NST;
+        uint8_t* st = smem + s * STAGE;
         if (it >= NST) {
           if (!dead) dead = !mbar_wait(&empty[s], ((it / NST) - 1) & 1, lim);
         } else if (nA > 0) {
           if (!dead) dead = !mbar_wait(sdone, 0, lim);  // phase A is done with every stage
         }
-        mbar_arrive_expect_tx(&full[s], 3 * TILE);
-        uint8_t* st = smem + s * STAGE;
+        mbar_arrive_expect_tx(&full[s], 2 * TILE);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
           tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, t0, bh);
           tma_load_3d(&tmK, &full[s], st + TILE + kb * C * 128, kb * 64, t0, bh);
-          tma_load_3d(&tmV, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, t0, bh);
         }
+        if (it >= NST && !dead) dead = !mbar_wait(&emptyV[s], ((it / NST) - 1) & 1, lim);
+        mbar_arrive_expect_tx(&fullV[s], TILE);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) tma_load_3d(&tmV, &fullV[s], st + 2 * TILE + kb * C * 128, kb * 64, t0, bh);
       }
-      for (int it = max(0, nB - NST); it < nB; ++it) mbar_wait(&full[it % NST], (it / NST) & 1, lim);
+      for (int it = max(0, nB - NST); it < nB; ++it) {
+        mbar_wait(&full[it % NST], (it / NST) & 1, lim);
+        mbar_wait(&fullV[it % NST], (it / NST) & 1, lim);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
@@ -286,6 +300,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         tc_commit(sc_full);
         if (!dead) dead = !mbar_wait(kt_ready, it & 1, lim);
         if (!dead) dead = !mbar_wait(wbf_ready, it & 1, lim);
+        if (!dead) dead = !mbar_wait(&fullV[s], (it / NST) & 1, lim);
         tc_fence_after();
         // (3) first: it needs only this tile's K1/K2 and the rewritten W, M
 #pragma unroll
@@ -303,6 +318,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           mma_bf16_ss(t_o, d_qt + k_step(C, kk), d_mbf + k_step(D, kk), ID_O_K, 1);
         }
         tc_commit(sdone);
+        tc_commit(&empty[s]);  // Q and K of this tile are read
         if (!dead) dead = !mbar_wait(p_ready, it & 1, lim);
         tc_fence_after();
 #pragma unroll
@@ -325,7 +341,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         for (int kb = 0; kb < D / 64; ++kb) tma_store_3d(&tmO, sv + kb * C * 128, kb * 64, t0, bh);
         bulk_commit();
         bulk_wait_read0();
-        mbar_arrive(&empty[s]);
+        mbar_arrive(&emptyV[s]);
       }
       bulk_wait0();
     }
@@ -703,9 +719,6 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
     }
 
     // ---- phase B
-    // Per tile: Step W, Step P, Step O.  (O is staged in the tile's V slot, so
-    // the stage is refilled only after Step O; doing the next Step W first
-    // delays that refill by more than it gains.)
     auto step_w = [&](int it) {
       const int s = it % NST;
       const int n = min(C, p.T - (chunk0 + it) * C);
@@ -811,10 +824,17 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         mbar_arrive(&staged[it % NST]);
       }
     };
+    // Order: the next tile's Step W as soon as this tile's readout is done
+    // (it gates the next MMAs), then this tile's Step O (its readout frees
+    // O in TMEM for the next (2)), then the next tile's Step P.
+    if (nB > 0) {
+      step_w(0);
+      step_p(0);
+    }
     for (int it = 0; it < nB; ++it) {
-      step_w(it);
-      step_p(it);
+      if (it + 1 < nB) step_w(it + 1);
       step_o(it);
+      if (it + 1 < nB) step_p(it + 1);
     }
 
     // final state (last segment)
