@@ -180,6 +180,36 @@ TTT_LA_API size_t ttt_la_host_staging_size(const ttt_la_args *args);
 TTT_LA_API ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args *args, void *device_buf,
                                                      size_t device_bytes, void *stream);
 
+/* Splitting one sequence over several devices along T (one exchange step).
+ * A run of tokens acts on the carried state as the affine map
+ *   (W, M) -> (W - G M + dW, B M + dM),
+ * with dW, dM the state the run leaves from W = M = 0, G = sum_t eta_t beta^t
+ * (t = 1..L over the run) and B = beta^L ("Test-Time Training with KV Binding
+ * Is Secretly Linear Attention", thelatestinai.com listing, Table 2: Variant 3
+ * carries (W, M); Variants 4-5 carry W alone, G = 0, B = 1).  A device holding
+ * tokens [t0, t1) of every sequence computes its run's map, the maps are
+ * exchanged (all-gather), and each device composes the maps of the runs
+ * before its own onto W_0, M_0 to get its start state, then calls
+ * ttt_la_forward_chunked from it.
+ *
+ * ttt_la_segment_map: args as for ttt_la_forward_chunked over the device's
+ * run (T = its length); state_in/mom_in/state_out/mom_out are ignored and
+ * args->o is scratch (written, contents unspecified).  Writes dW
+ * [B,H,d_v,d_k] fp32 and, with momentum, dM [B,H,d_v,d_k] fp32 and GB
+ * [B,H,2] fp32 = (G, B); dM and GB may be NULL without momentum.  Device
+ * pointers, 16-byte aligned.  Errors as ttt_la_forward_chunked.
+ *
+ * ttt_la_compose_maps: applies maps 0..nmaps-1 in order to (W0, M0) for BH
+ * heads: dW, dM [nmaps,BH,d_v,d_k] and GB [nmaps,BH,2] as written by
+ * ttt_la_segment_map (dM and GB both NULL: maps without momentum).  W0, M0
+ * [BH,d_v,d_k] may be NULL (zeros).  Writes W_out and, if not NULL, M_out
+ * [BH,d_v,d_k].  nmaps = 0 copies (W0, M0).  TTT_LA_ERR_INVALID_ARG for bad
+ * sizes or exactly one of dM, GB given. */
+TTT_LA_API ttt_la_status ttt_la_segment_map(const ttt_la_args *args, float *dW, float *dM, float *GB, void *stream);
+TTT_LA_API ttt_la_status ttt_la_compose_maps(int32_t nmaps, int32_t BH, int32_t d_v, int32_t d_k, const float *dW,
+                                             const float *dM, const float *GB, const float *W0, const float *M0,
+                                             float *W_out, float *M_out, void *stream);
+
 /* Synchronises `stream`, returns the device status word (TTT_LA_OK or
  * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
 TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);

@@ -52,6 +52,8 @@ SIGNATURES = [
     ("ttt_la_host_staging_size", _c_sz, [ctypes.POINTER(TttArgs)]),
     ("ttt_la_forward_chunked_host", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp, _c_sz, _c_vp]),
     ("ttt_la_forward_recurrent", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
+    ("ttt_la_segment_map", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp, _c_vp, _c_vp, _c_vp]),
+    ("ttt_la_compose_maps", ctypes.c_int, [ctypes.c_int32] * 4 + [_c_vp] * 8),
     ("ttt_la_decode_step", ctypes.c_int, [ctypes.POINTER(TttDecodeArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
     ("ttt_la_set_wait_limit_ns", ctypes.c_int, [ctypes.c_int64]),
@@ -209,6 +211,49 @@ def forward_chunked_host(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=Fal
            L.ttt_la_forward_chunked_host(ctypes.byref(a), ctypes.c_void_p(staging.data_ptr()),
                                          staging.numel() * staging.element_size(), _stream_handle(stream)))
     return o, staging
+
+
+def segment_map(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, chunk=64, segments=0, scratch=None,
+                workspace=None, stream=None):
+    """Affine map of this run of tokens on the carried state
+    (ttt_la_segment_map): returns (dW, dM, GB) with dW, dM [B,H,d_v,d_k] and
+    GB [B,H,2] = (G, B); dM and GB are None without momentum.  `scratch`
+    ([B,H,T,d_v] like v) receives throwaway outputs."""
+    _check_shapes(q, k, v, eta, None, None)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if scratch is None else scratch
+    dW = torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32)
+    dM = GB = None
+    if beta != 0:
+        dM = torch.empty_like(dW)
+        GB = torch.empty(B, H, 2, device=q.device, dtype=torch.float32)
+    a = _seq_args(q, k, v, eta, eta_const, beta, ascent, chunk, segments, None, None, o, None, None)
+    L = lib()
+    need = L.ttt_la_workspace_size(ctypes.byref(a))
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check("ttt_la_segment_map", L.ttt_la_segment_map(ctypes.byref(a), _ptr(dW), _ptr(dM), _ptr(GB),
+                                                      _stream_handle(stream)))
+    return dW, dM, GB
+
+
+def compose_maps(dW, dM=None, GB=None, W0=None, M0=None, stream=None):
+    """Applies maps 0..n-1 in order to (W0, M0) (ttt_la_compose_maps): dW, dM
+    [n,B,H,d_v,d_k], GB [n,B,H,2] (dM, GB None: no momentum); W0, M0
+    [B,H,d_v,d_k] or None (zeros).  Returns (W, M); M is None when neither
+    dM nor M0 is given."""
+    n = dW.shape[0]
+    B, H, dv, dk = dW.shape[1:]
+    _need_cuda(dW, dM, GB, W0, M0)
+    W = torch.empty(B, H, dv, dk, device=dW.device, dtype=torch.float32)
+    M = torch.empty_like(W) if (dM is not None or M0 is not None) else None
+    _check("ttt_la_compose_maps", lib().ttt_la_compose_maps(
+        n, B * H, dv, dk, _ptr(dW), _ptr(dM), _ptr(GB), _ptr(W0), _ptr(M0), _ptr(W), _ptr(M),
+        _stream_handle(stream)))
+    return W, M
 
 
 def workspace_bytes(q, v, chunk=64, beta=0.0, segments=0):

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "recurrent.cuh"
+#include "seqshard.cuh"
 
 namespace {
 
@@ -516,6 +517,54 @@ ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args* a, void* device_buf
       cudaStreamWaitEvent(st, hp->join_in, 0) != cudaSuccess || cudaStreamWaitEvent(st, hp->join_out, 0) != cudaSuccess)
     return TTT_LA_ERR_CUDA;
   return TTT_LA_OK;
+}
+
+ttt_la_status ttt_la_segment_map(const ttt_la_args* a, float* dW, float* dM, float* GB, void* stream) {
+  ttt_la_status s = check_seq(a);
+  if (s != TTT_LA_OK) return s;
+  const bool mom = a->beta != 0.f;
+  if (!dW || (mom && (!dM || !GB)) || !aligned16(dW) || (dM && !aligned16(dM))) return TTT_LA_ERR_INVALID_ARG;
+  // The map's state part is the forward's final state from W = M = 0.
+  ttt_la_args b = *a;
+  b.state_in = nullptr;
+  b.mom_in = nullptr;
+  b.state_out = dW;
+  b.mom_out = mom ? dM : nullptr;
+  s = ttt_la_forward_chunked(&b, stream);
+  if (s != TTT_LA_OK || !mom) return s;
+  ttt::MapScalarParams p;
+  p.BH = a->B * a->H;
+  p.T = a->T;
+  p.eta = a->eta;
+  p.eta_const = a->eta_const;
+  p.beta = a->beta;
+  p.GB = GB;
+  const int blocks = (p.BH * 32 + 255) / 256;
+  ttt::segment_scalars_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launched();
+}
+
+ttt_la_status ttt_la_compose_maps(int32_t nmaps, int32_t BH, int32_t d_v, int32_t d_k, const float* dW,
+                                  const float* dM, const float* GB, const float* W0, const float* M0, float* W_out,
+                                  float* M_out, void* stream) {
+  if (nmaps < 0 || BH < 1 || d_v < 1 || d_k < 1 || !W_out || (nmaps > 0 && !dW)) return TTT_LA_ERR_INVALID_ARG;
+  if ((dM == nullptr) != (GB == nullptr)) return TTT_LA_ERR_INVALID_ARG;
+  if (static_cast<long long>(BH) * d_v * d_k >= (1ll << 40)) return TTT_LA_ERR_INVALID_ARG;
+  ttt::ComposeParams p;
+  p.nmaps = nmaps;
+  p.DD = d_v * d_k;
+  p.n = static_cast<long long>(BH) * p.DD;
+  p.dW = dW;
+  p.dM = dM;
+  p.GB = GB;
+  p.W0 = W0;
+  p.M0 = M0;
+  p.W_out = W_out;
+  p.M_out = M_out;
+  const long long want = (p.n + 255) / 256;
+  const int blocks = static_cast<int>(std::min<long long>(want, static_cast<long long>(sm_count()) * 8));
+  ttt::compose_maps_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launched();
 }
 
 ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {

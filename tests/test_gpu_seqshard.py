@@ -1,0 +1,79 @@
+"""GPU checks of the sequence split along T: each run's affine map
+(ttt_la_segment_map), the composition of maps (ttt_la_compose_maps) and the
+forward from a composed start state reproduce the float64 oracle run over
+the whole sequence.  The ranks are simulated one after the other on one GPU;
+the exchange itself is covered on CPU ranks in test_multi_rank.py."""
+import math
+
+import pytest
+import torch
+
+from synth import make_qkv
+from tests.gpu_util import assert_bf16, assert_f32, oracle_forward
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from test_layers_causal_b200 import _abi, seqshard
+
+
+def _inputs(B, H, T, d, dtype, seed, token_eta=True):
+    q, k, v, z = make_qkv((B, H), T, d, d, seed)
+    eta = (torch.sigmoid(z) / math.sqrt(d)).float().cuda() if token_eta else None
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    return (*(x.to(dt).contiguous().cuda() for x in (q, k, v)), eta)
+
+
+@pytest.mark.parametrize("beta,ascent,token_eta", [(0.0, False, True), (0.9, False, True), (0.5, True, False),
+                                                   (0.0, True, False)])
+@pytest.mark.parametrize("world", [2, 3])
+def test_runs_compose_to_the_whole_sequence(beta, ascent, token_eta, world):
+    B, H, T, d = 2, 2, 3 * 64 * 2 + 41, 64
+    q, k, v, eta = _inputs(B, H, T, d, "bf16", 190 + world, token_eta)
+    ec = 1.0 / math.sqrt(d)
+    g = torch.Generator().manual_seed(21)
+    S0 = (0.1 * torch.randn(B, H, d, d, generator=g)).cuda()
+    M0 = (0.1 * torch.randn(B, H, d, d, generator=g)).cuda() if beta else None
+    kw = dict(eta_const=ec, beta=beta, ascent=ascent, chunk=64)
+    sl = [seqshard.token_slice(T, r, world) for r in range(world)]
+    run = lambda x, s: None if x is None else x[:, :, s].contiguous()  # noqa: E731
+    maps = [_abi.segment_map(run(q, s), run(k, s), run(v, s), run(eta, s), **kw) for s in sl]
+    dW = torch.stack([m[0] for m in maps])
+    dM = torch.stack([m[1] for m in maps]) if beta else None
+    GB = torch.stack([m[2] for m in maps]) if beta else None
+    outs = []
+    for r, s in enumerate(sl):
+        W0, M0r = _abi.compose_maps(dW[:r], None if dM is None else dM[:r], None if GB is None else GB[:r], S0, M0)
+        o, _, _ = _abi.forward_chunked(run(q, s), run(k, s), run(v, s), run(eta, s), state_in=W0,
+                                       mom_in=M0r if beta else None, return_state=False, **kw)
+        outs.append(o)
+    W_T, M_T = _abi.compose_maps(dW, dM, GB, S0, M0)
+    torch.cuda.synchronize()
+    o_ref, W_ref, M_ref = oracle_forward(q, k, v, eta, ec, beta, ascent, S0, M0)
+    assert_bf16(torch.cat(outs, dim=2), o_ref, "o")
+    assert_bf16(W_T, W_ref, "W_T")
+    if beta:
+        assert_bf16(M_T, M_ref, "M_T")
+
+
+def test_compose_is_exact_elementwise_and_module_world_one():
+    """compose_maps against the map formula on random maps (fp32 both sides,
+    same operation order), and the module at world size 1 (no exchange)."""
+    g = torch.Generator().manual_seed(5)
+    n, B, H, d = 3, 2, 3, 32
+    dW, dM = (torch.randn(n, B, H, d, d, generator=g).cuda() for _ in range(2))
+    GB = torch.rand(n, B, H, 2, generator=g).cuda()
+    W0, M0 = (torch.randn(B, H, d, d, generator=g).cuda() for _ in range(2))
+    W, M = _abi.compose_maps(dW, dM, GB, W0, M0)
+    w, m = W0.clone(), M0.clone()
+    for j in range(n):
+        G_, B_ = GB[j, ..., 0, None, None], GB[j, ..., 1, None, None]
+        w = torch.addcmul(w, -G_.expand_as(m), m) + dW[j]
+        m = torch.addcmul(dM[j], B_.expand_as(m), m)
+    assert_f32(W, w.cpu().double().numpy(), "W")
+    assert_f32(M, m.cpu().double().numpy(), "M")
+    q, k, v, eta = _inputs(1, 2, 200, 64, "bf16", 99)
+    o, W_T, _ = seqshard.forward_sequence_sharded(q, k, v, eta, chunk=64)
+    o_ref, W_ref, _ = oracle_forward(q, k, v, eta, 1.0 / 8)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(W_T, W_ref, "W_T")

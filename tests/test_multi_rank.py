@@ -7,6 +7,7 @@ import socket
 
 import numpy as np
 import pytest
+import torch
 import torch.multiprocessing as mp
 
 
@@ -61,6 +62,86 @@ def _shard_worker(rank, world, port, outq):
     ranks.finalize(info)
 
 
+def _oracle_backend():
+    """The three operations of the sequence split computed by the float64
+    oracle, so the orchestration (slicing, all-gather, which maps compose
+    where) runs on CPU ranks.  The map's scalars come from the recurrence
+    itself: G from how M_0 = 1 enters W, B from how it decays."""
+    import oracle
+    from test_layers_causal_b200.seqshard import Backend
+
+    f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
+
+    def seg_map(q, k, v, eta, eta_const=None, beta=0.0, ascent=False, chunk=64):
+        e = f(eta) if eta is not None else eta_const
+        _, W, M = oracle.ttt_recurrence_f64(f(q), f(k), f(v), e, beta=beta, ascent=ascent)
+        if not beta:
+            return torch.from_numpy(W), None, None
+        ones = np.ones_like(W)
+        _, W1, M1 = oracle.ttt_recurrence_f64(f(q), f(k), f(v), e, beta=beta, ascent=ascent, M0=ones)
+        G = -(W1 - W).mean(axis=(-2, -1))
+        B = (M1 - M).mean(axis=(-2, -1))
+        return torch.from_numpy(W), torch.from_numpy(M), torch.from_numpy(np.stack([G, B], -1))
+
+    def compose(dW, dM, GB, W0, M0):
+        w = f(W0) if W0 is not None else np.zeros(dW.shape[1:])
+        m = f(M0) if M0 is not None else np.zeros(dW.shape[1:])
+        for j in range(dW.shape[0]):
+            G = f(GB[j])[..., 0, None, None] if GB is not None else 0.0
+            B = f(GB[j])[..., 1, None, None] if GB is not None else 1.0
+            w = w - G * m + f(dW[j])
+            m = B * m + f(dM[j]) if dM is not None else m
+        return torch.from_numpy(w), torch.from_numpy(m)
+
+    def forward(q, k, v, eta, state_in=None, mom_in=None, return_state=False, eta_const=None, beta=0.0,
+                ascent=False, chunk=64):
+        e = f(eta) if eta is not None else eta_const
+        o, W, M = oracle.ttt_recurrence_f64(f(q), f(k), f(v), e, beta=beta, ascent=ascent, S0=f(state_in),
+                                            M0=f(mom_in))
+        return torch.from_numpy(o), torch.from_numpy(W), torch.from_numpy(M)
+
+    return Backend(segment_map=seg_map, compose_maps=compose, forward=forward)
+
+
+def _seqshard_worker(rank, world, port, outq):
+    _env(rank, world, port)
+    import torch.distributed as dist
+
+    import oracle
+    from synth import make_qkv
+    from test_layers_causal_b200 import ranks, seqshard
+    info = ranks.init(backend="gloo", timeout_s=60)
+    B, H, T, d = 2, 2, 53, 6
+    q, k, v, z = make_qkv((B, H), T, d, d, seed=41)  # every rank draws the whole sequence
+    eta = torch.sigmoid(z) / d ** 0.5
+    g = torch.Generator().manual_seed(3)
+    S0, M0 = 0.2 * torch.randn(B, H, d, d, generator=g), 0.2 * torch.randn(B, H, d, d, generator=g)
+    res = {}
+    for beta in (0.0, 0.9):
+        sl = seqshard.token_slice(T, info.rank, info.world)
+        loc = lambda x: x[:, :, sl].contiguous()  # noqa: E731
+        o, W_T, M_T = seqshard.forward_sequence_sharded(
+            loc(q), loc(k), loc(v), loc(eta), rank=info.rank, world=info.world, beta=beta,
+            state_in=S0.double(), mom_in=M0.double() if beta else None, backend=_oracle_backend())
+        parts = [None] * info.world
+        dist.all_gather_object(parts, (sl.start, sl.stop, o.numpy(), W_T.numpy(),
+                                       None if M_T is None else M_T.numpy()))
+        f = lambda t: t.double().numpy()  # noqa: E731
+        o_ref, W_ref, M_ref = oracle.ttt_recurrence_f64(f(q), f(k), f(v), f(eta), beta=beta, S0=f(S0),
+                                                        M0=f(M0) if beta else None)
+        err = 0.0
+        covered = np.zeros(T, dtype=int)
+        for a, b, o_p, W_p, M_p in parts:
+            covered[a:b] += 1
+            err = max(err, np.abs(o_p - o_ref[:, :, a:b]).max(), np.abs(W_p - W_ref).max())
+            if beta:
+                err = max(err, np.abs(M_p - M_ref).max())
+        res[beta] = (err, covered.tolist())
+    if info.rank == 0:
+        outq.put(res)
+    ranks.finalize(info)
+
+
 def _run(fn, world=2):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -102,3 +183,14 @@ def test_local_slice_partitions_the_batch(B, world):
         sl = ranks.local_slice(B, r, world)
         seen.extend(range(B)[sl])
     assert seen == list(range(B))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_split_over_ranks_matches_the_whole_sequence(world):
+    """Two or three CPU ranks each hold a contiguous run of every sequence;
+    after the all-gather of the runs' maps and the composition, every run's
+    output and the final (W, M) equal the whole-sequence recurrence."""
+    (res,) = _run(_seqshard_worker, world=world)
+    for beta, (err, covered) in res.items():
+        assert covered == [1] * 53, beta
+        assert err < 1e-12, (beta, err)
