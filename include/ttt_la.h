@@ -168,11 +168,17 @@ TTT_LA_API ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args *args,
  * staging buffers in `device_buf` (caller-owned device memory, 16-byte
  * aligned, at least ttt_la_host_staging_size(args) bytes).  Each piece runs
  * ttt_la_forward_chunked, so results agree with it up to the rounding of a
- * different segment split.  Ordering follows `stream`: the copies start after
- * the work already queued on it, and work queued on it after this call starts
- * only once every output has reached host memory.  Returns once everything is
- * queued (the host buffers must stay valid, and the inputs unchanged, until
- * then).  Calls whose executions overlap must not share `device_buf`.
+ * different segment split.  Ordering: copies in start as soon as the staging
+ * set they fill is free (the last forward that read it has finished, in this
+ * call or an earlier one on the device), possibly before earlier work on
+ * `stream` has finished, so the host inputs must be final when the call is
+ * made; the forwards and copies out follow the work already queued on
+ * `stream`, and work queued on it after this call starts only once every
+ * output has reached host memory.  Returns once everything is queued (the
+ * host inputs must stay valid and unchanged until `stream` passes this call).
+ * Calls on one device are ordered with one another through the library's
+ * shared copy streams; `device_buf` must not be used by anything else while
+ * such a call may still run.
  * Errors: as ttt_la_forward_chunked, plus TTT_LA_ERR_INVALID_ARG for a
  * missing, misaligned or short `device_buf`.  The paper has no counterpart of
  * this entry point; it is the end-to-end path for callers with host data. */

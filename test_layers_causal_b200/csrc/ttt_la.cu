@@ -482,15 +482,17 @@ ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args* a, void* device_buf
     return cudaMemcpyAsync(static_cast<uint8_t*>(dst) + row * first, base + src, row * cnt, cudaMemcpyDeviceToHost,
                            hp->s_out) == cudaSuccess;
   };
-  // fork: the copy streams start after the caller's earlier work
-  if (cudaEventRecord(hp->fork, st) != cudaSuccess || cudaStreamWaitEvent(hp->s_in, hp->fork, 0) != cudaSuccess ||
-      cudaStreamWaitEvent(hp->s_out, hp->fork, 0) != cudaSuccess)
+  // fork: copies out start after the caller's earlier work.  Copies in need
+  // only their staging set to be free (the last forward that read it, of
+  // this call or an earlier one), so a call's first copies overlap the end
+  // of the previous call.
+  if (cudaEventRecord(hp->fork, st) != cudaSuccess || cudaStreamWaitEvent(hp->s_out, hp->fork, 0) != cudaSuccess)
     return TTT_LA_ERR_CUDA;
   for (int j = 0; j < L.pieces; ++j) {
     const int b = j & 1, first = j * L.per, cnt = std::min(L.per, bh - first);
     uint8_t* base = static_cast<uint8_t*>(device_buf) + b * L.set_bytes;
-    // copy in, once the forward of piece j-2 has finished reading this set
-    if (j >= 2 && cudaStreamWaitEvent(hp->s_in, hp->done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    // copy in, once the last forward that read this set has finished
+    if (cudaStreamWaitEvent(hp->s_in, hp->done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
     if (!h2d(L.q, a->q, qrow, first, cnt, base) || !h2d(L.k, a->k, qrow, first, cnt, base) ||
         !h2d(L.v, a->v, vrow, first, cnt, base) || !h2d(L.eta, a->eta, erow, first, cnt, base) ||
         !h2d(L.s_in, a->state_in, srow, first, cnt, base) || !h2d(L.m_in, a->mom_in, srow, first, cnt, base) ||
@@ -499,7 +501,7 @@ ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args* a, void* device_buf
     // forward on the caller's stream, once the inputs are in and piece j-2's
     // outputs have left this set
     if (cudaStreamWaitEvent(st, hp->in_ready[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
-    if (j >= 2 && cudaStreamWaitEvent(st, hp->out_done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    if (cudaStreamWaitEvent(st, hp->out_done[b], 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
     const ttt_la_args pa = piece_args(a, L, cnt, base);
     s = ttt_la_forward_chunked(&pa, st);
     if (s != TTT_LA_OK) return s;
