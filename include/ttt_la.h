@@ -44,6 +44,12 @@
  *    TTT_LA_ERR_TIMEOUT in the library's device status word, the kernel
  *    drains its own copies, frees its tensor memory and returns;
  *    ttt_la_get_last_device_status reads (and clears) that word.
+ *  - The chunked forward splits long sequences into segments whose blocks
+ *    exchange segment states through the workspace.  When the grid fits in
+ *    one wave of resident blocks, the blocks of a head can wait for one
+ *    another: other work running at the same time on the device delays them,
+ *    and a delay beyond the wait limit (ttt_la_set_wait_limit_ns, default
+ *    1 s) ends the call with TTT_LA_ERR_TIMEOUT rather than a hang.
  *  - o must not alias q, k, v, eta or the states.  state_out may equal
  *    state_in (in place), and mom_out may equal mom_in.
  */
