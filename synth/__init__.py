@@ -21,7 +21,7 @@ import math
 
 import torch
 
-__all__ = ["LayerCase", "CONFIGS", "make_case", "make_qkv", "get_config"]
+__all__ = ["LayerCase", "CONFIGS", "make_case", "make_qkv", "get_config", "make_feature_weights"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -129,3 +129,16 @@ def make_decode_inputs(device="cuda", N=None, H=None, prefill=None, steps=None, 
     pq, pk, pv = draw(N, H, T, d, unit=True), draw(N, H, T, d, unit=True), draw(N, H, T, d, unit=False)
     sq, sk, sv = draw(S, N, H, d, unit=True), draw(S, N, H, d, unit=True), draw(S, N, H, d, unit=False)
     return dict(prefill=(pq, pk, pv), steps=(sq, sk, sv), eta_const=1.0 / math.sqrt(d))
+
+
+def make_feature_weights(H, d_in, d_out, seed, dtype=torch.bfloat16, device="cpu"):
+    """Seeded stand-ins for the frozen gated layer of the feature map,
+    phi(x) = silu(W1 x) * (W3 x): W1 and W3 [H, d_out, d_in] with N(0, 1)
+    entries, drawn in fp32 in the order W1, W3 from one generator and rounded
+    to `dtype`.  With unit-norm q and k every pre-activation is then N(0, 1),
+    the range where the gate is neither linear nor saturated."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    W1 = torch.randn(H, d_out, d_in, generator=g, device=device)
+    W3 = torch.randn(H, d_out, d_in, generator=g, device=device)
+    return W1.to(dtype).contiguous(), W3.to(dtype).contiguous()
