@@ -253,6 +253,72 @@ def decode_measure(ttt, dev, peaks):
             "tokens_per_s": sq.shape[1] / (us * 1e-6), "gpu_launches": n}
 
 
+def phi_measure(ttt, dev, peaks, reps=100):
+    """The layer whose fast weight is the last layer of a frozen gated MLP,
+    on the llm_d64 shape (B4 H16 T4096, per-token eta): phi(q), phi(k) =
+    silu(W1 x) * (W3 x) with d_in = d_out = 64 (one feature-map launch for
+    both), then the chunked forward on (phi(q), phi(k), v).  Four rotating
+    input sets (512 MB) keep consecutive steps out of L2; one CUDA graph holds
+    a step on each set."""
+    from synth import make_feature_weights
+    c = CONFIGS["llm_d64"]
+    x = make_case(c)
+    W1, W3 = (w.to(dev) for w in make_feature_weights(c.H, c.d_k, c.d_k, 7))
+    B, H, T, d = c.B, c.H, c.T, c.d_k
+    sets = []
+    for _ in range(4):
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        eta = x["eta"].to(dev)
+        fq, fk = torch.empty_like(q), torch.empty_like(k)
+        o = torch.empty_like(v)
+        S = torch.empty(B, H, d, d, device=dev, dtype=torch.float32)
+        sets.append((q, k, v, eta, fq, fk, o, S))
+    work = torch.empty(max(ttt.workspace_bytes(sets[0][0], sets[0][2], chunk=c.chunk), 16), dtype=torch.uint8,
+                       device=dev)
+
+    def phi_only(i):
+        q, k, _, _, fq, fk, _, _ = sets[i]
+        ttt.feature_map([q, k], W1, W3, out=[fq, fk])
+
+    def layer(i):
+        q, k, v, eta, fq, fk, o, S = sets[i]
+        ttt.feature_map([q, k], W1, W3, out=[fq, fk])
+        ttt.forward_chunked(fq, fk, v, eta, eta_const=x["eta_const"], chunk=c.chunk, out=o, state_out=S,
+                            workspace=work)
+
+    def timed(fn):
+        for i in range(4):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(4):
+                fn(i)
+        for _ in range(3):
+            g.replay()
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / (4 * reps)
+
+    phi_us = timed(phi_only)
+    layer_us = timed(layer)
+    if ttt.device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait")
+    n_tok = B * H * T
+    phi_bytes = 2 * n_tok * d * 2 + 2 * n_tok * d * 2 + 2 * H * d * d * 2
+    gbs = phi_bytes / (phi_us * 1e-6) / 1e9
+    return {"workload": "llm_d64 with the frozen gated-MLP feature map (d_in 64 -> d_out 64)",
+            "phi_us": phi_us, "phi_bytes": phi_bytes, "phi_hbm_gbs": gbs, "phi_frac": gbs / peaks["hbm_gbs"],
+            "layer_us_per_step": layer_us, "tokens_per_s": B * T / (layer_us * 1e-6),
+            "gpu_launches_per_step": 2}
+
+
 def workload_config(c, args):
     return {"workload": c.name, "B": c.B, "H": c.H, "T": c.T, "d_k": c.d_k, "d_v": c.d_v,
             "chunk": args.chunk or c.chunk, "eta": "per-token" if c.eta_mode == "token" else "constant",
@@ -396,6 +462,9 @@ def run_ours(args, c, ws, rank, local, info):
         del sets, graphs
         torch.cuda.empty_cache()
         line["decode"] = decode_measure(ttt, dev, peaks)
+    if not args.no_phi:
+        torch.cuda.empty_cache()
+        line["phi_layer"] = phi_measure(ttt, dev, peaks)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(c, c.B * c.H if args.cpu_heads == 0 else args.cpu_heads)
     if rank == 0:
@@ -404,7 +473,8 @@ def run_ours(args, c, ws, rank, local, info):
 
 def profile_run(args):
     """Plain launches (no graphs, no timing) for ncu: --warmup + --steps calls
-    of the workload's forward, or of the decode step on a random 256 MiB state."""
+    of the workload's forward, of the decode step on a random 256 MiB state,
+    or (phi) of the feature map plus chunked forward on the llm_d64 shape."""
     import test_layers_causal_b200 as ttt
     dev = torch.device("cuda", 0)
     if args.workload == "decode":
@@ -415,6 +485,14 @@ def profile_run(args):
         q, k, v = (torch.randn(N, H, d, generator=g, device=dev).to(torch.bfloat16) for _ in range(3))
         for _ in range(args.warmup + args.steps):
             ttt.decode_step(q, k, v, S, eta_const=1.0 / math.sqrt(d))
+    elif args.workload == "phi":
+        from synth import make_feature_weights
+        c = CONFIGS["llm_d64"]
+        x = make_case(c)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        W1, W3 = (w.to(dev) for w in make_feature_weights(c.H, c.d_k, c.d_k, 7))
+        for _ in range(args.warmup + args.steps):
+            ttt.forward_chunked_phi(q, k, v, W1, W3, x["eta"].to(dev), eta_const=x["eta_const"], chunk=c.chunk)
     else:
         c = CONFIGS[args.workload]
         x = make_case(c)
@@ -435,7 +513,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llm_d64", choices=sorted(CONFIGS) + ["decode"])
+    ap.add_argument("--workload", default="llm_d64", choices=sorted(CONFIGS) + ["decode", "phi"])
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--sets", type=int, default=4)
@@ -443,14 +521,15 @@ def main():
     ap.add_argument("--cpu-heads", type=int, default=0, help="cpu_baseline sample; 0 = the whole layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-phi", action="store_true", help="skip the feature-map layer measurement")
     ap.add_argument("--profile-run", action="store_true",
                     help="plain launches for a profiler: no graphs, timing, decode or CPU baseline")
     args = ap.parse_args()
     if args.profile_run:
         profile_run(args)
         return
-    if args.workload == "decode":
-        raise SystemExit("decode is measured inside every chunked run (the 'decode' object)")
+    if args.workload in ("decode", "phi"):
+        raise SystemExit(f"{args.workload} is measured inside every chunked run (its own object in the line)")
     c = CONFIGS[args.workload]
     if c.dtype != "bf16":
         raise SystemExit("bench workloads are the bf16 layers")

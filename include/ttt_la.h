@@ -222,6 +222,38 @@ TTT_LA_API ttt_la_status ttt_la_compose_maps(int32_t nmaps, int32_t BH, int32_t 
                                              const float *dM, const float *GB, const float *W0, const float *M0,
                                              float *W_out, float *M_out, void *stream);
 
+/* Frozen-MLP feature map of the keys and queries (Variants 1-2 of Table 2 in
+ * the thelatestinai.com listing: the inner loop updates only the fast-weight
+ * network's last layer, so the layers before it are fixed for the sequence
+ * and act as the feature map phi of the (phi(Q) phi(K)^T) V form, kualia.ai
+ * explainer, section "The Linear Attention Equivalence").  The frozen part is
+ * one gated hidden layer of the "GLU Variants Improve Transformer" (SwiGLU)
+ * form, applied per token:
+ *
+ *   phi(x) = silu(W1[h] x) * (W3[h] x),   silu(a) = a / (1 + exp(-a)),
+ *
+ * with fp32 accumulation and the result rounded to bf16.  The linear fast
+ * weight is then trained on phi(k) and read with phi(q): call
+ * ttt_la_forward_chunked (or the recurrent / decode forms) with q := phi(q),
+ * k := phi(k), d_k := d_out.
+ *
+ * Fields: x[i], y[i] for i < n_inputs (1 or 2; typically q and k in one
+ * launch).  x[i]: [B,H,T,d_in] bf16; y[i]: [B,H,T,d_out] bf16, written;
+ * w1, w3: [H,d_out,d_in] bf16 (row o of w1[h] gives hidden unit o), shared by
+ * every input.  (d_in, d_out) in {64,128} x {64,128}; other widths return
+ * TTT_LA_ERR_UNSUPPORTED.  Device pointers, 16-byte aligned; y[i] must not
+ * overlap any x[j] or the weights.  One launch, asynchronous on `stream`;
+ * errors as ttt_la_forward_chunked. */
+typedef struct ttt_la_feature_args {
+  int32_t B, H, T, d_in, d_out;
+  int32_t n_inputs;
+  const void *x[2];
+  void *y[2];
+  const void *w1, *w3;
+} ttt_la_feature_args;
+
+TTT_LA_API ttt_la_status ttt_la_feature_map(const ttt_la_feature_args *args, void *stream);
+
 /* Synchronises `stream`, returns the device status word (TTT_LA_OK or
  * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
 TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);

@@ -3,13 +3,16 @@
 The C ABI lives in ``include/ttt_la.h`` and ``libttt_la.so`` (built in-tree by
 ``python -m test_layers_causal_b200.build``); this package is its thin Python
 binding.  Entry points: ``forward_chunked``, ``forward_recurrent``,
-``decode_step``, ``segment_map`` and ``compose_maps`` (see ``_abi``),
+``decode_step``, ``segment_map``, ``compose_maps``, ``feature_map`` (the
+frozen gated-MLP feature map of keys and queries) and ``forward_chunked_phi``
+(feature map, then the chunked forward) (see ``_abi``),
 ``forward_chunked_host`` (host buffers in, host buffers out, for end-to-end
 timing) and ``forward_sequence_sharded`` (one sequence split over ranks along
 T, see ``seqshard``).
 """
 from ._abi import (  # noqa: F401
-    TttError, compose_maps, decode_step, device_status, forward_chunked, forward_recurrent, lib, segment_map,
+    TttError, compose_maps, decode_step, device_status, feature_map, forward_chunked, forward_chunked_phi,
+    forward_recurrent, lib, segment_map,
     selftest_wait_timeout, set_wait_limit_ns, status_string, version, workspace_bytes,
 )
 from .host import forward_chunked_host  # noqa: F401

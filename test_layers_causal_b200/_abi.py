@@ -44,6 +44,14 @@ class TttDecodeArgs(ctypes.Structure):
     ]
 
 
+class TttFeatureArgs(ctypes.Structure):
+    """Mirror of ``ttt_la_feature_args``."""
+    _fields_ = [
+        ("B", _c_i32), ("H", _c_i32), ("T", _c_i32), ("d_in", _c_i32), ("d_out", _c_i32), ("n_inputs", _c_i32),
+        ("x", _c_vp * 2), ("y", _c_vp * 2), ("w1", _c_vp), ("w3", _c_vp),
+    ]
+
+
 # (name, restype, argtypes) for every symbol of include/ttt_la.h
 SIGNATURES = [
     ("ttt_la_workspace_size", _c_sz, [ctypes.POINTER(TttArgs)]),
@@ -55,6 +63,7 @@ SIGNATURES = [
     ("ttt_la_segment_map", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp, _c_vp, _c_vp, _c_vp]),
     ("ttt_la_compose_maps", ctypes.c_int, [ctypes.c_int32] * 4 + [_c_vp] * 8),
     ("ttt_la_decode_step", ctypes.c_int, [ctypes.POINTER(TttDecodeArgs), _c_vp]),
+    ("ttt_la_feature_map", ctypes.c_int, [ctypes.POINTER(TttFeatureArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
     ("ttt_la_set_wait_limit_ns", ctypes.c_int, [ctypes.c_int64]),
     ("ttt_la_selftest_wait_timeout", ctypes.c_int, [ctypes.c_int64, _c_vp]),
@@ -254,6 +263,50 @@ def compose_maps(dW, dM=None, GB=None, W0=None, M0=None, stream=None):
         n, B * H, dv, dk, _ptr(dW), _ptr(dM), _ptr(GB), _ptr(W0), _ptr(M0), _ptr(W), _ptr(M),
         _stream_handle(stream)))
     return W, M
+
+
+def feature_map(xs, W1, W3, out=None, stream=None):
+    """phi(x) = silu(W1 x) * (W3 x) of one or two bf16 inputs in one launch
+    (ttt_la_feature_map).  xs: a tensor or a sequence of one or two tensors
+    [B,H,T,d_in]; W1, W3: bf16 [H,d_out,d_in].  Returns a list of bf16
+    [B,H,T,d_out] tensors (written into `out` when given)."""
+    xs = [xs] if torch.is_tensor(xs) else list(xs)
+    if not 1 <= len(xs) <= 2:
+        raise ValueError("one or two inputs")
+    x0 = xs[0]
+    if x0.dim() != 4 or any(x.shape != x0.shape for x in xs):
+        raise ValueError("inputs must share one [B,H,T,d_in] shape")
+    B, H, T, d_in = x0.shape
+    if W1.dim() != 3 or W1.shape != W3.shape or W1.shape[0] != H or W1.shape[2] != d_in:
+        raise ValueError("W1, W3 must be [H,d_out,d_in]")
+    if any(t.dtype != torch.bfloat16 for t in (*xs, W1, W3)):
+        raise TypeError("the feature map takes bf16 inputs and weights")
+    if not all(t.is_contiguous() for t in (*xs, W1, W3)):
+        raise ValueError("inputs and weights must be contiguous")
+    _need_cuda(*xs, W1, W3)
+    d_out = W1.shape[1]
+    ys = list(out) if out is not None else [torch.empty(B, H, T, d_out, device=x0.device, dtype=torch.bfloat16)
+                                            for _ in xs]
+    if len(ys) != len(xs) or any(y.shape != (B, H, T, d_out) or y.dtype != torch.bfloat16 or not y.is_contiguous()
+                                 for y in ys):
+        raise ValueError("out: one contiguous bf16 [B,H,T,d_out] tensor per input")
+    a = TttFeatureArgs()
+    a.B, a.H, a.T, a.d_in, a.d_out, a.n_inputs = B, H, T, d_in, d_out, len(xs)
+    for i, (x, y) in enumerate(zip(xs, ys)):
+        a.x[i] = x.data_ptr()
+        a.y[i] = y.data_ptr()
+    a.w1, a.w3 = W1.data_ptr(), W3.data_ptr()
+    _check("ttt_la_feature_map", lib().ttt_la_feature_map(ctypes.byref(a), _stream_handle(stream)))
+    return ys
+
+
+def forward_chunked_phi(q, k, v, W1, W3, eta=None, **kw):
+    """The layer whose fast weight is the last layer of a frozen gated MLP:
+    phi(q), phi(k) by ttt_la_feature_map (one launch for both), then the
+    chunked forward on (phi(q), phi(k), v) with d_k = d_out.  Keyword
+    arguments as forward_chunked.  Returns forward_chunked's (o, S, M)."""
+    fq, fk = feature_map([q, k], W1, W3, stream=kw.get("stream"))
+    return forward_chunked(fq, fk, v, eta, **kw)
 
 
 def workspace_bytes(q, v, chunk=64, beta=0.0, segments=0):

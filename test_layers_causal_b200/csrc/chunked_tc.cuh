@@ -103,10 +103,7 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int C, int kk) {
   return sdesc_sw128(base + static_cast<uint32_t>(kk * 2048), static_cast<uint32_t>(C * 128), 1024);
 }
 
-// Offsets (in the descriptor's 16-byte address units) of k-step kk.
-__host__ __device__ constexpr uint64_t k_step(int rows, int kk) {
-  return static_cast<uint64_t>(((kk >> 2) * rows * 128 + (kk & 3) * 32) >> 4);
-}
+// Offset (in the descriptor's 16-byte address units) of the MN-major step kk.
 __host__ __device__ constexpr uint64_t mn_step(int kk) { return static_cast<uint64_t>(kk * 2048 >> 4); }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -134,11 +131,6 @@ __device__ __noinline__ unsigned wait_geq(const unsigned* p, unsigned target, ui
   }
 }
 
-// 16-byte store to a shared-memory address (32-bit: half the address
-// registers of a generic pointer).
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
 
 // Packs 32 fp32 values (as raw bits) into bf16 and writes them as four
 // 16-byte units of row `row` of a 128B-swizzled K-major tile (shared address

@@ -246,10 +246,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((static_cast<uint32_t>(M) >> 4) << 24); // M / 16
 }
 
+// K-major operand stored as 64-element k-blocks of `rows` 128-byte rows
+// (SW128): offset, in the descriptor's 16-byte address units, of the 16-wide
+// k-step kk (block kk / 4, (kk % 4) * 32 bytes into each row).
+__host__ __device__ constexpr uint64_t k_step(int rows, int kk) {
+  return static_cast<uint64_t>(((kk >> 2) * rows * 128 + (kk & 3) * 32) >> 4);
+}
+
 // Byte offset of the 16-byte unit `c16` (0..7) of row `row` inside a
 // 128B-swizzled block whose rows are 128 bytes.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t c16) {
   return row * 128u + ((c16 ^ (row & 7u)) << 4);
+}
+
+// 16-byte store to a shared-memory address (32-bit: half the address
+// registers of a generic pointer).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

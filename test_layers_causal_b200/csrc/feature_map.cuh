@@ -1,0 +1,265 @@
+// feature_map.cuh -- the frozen feature map phi(x) = silu(W1 x) * (W3 x) of
+// keys and queries, on the fifth-generation tensor cores (sm_100a).
+//
+// Variants 1-2 of Table 2 in the thelatestinai.com listing of "Test-Time
+// Training with KV Binding Is Secretly Linear Attention" update only the last
+// layer of the fast-weight MLP, so the layers before it are fixed for the
+// sequence and act as a feature map of the keys and queries.  Here that fixed
+// part is one gated hidden layer of the "GLU Variants Improve Transformer"
+// form; per head h and token,
+//   phi(x) = silu(W1[h] x) * (W3[h] x),   silu(a) = a / (1 + exp(-a)).
+//
+// Design.  A tile is 128 tokens of one (input, b, h).  W1[h] and W3[h] are
+// stacked into one K-major B operand [W1; W3] of 2 d_out rows, so a single
+// chain of d_in / 16 MMAs writes [x W1^T | x W3^T] (128 lanes x 2 d_out fp32
+// columns) into TMEM.  TMEM holds two such accumulators: the epilogue of one
+// tile overlaps the MMAs of the next, and the x stages keep NST tiles of
+// loads in flight.  The grid is persistent, one CTA per SM, and walks the
+// tiles in head-major order in contiguous ranges, so a CTA's tiles mostly
+// share one head and its stacked weights stay in shared memory.
+//
+// Warp roles (320 threads):
+//   warp 0     TMA producer: the stacked weights on a head change, x tiles
+//   warp 1     MMA issuer; owns the TMEM allocation
+//   warps 2-9  epilogue: warp w reads TMEM lane quadrant w % 4 and half
+//              (w - 2) / 4 of the output columns, applies the gate, rounds to
+//              bf16 into a double-buffered 128B-swizzled tile; one thread
+//              issues the TMA stores (rows past T are clipped by the map).
+//
+// Bound: HBM.  Per token it reads d_in and writes d_out bf16 values; the
+// weights (2 d_out d_in bf16 per head) come from L2.
+#pragma once
+#include "common.cuh"
+
+namespace ttt {
+
+struct FmapParams {
+  int H, B, T;
+  int ntile;    // 128-token tiles per sequence
+  int ninputs;  // 1 or 2
+  int total;    // H * ninputs * B * ntile
+  uint64_t limit_ns;
+};
+
+template <int DIN, int DOUT>
+struct FmapCfg {
+  static_assert(DIN == 64 || DIN == 128, "input width");
+  static_assert(DOUT == 64 || DOUT == 128, "output width");
+  static constexpr int ROWS = 128;            // tokens per tile (MMA M)
+  static constexpr int N = 2 * DOUT;          // [W1; W3] rows (MMA N)
+  static constexpr int XT = ROWS * DIN * 2;   // x tile bytes
+  static constexpr int WT = N * DIN * 2;      // stacked weight bytes
+  static constexpr int YT = ROWS * DOUT * 2;  // output tile bytes
+  static constexpr int fits(int nst) { return 1024 + WT + nst * XT + 2 * YT + 256 <= 232448; }
+  static constexpr int NST = fits(4) ? 4 : (fits(3) ? 3 : 2);
+  static constexpr int OFF_X = WT;
+  static constexpr int OFF_Y = OFF_X + NST * XT;
+  static constexpr int OFF_BAR = OFF_Y + 2 * YT;
+  static constexpr int NBAR = 2 * NST + 7;    // full, empty, w_full, w_empty, acc_full[2], acc_empty[2], drain
+  static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+  static constexpr int TCOLS = 2 * N;         // two accumulators: 256 or 512 columns
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int CW = DOUT / 2;         // output columns per epilogue thread
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+// silu(a) * b = a b / (1 + e^-a).  The exponent is clamped at 80 so that the
+// denominator stays below 2^126, the range of the fast division; past the
+// clamp the quotient is below 1e-33 of a b anyway.
+__device__ __forceinline__ float swiglu(float a, float b) {
+  return __fdividef(a * b, 1.f + __expf(-fmaxf(a, -80.f)));
+}
+
+template <int DIN, int DOUT>
+__global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
+    feature_map_kernel(const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmX1,
+                       const __grid_constant__ CUtensorMap tmY0, const __grid_constant__ CUtensorMap tmY1,
+                       const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW3,
+                       const FmapParams p) {
+  using Cfg = FmapCfg<DIN, DOUT>;
+  constexpr int NST = Cfg::NST, ROWS = Cfg::ROWS, N = Cfg::N;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint64_t* full = bars;                 // [NST] x tile landed
+  uint64_t* empty = bars + NST;          // [NST] x stage consumed by the MMAs
+  uint64_t* w_full = bars + 2 * NST;     // stacked weights landed
+  uint64_t* w_empty = w_full + 1;        // MMAs on the previous weights done
+  uint64_t* acc_full = w_full + 2;       // [2] accumulator written
+  uint64_t* acc_empty = w_full + 4;      // [2] accumulator read out
+  uint64_t* drain = w_full + 6;          // every MMA of this CTA done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.limit_ns;
+  // Contiguous range of tiles, head-major: tile i -> (head, input, b, t).
+  const int lo = static_cast<int>(static_cast<long long>(blockIdx.x) * p.total / gridDim.x);
+  const int hi = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.total / gridDim.x);
+  const int per_head = p.ninputs * p.B * p.ntile;
+  auto head_of = [&](int i) { return i / per_head; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(w_full, 1);
+    mbar_init(w_empty, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], Cfg::EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::TCOLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX0);
+    prefetch_tmap(&tmX1);
+    prefetch_tmap(&tmY0);
+    prefetch_tmap(&tmY1);
+    prefetch_tmap(&tmW1);
+    prefetch_tmap(&tmW3);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer --
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();  // x is read once
+      bool dead = false;
+      int cur = -1, nw = 0;
+      for (int i = lo, li = 0; i < hi && !dead; ++i, ++li) {
+        const int head = head_of(i), r = i % per_head;
+        const int inp = r / (p.B * p.ntile), b = (r / p.ntile) % p.B, t = r % p.ntile;
+        if (head != cur) {
+          if (nw > 0) dead = !mbar_wait(w_empty, (nw - 1) & 1, lim);
+          if (dead) break;
+          mbar_arrive_expect_tx(w_full, Cfg::WT);
+#pragma unroll
+          for (int kb = 0; kb < DIN / 64; ++kb) {
+            tma_load_3d(&tmW1, w_full, smem + kb * N * 128, kb * 64, 0, head);
+            tma_load_3d(&tmW3, w_full, smem + kb * N * 128 + DOUT * 128, kb * 64, 0, head);
+          }
+          cur = head;
+          ++nw;
+        }
+        const int s = li % NST;
+        if (li >= NST) dead = !mbar_wait(&empty[s], ((li / NST) - 1) & 1, lim);
+        if (dead) break;
+        mbar_arrive_expect_tx(&full[s], Cfg::XT);
+        const CUtensorMap* mx = inp ? &tmX1 : &tmX0;
+        uint8_t* xs = smem + Cfg::OFF_X + s * Cfg::XT;
+#pragma unroll
+        for (int kb = 0; kb < DIN / 64; ++kb)
+          tma_load_3d_hint(mx, &full[s], xs + kb * ROWS * 128, kb * 64, t * ROWS, b * p.H + head, pol);
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t ID = idesc_bf16_f32(ROWS, N, false, false);
+      const uint64_t dw = sdesc_sw128(sbase, 16, 1024);
+      bool dead = false;
+      int cur = -1, nw = 0;
+      for (int i = lo, li = 0; i < hi && !dead; ++i, ++li) {
+        const int head = head_of(i);
+        if (head != cur) {
+          if (nw > 0) tc_commit(w_empty);
+          dead = !mbar_wait(w_full, nw & 1, lim);
+          if (dead) break;
+          cur = head;
+          ++nw;
+        }
+        const int s = li % NST, a = li & 1;
+        dead = !mbar_wait(&full[s], (li / NST) & 1, lim);
+        if (!dead && li >= 2) dead = !mbar_wait(&acc_empty[a], ((li >> 1) - 1) & 1, lim);
+        if (dead) break;
+        tc_fence_after();
+        const uint64_t dx = sdesc_sw128(sbase + Cfg::OFF_X + s * Cfg::XT, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < DIN / 16; ++kk)
+          mma_bf16_ss(tmem + a * N, dx + k_step(ROWS, kk), dw + k_step(N, kk), ID, kk > 0 ? 1u : 0u);
+        tc_commit(&empty[s]);
+        tc_commit(&acc_full[a]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, lim);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int ew = warp - 2, quad = warp & 3, half = ew >> 2;
+    const int row = quad * 32 + lane;
+    const bool issuer = (ew == 0 && lane == 0);
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    bool dead = false;
+    for (int i = lo, li = 0; i < hi; ++i, ++li) {
+      const int head = head_of(i), r = i % per_head;
+      const int inp = r / (p.B * p.ntile), b = (r / p.ntile) % p.B, t = r % p.ntile;
+      const int a = li & 1;
+      if (!dead) dead = !mbar_wait(&acc_full[a], (li >> 1) & 1, lim);
+      dead = __any_sync(0xffffffffu, dead);
+      uint32_t out[Cfg::CW / 2];
+      if (!dead) {
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < Cfg::CW / 32; ++j) {
+          uint32_t ra[32], rb[32];
+          const uint32_t tb = tmem + a * N + lane_off + half * Cfg::CW + j * 32;
+          tmem_ld32(tb, ra);
+          tmem_ld32(tb + DOUT, rb);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            out[16 * j + e] = pack_bf16x2(swiglu(__uint_as_float(ra[2 * e]), __uint_as_float(rb[2 * e])),
+                                          swiglu(__uint_as_float(ra[2 * e + 1]), __uint_as_float(rb[2 * e + 1])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[a]);
+      }
+      // The tile buffer was last stored from two tiles ago: its TMA store must
+      // have finished reading it.
+      if (issuer) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * Cfg::EPI_WARPS) : "memory");
+      const uint32_t ys = sbase + Cfg::OFF_Y + a * Cfg::YT;
+      if (!dead) {
+#pragma unroll
+        for (int j = 0; j < Cfg::CW / 32; ++j) {
+          const int c0 = half * Cfg::CW + j * 32;
+          const uint32_t blk = ys + (c0 >> 6) * (ROWS * 128);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(blk + sw128_off(row, ((c0 & 63) >> 3) + q), out[16 * j + 4 * q], out[16 * j + 4 * q + 1],
+                         out[16 * j + 4 * q + 2], out[16 * j + 4 * q + 3]);
+        }
+        fence_async_smem();
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * Cfg::EPI_WARPS) : "memory");
+      if (issuer && !dead) {
+        const CUtensorMap* my = inp ? &tmY1 : &tmY0;
+#pragma unroll
+        for (int blk = 0; blk < DOUT / 64; ++blk)
+          tma_store_3d(my, smem + Cfg::OFF_Y + a * Cfg::YT + blk * ROWS * 128, blk * 64, t * ROWS, b * p.H + head);
+        bulk_commit();
+      }
+    }
+    if (issuer) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::TCOLS);
+}
+
+}  // namespace ttt

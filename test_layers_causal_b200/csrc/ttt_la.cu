@@ -18,6 +18,7 @@
 #include "chunked_tc_mom.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "feature_map.cuh"
 #include "recurrent.cuh"
 #include "seqshard.cuh"
 
@@ -342,6 +343,67 @@ ttt_la_status decode_dk(const ttt_la_decode_args* a, cudaStream_t st) {
   }
 }
 
+// ----------------------------------------------------------- feature map ----
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+ttt_la_status check_feature(const ttt_la_feature_args* a) {
+  if (!a) return TTT_LA_ERR_INVALID_ARG;
+  if (a->B < 1 || a->H < 1 || a->T < 1 || a->d_in < 1 || a->d_out < 1) return TTT_LA_ERR_INVALID_ARG;
+  if (a->n_inputs != 1 && a->n_inputs != 2) return TTT_LA_ERR_INVALID_ARG;
+  if (!a->w1 || !a->w3 || !aligned16(a->w1) || !aligned16(a->w3)) return TTT_LA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(a->B) * a->H;
+  const long long ntile = (a->T + 127) / 128;
+  if (bh > (1 << 30) || static_cast<long long>(a->T) * std::max(a->d_in, a->d_out) * bh > (1ll << 40) ||
+      bh * ntile * a->n_inputs >= (1ll << 31))
+    return TTT_LA_ERR_INVALID_ARG;
+  const size_t xb = static_cast<size_t>(bh) * a->T * a->d_in * 2, yb = static_cast<size_t>(bh) * a->T * a->d_out * 2;
+  const size_t wb = static_cast<size_t>(a->H) * a->d_out * a->d_in * 2;
+  for (int i = 0; i < a->n_inputs; ++i) {
+    if (!a->x[i] || !a->y[i] || !aligned16(a->x[i]) || !aligned16(a->y[i])) return TTT_LA_ERR_INVALID_ARG;
+    if (overlaps(a->y[i], yb, a->w1, wb) || overlaps(a->y[i], yb, a->w3, wb)) return TTT_LA_ERR_INVALID_ARG;
+    for (int j = 0; j < a->n_inputs; ++j)
+      if (overlaps(a->y[i], yb, a->x[j], xb) || (j != i && overlaps(a->y[i], yb, a->y[j], yb)))
+        return TTT_LA_ERR_INVALID_ARG;
+  }
+  if ((a->d_in != 64 && a->d_in != 128) || (a->d_out != 64 && a->d_out != 128)) return TTT_LA_ERR_UNSUPPORTED;
+  return TTT_LA_OK;
+}
+
+template <int DIN, int DOUT>
+ttt_la_status launch_feature(const ttt_la_feature_args* a, cudaStream_t st) {
+  using Cfg = ttt::FmapCfg<DIN, DOUT>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::feature_map_kernel<DIN, DOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
+  const int bh = a->B * a->H;
+  CUtensorMap mx[2], my[2], m1, m3;
+  for (int i = 0; i < 2; ++i) {
+    const int j = i < a->n_inputs ? i : 0;  // a single input fills both slots
+    if (!make_map(&mx[i], a->x[j], bh, a->T, DIN, Cfg::ROWS) || !make_map(&my[i], a->y[j], bh, a->T, DOUT, Cfg::ROWS))
+      return TTT_LA_ERR_CUDA;
+  }
+  if (!make_map(&m1, a->w1, a->H, DOUT, DIN, DOUT) || !make_map(&m3, a->w3, a->H, DOUT, DIN, DOUT))
+    return TTT_LA_ERR_CUDA;
+  ttt::FmapParams p;
+  p.H = a->H;
+  p.B = a->B;
+  p.T = a->T;
+  p.ntile = (a->T + Cfg::ROWS - 1) / Cfg::ROWS;
+  p.ninputs = a->n_inputs;
+  p.total = a->H * a->n_inputs * a->B * p.ntile;
+  p.limit_ns = g_limit_ns;
+  const int grid = std::min(p.total, sm_count());
+  ttt::feature_map_kernel<DIN, DOUT><<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mx[0], mx[1], my[0], my[1], m1, m3, p);
+  return launched();
+}
+
 // Scratch of ttt_la_forward_chunked_noalloc: one fixed array per device,
 // shared by every call on that device (see include/ttt_la.h).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TTT_LA_STATIC_SCRATCH_BYTES];
@@ -567,6 +629,14 @@ ttt_la_status ttt_la_compose_maps(int32_t nmaps, int32_t BH, int32_t d_v, int32_
   const int blocks = static_cast<int>(std::min<long long>(want, static_cast<long long>(sm_count()) * 8));
   ttt::compose_maps_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
   return launched();
+}
+
+ttt_la_status ttt_la_feature_map(const ttt_la_feature_args* a, void* stream) {
+  const ttt_la_status s = check_feature(a);
+  if (s != TTT_LA_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a->d_in == 64) return a->d_out == 64 ? launch_feature<64, 64>(a, st) : launch_feature<64, 128>(a, st);
+  return a->d_out == 64 ? launch_feature<128, 64>(a, st) : launch_feature<128, 128>(a, st);
 }
 
 ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {

@@ -58,6 +58,9 @@ int main(void) {
   P(ttt_la_args, state_in); P(ttt_la_args, o); P(ttt_la_args, workspace_bytes);
   P(ttt_la_decode_args, q); P(ttt_la_decode_args, eta_const); P(ttt_la_decode_args, state);
   P(ttt_la_decode_args, o);
+  printf("ttt_la_feature_args %zu\n", sizeof(ttt_la_feature_args));
+  P(ttt_la_feature_args, n_inputs); P(ttt_la_feature_args, x); P(ttt_la_feature_args, y);
+  P(ttt_la_feature_args, w1); P(ttt_la_feature_args, w3);
   return 0;
 }
 """
@@ -70,10 +73,13 @@ int main(void) {
     vals = dict(l.split() for l in lines if l.strip())
     assert int(vals["ttt_la_args"]) == ctypes.sizeof(abi.TttArgs)
     assert int(vals["ttt_la_decode_args"]) == ctypes.sizeof(abi.TttDecodeArgs)
+    assert int(vals["ttt_la_feature_args"]) == ctypes.sizeof(abi.TttFeatureArgs)
+    classes = {"ttt_la_args": abi.TttArgs, "ttt_la_decode_args": abi.TttDecodeArgs,
+               "ttt_la_feature_args": abi.TttFeatureArgs}
     for key, v in vals.items():
         if "." in key:
             struct, field = key.split(".")
-            cls = abi.TttArgs if struct == "ttt_la_args" else abi.TttDecodeArgs
+            cls = classes[struct]
             assert getattr(cls, field).offset == int(v), key
 
 
@@ -138,6 +144,47 @@ def test_decode_validation(abi):
     d.state, d.N = 0x50000, 0
     assert L.ttt_la_decode_step(ctypes.byref(d), None) == abi.ERR_INVALID_ARG
     assert L.ttt_la_decode_step(None, None) == abi.ERR_INVALID_ARG
+
+
+def _feature_args(abi, B=2, H=4, T=300, d_in=64, d_out=64, n=2):
+    f = abi.TttFeatureArgs()
+    f.B, f.H, f.T, f.d_in, f.d_out, f.n_inputs = B, H, T, d_in, d_out, n
+    # fake, disjoint, 16-byte aligned device addresses: nothing is launched
+    # because every case below fails a host-side check
+    f.x[0], f.x[1], f.y[0], f.y[1] = 0x1000000, 0x2000000, 0x3000000, 0x4000000
+    f.w1, f.w3 = 0x5000000, 0x5100000
+    return f
+
+
+def test_feature_map_validation(abi):
+    L = abi.lib()
+    call = lambda f: L.ttt_la_feature_map(ctypes.byref(f), None)  # noqa: E731
+    assert L.ttt_la_feature_map(None, None) == abi.ERR_INVALID_ARG
+    for field, val in [("B", 0), ("T", 0), ("H", -1), ("n_inputs", 0), ("n_inputs", 3)]:
+        f = _feature_args(abi)
+        setattr(f, field, val)
+        assert call(f) == abi.ERR_INVALID_ARG, field
+    f = _feature_args(abi)
+    f.x[1] = 0x2000008  # misaligned input
+    assert call(f) == abi.ERR_INVALID_ARG
+    f = _feature_args(abi)
+    f.w3 = 0  # missing weight
+    assert call(f) == abi.ERR_INVALID_ARG
+    f = _feature_args(abi)
+    f.y[0] = f.x[1] + 4096  # output overlaps an input
+    assert call(f) == abi.ERR_INVALID_ARG
+    f = _feature_args(abi)
+    f.y[1] = f.y[0] + 4096  # the two outputs overlap
+    assert call(f) == abi.ERR_INVALID_ARG
+    f = _feature_args(abi)
+    f.y[0] = f.w1 - 16  # output runs into the weights
+    assert call(f) == abi.ERR_INVALID_ARG
+    for d_in, d_out in [(32, 64), (64, 96), (256, 128)]:
+        assert call(_feature_args(abi, d_in=d_in, d_out=d_out)) == abi.ERR_UNSUPPORTED
+    # a single input leaves the second slots unused: junk there is ignored
+    f = _feature_args(abi, n=1, d_in=32)
+    f.x[1], f.y[1] = 0x7, 0x3000000
+    assert call(f) == abi.ERR_UNSUPPORTED
 
 
 def test_workspace_query(abi):
