@@ -64,13 +64,16 @@ def executed_flops(c, B, H, T, chunk):
     return B * H * T * per
 
 
+CHUNKED_SOURCES = ("chunked_tc.cuh", "chunked_tc_mom.cuh", "common.cuh", "ttt_la.cu")
+
+
 def src_hash():
-    """Hash of the kernel sources and their launch planner (the device code in
-    csrc/*.cuh and ttt_la.cu; the host-buffer pipeline does not change what a
-    kernel launch reads or writes)."""
+    """Hash of the chunked kernels' sources and their launch planner (the files
+    they are compiled and planned from; the other kernels' headers and the
+    host-buffer pipeline do not change what a chunked launch reads or writes)."""
     h = hashlib.sha1()
     cdir = os.path.join(ROOT, "test_layers_causal_b200", "csrc")
-    for f in sorted(x for x in os.listdir(cdir) if x.endswith(".cuh") or x == "ttt_la.cu"):
+    for f in CHUNKED_SOURCES:
         with open(os.path.join(cdir, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]

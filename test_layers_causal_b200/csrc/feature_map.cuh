@@ -12,19 +12,21 @@
 // Design.  A tile is 128 tokens of one (input, b, h).  W1[h] and W3[h] are
 // stacked into one K-major B operand [W1; W3] of 2 d_out rows, so a single
 // chain of d_in / 16 MMAs writes [x W1^T | x W3^T] (128 lanes x 2 d_out fp32
-// columns) into TMEM.  TMEM holds two such accumulators: the epilogue of one
-// tile overlaps the MMAs of the next, and the x stages keep NST tiles of
-// loads in flight.  The grid is persistent, one CTA per SM, and walks the
-// tiles in head-major order in contiguous ranges, so a CTA's tiles mostly
-// share one head and its stacked weights stay in shared memory.
+// columns) into TMEM.  TMEM holds two (d_out 128) or four (d_out 64) such
+// accumulators, so the epilogue of one tile overlaps the MMAs of the next
+// ones, and up to eight x stages keep that many tiles of loads in flight.  The
+// grid is persistent, one CTA per SM, and walks the tiles in head-major order
+// in contiguous ranges, so a CTA's tiles mostly share one head and its stacked
+// weights stay in shared memory.
 //
-// Warp roles (320 threads):
+// Warp roles (576 threads):
 //   warp 0     TMA producer: the stacked weights on a head change, x tiles
 //   warp 1     MMA issuer; owns the TMEM allocation
-//   warps 2-9  epilogue: warp w reads TMEM lane quadrant w % 4 and half
-//              (w - 2) / 4 of the output columns, applies the gate, rounds to
-//              bf16 into a double-buffered 128B-swizzled tile; one thread
-//              issues the TMA stores (rows past T are clipped by the map).
+//   warps 2-17 epilogue, two groups of eight taking alternate tiles: a warp
+//              reads one TMEM lane quadrant and half of the output columns,
+//              applies the gate and rounds to bf16 into its group's
+//              128B-swizzled tile; one thread of the group stores the tile
+//              with TMA (rows past T are clipped by the map).
 //
 // Bound: HBM.  Per token it reads d_in and writes d_out bf16 values; the
 // weights (2 d_out d_in bf16 per head) come from L2.
@@ -51,24 +53,47 @@ struct FmapCfg {
   static constexpr int WT = N * DIN * 2;      // stacked weight bytes
   static constexpr int YT = ROWS * DOUT * 2;  // output tile bytes
   static constexpr int fits(int nst) { return 1024 + WT + nst * XT + 2 * YT + 256 <= 232448; }
-  static constexpr int NST = fits(4) ? 4 : (fits(3) ? 3 : 2);
+  // as many x stages as shared memory holds, up to 8 (bytes in flight per SM)
+  static constexpr int NST = fits(8) ? 8 : fits(6) ? 6 : fits(5) ? 5 : fits(4) ? 4 : fits(3) ? 3 : 2;
+  static constexpr int NACC = 512 / N;        // accumulators in TMEM: 4 (d_out 64) or 2 (d_out 128)
   static constexpr int OFF_X = WT;
   static constexpr int OFF_Y = OFF_X + NST * XT;
   static constexpr int OFF_BAR = OFF_Y + 2 * YT;
-  static constexpr int NBAR = 2 * NST + 7;    // full, empty, w_full, w_empty, acc_full[2], acc_empty[2], drain
+  static constexpr int NBAR = 2 * NST + 3 + 2 * NACC;  // full, empty, w_full, w_empty, drain, acc_full, acc_empty
   static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
-  static constexpr int TCOLS = 2 * N;         // two accumulators: 256 or 512 columns
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int TCOLS = NACC * N;      // all 512 columns
+  static constexpr int EPI_WARPS = 16;        // two groups of eight
+  static constexpr int GROUP_WARPS = 8;       // the warps that read one tile
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int CW = DOUT / 2;         // output columns per epilogue thread
+  static constexpr int CW = DOUT / 2;         // output columns per epilogue thread and tile
+  static constexpr int SUBS = CW / 32;        // 32-column pieces of them
   static_assert(SMEM <= 232448, "shared memory");
 };
 
+// Named barrier `id` over `n` threads (the epilogue groups).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// 1 / d for 1 <= d < 2^126 on the FMA pipe, leaving the special-function
+// unit (which bounds this kernel: it also evaluates e^-a) one operation per
+// element.  Newton-Raphson for the reciprocal, r <- r + r (1 - d r), from
+// the seed obtained by subtracting the bit pattern of d from 0x7F000000: for
+// d = 2^E m, 1 <= m < 2, that seed is 2^(-E-1) (3 - m), which lies in
+// [1/d, 1.125/d].  Each step squares the relative error: 2^-3, 2^-6, 2^-12,
+// 2^-24, so three steps reach single precision.
+__device__ __forceinline__ float recip_newton(float d) {
+  float r = __int_as_float(0x7F000000 - __float_as_int(d));
+#pragma unroll
+  for (int k = 0; k < 3; ++k) r = fmaf(r, fmaf(-d, r, 1.f), r);
+  return r;
+}
+
 // silu(a) * b = a b / (1 + e^-a).  The exponent is clamped at 80 so that the
-// denominator stays below 2^126, the range of the fast division; past the
-// clamp the quotient is below 1e-33 of a b anyway.
+// denominator stays below 2^116, inside the reciprocal's range; past the
+// clamp the quotient is below 1e-34 of a b anyway.
 __device__ __forceinline__ float swiglu(float a, float b) {
-  return __fdividef(a * b, 1.f + __expf(-fmaxf(a, -80.f)));
+  return (a * b) * recip_newton(1.f + __expf(-fmaxf(a, -80.f)));
 }
 
 template <int DIN, int DOUT>
@@ -88,9 +113,9 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
   uint64_t* empty = bars + NST;          // [NST] x stage consumed by the MMAs
   uint64_t* w_full = bars + 2 * NST;     // stacked weights landed
   uint64_t* w_empty = w_full + 1;        // MMAs on the previous weights done
-  uint64_t* acc_full = w_full + 2;       // [2] accumulator written
-  uint64_t* acc_empty = w_full + 4;      // [2] accumulator read out
-  uint64_t* drain = w_full + 6;          // every MMA of this CTA done
+  uint64_t* drain = w_full + 2;          // every MMA of this CTA done
+  uint64_t* acc_full = w_full + 3;       // [NACC] accumulator written
+  uint64_t* acc_empty = acc_full + Cfg::NACC;  // [NACC] accumulator read out
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,9 +133,9 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
     }
     mbar_init(w_full, 1);
     mbar_init(w_empty, 1);
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < Cfg::NACC; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], Cfg::EPI_WARPS);
+      mbar_init(&acc_empty[a], Cfg::GROUP_WARPS);  // one arrival per warp of the reading group
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -180,9 +205,9 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
           cur = head;
           ++nw;
         }
-        const int s = li % NST, a = li & 1;
+        const int s = li % NST, a = li % Cfg::NACC;
         dead = !mbar_wait(&full[s], (li / NST) & 1, lim);
-        if (!dead && li >= 2) dead = !mbar_wait(&acc_empty[a], ((li >> 1) - 1) & 1, lim);
+        if (!dead && li >= Cfg::NACC) dead = !mbar_wait(&acc_empty[a], ((li / Cfg::NACC) - 1) & 1, lim);
         if (dead) break;
         tc_fence_after();
         const uint64_t dx = sdesc_sw128(sbase + Cfg::OFF_X + s * Cfg::XT, 16, 1024);
@@ -197,59 +222,59 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue --
-    const int ew = warp - 2, quad = warp & 3, half = ew >> 2;
+    // Two groups of eight warps take alternate tiles, so one group's TMEM
+    // reads, barriers and store overlap the other's arithmetic.  In a group,
+    // warp w reads lane quadrant w % 4 and half (w / 4) % 2 of the output
+    // columns; the group shares one 128B-swizzled output tile, stored by one
+    // thread after a group barrier.
+    const int ew = warp - 2, grp = ew >> 3, quad = warp & 3, half = (ew >> 2) & 1;
     const int row = quad * 32 + lane;
-    const bool issuer = (ew == 0 && lane == 0);
+    const bool issuer = ((ew & 7) == 0 && lane == 0);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    bool dead = false;
-    for (int i = lo, li = 0; i < hi; ++i, ++li) {
+    const uint32_t ys = sbase + Cfg::OFF_Y + grp * Cfg::YT;
+    bool dead = false;  // warp-uniform: a wait ran out, later tiles are skipped
+    for (int i = lo + grp, li = grp; i < hi; i += 2, li += 2) {
       const int head = head_of(i), r = i % per_head;
       const int inp = r / (p.B * p.ntile), b = (r / p.ntile) % p.B, t = r % p.ntile;
-      const int a = li & 1;
-      if (!dead) dead = !mbar_wait(&acc_full[a], (li >> 1) & 1, lim);
-      dead = __any_sync(0xffffffffu, dead);
-      uint32_t out[Cfg::CW / 2];
-      if (!dead) {
+      const int a = li % Cfg::NACC;
+      // every thread of the group reaches both barriers of every tile: a
+      // timed-out wait only skips the work
+      if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (li / Cfg::NACC) & 1, lim));
+      const bool ok = !dead;
+      // the group's tile buffer: its previous store must have read it
+      if (issuer) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      named_bar_sync(1 + grp, 32 * Cfg::GROUP_WARPS);
+      if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < Cfg::CW / 32; ++j) {
-          uint32_t ra[32], rb[32];
-          const uint32_t tb = tmem + a * N + lane_off + half * Cfg::CW + j * 32;
+        for (int j = 0; j < Cfg::SUBS; ++j) {
+          uint32_t ra[32], rb[32], out[16];
+          const int c0 = half * Cfg::CW + j * 32;
+          const uint32_t tb = tmem + a * N + lane_off + c0;
           tmem_ld32(tb, ra);
           tmem_ld32(tb + DOUT, rb);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            out[16 * j + e] = pack_bf16x2(swiglu(__uint_as_float(ra[2 * e]), __uint_as_float(rb[2 * e])),
-                                          swiglu(__uint_as_float(ra[2 * e + 1]), __uint_as_float(rb[2 * e + 1])));
+            out[e] = pack_bf16x2(swiglu(__uint_as_float(ra[2 * e]), __uint_as_float(rb[2 * e])),
+                                 swiglu(__uint_as_float(ra[2 * e + 1]), __uint_as_float(rb[2 * e + 1])));
+          const uint32_t blk = ys + (c0 >> 6) * (ROWS * 128);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(blk + sw128_off(row, ((c0 & 63) >> 3) + q), out[4 * q], out[4 * q + 1], out[4 * q + 2],
+                         out[4 * q + 3]);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[a]);
-      }
-      // The tile buffer was last stored from two tiles ago: its TMA store must
-      // have finished reading it.
-      if (issuer) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * Cfg::EPI_WARPS) : "memory");
-      const uint32_t ys = sbase + Cfg::OFF_Y + a * Cfg::YT;
-      if (!dead) {
-#pragma unroll
-        for (int j = 0; j < Cfg::CW / 32; ++j) {
-          const int c0 = half * Cfg::CW + j * 32;
-          const uint32_t blk = ys + (c0 >> 6) * (ROWS * 128);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            st_shared_v4(blk + sw128_off(row, ((c0 & 63) >> 3) + q), out[16 * j + 4 * q], out[16 * j + 4 * q + 1],
-                         out[16 * j + 4 * q + 2], out[16 * j + 4 * q + 3]);
-        }
         fence_async_smem();
       }
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * Cfg::EPI_WARPS) : "memory");
-      if (issuer && !dead) {
+      named_bar_sync(1 + grp, 32 * Cfg::GROUP_WARPS);
+      if (issuer && ok) {
         const CUtensorMap* my = inp ? &tmY1 : &tmY0;
 #pragma unroll
         for (int blk = 0; blk < DOUT / 64; ++blk)
-          tma_store_3d(my, smem + Cfg::OFF_Y + a * Cfg::YT + blk * ROWS * 128, blk * 64, t * ROWS, b * p.H + head);
+          tma_store_3d(my, smem + Cfg::OFF_Y + grp * Cfg::YT + blk * ROWS * 128, blk * 64, t * ROWS, b * p.H + head);
         bulk_commit();
       }
     }

@@ -52,18 +52,23 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH][T][d] bf16 tensor, boxes of 64 elements x `rows` tokens, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int BH, int T, int d, int rows) {
+// [BH][T][d] bf16 tensor, boxes of `cols` elements x `rows` tokens.
+bool make_map_box(CUtensorMap* m, const void* base, int BH, int T, int d, int cols, int rows,
+                  CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(T) * d * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(cols), static_cast<cuuint32_t>(rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+// Boxes of 64 elements x `rows` tokens, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int BH, int T, int d, int rows) {
+  return make_map_box(m, base, BH, T, d, 64, rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // ------------------------------------------------------ argument checks ----

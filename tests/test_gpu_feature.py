@@ -29,6 +29,13 @@ if torch.cuda.is_available():
 WIDTHS = [(64, 64), (64, 128), (128, 64), (128, 128)]
 
 
+@pytest.fixture(autouse=True)
+def _no_timed_out_wait():
+    """Every test also requires that no in-kernel wait ran out."""
+    yield
+    assert _abi.device_status() == _abi.OK
+
+
 def _x(B, H, T, d, seed):
     q, k, _, _ = make_qkv((B, H), T, d, d, seed, with_z=False)
     return q.to(torch.bfloat16).contiguous().cuda(), k.to(torch.bfloat16).contiguous().cuda()
@@ -82,6 +89,20 @@ def test_feature_map_head_changes_inside_a_block(H, B, T):
     q, k = _x(B, H, T, 128, 30 + H)
     W1, W3 = _weights(H, 128, 64, 31)
     yq, yk = _abi.feature_map([q, k], W1, W3)
+    torch.cuda.synchronize()
+    _assert_phi(yq, q, W1, W3, "phi(q)")
+    _assert_phi(yk, k, W1, W3, "phi(k)")
+
+
+@pytest.mark.parametrize("d_in,d_out", WIDTHS)
+def test_feature_map_many_tiles_per_block(d_in, d_out):
+    """About seven tiles per block (1024 tiles over the persistent grid): every
+    TMEM accumulator and output buffer is reused several times."""
+    B, H, T = 1, 8, 8192
+    q, k = _x(B, H, T, d_in, 35)
+    W1, W3 = _weights(H, d_in, d_out, 36)
+    ys = [torch.full((B, H, T, d_out), float("nan"), device="cuda", dtype=torch.bfloat16) for _ in range(2)]
+    yq, yk = _abi.feature_map([q, k], W1, W3, out=ys)
     torch.cuda.synchronize()
     _assert_phi(yq, q, W1, W3, "phi(q)")
     _assert_phi(yk, k, W1, W3, "phi(k)")
