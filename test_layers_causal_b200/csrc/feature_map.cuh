@@ -52,13 +52,16 @@ struct FmapCfg {
   static constexpr int XT = ROWS * DIN * 2;   // x tile bytes
   static constexpr int WT = N * DIN * 2;      // stacked weight bytes
   static constexpr int YT = ROWS * DOUT * 2;  // output tile bytes
-  static constexpr int fits(int nst) { return 1024 + WT + nst * XT + 2 * YT + 256 <= 232448; }
+  static constexpr int fits(int nst, int yb) { return 1024 + WT + nst * XT + 2 * yb * YT + 256 <= 232448; }
+  // output tiles per epilogue group: two (the next tile is written while the
+  // last one is stored) when that still leaves four x stages
+  static constexpr int YB = fits(4, 2) ? 2 : 1;
   // as many x stages as shared memory holds, up to 8 (bytes in flight per SM)
-  static constexpr int NST = fits(8) ? 8 : fits(6) ? 6 : fits(5) ? 5 : fits(4) ? 4 : fits(3) ? 3 : 2;
+  static constexpr int NST = fits(8, YB) ? 8 : fits(6, YB) ? 6 : fits(5, YB) ? 5 : fits(4, YB) ? 4 : fits(3, YB) ? 3 : 2;
   static constexpr int NACC = 512 / N;        // accumulators in TMEM: 4 (d_out 64) or 2 (d_out 128)
   static constexpr int OFF_X = WT;
   static constexpr int OFF_Y = OFF_X + NST * XT;
-  static constexpr int OFF_BAR = OFF_Y + 2 * YT;
+  static constexpr int OFF_BAR = OFF_Y + 2 * YB * YT;
   static constexpr int NBAR = 2 * NST + 3 + 2 * NACC;  // full, empty, w_full, w_empty, drain, acc_full, acc_empty
   static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
   static constexpr int TCOLS = NACC * N;      // all 512 columns
@@ -231,18 +234,19 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
     const int row = quad * 32 + lane;
     const bool issuer = ((ew & 7) == 0 && lane == 0);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t ys = sbase + Cfg::OFF_Y + grp * Cfg::YT;
+    const uint32_t ys0 = Cfg::OFF_Y + grp * Cfg::YB * Cfg::YT;  // the group's output tiles
     bool dead = false;  // warp-uniform: a wait ran out, later tiles are skipped
     for (int i = lo + grp, li = grp; i < hi; i += 2, li += 2) {
       const int head = head_of(i), r = i % per_head;
       const int inp = r / (p.B * p.ntile), b = (r / p.ntile) % p.B, t = r % p.ntile;
       const int a = li % Cfg::NACC;
+      const uint32_t yoff = ys0 + ((li >> 1) % Cfg::YB) * Cfg::YT, ys = sbase + yoff;
       // every thread of the group reaches both barriers of every tile: a
       // timed-out wait only skips the work
       if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (li / Cfg::NACC) & 1, lim));
       const bool ok = !dead;
-      // the group's tile buffer: its previous store must have read it
-      if (issuer) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      // this output tile's previous store (YB tiles of the group ago) must have read it
+      if (issuer) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(Cfg::YB - 1) : "memory");
       named_bar_sync(1 + grp, 32 * Cfg::GROUP_WARPS);
       if (ok) {
         tc_fence_after();
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
         const CUtensorMap* my = inp ? &tmY1 : &tmY0;
 #pragma unroll
         for (int blk = 0; blk < DOUT / 64; ++blk)
-          tma_store_3d(my, smem + Cfg::OFF_Y + grp * Cfg::YT + blk * ROWS * 128, blk * 64, t * ROWS, b * p.H + head);
+          tma_store_3d(my, smem + yoff + blk * ROWS * 128, blk * 64, t * ROWS, b * p.H + head);
         bulk_commit();
       }
     }
