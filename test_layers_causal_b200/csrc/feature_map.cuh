@@ -78,25 +78,46 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// 1 / d for 1 <= d < 2^126 on the FMA pipe, leaving the special-function
-// unit (which bounds this kernel: it also evaluates e^-a) one operation per
-// element.  Newton-Raphson for the reciprocal, r <- r + r (1 - d r), from
-// the seed obtained by subtracting the bit pattern of d from 0x7F000000: for
-// d = 2^E m, 1 <= m < 2, that seed is 2^(-E-1) (3 - m), which lies in
-// [1/d, 1.125/d].  Each step squares the relative error: 2^-3, 2^-6, 2^-12,
-// 2^-24, so three steps reach single precision.
-__device__ __forceinline__ float recip_newton(float d) {
-  float r = __int_as_float(0x7F000000 - __float_as_int(d));
-#pragma unroll
-  for (int k = 0; k < 3; ++k) r = fmaf(r, fmaf(-d, r, 1.f), r);
-  return r;
+// Packed fp32 arithmetic (sm_100): one instruction applies the operation to
+// both halves of a pair, each rounded to nearest as the scalar form would be.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
-// silu(a) * b = a b / (1 + e^-a).  The exponent is clamped at 80 so that the
-// denominator stays below 2^116, inside the reciprocal's range; past the
-// clamp the quotient is below 1e-34 of a b anyway.
-__device__ __forceinline__ float swiglu(float a, float b) {
-  return (a * b) * recip_newton(1.f + __expf(-fmaxf(a, -80.f)));
+// silu(a) * b = a b / (1 + e^-a) for a pair of elements, packed as bf16x2.
+// e^-a comes from the special-function unit, which bounded the first
+// version of this kernel; the reciprocal stays on the FMA pipe: Newton-
+// Raphson, r <- r + r (1 - d r), from the seed obtained by subtracting the bit
+// pattern of d from 0x7F000000.  For d = 2^E m, 1 <= m < 2, that seed is
+// 2^(-E-1) (3 - m), within [1/d, 1.125/d]; each step squares the relative
+// error (2^-3, 2^-6, 2^-12, 2^-24), so three steps reach single precision.
+// The exponent is clamped at 80 so that d < 2^116 stays in the seed's range;
+// past the clamp the quotient is below 1e-34 of a b anyway.  The work runs on
+// negated denominators, nd = -(1 + e), so that 1 - d r is one fused step.
+__device__ __forceinline__ uint32_t swiglu2_bf16(float a0, float a1, float b0, float b1) {
+  const float2 e = make_float2(__expf(-fmaxf(a0, -80.f)), __expf(-fmaxf(a1, -80.f)));
+  const float2 m1 = make_float2(-1.f, -1.f), one = make_float2(1.f, 1.f);
+  const float2 nd = fma2(e, m1, m1);  // -(1 + e)
+  // seed of 1/d from -d: 0x7F000000 - bits(d) = 0xFF000000 - bits(-d) (mod 2^32)
+  float2 r = make_float2(__uint_as_float(0xFF000000u - __float_as_uint(nd.x)),
+                         __uint_as_float(0xFF000000u - __float_as_uint(nd.y)));
+#pragma unroll
+  for (int k = 0; k < 3; ++k) r = fma2(r, fma2(nd, r, one), r);
+  const float2 y = mul2(mul2(make_float2(a0, a1), make_float2(b0, b1)), r);
+  return pack_bf16x2(y.x, y.y);
 }
 
 template <int DIN, int DOUT>
@@ -250,7 +271,7 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
       named_bar_sync(1 + grp, 32 * Cfg::GROUP_WARPS);
       if (ok) {
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < Cfg::SUBS; ++j) {
           uint32_t ra[32], rb[32], out[16];
           const int c0 = half * Cfg::CW + j * 32;
@@ -260,8 +281,8 @@ __global__ void __launch_bounds__(FmapCfg<DIN, DOUT>::THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            out[e] = pack_bf16x2(swiglu(__uint_as_float(ra[2 * e]), __uint_as_float(rb[2 * e])),
-                                 swiglu(__uint_as_float(ra[2 * e + 1]), __uint_as_float(rb[2 * e + 1])));
+            out[e] = swiglu2_bf16(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1]),
+                                  __uint_as_float(rb[2 * e]), __uint_as_float(rb[2 * e + 1]));
           const uint32_t blk = ys + (c0 >> 6) * (ROWS * 128);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
