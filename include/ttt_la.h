@@ -254,6 +254,53 @@ typedef struct ttt_la_feature_args {
 
 TTT_LA_API ttt_la_status ttt_la_feature_map(const ttt_la_feature_args *args, void *stream);
 
+/* Backward of the layer (the gradient needed to train it, Figure 4 of the
+ * thelatestinai.com listing).  Given the forward's inputs and the upstream
+ * gradients dL/do (and optionally dL/dW_T, dL/dM_T on the final states), it
+ * writes dL/dq, dL/dk, dL/dv, the per-token dL/deta_t and dL/dW_0, dL/dM_0.
+ * Over the tokens in reverse, with G_t = dL/dW_t and H_t = dL/dM_t:
+ *   G_t = G_{t+1} + do_t q_t^T (G_{T+1} = dL/dW_T);  dq_t = W_t^T do_t
+ *   momentum: H_t = beta H_{t+1} - eta_t G_t (H_T = dL/dM_T - eta_T G_T),
+ *             dv_t = -sigma H_t k_t, dk_t = -sigma H_t^T v_t, deta_t = -<G_t, M_t>
+ *   plain:    dv_t = sigma eta_t G_t k_t, dk_t = sigma eta_t G_t^T v_t,
+ *             deta_t = sigma v_t^T G_t k_t
+ *   dW_0 = G_1, dM_0 = beta H_1 (zero without momentum).
+ *
+ * Fields: the forward's B, H, T, d_k, d_v, dtype, q, k, v, eta, eta_const,
+ * beta, ascent, state_in (W_0), mom_in (M_0) exactly as in ttt_la_args.
+ * grad_o: [B,H,T,d_v] dtype.  grad_state, grad_mom: [B,H,d_v,d_k] fp32 or
+ * NULL (zero).  Outputs: grad_q, grad_k [B,H,T,d_k] and grad_v [B,H,T,d_v]
+ * in dtype (required); grad_eta [B,H,T] fp32 (per token, also when eta is
+ * NULL: its sum is dL/deta_const), grad_state_in, grad_mom_in [B,H,d_v,d_k]
+ * fp32, each optional (NULL: not written).  Device pointers, 16-byte aligned;
+ * outputs must not overlap the inputs.  The workspace holds state
+ * checkpoints every 32 tokens and one chunk's state history per (b,h):
+ * ttt_la_backward_workspace_size bytes.
+ *
+ * ttt_la_backward_recurrent computes it token by token in fp32 with one
+ * block per (b,h).  d_k must be 32, 64 or 128 and d_v at most 512, 256 or 128
+ * respectively; other sizes return TTT_LA_ERR_UNSUPPORTED.  Errors as
+ * ttt_la_forward_chunked; a workspace smaller than the size query returns
+ * TTT_LA_ERR_INVALID_ARG. */
+typedef struct ttt_la_grad_args {
+  int32_t B, H, T, d_k, d_v;
+  int32_t dtype;            /* ttt_la_dtype of q, k, v, grad_o and grad_q/k/v */
+  const void *q, *k, *v;
+  const float *eta;
+  float eta_const, beta;
+  int32_t ascent;
+  const float *state_in, *mom_in;
+  const void *grad_o;
+  const float *grad_state, *grad_mom;
+  void *grad_q, *grad_k, *grad_v;
+  float *grad_eta, *grad_state_in, *grad_mom_in;
+  void *workspace;
+  size_t workspace_bytes;
+} ttt_la_grad_args;
+
+TTT_LA_API size_t ttt_la_backward_workspace_size(const ttt_la_grad_args *args);
+TTT_LA_API ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args *args, void *stream);
+
 /* Synchronises `stream`, returns the device status word (TTT_LA_OK or
  * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
 TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);

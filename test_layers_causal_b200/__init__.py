@@ -5,13 +5,15 @@ The C ABI lives in ``include/ttt_la.h`` and ``libttt_la.so`` (built in-tree by
 binding.  Entry points: ``forward_chunked``, ``forward_recurrent``,
 ``decode_step``, ``segment_map``, ``compose_maps``, ``feature_map`` (the
 frozen gated-MLP feature map of keys and queries) and ``forward_chunked_phi``
-(feature map, then the chunked forward) (see ``_abi``),
+(feature map, then the chunked forward), ``backward_recurrent`` (the
+layer's gradient) (see ``_abi``),
 ``forward_chunked_host`` (host buffers in, host buffers out, for end-to-end
 timing) and ``forward_sequence_sharded`` (one sequence split over ranks along
 T, see ``seqshard``).
 """
 from ._abi import (  # noqa: F401
-    TttError, compose_maps, decode_step, device_status, feature_map, forward_chunked, forward_chunked_phi,
+    TttError, backward_recurrent, compose_maps, decode_step, device_status, feature_map, forward_chunked,
+    forward_chunked_phi,
     forward_recurrent, lib, segment_map,
     selftest_wait_timeout, set_wait_limit_ns, status_string, version, workspace_bytes,
 )

@@ -52,6 +52,20 @@ class TttFeatureArgs(ctypes.Structure):
     ]
 
 
+class TttGradArgs(ctypes.Structure):
+    """Mirror of ``ttt_la_grad_args``."""
+    _fields_ = [
+        ("B", _c_i32), ("H", _c_i32), ("T", _c_i32), ("d_k", _c_i32), ("d_v", _c_i32), ("dtype", _c_i32),
+        ("q", _c_vp), ("k", _c_vp), ("v", _c_vp), ("eta", _c_vp),
+        ("eta_const", _c_f32), ("beta", _c_f32), ("ascent", _c_i32),
+        ("state_in", _c_vp), ("mom_in", _c_vp),
+        ("grad_o", _c_vp), ("grad_state", _c_vp), ("grad_mom", _c_vp),
+        ("grad_q", _c_vp), ("grad_k", _c_vp), ("grad_v", _c_vp),
+        ("grad_eta", _c_vp), ("grad_state_in", _c_vp), ("grad_mom_in", _c_vp),
+        ("workspace", _c_vp), ("workspace_bytes", _c_sz),
+    ]
+
+
 # (name, restype, argtypes) for every symbol of include/ttt_la.h
 SIGNATURES = [
     ("ttt_la_workspace_size", _c_sz, [ctypes.POINTER(TttArgs)]),
@@ -64,6 +78,8 @@ SIGNATURES = [
     ("ttt_la_compose_maps", ctypes.c_int, [ctypes.c_int32] * 4 + [_c_vp] * 8),
     ("ttt_la_decode_step", ctypes.c_int, [ctypes.POINTER(TttDecodeArgs), _c_vp]),
     ("ttt_la_feature_map", ctypes.c_int, [ctypes.POINTER(TttFeatureArgs), _c_vp]),
+    ("ttt_la_backward_workspace_size", _c_sz, [ctypes.POINTER(TttGradArgs)]),
+    ("ttt_la_backward_recurrent", ctypes.c_int, [ctypes.POINTER(TttGradArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
     ("ttt_la_set_wait_limit_ns", ctypes.c_int, [ctypes.c_int64]),
     ("ttt_la_selftest_wait_timeout", ctypes.c_int, [ctypes.c_int64, _c_vp]),
@@ -307,6 +323,39 @@ def forward_chunked_phi(q, k, v, W1, W3, eta=None, **kw):
     arguments as forward_chunked.  Returns forward_chunked's (o, S, M)."""
     fq, fk = feature_map([q, k], W1, W3, stream=kw.get("stream"))
     return forward_chunked(fq, fk, v, eta, **kw)
+
+
+def backward_recurrent(q, k, v, grad_o, eta=None, eta_const=None, beta=0.0, ascent=False, state_in=None,
+                       mom_in=None, grad_state=None, grad_mom=None, workspace=None, stream=None):
+    """Gradients of the layer (ttt_la_backward_recurrent): returns a dict with
+    dq, dk, dv (dtype of q), deta [B,H,T] fp32 (per token), dW0 and dM0
+    [B,H,d_v,d_k] fp32 (dM0 None without momentum)."""
+    _check_shapes(q, k, v, eta, state_in, mom_in)
+    if grad_o.shape != v.shape or grad_o.dtype != v.dtype or not grad_o.is_contiguous():
+        raise ValueError("grad_o must match v")
+    _need_cuda(q, k, v, grad_o, eta, state_in, mom_in, grad_state, grad_mom)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               deta=torch.empty(B, H, T, device=q.device, dtype=torch.float32),
+               dW0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32),
+               dM0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32) if beta else None)
+    a = TttGradArgs()
+    a.B, a.H, a.T, a.d_k, a.d_v, a.dtype = B, H, T, dk, dv, _dtype_code(q)
+    a.q, a.k, a.v, a.eta = q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(eta)
+    a.eta_const = (1.0 / math.sqrt(dk)) if eta_const is None else float(eta_const)
+    a.beta, a.ascent = float(beta), int(bool(ascent))
+    a.state_in, a.mom_in = _ptr(state_in), _ptr(mom_in)
+    a.grad_o, a.grad_state, a.grad_mom = grad_o.data_ptr(), _ptr(grad_state), _ptr(grad_mom)
+    a.grad_q, a.grad_k, a.grad_v = out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr()
+    a.grad_eta, a.grad_state_in, a.grad_mom_in = _ptr(out["deta"]), _ptr(out["dW0"]), _ptr(out["dM0"])
+    L = lib()
+    need = L.ttt_la_backward_workspace_size(ctypes.byref(a))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check("ttt_la_backward_recurrent", L.ttt_la_backward_recurrent(ctypes.byref(a), _stream_handle(stream)))
+    return out
 
 
 def workspace_bytes(q, v, chunk=64, beta=0.0, segments=0):

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "../../include/ttt_la.h"
+#include "backward.cuh"
 #include "chunked_simt.cuh"
 #include "chunked_tc.cuh"
 #include "chunked_tc_mom.cuh"
@@ -409,6 +410,101 @@ ttt_la_status launch_feature(const ttt_la_feature_args* a, cudaStream_t st) {
   return launched();
 }
 
+// -------------------------------------------------------------- backward ----
+int bwd_max_dv(int dk) { return dk == 32 ? 512 : dk == 64 ? 256 : 128; }  // 32 warps x rows per warp
+int bwd_nck(int T) { return (T + ttt::BwdShape<32>::CK - 1) / ttt::BwdShape<32>::CK; }
+size_t bwd_ws_bytes(const ttt_la_grad_args* a) {
+  const size_t ns = a->beta != 0.f ? 2 : 1;
+  const size_t per = (static_cast<size_t>(bwd_nck(a->T)) + ttt::BwdShape<32>::CK) * ns * a->d_v * a->d_k;
+  return static_cast<size_t>(a->B) * a->H * per * sizeof(float);
+}
+
+ttt_la_status check_grad(const ttt_la_grad_args* a) {
+  if (!a) return TTT_LA_ERR_INVALID_ARG;
+  if (a->B < 1 || a->H < 1 || a->T < 1 || a->d_k < 1 || a->d_v < 1) return TTT_LA_ERR_INVALID_ARG;
+  if (a->dtype != TTT_LA_F32 && a->dtype != TTT_LA_BF16) return TTT_LA_ERR_INVALID_ARG;
+  if (!(a->beta >= 0.f && a->beta < 1.f)) return TTT_LA_ERR_INVALID_ARG;
+  const void* need[] = {a->q, a->k, a->v, a->grad_o, a->grad_q, a->grad_k, a->grad_v};
+  for (const void* x : need)
+    if (!x || !aligned16(x)) return TTT_LA_ERR_INVALID_ARG;
+  const void* opt[] = {a->eta, a->state_in, a->mom_in, a->grad_state, a->grad_mom, a->grad_eta,
+                       a->grad_state_in, a->grad_mom_in, a->workspace};
+  for (const void* x : opt)
+    if (x && !aligned16(x)) return TTT_LA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(a->B) * a->H;
+  if (bh > (1 << 30) || static_cast<long long>(a->T) * std::max(a->d_k, a->d_v) * bh > (1ll << 40))
+    return TTT_LA_ERR_INVALID_ARG;
+  const size_t el = a->dtype == TTT_LA_F32 ? 4 : 2;
+  const size_t nk = static_cast<size_t>(bh) * a->T * a->d_k * el, nv = static_cast<size_t>(bh) * a->T * a->d_v * el;
+  const size_t ns = static_cast<size_t>(bh) * a->d_v * a->d_k * 4, ne = static_cast<size_t>(bh) * a->T * 4;
+  const void* outs[] = {a->grad_q, a->grad_k, a->grad_v, a->grad_eta, a->grad_state_in, a->grad_mom_in};
+  const size_t osz[] = {nk, nk, nv, ne, ns, ns};
+  const void* ins[] = {a->q, a->k, a->v, a->grad_o, a->eta, a->state_in, a->mom_in, a->grad_state, a->grad_mom};
+  const size_t isz[] = {nk, nk, nv, nv, ne, ns, ns, ns, ns};
+  for (int i = 0; i < 6; ++i) {
+    if (!outs[i]) continue;
+    for (int j = 0; j < 9; ++j)
+      if (ins[j] && overlaps(outs[i], osz[i], ins[j], isz[j])) return TTT_LA_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (outs[j] && overlaps(outs[i], osz[i], outs[j], osz[j])) return TTT_LA_ERR_INVALID_ARG;
+  }
+  if (a->d_k != 32 && a->d_k != 64 && a->d_k != 128) return TTT_LA_ERR_UNSUPPORTED;
+  if (a->d_v > bwd_max_dv(a->d_k)) return TTT_LA_ERR_UNSUPPORTED;
+  if (!a->workspace || a->workspace_bytes < bwd_ws_bytes(a)) return TTT_LA_ERR_INVALID_ARG;
+  return TTT_LA_OK;
+}
+
+template <int DK, typename T, bool MOM>
+ttt_la_status launch_backward(const ttt_la_grad_args* a, cudaStream_t st) {
+  using Sh = ttt::BwdShape<DK>;
+  const size_t smem = ttt::bwd_smem_floats(DK, a->d_v, Sh::CK) * sizeof(float);
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::backward_recurrent_kernel<DK, T, MOM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             232448) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
+  ttt::BwdParams p;
+  p.BH = a->B * a->H;
+  p.T = a->T;
+  p.dk = a->d_k;
+  p.dv = a->d_v;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.eta = a->eta;
+  p.eta_const = a->eta_const;
+  p.beta = a->beta;
+  p.sigma = a->ascent ? -1.f : 1.f;
+  p.S_in = a->state_in;
+  p.M_in = a->mom_in;
+  p.dO = a->grad_o;
+  p.dS = a->grad_state;
+  p.dM = a->grad_mom;
+  p.dq = a->grad_q;
+  p.dk_out = a->grad_k;
+  p.dv_out = a->grad_v;
+  p.deta = a->grad_eta;
+  p.dS_in = a->grad_state_in;
+  p.dM_in = a->grad_mom_in;
+  p.nck = bwd_nck(a->T);
+  const size_t ns = MOM ? 2 : 1;
+  p.ckpt = static_cast<float*>(a->workspace);
+  p.hist = p.ckpt + static_cast<size_t>(p.BH) * p.nck * ns * a->d_v * a->d_k;
+  const int warps = (a->d_v + Sh::ROWS_PER_WARP - 1) / Sh::ROWS_PER_WARP;
+  ttt::backward_recurrent_kernel<DK, T, MOM><<<p.BH, 32 * warps, smem, st>>>(p);
+  return launched();
+}
+template <typename T, bool MOM>
+ttt_la_status backward_dk(const ttt_la_grad_args* a, cudaStream_t st) {
+  switch (a->d_k) {
+    case 32: return launch_backward<32, T, MOM>(a, st);
+    case 64: return launch_backward<64, T, MOM>(a, st);
+    default: return launch_backward<128, T, MOM>(a, st);
+  }
+}
+
 // Scratch of ttt_la_forward_chunked_noalloc: one fixed array per device,
 // shared by every call on that device (see include/ttt_la.h).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TTT_LA_STATIC_SCRATCH_BYTES];
@@ -642,6 +738,20 @@ ttt_la_status ttt_la_feature_map(const ttt_la_feature_args* a, void* stream) {
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (a->d_in == 64) return a->d_out == 64 ? launch_feature<64, 64>(a, st) : launch_feature<64, 128>(a, st);
   return a->d_out == 64 ? launch_feature<128, 64>(a, st) : launch_feature<128, 128>(a, st);
+}
+
+size_t ttt_la_backward_workspace_size(const ttt_la_grad_args* a) {
+  if (!a || a->B < 1 || a->H < 1 || a->T < 1 || a->d_k < 1 || a->d_v < 1) return 0;
+  return bwd_ws_bytes(a);
+}
+
+ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args* a, void* stream) {
+  const ttt_la_status s = check_grad(a);
+  if (s != TTT_LA_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool mom = a->beta != 0.f;
+  if (a->dtype == TTT_LA_F32) return mom ? backward_dk<float, true>(a, st) : backward_dk<float, false>(a, st);
+  return mom ? backward_dk<__nv_bfloat16, true>(a, st) : backward_dk<__nv_bfloat16, false>(a, st);
 }
 
 ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {

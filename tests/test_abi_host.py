@@ -61,6 +61,10 @@ int main(void) {
   printf("ttt_la_feature_args %zu\n", sizeof(ttt_la_feature_args));
   P(ttt_la_feature_args, n_inputs); P(ttt_la_feature_args, x); P(ttt_la_feature_args, y);
   P(ttt_la_feature_args, w1); P(ttt_la_feature_args, w3);
+  printf("ttt_la_grad_args %zu\n", sizeof(ttt_la_grad_args));
+  P(ttt_la_grad_args, q); P(ttt_la_grad_args, eta_const); P(ttt_la_grad_args, state_in);
+  P(ttt_la_grad_args, grad_o); P(ttt_la_grad_args, grad_q); P(ttt_la_grad_args, grad_eta);
+  P(ttt_la_grad_args, grad_mom_in); P(ttt_la_grad_args, workspace_bytes);
   return 0;
 }
 """
@@ -74,8 +78,9 @@ int main(void) {
     assert int(vals["ttt_la_args"]) == ctypes.sizeof(abi.TttArgs)
     assert int(vals["ttt_la_decode_args"]) == ctypes.sizeof(abi.TttDecodeArgs)
     assert int(vals["ttt_la_feature_args"]) == ctypes.sizeof(abi.TttFeatureArgs)
+    assert int(vals["ttt_la_grad_args"]) == ctypes.sizeof(abi.TttGradArgs)
     classes = {"ttt_la_args": abi.TttArgs, "ttt_la_decode_args": abi.TttDecodeArgs,
-               "ttt_la_feature_args": abi.TttFeatureArgs}
+               "ttt_la_feature_args": abi.TttFeatureArgs, "ttt_la_grad_args": abi.TttGradArgs}
     for key, v in vals.items():
         if "." in key:
             struct, field = key.split(".")
@@ -185,6 +190,42 @@ def test_feature_map_validation(abi):
     f = _feature_args(abi, n=1, d_in=32)
     f.x[1], f.y[1] = 0x7, 0x3000000
     assert call(f) == abi.ERR_UNSUPPORTED
+
+
+def _grad_args(abi, B=2, H=2, T=100, dk=64, dv=64, beta=0.0):
+    g = abi.TttGradArgs()
+    g.B, g.H, g.T, g.d_k, g.d_v, g.dtype, g.beta = B, H, T, dk, dv, abi.BF16, beta
+    # fake, disjoint, 16-byte aligned addresses: every case below fails a host check
+    g.q, g.k, g.v, g.grad_o = 0x1000000, 0x2000000, 0x3000000, 0x4000000
+    g.grad_q, g.grad_k, g.grad_v = 0x5000000, 0x6000000, 0x7000000
+    g.workspace = 0x10000000
+    g.workspace_bytes = abi.lib().ttt_la_backward_workspace_size(ctypes.byref(g))
+    return g
+
+
+def test_backward_workspace_and_validation(abi):
+    L = abi.lib()
+    call = lambda g: L.ttt_la_backward_recurrent(ctypes.byref(g), None)  # noqa: E731
+    size = lambda g: L.ttt_la_backward_workspace_size(ctypes.byref(g))  # noqa: E731
+    # checkpoints every 32 tokens plus one chunk of history, W (and M) per head
+    g = _grad_args(abi, T=100)
+    assert size(g) == 2 * 2 * (4 + 32) * 1 * 64 * 64 * 4
+    assert size(_grad_args(abi, T=100, beta=0.9)) == 2 * 2 * (4 + 32) * 2 * 64 * 64 * 4
+    assert L.ttt_la_backward_workspace_size(None) == 0
+    assert L.ttt_la_backward_recurrent(None, None) == abi.ERR_INVALID_ARG
+    for field, val in [("T", 0), ("B", 0), ("beta", 1.0), ("beta", -0.1), ("grad_o", 0), ("grad_v", 0x7000008),
+                       ("workspace_bytes", 16)]:
+        g = _grad_args(abi)
+        setattr(g, field, val)
+        assert call(g) == abi.ERR_INVALID_ARG, field
+    g = _grad_args(abi)
+    g.grad_q = g.q + 64  # output overlaps an input
+    assert call(g) == abi.ERR_INVALID_ARG
+    g = _grad_args(abi)
+    g.grad_eta = g.grad_k + 256  # two outputs overlap
+    assert call(g) == abi.ERR_INVALID_ARG
+    for dk, dv in [(48, 64), (128, 256), (64, 512)]:
+        assert call(_grad_args(abi, dk=dk, dv=dv)) == abi.ERR_UNSUPPORTED
 
 
 def test_workspace_query(abi):
