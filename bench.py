@@ -322,6 +322,34 @@ def phi_measure(ttt, dev, peaks, reps=100):
             "gpu_launches_per_step": 2}
 
 
+def backward_measure(ttt, dev, reps=5):
+    """The layer's backward (ttt_la_backward_recurrent) on the llm_d64 inputs
+    (B4 H16 T4096 d64, per-token eta) with a seeded upstream gradient: dq,
+    dk, dv, per-token deta and dW0.  CUDA events over `reps` calls after one
+    warm-up call."""
+    c = CONFIGS["llm_d64"]
+    x = make_case(c)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    eta = x["eta"].to(dev)
+    g = torch.Generator(device=dev).manual_seed(11)
+    dO = torch.randn(v.shape, generator=g, device=dev).to(v.dtype)
+    out = ttt.backward_recurrent(q, k, v, dO, eta, eta_const=x["eta_const"])
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        out = ttt.backward_recurrent(q, k, v, dO, eta, eta_const=x["eta_const"])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del out
+    if ttt.device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait")
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    return {"workload": "llm_d64 backward (recurrent form, one block per head)", "us_per_call": us,
+            "tokens_per_s": c.B * c.T / (us * 1e-6), "gpu_launches_per_call": 1}
+
+
 def workload_config(c, args):
     return {"workload": c.name, "B": c.B, "H": c.H, "T": c.T, "d_k": c.d_k, "d_v": c.d_v,
             "chunk": args.chunk or c.chunk, "eta": "per-token" if c.eta_mode == "token" else "constant",
@@ -468,6 +496,9 @@ def run_ours(args, c, ws, rank, local, info):
     if not args.no_phi:
         torch.cuda.empty_cache()
         line["phi_layer"] = phi_measure(ttt, dev, peaks)
+    if not args.no_backward:
+        torch.cuda.empty_cache()
+        line["backward"] = backward_measure(ttt, dev)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(c, c.B * c.H if args.cpu_heads == 0 else args.cpu_heads)
     if rank == 0:
@@ -525,6 +556,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-phi", action="store_true", help="skip the feature-map layer measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--profile-run", action="store_true",
                     help="plain launches for a profiler: no graphs, timing, decode or CPU baseline")
     args = ap.parse_args()
