@@ -75,3 +75,29 @@ def test_zero_learning_rate_and_linearity():
                              S0=x["S0"])
         for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
             np.testing.assert_allclose(b[n], -2.5 * a[n], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("ascent", [False, True])
+def test_plain_gradient_is_three_forward_passes(ascent):
+    """Without momentum the backward is three runs of the forward layer:
+      dq_t = W_t^T do_t            forward on (q=dO, k=v, v=k), W_0 -> W_0^T
+      u_t  = G_t k_t               forward on the reversed sequence of (q=k, k=q, v=dO),
+                                   eta = 1, descent, starting from dL/dW_T
+      r_t  = G_t^T v_t             the same with (q=v, k=dO, v=q), starting from dL/dW_T^T
+    then dv = sigma eta u, dk = sigma eta r, deta = sigma v . u, and dW_0 is the
+    second run's final state.  An independent route to the same numbers."""
+    x = _rand(6, T=9, dk=4, dv=4)
+    s = -1.0 if ascent else 1.0
+    g = ttt_backward_f64(x["q"], x["k"], x["v"], x["eta"], x["dO"], x["dW"], ascent=ascent, S0=x["S0"])
+    tr = lambda m: np.swapaxes(m, -1, -2)  # noqa: E731
+    rev = lambda a: a[..., ::-1, :]  # noqa: E731
+    dq, _, _ = ttt_recurrence_f64(x["dO"], x["v"], x["k"], x["eta"], ascent=ascent, S0=tr(x["S0"]))
+    u_rev, G1, _ = ttt_recurrence_f64(rev(x["k"]), rev(x["q"]), rev(x["dO"]), 1.0, S0=x["dW"])
+    r_rev, _, _ = ttt_recurrence_f64(rev(x["v"]), rev(x["dO"]), rev(x["q"]), 1.0, S0=tr(x["dW"]))
+    u, r = rev(u_rev), rev(r_rev)
+    e = x["eta"][..., None]
+    np.testing.assert_allclose(g["dq"], dq, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dv"], s * e * u, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dk"], s * e * r, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["deta"], s * np.sum(x["v"] * u, axis=-1), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dW0"], G1, rtol=1e-12, atol=1e-12)
