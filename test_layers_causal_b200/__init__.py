@@ -18,4 +18,4 @@ from ._abi import (  # noqa: F401
     selftest_wait_timeout, set_wait_limit_ns, status_string, version, workspace_bytes,
 )
 from .host import forward_chunked_host  # noqa: F401
-from .seqshard import forward_sequence_sharded, token_slice  # noqa: F401
+from .seqshard import backward_sequence_sharded, forward_sequence_sharded, token_slice  # noqa: F401

@@ -100,7 +100,12 @@ def _oracle_backend():
                                             M0=f(mom_in))
         return torch.from_numpy(o), torch.from_numpy(W), torch.from_numpy(M)
 
-    return Backend(segment_map=seg_map, compose_maps=compose, forward=forward)
+    def backward(q, k, v, dO, eta, eta_const=None, ascent=False, state_in=None, grad_state=None):
+        e = f(eta) if eta is not None else eta_const
+        r = oracle.ttt_backward_f64(f(q), f(k), f(v), e, f(dO), f(grad_state), ascent=ascent, S0=f(state_in))
+        return {n: torch.from_numpy(np.ascontiguousarray(x)) for n, x in r.items()}
+
+    return Backend(segment_map=seg_map, compose_maps=compose, forward=forward, backward=backward)
 
 
 def _seqshard_worker(rank, world, port, outq):
@@ -137,6 +142,45 @@ def _seqshard_worker(rank, world, port, outq):
             if beta:
                 err = max(err, np.abs(M_p - M_ref).max())
         res[beta] = (err, covered.tolist())
+    if info.rank == 0:
+        outq.put(res)
+    ranks.finalize(info)
+
+
+def _seqshard_bwd_worker(rank, world, port, outq):
+    _env(rank, world, port)
+    import torch.distributed as dist
+
+    import oracle
+    from synth import make_qkv
+    from test_layers_causal_b200 import ranks, seqshard
+    info = ranks.init(backend="gloo", timeout_s=60)
+    B, H, T, d = 2, 2, 47, 5
+    q, k, v, z = make_qkv((B, H), T, d, d, seed=43)  # every rank draws the whole sequence
+    eta = torch.sigmoid(z) / d ** 0.5
+    g = torch.Generator().manual_seed(4)
+    S0, dW_T = 0.2 * torch.randn(B, H, d, d, generator=g), torch.randn(B, H, d, d, generator=g)
+    dO = torch.randn(B, H, T, d, generator=g)
+    sl = seqshard.token_slice(T, info.rank, info.world)
+    loc = lambda x: x[:, :, sl].contiguous()  # noqa: E731
+    res = {}
+    for ascent in (False, True):
+        dq, dk, dv, deta, dW0 = seqshard.backward_sequence_sharded(
+            loc(q), loc(k), loc(v), loc(dO), loc(eta), rank=info.rank, world=info.world, ascent=ascent,
+            state_in=S0.double(), grad_state=dW_T.double(), backend=_oracle_backend())
+        parts = [None] * info.world
+        dist.all_gather_object(parts, (sl.start, sl.stop, dq.numpy(), dk.numpy(), dv.numpy(), deta.numpy(),
+                                       dW0.numpy()))
+        f = lambda t: t.double().numpy()  # noqa: E731
+        ref = oracle.ttt_backward_f64(f(q), f(k), f(v), f(eta), f(dO), f(dW_T), ascent=ascent, S0=f(S0))
+        err = 0.0
+        covered = np.zeros(T, dtype=int)
+        for a, b, dq_p, dk_p, dv_p, de_p, dW0_p in parts:
+            covered[a:b] += 1
+            err = max(err, np.abs(dq_p - ref["dq"][:, :, a:b]).max(), np.abs(dk_p - ref["dk"][:, :, a:b]).max(),
+                      np.abs(dv_p - ref["dv"][:, :, a:b]).max(), np.abs(de_p - ref["deta"][:, :, a:b]).max(),
+                      np.abs(dW0_p - ref["dW0"]).max())
+        res[ascent] = (err, covered.tolist())
     if info.rank == 0:
         outq.put(res)
     ranks.finalize(info)
@@ -194,3 +238,15 @@ def test_sequence_split_over_ranks_matches_the_whole_sequence(world):
     for beta, (err, covered) in res.items():
         assert covered == [1] * 53, beta
         assert err < 1e-12, (beta, err)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_backward_sequence_split_over_ranks_matches_the_whole_sequence(world):
+    """The backward without momentum over two or three CPU ranks: each rank's
+    dq, dk, dv, deta for its run and the common dL/dW_0 equal the
+    whole-sequence gradient oracle (one all-gather of start maps, one of the
+    runs' do q^T sums)."""
+    (res,) = _run(_seqshard_bwd_worker, world=world)
+    for ascent, (err, covered) in res.items():
+        assert covered == [1] * 47, ascent
+        assert err < 1e-12, (ascent, err)
