@@ -115,25 +115,6 @@ ttt::SeqParams seq_params(const ttt_la_args* a) {
 
 ttt_la_status launched() { return cudaGetLastError() == cudaSuccess ? TTT_LA_OK : TTT_LA_ERR_CUDA; }
 
-// Dynamic shared memory a kernel may use beyond the 48 KB default.  The
-// attribute belongs to each device's context, so it is granted once per
-// device: `granted` is the launcher's own [kMaxDevices] record of the bytes
-// already granted on each device.
-constexpr int kMaxDevices = 64;
-std::mutex g_attr_mu;
-template <typename K>
-bool grant_smem(K* kernel, size_t* granted, size_t bytes) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  std::lock_guard<std::mutex> lock(g_attr_mu);
-  if (granted[dev] >= bytes) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
-      cudaSuccess)
-    return false;
-  granted[dev] = bytes;
-  return true;
-}
-
 // ------------------------------------------------------------ recurrent ----
 template <int DK, typename T, bool MOM>
 ttt_la_status launch_recurrent(const ttt_la_args* a, cudaStream_t st) {
@@ -218,8 +199,13 @@ size_t tc_ws_bytes(int bh, int nseg, int D) {
 template <int C, int D>
 ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
   using Cfg = ttt::TcCfg<C, D>;
-  static size_t granted[kMaxDevices] = {};
-  if (!grant_smem(ttt::chunked_tc_kernel<C, D>, granted, Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+        cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
   const int bh = a->B * a->H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
@@ -252,9 +238,14 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
 
 template <bool MOM>
 ttt_la_status launch_simt(const ttt_la_args* a, const ttt::SimtShape& sh, cudaStream_t st) {
-  static size_t granted[kMaxDevices] = {};
+  static size_t attr_bytes = 0;
   const size_t bytes = sh.bytes();
-  if (bytes > 48 * 1024 && !grant_smem(ttt::chunked_simt_f32_kernel<MOM>, granted, bytes)) return TTT_LA_ERR_CUDA;
+  if (bytes > 48 * 1024 && bytes > attr_bytes) {
+    if (cudaFuncSetAttribute(ttt::chunked_simt_f32_kernel<MOM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes)) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_bytes = bytes;
+  }
   ttt::chunked_simt_f32_kernel<MOM><<<a->B * a->H, 256, bytes, st>>>(seq_params(a), sh);
   return launched();
 }
@@ -278,8 +269,13 @@ template <int D>
 ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
   using Cfg = ttt::TcMomCfg<D>;
   constexpr int C = Cfg::C;
-  static size_t granted[kMaxDevices] = {};
-  if (!grant_smem(ttt::chunked_tc_mom_kernel<D>, granted, Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::chunked_tc_mom_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
   const int bh = a->B * a->H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
@@ -385,8 +381,13 @@ ttt_la_status check_feature(const ttt_la_feature_args* a) {
 template <int DIN, int DOUT>
 ttt_la_status launch_feature(const ttt_la_feature_args* a, cudaStream_t st) {
   using Cfg = ttt::FmapCfg<DIN, DOUT>;
-  static size_t granted[kMaxDevices] = {};
-  if (!grant_smem(ttt::feature_map_kernel<DIN, DOUT>, granted, Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::feature_map_kernel<DIN, DOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
   const int bh = a->B * a->H;
   CUtensorMap mx[2], my[2], m1, m3;
   for (int i = 0; i < 2; ++i) {
@@ -457,9 +458,13 @@ template <int DK, typename T, bool MOM>
 ttt_la_status launch_backward(const ttt_la_grad_args* a, cudaStream_t st) {
   using Sh = ttt::BwdShape<DK>;
   const size_t smem = ttt::bwd_smem_floats(DK, a->d_v, Sh::CK) * sizeof(float);
-  static size_t granted[kMaxDevices] = {};
-  if (smem > 48 * 1024 && !grant_smem(ttt::backward_recurrent_kernel<DK, T, MOM>, granted, smem))
-    return TTT_LA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(ttt::backward_recurrent_kernel<DK, T, MOM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             232448) != cudaSuccess)
+      return TTT_LA_ERR_CUDA;
+    attr_done = true;
+  }
   ttt::BwdParams p;
   p.BH = a->B * a->H;
   p.T = a->T;
@@ -509,6 +514,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[TTT_LA_STATIC_S
 // looked up with cudaGetSymbolAddress once per device (that device current)
 // and cached.  Returns nullptr when the lookup fails.
 void* noalloc_scratch_ptr() {
+  constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static void* ptrs[kMaxDevices] = {};
   int dev = -1;
