@@ -17,17 +17,19 @@ The arithmetic runs in the library; this module only moves tensors and
 orders the calls.  The `backend` argument exists so that the orchestration
 can be exercised on CPU ranks with a substitute for the library.
 
-The backward (without momentum) has one exchange too.  The gradient with
-respect to the state at the end of run r is
-    G_end_r = dL/dW_T + sum over later runs r' of B_r',   B_r' = sum_{t in r'} do_t q_t^T,
-and B_r is what the backward of run r returns as dL/dW_0 when no gradient
-enters its final state.  So each rank
+The backward has one exchange too.  A run's backward is affine in the
+gradients entering its end, and the linear part is the adjoint of the run's
+forward map: per head a multiple of the identity,
+    (G, H) -> (G, P H - G_run G)      (P = beta^L; without momentum only G),
+so each rank
   1. rebuilds its start state as in the forward (maps, all-gather, compose),
-  2. runs its backward from a zero final-state gradient to get B_r,
-  3. all-gathers the B's (d_v x d_k fp32 per head) and sums the later ones
-     onto dL/dW_T (ttt_la_compose_maps with plain maps),
-  4. runs its backward again from that end gradient for dq, dk, dv, deta.
-dL/dW_0 of the whole sequence is dL/dW_T plus all the B's.
+  2. runs its backward with no gradient entering its end; the dL/dW_0,
+     dL/dM_0 it returns are the run's constant term (B_W, B_M),
+  3. all-gathers them (d_v x d_k fp32 per head, one or two),
+  4. folds the later runs' adjoint maps onto (dL/dW_T, dL/dM_T) with
+     ttt_la_compose_maps (whose elementwise form w - G m + dW, B m + dM
+     expresses both steps with per-head scalars),
+  5. runs its backward again from that end gradient for dq, dk, dv, deta.
 """
 from __future__ import annotations
 
@@ -91,20 +93,58 @@ def forward_sequence_sharded(q, k, v, eta=None, *, rank=0, world=1, eta_const=No
     return o, W_T, (M_T if beta else None)
 
 
-def backward_sequence_sharded(q, k, v, dO, eta=None, *, rank=0, world=1, eta_const=None, ascent=False, chunk=64,
-                              state_in=None, grad_state=None, backend: Backend = LIBRARY):
-    """Backward of the layer without momentum for this rank's run of every
-    sequence (see token_slice).  q, k, v, dO, eta: this run's tokens;
-    state_in = W_0 and grad_state = dL/dW_T [B,H,d_v,d_k] (the same on every
-    rank) or None.  Returns (dq, dk, dv, deta) for this run and dL/dW_0 of the
-    whole sequence (identical on every rank)."""
-    dW, _, _ = backend.segment_map(q, k, v, eta, eta_const=eta_const, beta=0.0, ascent=ascent, chunk=chunk)
+def _stack_gb(G, P):
+    """[1, B, H, 2] map scalars (G, P) for ttt_la_compose_maps."""
+    return torch.stack([G, P], dim=-1).unsqueeze(0).contiguous()
+
+
+def backward_sequence_sharded(q, k, v, dO, eta=None, *, rank=0, world=1, eta_const=None, beta=0.0, ascent=False,
+                              chunk=64, state_in=None, mom_in=None, grad_state=None, grad_mom=None,
+                              backend: Backend = LIBRARY):
+    """Backward of the layer for this rank's run of every sequence (see
+    token_slice).  q, k, v, dO, eta: this run's tokens; state_in, mom_in =
+    W_0, M_0 and grad_state, grad_mom = dL/dW_T, dL/dM_T [B,H,d_v,d_k] (the
+    same on every rank) or None.  Returns (dq, dk, dv, deta) for this run and
+    (dL/dW_0, dL/dM_0) of the whole sequence (identical on every rank; dL/dM_0
+    is None without momentum).
+
+    The gradients entering run r's end: G_end_r = dL/dW_T + sum_{r' > r} B_W,r'
+    (W's gradient passes a run unchanged plus the run's own do q^T sums), and
+    with momentum H_end_r from the adjoint of each later run's map,
+        H <- P_r' H - G_r' G_end_r' + B_M,r'      (r' = last run down to r + 1),
+    where (G_r', P_r') are the run's map scalars (G and beta^L of
+    ttt_la_segment_map) and (B_W,r', B_M,r') the dL/dW_0, dL/dM_0 of run r''s
+    backward with no gradient entering its end."""
+    kw = dict(eta_const=eta_const, beta=beta, ascent=ascent)
+    dW, dM, GB = backend.segment_map(q, k, v, eta, chunk=chunk, **kw)
     dW_all = _all_gather(dW, world)
-    W0, _ = backend.compose_maps(dW_all[:rank], None, None, state_in, None)
-    kw = dict(eta_const=eta_const, ascent=ascent, state_in=W0)
-    own = backend.backward(q, k, v, dO, eta, **kw)["dW0"]  # B_r = sum over this run of do q^T
-    own_all = _all_gather(own, world)
-    G_end, _ = backend.compose_maps(own_all[rank + 1:], None, None, grad_state, None)
-    g = backend.backward(q, k, v, dO, eta, grad_state=G_end, **kw)
-    dW0, _ = backend.compose_maps(own_all, None, None, grad_state, None)
-    return g["dq"], g["dk"], g["dv"], g["deta"], dW0
+    dM_all = _all_gather(dM, world) if dM is not None else None
+    GB_all = _all_gather(GB, world) if GB is not None else None
+    W0, M0 = backend.compose_maps(dW_all[:rank], None if dM_all is None else dM_all[:rank],
+                                  None if GB_all is None else GB_all[:rank], state_in, mom_in)
+    bk = dict(kw, state_in=W0, mom_in=M0 if beta else None)
+    z = backend.backward(q, k, v, dO, eta, **bk)  # this run with no gradient entering its end
+    BW_all = _all_gather(z["dW0"], world)
+    BM_all = _all_gather(z["dM0"], world) if beta else None
+
+    def g_end(r):  # dL/dW at the end of run r
+        return backend.compose_maps(BW_all[r + 1:], None, None, grad_state, None)[0]
+
+    def h_fold(r_stop):  # dL/dM at the end of run r_stop (r_stop = -1: at the start of run 0)
+        H = grad_mom if grad_mom is not None else torch.zeros_like(BW_all[0])
+        for r2 in range(world - 1, r_stop, -1):
+            G2, P2 = GB_all[r2][..., 0], GB_all[r2][..., 1]
+            zero = torch.zeros_like(BW_all[0])
+            # C = B_M - G G_end, then H = P H + C (the W channel of the map is idle)
+            C, _ = backend.compose_maps(zero.unsqueeze(0), zero.unsqueeze(0), _stack_gb(G2, torch.ones_like(P2)),
+                                        BM_all[r2], g_end(r2))
+            _, H = backend.compose_maps(zero.unsqueeze(0), C.unsqueeze(0), _stack_gb(torch.zeros_like(G2), P2),
+                                        zero, H)
+        return H
+
+    G_end = g_end(rank)
+    H_end = h_fold(rank) if beta else None
+    g = backend.backward(q, k, v, dO, eta, grad_state=G_end, grad_mom=H_end, **bk)
+    dW0 = backend.compose_maps(BW_all, None, None, grad_state, None)[0]
+    dM0 = h_fold(-1) if beta else None
+    return g["dq"], g["dk"], g["dv"], g["deta"], dW0, dM0

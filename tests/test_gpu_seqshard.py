@@ -114,8 +114,29 @@ def test_backward_runs_compose_to_the_whole_sequence(world):
         assert_bf16(torch.cat([p[n] for p in parts], dim=2), ref[n], n)
     assert_bf16(dW0, ref["dW0"], "dW0")
     if world == 1:  # the module itself, no exchange
-        dq, dk, dv, deta, dW0m = seqshard.backward_sequence_sharded(q, k, v, dO, eta, eta_const=ec, state_in=S0,
-                                                                    grad_state=dW_T)
+        dq, dk, dv, deta, dW0m, dM0m = seqshard.backward_sequence_sharded(q, k, v, dO, eta, eta_const=ec,
+                                                                          state_in=S0, grad_state=dW_T)
+        assert dM0m is None
         torch.cuda.synchronize()
         assert_bf16(dq, ref["dq"], "module dq")
         assert_bf16(dW0m, ref["dW0"], "module dW0")
+
+
+def test_backward_module_with_momentum_world_one():
+    """backward_sequence_sharded with momentum on one rank: the adjoint fold
+    of its own run (ttt_la_compose_maps with per-head scalars) gives dL/dM_0,
+    and the run's gradients equal the whole-sequence oracle."""
+    B, H, T, d = 2, 2, 2 * 64 + 9, 64
+    q, k, v, eta = _inputs(B, H, T, d, "bf16", 230)
+    g = torch.Generator().manual_seed(23)
+    S0, M0 = ((0.1 * torch.randn(B, H, d, d, generator=g)).cuda() for _ in range(2))
+    dW_T, dM_T = (torch.randn(B, H, d, d, generator=g).cuda() for _ in range(2))
+    dO = torch.randn(B, H, T, d, generator=g).to(torch.bfloat16).cuda()
+    ec = 1.0 / math.sqrt(d)
+    dq, dk, dv, deta, dW0, dM0 = seqshard.backward_sequence_sharded(
+        q, k, v, dO, eta, eta_const=ec, beta=0.9, state_in=S0, mom_in=M0, grad_state=dW_T, grad_mom=dM_T)
+    torch.cuda.synchronize()
+    ref = oracle.ttt_backward_f64(f64(q), f64(k), f64(v), f64(eta), f64(dO), f64(dW_T), f64(dM_T), beta=0.9,
+                                  S0=f64(S0), M0=f64(M0))
+    for n, x in (("dq", dq), ("dk", dk), ("dv", dv), ("deta", deta), ("dW0", dW0), ("dM0", dM0)):
+        assert_bf16(x, ref[n], n)

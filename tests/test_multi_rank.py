@@ -100,9 +100,11 @@ def _oracle_backend():
                                             M0=f(mom_in))
         return torch.from_numpy(o), torch.from_numpy(W), torch.from_numpy(M)
 
-    def backward(q, k, v, dO, eta, eta_const=None, ascent=False, state_in=None, grad_state=None):
+    def backward(q, k, v, dO, eta, eta_const=None, beta=0.0, ascent=False, state_in=None, mom_in=None,
+                 grad_state=None, grad_mom=None):
         e = f(eta) if eta is not None else eta_const
-        r = oracle.ttt_backward_f64(f(q), f(k), f(v), e, f(dO), f(grad_state), ascent=ascent, S0=f(state_in))
+        r = oracle.ttt_backward_f64(f(q), f(k), f(v), e, f(dO), f(grad_state), f(grad_mom), beta=beta,
+                                    ascent=ascent, S0=f(state_in), M0=f(mom_in))
         return {n: torch.from_numpy(np.ascontiguousarray(x)) for n, x in r.items()}
 
     return Backend(segment_map=seg_map, compose_maps=compose, forward=forward, backward=backward)
@@ -159,28 +161,32 @@ def _seqshard_bwd_worker(rank, world, port, outq):
     q, k, v, z = make_qkv((B, H), T, d, d, seed=43)  # every rank draws the whole sequence
     eta = torch.sigmoid(z) / d ** 0.5
     g = torch.Generator().manual_seed(4)
-    S0, dW_T = 0.2 * torch.randn(B, H, d, d, generator=g), torch.randn(B, H, d, d, generator=g)
+    S0, M0, dW_T, dM_T = (0.2 * torch.randn(B, H, d, d, generator=g) for _ in range(4))
     dO = torch.randn(B, H, T, d, generator=g)
     sl = seqshard.token_slice(T, info.rank, info.world)
     loc = lambda x: x[:, :, sl].contiguous()  # noqa: E731
+    f = lambda t: t.double().numpy()  # noqa: E731
     res = {}
-    for ascent in (False, True):
-        dq, dk, dv, deta, dW0 = seqshard.backward_sequence_sharded(
-            loc(q), loc(k), loc(v), loc(dO), loc(eta), rank=info.rank, world=info.world, ascent=ascent,
-            state_in=S0.double(), grad_state=dW_T.double(), backend=_oracle_backend())
+    for beta, ascent in ((0.0, False), (0.0, True), (0.8, False), (0.6, True)):
+        mom = dict(mom_in=M0.double(), grad_mom=dM_T.double()) if beta else {}
+        dq, dk, dv, deta, dW0, dM0 = seqshard.backward_sequence_sharded(
+            loc(q), loc(k), loc(v), loc(dO), loc(eta), rank=info.rank, world=info.world, beta=beta, ascent=ascent,
+            state_in=S0.double(), grad_state=dW_T.double(), backend=_oracle_backend(), **mom)
         parts = [None] * info.world
         dist.all_gather_object(parts, (sl.start, sl.stop, dq.numpy(), dk.numpy(), dv.numpy(), deta.numpy(),
-                                       dW0.numpy()))
-        f = lambda t: t.double().numpy()  # noqa: E731
-        ref = oracle.ttt_backward_f64(f(q), f(k), f(v), f(eta), f(dO), f(dW_T), ascent=ascent, S0=f(S0))
+                                       dW0.numpy(), None if dM0 is None else dM0.numpy()))
+        ref = oracle.ttt_backward_f64(f(q), f(k), f(v), f(eta), f(dO), f(dW_T), f(dM_T) if beta else None,
+                                      beta=beta, ascent=ascent, S0=f(S0), M0=f(M0) if beta else None)
         err = 0.0
         covered = np.zeros(T, dtype=int)
-        for a, b, dq_p, dk_p, dv_p, de_p, dW0_p in parts:
+        for a, b, dq_p, dk_p, dv_p, de_p, dW0_p, dM0_p in parts:
             covered[a:b] += 1
             err = max(err, np.abs(dq_p - ref["dq"][:, :, a:b]).max(), np.abs(dk_p - ref["dk"][:, :, a:b]).max(),
                       np.abs(dv_p - ref["dv"][:, :, a:b]).max(), np.abs(de_p - ref["deta"][:, :, a:b]).max(),
                       np.abs(dW0_p - ref["dW0"]).max())
-        res[ascent] = (err, covered.tolist())
+            if beta:
+                err = max(err, np.abs(dM0_p - ref["dM0"]).max())
+        res[(beta, ascent)] = (err, covered.tolist())
     if info.rank == 0:
         outq.put(res)
     ranks.finalize(info)
@@ -242,11 +248,12 @@ def test_sequence_split_over_ranks_matches_the_whole_sequence(world):
 
 @pytest.mark.parametrize("world", [2, 3])
 def test_backward_sequence_split_over_ranks_matches_the_whole_sequence(world):
-    """The backward without momentum over two or three CPU ranks: each rank's
-    dq, dk, dv, deta for its run and the common dL/dW_0 equal the
-    whole-sequence gradient oracle (one all-gather of start maps, one of the
-    runs' do q^T sums)."""
+    """The backward over two or three CPU ranks, with and without momentum:
+    each rank's dq, dk, dv, deta for its run and the common dL/dW_0, dL/dM_0
+    equal the whole-sequence gradient oracle (one all-gather of the forward
+    maps, one of the runs' constant terms, the later runs' adjoint maps
+    folded onto the final-state gradients)."""
     (res,) = _run(_seqshard_bwd_worker, world=world)
-    for ascent, (err, covered) in res.items():
-        assert covered == [1] * 47, ascent
-        assert err < 1e-12, (ascent, err)
+    for key, (err, covered) in res.items():
+        assert covered == [1] * 47, key
+        assert err < 1e-11, (key, err)
