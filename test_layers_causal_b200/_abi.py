@@ -333,6 +333,10 @@ def backward_recurrent(q, k, v, grad_o, eta=None, eta_const=None, beta=0.0, asce
     _check_shapes(q, k, v, eta, state_in, mom_in)
     if grad_o.shape != v.shape or grad_o.dtype != v.dtype or not grad_o.is_contiguous():
         raise ValueError("grad_o must match v")
+    state_shape = (q.shape[0], q.shape[1], v.shape[-1], q.shape[-1])
+    for t in (grad_state, grad_mom):
+        if t is not None and (t.shape != state_shape or t.dtype != torch.float32):
+            raise ValueError("grad_state / grad_mom must be fp32 [B,H,d_v,d_k]")
     _need_cuda(q, k, v, grad_o, eta, state_in, mom_in, grad_state, grad_mom)
     B, H, T, dk = q.shape
     dv = v.shape[-1]
