@@ -270,8 +270,17 @@ def compose_maps(dW, dM=None, GB=None, W0=None, M0=None, stream=None):
     [n,B,H,d_v,d_k], GB [n,B,H,2] (dM, GB None: no momentum); W0, M0
     [B,H,d_v,d_k] or None (zeros).  Returns (W, M); M is None when neither
     dM nor M0 is given."""
+    if dW.dim() != 5:
+        raise ValueError("dW must be [n,B,H,d_v,d_k]")
     n = dW.shape[0]
     B, H, dv, dk = dW.shape[1:]
+    if (dM is None) != (GB is None):
+        raise ValueError("dM and GB come together (maps with momentum) or not at all")
+    for t, shape in ((dM, dW.shape), (GB, (n, B, H, 2)), (W0, (B, H, dv, dk)), (M0, (B, H, dv, dk))):
+        if t is not None and (tuple(t.shape) != tuple(shape) or t.dtype != torch.float32):
+            raise ValueError(f"compose_maps: expected fp32 {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+    if dW.dtype != torch.float32:
+        raise ValueError("dW must be fp32")
     _need_cuda(dW, dM, GB, W0, M0)
     W = torch.empty(B, H, dv, dk, device=dW.device, dtype=torch.float32)
     M = torch.empty_like(W) if (dM is not None or M0 is not None) else None
