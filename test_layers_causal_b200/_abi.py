@@ -179,9 +179,19 @@ def _check_shapes(q, k, v, eta, state_in, mom_in):
     _need_cuda(q, k, v, eta, state_in, mom_in)
 
 
+def _check_buf(t, shape, dtype, name):
+    """A caller-supplied buffer must have exactly the shape and dtype the
+    library will write: a smaller one would be written past its end."""
+    if t is not None and (tuple(t.shape) != tuple(shape) or t.dtype != dtype):
+        raise ValueError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
 def _alloc_outputs(q, v, beta, return_state, out, state_out=None, mom_out=None):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
+    _check_buf(out, v.shape, v.dtype, "out")
+    _check_buf(state_out, (B, H, dv, dk), torch.float32, "state_out")
+    _check_buf(mom_out, (B, H, dv, dk), torch.float32, "mom_out")
     o = torch.empty_like(v) if out is None else out
     S = M = None
     if return_state:
@@ -199,6 +209,7 @@ def forward_chunked(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, c
     `state_out`, `mom_out` and `workspace` may be preallocated buffers."""
     _check_shapes(q, k, v, eta, state_in, mom_in)
     o, S, M = _alloc_outputs(q, v, beta, return_state, out, state_out, mom_out)
+    _need_cuda(o, S, M, workspace)
     a = _seq_args(q, k, v, eta, eta_const, beta, ascent, chunk, segments, state_in, mom_in, o, S, M)
     L = lib()
     need = L.ttt_la_workspace_size(ctypes.byref(a))
@@ -224,6 +235,11 @@ def forward_chunked_host(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=Fal
     for t in (q, k, v, eta, state_in, mom_in, out, state_out, mom_out):
         if t is not None and (t.is_cuda or not t.is_contiguous()):
             raise ValueError("forward_chunked_host takes contiguous host tensors")
+    B, H, T, dk = q.shape
+    _check_buf(out, v.shape, v.dtype, "out")
+    for t, name in ((state_in, "state_in"), (mom_in, "mom_in"), (state_out, "state_out"), (mom_out, "mom_out")):
+        _check_buf(t, (B, H, v.shape[-1], dk), torch.float32, name)
+    _check_buf(eta, (B, H, T), torch.float32, "eta")
     o = torch.empty(v.shape, dtype=v.dtype, pin_memory=True) if out is None else out
     a = _seq_args(q, k, v, eta, eta_const, beta, ascent, chunk, segments, state_in, mom_in, o, state_out, mom_out)
     L = lib()
@@ -247,6 +263,8 @@ def segment_map(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, chunk
     _check_shapes(q, k, v, eta, None, None)
     B, H, T, dk = q.shape
     dv = v.shape[-1]
+    _check_buf(scratch, v.shape, v.dtype, "scratch")
+    _need_cuda(scratch, workspace)
     o = torch.empty_like(v) if scratch is None else scratch
     dW = torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32)
     dM = GB = None
@@ -308,7 +326,7 @@ def feature_map(xs, W1, W3, out=None, stream=None):
         raise TypeError("the feature map takes bf16 inputs and weights")
     if not all(t.is_contiguous() for t in (*xs, W1, W3)):
         raise ValueError("inputs and weights must be contiguous")
-    _need_cuda(*xs, W1, W3)
+    _need_cuda(*xs, W1, W3, *(out or []))
     d_out = W1.shape[1]
     ys = list(out) if out is not None else [torch.empty(B, H, T, d_out, device=x0.device, dtype=torch.bfloat16)
                                             for _ in xs]
@@ -386,6 +404,7 @@ def forward_recurrent(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False,
     """Token-by-token forward (ttt_la_forward_recurrent).  Returns (o, W_T, M_T)."""
     _check_shapes(q, k, v, eta, state_in, mom_in)
     o, S, M = _alloc_outputs(q, v, beta, return_state, out)
+    _need_cuda(o)
     a = _seq_args(q, k, v, eta, eta_const, beta, ascent, 0, 0, state_in, mom_in, o, S, M)
     _check("ttt_la_forward_recurrent", lib().ttt_la_forward_recurrent(ctypes.byref(a), _stream_handle(stream)))
     return o, S, M
@@ -404,7 +423,11 @@ def decode_step(q, k, v, state, mom=None, eta=None, eta_const=None, beta=0.0, as
         raise ValueError("state must be fp32 [N,H,d_v,d_k]")
     if eta is not None and (eta.shape != (N, H) or eta.dtype != torch.float32):
         raise ValueError("eta must be fp32 [N,H]")
-    _need_cuda(q, k, v, state, mom, eta)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share a dtype")
+    _check_buf(mom, (N, H, dv, dk), torch.float32, "mom")
+    _check_buf(out, v.shape, v.dtype, "out")
+    _need_cuda(q, k, v, state, mom, eta, out)
     o = torch.empty_like(v) if out is None else out
     a = TttDecodeArgs()
     a.N, a.H, a.d_k, a.d_v, a.dtype = N, H, dk, dv, _dtype_code(q)

@@ -281,3 +281,23 @@ def test_host_staging_size_and_checks(abi):
     unsupported = _args(abi, d_k=96, d_v=96)
     assert L.ttt_la_forward_chunked_host(ctypes.byref(unsupported), ctypes.c_void_p(0x100000), 1 << 30, None) == \
         abi.ERR_UNSUPPORTED
+
+
+def test_binding_rejects_wrongly_shaped_buffers(abi):
+    """Caller buffers the library would write past the end of are refused in
+    the binding (checked here where no GPU is needed: host-buffer forward and
+    decode step argument checks run before any CUDA requirement)."""
+    import torch
+    q = torch.zeros(1, 2, 8, 32)
+    for kw in (dict(out=torch.zeros(1, 2, 8, 16)), dict(state_out=torch.zeros(1, 2, 32, 16)),
+               dict(mom_out=torch.zeros(1, 2, 32, 32, dtype=torch.float64)), dict(eta=torch.zeros(1, 2, 7))):
+        with pytest.raises(ValueError):
+            abi.forward_chunked_host(q, q, q, **kw)
+    x = torch.zeros(1, 2, 32)
+    S = torch.zeros(1, 2, 32, 32)
+    with pytest.raises(ValueError):
+        abi.decode_step(x, x, x, S, mom=torch.zeros(1, 2, 32, 16))
+    with pytest.raises(ValueError):
+        abi.decode_step(x, x, x, S, out=torch.zeros(1, 2, 16))
+    with pytest.raises(TypeError):
+        abi.decode_step(x, x.bfloat16(), x, S)
