@@ -172,41 +172,52 @@ def max_over_ranks(x, info):
 
 
 # --------------------------------------------------------------- oracle ----
-def oracle_sample(c, heads, rank_seed=0):
-    """Runs the float64 oracle on `heads` (b, h) sequences of the workload at
-    full length; returns (seconds, head-tokens)."""
-    import numpy as np
-
+def oracle_sample(c, heads, x=None):
+    """Runs the float64 oracle on the first `heads` (b, h) sequences of the
+    workload's inputs `x` (make_case(c) when None) at full length; returns
+    (seconds, head-tokens, o [heads, T, d_v])."""
     import oracle
-    x = make_case(c, B=1, H=heads)
-    f = lambda t: t.float().double().numpy()  # noqa: E731
+    x = make_case(c) if x is None else x
+    f = lambda t: t.float().double().reshape(-1, *t.shape[2:])[:heads].numpy()  # noqa: E731
     eta = f(x["eta"]) if x["eta"] is not None else x["eta_const"]
     t0 = time.perf_counter()
-    oracle.ttt_recurrence_f64(f(x["q"]), f(x["k"]), f(x["v"]), eta, beta=c.beta)
+    o, _, _ = oracle.ttt_recurrence_f64(f(x["q"]), f(x["k"]), f(x["v"]), eta, beta=c.beta)
     dt = time.perf_counter() - t0
-    del np
-    return dt, heads * c.T
+    return dt, heads * c.T, o
 
 
-def cpu_baseline(c, heads):
-    dt, head_tokens = oracle_sample(c, heads)
+def parity(o_gpu, o_ref, tol=2e-2):
+    """Worst relative Frobenius error over the sampled (b, h) sequences of the
+    GPU output against the oracle's."""
+    import numpy as np
+    g = o_gpu.float().double().reshape(-1, *o_gpu.shape[2:])[:o_ref.shape[0]].numpy()
+    err = np.linalg.norm(g - o_ref, axis=(1, 2)) / np.maximum(np.linalg.norm(o_ref, axis=(1, 2)), 1e-30)
+    worst = float(err.max())
+    return {"sequences": int(o_ref.shape[0]), "rel_frobenius_max": worst, "tolerance": tol, "pass": worst <= tol}
+
+
+def cpu_baseline(c, heads, x=None):
+    """The oracle timed on `heads` sequences of the workload's inputs; also
+    returns its outputs, for the parity check of the GPU result."""
+    dt, head_tokens, o_ref = oracle_sample(c, heads, x)
     total_head_tokens = c.B * c.H * c.T
     t_full = dt * total_head_tokens / head_tokens
     return {"value": c.B * c.T / t_full, "unit": "tokens/s", "cores": 1,
             "kind": "oracle",
-            "sample": f"{heads} of {c.B * c.H} (b,h) sequences at full length T={c.T} "
-                      f"({dt:.1f} s of single-threaded float64 numpy), scaled to the whole layer"}
+            "sample": f"{heads} of {c.B * c.H} (b,h) sequences of the benchmark's own inputs at full length "
+                      f"T={c.T} ({dt:.1f} s of single-threaded float64 numpy), scaled to the whole layer"}, o_ref
 
 
 def run_reference(args, c, ws, rank, info):
     if rank != 0:
         return
     heads = max(1, min(c.B * c.H, args.ref_heads))
+    x = make_case(c)
     for _ in range(args.warmup):
-        oracle_sample(c, heads)
+        oracle_sample(c, heads, x)
     times = []
     for _ in range(args.steps):
-        dt, _ = oracle_sample(c, heads)
+        dt, _, _ = oracle_sample(c, heads, x)
         times.append(dt * (c.B * c.H) / heads)
     t = sum(times) / len(times)
     val = c.B * c.T / t
@@ -216,8 +227,8 @@ def run_reference(args, c, ws, rank, info):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(c, args),
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: {heads} of {c.B * c.H} (b,h) sequences at full length, "
-                                   "scaled to the whole layer"},
+                         "sample": f"each step: the first {heads} of {c.B * c.H} (b,h) sequences of the "
+                                   "workload at full length, scaled to the whole layer"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -500,7 +511,9 @@ def run_ours(args, c, ws, rank, local, info):
         torch.cuda.empty_cache()
         line["backward"] = backward_measure(ttt, dev)
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(c, c.B * c.H if args.cpu_heads == 0 else args.cpu_heads)
+        line["cpu_baseline"], o_ref = cpu_baseline(c, c.B * c.H if args.cpu_heads == 0 else args.cpu_heads, x)
+        # the end-to-end run's output (public host-buffer API) against the oracle on the same inputs
+        line["parity"] = parity(oh, o_ref)
     if rank == 0:
         print(json.dumps(line), flush=True)
 

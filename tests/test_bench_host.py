@@ -53,3 +53,17 @@ def test_traffic_figure_needs_matching_sources(tmp_path, monkeypatch):
 @pytest.mark.parametrize("name", sorted(bench.CHUNKED_SOURCES))
 def test_hashed_sources_exist(name):
     assert os.path.exists(os.path.join(ROOT, "test_layers_causal_b200", "csrc", name))
+
+
+def test_parity_helper_against_the_oracle_samples():
+    """The bench's parity figure: fp32 rounding for the oracle's own output,
+    the relative error of a known perturbation otherwise."""
+    import torch
+    c = CONFIGS["tiny_f32"]
+    x = bench.make_case(c)
+    _, _, o_ref = bench.oracle_sample(c, 2, x)
+    o = torch.from_numpy(o_ref).reshape(c.B, c.H, c.T, c.d_v)
+    p = bench.parity(o, o_ref)
+    assert p["sequences"] == 2 and p["rel_frobenius_max"] < 1e-7 and p["pass"]  # fp32 rounding only
+    p = bench.parity(1.03 * o, o_ref)
+    assert abs(p["rel_frobenius_max"] - 0.03) < 1e-6 and not p["pass"]
