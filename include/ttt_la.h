@@ -301,6 +301,25 @@ typedef struct ttt_la_grad_args {
 TTT_LA_API size_t ttt_la_backward_workspace_size(const ttt_la_grad_args *args);
 TTT_LA_API ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args *args, void *stream);
 
+/* Chunk-parallel backward of the layer without momentum (beta == 0): the
+ * same gradients as ttt_la_backward_recurrent, from three runs of the chunked
+ * forward on the tensor cores.  With G_t = dL/dW_T + sum_{t' >= t} do_t' q_t'^T:
+ *   dq_t = W_t^T do_t   the forward on (q, k, v) := (do, v, k) from W_0^T;
+ *   G_t k_t, G_t^T v_t  the forward on the time-reversed sequences of
+ *                       (k, q, do) and (v, do, q), learning rate 1, from
+ *                       dL/dW_T and its transpose (the first run's final
+ *                       state is dL/dW_0);
+ *   dv_t = sigma eta_t G_t k_t, dk_t = sigma eta_t G_t^T v_t,
+ *   deta_t = sigma v_t . G_t k_t.
+ * bf16: d_k == d_v in {64, 128}; fp32: d_k, d_v multiples of 4 up to 128.
+ * beta != 0, mom_in or grad_mom: TTT_LA_ERR_UNSUPPORTED; grad_mom_in, if
+ * given, is zeroed.  The workspace (ttt_la_backward_chunked_workspace_size
+ * bytes) holds reversed copies of q, k, v and grad_o, the passes' outputs,
+ * the transposed states and one forward workspace.  Errors as
+ * ttt_la_backward_recurrent. */
+TTT_LA_API size_t ttt_la_backward_chunked_workspace_size(const ttt_la_grad_args *args);
+TTT_LA_API ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args *args, void *stream);
+
 /* Synchronises `stream`, returns the device status word (TTT_LA_OK or
  * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
 TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);

@@ -80,6 +80,8 @@ SIGNATURES = [
     ("ttt_la_feature_map", ctypes.c_int, [ctypes.POINTER(TttFeatureArgs), _c_vp]),
     ("ttt_la_backward_workspace_size", _c_sz, [ctypes.POINTER(TttGradArgs)]),
     ("ttt_la_backward_recurrent", ctypes.c_int, [ctypes.POINTER(TttGradArgs), _c_vp]),
+    ("ttt_la_backward_chunked_workspace_size", _c_sz, [ctypes.POINTER(TttGradArgs)]),
+    ("ttt_la_backward_chunked", ctypes.c_int, [ctypes.POINTER(TttGradArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
     ("ttt_la_set_wait_limit_ns", ctypes.c_int, [ctypes.c_int64]),
     ("ttt_la_selftest_wait_timeout", ctypes.c_int, [ctypes.c_int64, _c_vp]),
@@ -386,6 +388,39 @@ def backward_recurrent(q, k, v, grad_o, eta=None, eta_const=None, beta=0.0, asce
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("ttt_la_backward_recurrent", L.ttt_la_backward_recurrent(ctypes.byref(a), _stream_handle(stream)))
+    return out
+
+
+def backward_chunked(q, k, v, grad_o, eta=None, eta_const=None, ascent=False, state_in=None, grad_state=None,
+                     workspace=None, stream=None):
+    """Gradients of the layer without momentum from three chunked forward runs
+    (ttt_la_backward_chunked): returns a dict with dq, dk, dv (dtype of q),
+    deta [B,H,T] fp32 (per token) and dW0 [B,H,d_v,d_k] fp32."""
+    _check_shapes(q, k, v, eta, state_in, None)
+    if grad_o.shape != v.shape or grad_o.dtype != v.dtype:
+        raise ValueError("grad_o must match v")
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if grad_state is not None and (grad_state.shape != (B, H, dv, dk) or grad_state.dtype != torch.float32):
+        raise ValueError("grad_state must be fp32 [B,H,d_v,d_k]")
+    _need_cuda(q, k, v, grad_o, eta, state_in, grad_state, workspace)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               deta=torch.empty(B, H, T, device=q.device, dtype=torch.float32),
+               dW0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32))
+    a = TttGradArgs()
+    a.B, a.H, a.T, a.d_k, a.d_v, a.dtype = B, H, T, dk, dv, _dtype_code(q)
+    a.q, a.k, a.v, a.eta = q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(eta)
+    a.eta_const = (1.0 / math.sqrt(dk)) if eta_const is None else float(eta_const)
+    a.beta, a.ascent = 0.0, int(bool(ascent))
+    a.state_in, a.grad_o, a.grad_state = _ptr(state_in), grad_o.data_ptr(), _ptr(grad_state)
+    a.grad_q, a.grad_k, a.grad_v = out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr()
+    a.grad_eta, a.grad_state_in = out["deta"].data_ptr(), out["dW0"].data_ptr()
+    L = lib()
+    need = L.ttt_la_backward_chunked_workspace_size(ctypes.byref(a))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check("ttt_la_backward_chunked", L.ttt_la_backward_chunked(ctypes.byref(a), _stream_handle(stream)))
     return out
 
 

@@ -14,6 +14,7 @@
 
 #include "../../include/ttt_la.h"
 #include "backward.cuh"
+#include "backward_chunked.cuh"
 #include "chunked_simt.cuh"
 #include "chunked_tc.cuh"
 #include "chunked_tc_mom.cuh"
@@ -419,7 +420,8 @@ size_t bwd_ws_bytes(const ttt_la_grad_args* a) {
   return static_cast<size_t>(a->B) * a->H * per * sizeof(float);
 }
 
-ttt_la_status check_grad(const ttt_la_grad_args* a) {
+// Checks shared by both backward forms: sizes, pointers, alignment, overlaps.
+ttt_la_status check_grad_common(const ttt_la_grad_args* a) {
   if (!a) return TTT_LA_ERR_INVALID_ARG;
   if (a->B < 1 || a->H < 1 || a->T < 1 || a->d_k < 1 || a->d_v < 1) return TTT_LA_ERR_INVALID_ARG;
   if (a->dtype != TTT_LA_F32 && a->dtype != TTT_LA_BF16) return TTT_LA_ERR_INVALID_ARG;
@@ -448,6 +450,12 @@ ttt_la_status check_grad(const ttt_la_grad_args* a) {
     for (int j = 0; j < i; ++j)
       if (outs[j] && overlaps(outs[i], osz[i], outs[j], osz[j])) return TTT_LA_ERR_INVALID_ARG;
   }
+  return TTT_LA_OK;
+}
+
+ttt_la_status check_grad(const ttt_la_grad_args* a) {
+  const ttt_la_status s = check_grad_common(a);
+  if (s != TTT_LA_OK) return s;
   if (a->d_k != 32 && a->d_k != 64 && a->d_k != 128) return TTT_LA_ERR_UNSUPPORTED;
   if (a->d_v > bwd_max_dv(a->d_k)) return TTT_LA_ERR_UNSUPPORTED;
   if (!a->workspace || a->workspace_bytes < bwd_ws_bytes(a)) return TTT_LA_ERR_INVALID_ARG;
@@ -798,3 +806,195 @@ ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// Chunk-parallel backward without momentum: three runs of the chunked forward
+// (see backward_chunked.cuh) over scratch carved from the caller's workspace.
+namespace {
+struct BwdChunkedLayout {
+  size_t rev[4], u, r, w0t, dwt, fwd, total, fwd_bytes;
+};
+
+int bwdc_chunk(const ttt_la_grad_args* a) { return (a->dtype == TTT_LA_BF16 && a->d_k == 128) ? 128 : 64; }
+
+// Arguments of forward pass p: 0 gives dq, 1 gives u = G k (reversed order)
+// and dL/dW_0, 2 gives r = G^T v (reversed order).  rev[] are q, k, v, dO
+// reversed along T.
+ttt_la_args bwdc_pass(const ttt_la_grad_args* a, int p, void* const* rev, void* u, void* r, const float* w0t,
+                      const float* dwt) {
+  ttt_la_args f;
+  std::memset(&f, 0, sizeof f);
+  f.B = a->B;
+  f.H = a->H;
+  f.T = a->T;
+  f.dtype = a->dtype;
+  f.chunk = bwdc_chunk(a);
+  f.beta = 0.f;
+  if (p == 0) {  // W_t^T do_t: keys v, values k, from W_0^T, the layer's eta and sigma
+    f.d_k = a->d_v;
+    f.d_v = a->d_k;
+    f.q = a->grad_o;
+    f.k = a->v;
+    f.v = a->k;
+    f.eta = a->eta;
+    f.eta_const = a->eta_const;
+    f.ascent = a->ascent;
+    f.state_in = w0t;
+    f.o = a->grad_q;
+  } else if (p == 1) {  // G_t k_t: reversed (q, k, v) := (k, q, dO), eta = 1, from dL/dW_T
+    f.d_k = a->d_k;
+    f.d_v = a->d_v;
+    f.q = rev[1];
+    f.k = rev[0];
+    f.v = rev[3];
+    f.eta_const = 1.f;
+    f.state_in = a->grad_state;
+    f.state_out = a->grad_state_in;
+    f.o = u;
+  } else {  // G_t^T v_t: reversed (q, k, v) := (v, dO, q), eta = 1, from (dL/dW_T)^T
+    f.d_k = a->d_v;
+    f.d_v = a->d_k;
+    f.q = rev[2];
+    f.k = rev[3];
+    f.v = rev[0];
+    f.eta_const = 1.f;
+    f.state_in = dwt;
+    f.o = r;
+  }
+  return f;
+}
+
+BwdChunkedLayout bwdc_layout(const ttt_la_grad_args* a) {
+  BwdChunkedLayout L;
+  const size_t el = a->dtype == TTT_LA_F32 ? 4 : 2, bh = static_cast<size_t>(a->B) * a->H;
+  const size_t nk = align256(bh * a->T * a->d_k * el), nv = align256(bh * a->T * a->d_v * el);
+  const size_t ns = align256(bh * a->d_k * a->d_v * 4);
+  size_t off = 0;
+  const size_t sizes[4] = {nk, nk, nv, nv};
+  for (int i = 0; i < 4; ++i) {
+    L.rev[i] = off;
+    off += sizes[i];
+  }
+  L.u = off;
+  off += nv;
+  L.r = off;
+  off += nk;
+  L.w0t = off;
+  off += a->state_in ? ns : 0;
+  L.dwt = off;
+  off += a->grad_state ? ns : 0;
+  L.fwd = off;
+  L.fwd_bytes = 0;
+  void* none[4] = {nullptr, nullptr, nullptr, nullptr};
+  for (int p = 0; p < 3; ++p) {
+    ttt_la_args f = bwdc_pass(a, p, none, nullptr, nullptr, nullptr, nullptr);
+    L.fwd_bytes = std::max(L.fwd_bytes, ttt_la_workspace_size(&f));
+  }
+  L.total = off + align256(L.fwd_bytes);
+  return L;
+}
+
+ttt_la_status check_grad_chunked(const ttt_la_grad_args* a) {
+  const ttt_la_status s = check_grad_common(a);
+  if (s != TTT_LA_OK) return s;
+  if (a->beta != 0.f || a->mom_in || a->grad_mom) return TTT_LA_ERR_UNSUPPORTED;
+  if (a->dtype == TTT_LA_BF16 && !(a->d_k == a->d_v && (a->d_k == 64 || a->d_k == 128)))
+    return TTT_LA_ERR_UNSUPPORTED;
+  if (a->dtype == TTT_LA_F32 && (a->d_k % 4 || a->d_v % 4 || a->d_k > 128 || a->d_v > 128))
+    return TTT_LA_ERR_UNSUPPORTED;
+  if (!a->workspace || a->workspace_bytes < bwdc_layout(a).total) return TTT_LA_ERR_INVALID_ARG;
+  return TTT_LA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t ttt_la_backward_chunked_workspace_size(const ttt_la_grad_args* a) {
+  if (!a || a->B < 1 || a->H < 1 || a->T < 1 || a->d_k < 1 || a->d_v < 1) return 0;
+  return bwdc_layout(a).total;
+}
+
+ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
+  ttt_la_status s = check_grad_chunked(a);
+  if (s != TTT_LA_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const BwdChunkedLayout L = bwdc_layout(a);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  void* rev[4] = {ws + L.rev[0], ws + L.rev[1], ws + L.rev[2], ws + L.rev[3]};
+  float* w0t = a->state_in ? reinterpret_cast<float*>(ws + L.w0t) : nullptr;
+  float* dwt = a->grad_state ? reinterpret_cast<float*>(ws + L.dwt) : nullptr;
+  const int BH = a->B * a->H, el = a->dtype == TTT_LA_F32 ? 4 : 2;
+  const int grid = sm_count() * 4;
+
+  // q, k (rows of d_k) and v, dO (rows of d_v) reversed along T
+  for (int g = 0; g < 2; ++g) {
+    ttt::ReverseParams rp;
+    std::memset(&rp, 0, sizeof rp);
+    rp.n = 2;
+    rp.BH = BH;
+    rp.T = a->T;
+    rp.units = ((g == 0 ? a->d_k : a->d_v) * el) / 16;
+    rp.src[0] = static_cast<const uint4*>(g == 0 ? a->q : a->v);
+    rp.src[1] = static_cast<const uint4*>(g == 0 ? a->k : a->grad_o);
+    rp.dst[0] = static_cast<uint4*>(rev[2 * g]);
+    rp.dst[1] = static_cast<uint4*>(rev[2 * g + 1]);
+    ttt::reverse_tokens_kernel<<<grid, 256, 0, st>>>(rp);
+    if ((s = launched()) != TTT_LA_OK) return s;
+  }
+  // W_0^T and (dL/dW_T)^T
+  ttt::TransposeParams tp;
+  std::memset(&tp, 0, sizeof tp);
+  tp.BH = BH;
+  tp.R = a->d_v;
+  tp.C = a->d_k;
+  if (a->state_in) {
+    tp.src[tp.n] = a->state_in;
+    tp.dst[tp.n++] = w0t;
+  }
+  if (a->grad_state) {
+    tp.src[tp.n] = a->grad_state;
+    tp.dst[tp.n++] = dwt;
+  }
+  if (tp.n > 0) {
+    ttt::transpose_states_kernel<<<grid, 256, 0, st>>>(tp);
+    if ((s = launched()) != TTT_LA_OK) return s;
+  }
+  // the three forward passes
+  void* u = ws + L.u;
+  void* r = ws + L.r;
+  for (int p = 0; p < 3; ++p) {
+    ttt_la_args f = bwdc_pass(a, p, rev, u, r, w0t, dwt);
+    f.workspace = L.fwd_bytes ? ws + L.fwd : nullptr;
+    f.workspace_bytes = L.fwd_bytes;
+    if ((s = ttt_la_forward_chunked(&f, stream)) != TTT_LA_OK) return s;
+  }
+  // dv, dk, deta
+  ttt::FinishParams fp;
+  fp.BH = BH;
+  fp.T = a->T;
+  fp.dk = a->d_k;
+  fp.dv = a->d_v;
+  fp.u_rev = u;
+  fp.r_rev = r;
+  fp.v = a->v;
+  fp.eta = a->eta;
+  fp.eta_const = a->eta_const;
+  fp.sigma = a->ascent ? -1.f : 1.f;
+  fp.dk_out = a->grad_k;
+  fp.dv_out = a->grad_v;
+  fp.deta = a->grad_eta;
+  const long long warps = static_cast<long long>(BH) * a->T;
+  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+  if (a->dtype == TTT_LA_F32)
+    ttt::backward_finish_kernel<float><<<blocks, 256, 0, st>>>(fp);
+  else
+    ttt::backward_finish_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(fp);
+  if ((s = launched()) != TTT_LA_OK) return s;
+  if (a->grad_mom_in &&
+      cudaMemsetAsync(a->grad_mom_in, 0, static_cast<size_t>(BH) * a->d_v * a->d_k * sizeof(float), st) !=
+          cudaSuccess)
+    return TTT_LA_ERR_CUDA;
+  return TTT_LA_OK;
+}
+
+}  // extern "C"
+

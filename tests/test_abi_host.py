@@ -301,3 +301,28 @@ def test_binding_rejects_wrongly_shaped_buffers(abi):
         abi.decode_step(x, x, x, S, out=torch.zeros(1, 2, 16))
     with pytest.raises(TypeError):
         abi.decode_step(x, x.bfloat16(), x, S)
+
+
+def test_backward_chunked_workspace_and_validation(abi):
+    L = abi.lib()
+    call = lambda g: L.ttt_la_backward_chunked(ctypes.byref(g), None)  # noqa: E731
+    size = lambda g: L.ttt_la_backward_chunked_workspace_size(ctypes.byref(g))  # noqa: E731
+    g = _grad_args(abi, T=100)
+    seq = 2 * 2 * 100 * 64 * 2  # one reversed bf16 tensor
+    assert size(g) >= 6 * seq  # four reversed inputs and the two passes' outputs
+    g.state_in, g.grad_state = 0x8000000, 0x9000000
+    assert size(g) >= 6 * seq + 2 * 2 * 2 * 64 * 64 * 4  # plus the two transposed states
+    assert L.ttt_la_backward_chunked_workspace_size(None) == 0
+    assert L.ttt_la_backward_chunked(None, None) == abi.ERR_INVALID_ARG
+    # momentum is the recurrent form's
+    for field, val in [("beta", 0.9), ("mom_in", 0xA000000), ("grad_mom", 0xB000000)]:
+        g = _grad_args(abi)
+        setattr(g, field, val)
+        g.workspace_bytes = 1 << 40
+        assert call(g) == abi.ERR_UNSUPPORTED, field
+    g = _grad_args(abi, dk=64, dv=128)  # the bf16 tensor-core forward wants d_k == d_v
+    g.workspace_bytes = 1 << 40
+    assert call(g) == abi.ERR_UNSUPPORTED
+    g = _grad_args(abi)
+    g.workspace_bytes = size(g) - 256
+    assert call(g) == abi.ERR_INVALID_ARG

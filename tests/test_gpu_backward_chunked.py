@@ -1,0 +1,82 @@
+"""GPU parity of the chunk-parallel backward without momentum
+(ttt_la_backward_chunked: three runs of the chunked forward) against the
+float64 gradient oracle and against the recurrent backward.
+
+Skipped until these have run on a B200.  Its orchestration (which pass reads
+which tensors, the reversals, transposes and the final scaling) was checked
+on CPU with the forward oracle in place of the chunked kernel.
+
+Tolerances: bf16 inputs, relative Frobenius error <= 2e-2 per (b, h) slice
+and overall; fp32 inputs (the fp32 chunked forward), max-rel <= 1e-4.
+"""
+import math
+
+import pytest
+import torch
+
+import oracle
+from synth import make_qkv
+from tests.gpu_util import assert_bf16, assert_f32, f64
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="not yet run on a B200")]
+
+if torch.cuda.is_available():
+    from test_layers_causal_b200 import _abi
+
+
+@pytest.fixture(autouse=True)
+def _no_timed_out_wait():
+    yield
+    assert _abi.device_status() == _abi.OK
+
+
+def _case(B, H, T, dk, dv, dtype, seed, token_eta=True, states=True):
+    q, k, v, z = make_qkv((B, H), T, dk, dv, seed)
+    g = torch.Generator().manual_seed(seed + 2000)
+    dO = torch.randn(B, H, T, dv, generator=g)
+    S0 = 0.3 * torch.randn(B, H, dv, dk, generator=g) if states else None
+    dW = torch.randn(B, H, dv, dk, generator=g) if states else None
+    eta = (torch.sigmoid(z) / math.sqrt(dk)).float() if token_eta else None
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    dev = lambda x: None if x is None else x.contiguous().cuda()  # noqa: E731
+    return dict(q=dev(q.to(dt)), k=dev(k.to(dt)), v=dev(v.to(dt)), dO=dev(dO.to(dt)), eta=dev(eta), S0=dev(S0),
+                dW=dev(dW), ec=1.0 / math.sqrt(dk))
+
+
+def _ref(x, ascent):
+    e = f64(x["eta"]) if x["eta"] is not None else x["ec"]
+    return oracle.ttt_backward_f64(f64(x["q"]), f64(x["k"]), f64(x["v"]), e, f64(x["dO"]), f64(x["dW"]),
+                                   ascent=ascent, S0=f64(x["S0"]))
+
+
+@pytest.mark.parametrize("d,T,token_eta,ascent,states", [(64, 300, True, False, True), (128, 257, False, True, True),
+                                                         (64, 64, True, False, False), (128, 1, True, False, True)])
+def test_backward_chunked_bf16_matches_oracle(d, T, token_eta, ascent, states):
+    x = _case(2, 3, T, d, d, "bf16", 90 + d + T, token_eta, states)
+    g = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], eta_const=x["ec"], ascent=ascent,
+                              state_in=x["S0"], grad_state=x["dW"])
+    torch.cuda.synchronize()
+    ref = _ref(x, ascent)
+    for n in ("dq", "dk", "dv", "deta", "dW0"):
+        assert_bf16(g[n], ref[n], n)
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 48)])
+def test_backward_chunked_f32_matches_oracle(dk, dv):
+    x = _case(2, 2, 150, dk, dv, "f32", 120 + dk + dv)
+    g = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], eta_const=x["ec"], state_in=x["S0"],
+                              grad_state=x["dW"])
+    torch.cuda.synchronize()
+    ref = _ref(x, False)
+    for n in ("dq", "dk", "dv", "deta", "dW0"):
+        assert_f32(g[n], ref[n], n)
+
+
+def test_backward_chunked_agrees_with_recurrent_at_llm_shape():
+    """B4 H16 T4096 d64, per-token eta: the two backward forms agree."""
+    x = _case(4, 16, 4096, 64, 64, "bf16", 140)
+    a = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], state_in=x["S0"], grad_state=x["dW"])
+    b = _abi.backward_recurrent(x["q"], x["k"], x["v"], x["dO"], x["eta"], state_in=x["S0"], grad_state=x["dW"])
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dW0"):
+        assert_bf16(a[n], f64(b[n]), n)
