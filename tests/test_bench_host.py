@@ -67,3 +67,12 @@ def test_parity_helper_against_the_oracle_samples():
     assert p["sequences"] == 2 and p["rel_frobenius_max"] < 1e-7 and p["pass"]  # fp32 rounding only
     p = bench.parity(1.03 * o, o_ref)
     assert abs(p["rel_frobenius_max"] - 0.03) < 1e-6 and not p["pass"]
+
+
+def test_cpu_baseline_returns_the_line_object_and_its_outputs():
+    c = CONFIGS["tiny_f32"]
+    x = bench.make_case(c)
+    line, o_ref = bench.cpu_baseline(c, 2, x)
+    assert line["kind"] == "oracle" and line["cores"] == 1 and line["unit"] == "tokens/s" and line["value"] > 0
+    assert "2 of 2" in line["sample"]
+    assert o_ref.shape == (2, c.T, c.d_v)
