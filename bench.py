@@ -5,8 +5,11 @@
 
 A step is one chunked forward of the whole layer (all heads, all tokens, final
 state) over one batch of synthetic inputs already resident in HBM.  Default
-workload: the LLM-shaped layer (B=4, H=16, T=4096, d=64, bf16, per-token
-learning rate, chunk 64).  Prints ONE JSON line on rank 0.
+workload: the long-context layer the tensor-peak fraction is quoted on (B=1,
+H=8, T=65536, d=128, bf16, constant learning rate, chunk 128).  The same line
+carries the chunk sweep (64, 128), the LLM-shaped and momentum layers, the
+decode step, the feature-mapped layer and the backward as sub-objects.
+Prints ONE JSON line on rank 0.
 
 Multi-GPU (torchrun): every rank runs its own batch (independent sequences,
 no collective on the data path: weak scaling); value = tokens of all ranks /
@@ -172,66 +175,166 @@ def max_over_ranks(x, info):
 
 
 # --------------------------------------------------------------- oracle ----
-def oracle_sample(c, heads, x=None):
-    """Runs the float64 oracle on the first `heads` (b, h) sequences of the
-    workload's inputs `x` (make_case(c) when None) at full length; returns
-    (seconds, head-tokens, o [heads, T, d_v])."""
+# Tokens of every (b, h) sequence in one bounded oracle sample: the reference
+# arm's steps (about 1 s of float64 work each) and the cpu_baseline leg (about
+# 5-10 s).  The oracle's cost per token is constant, so its tokens/s over a
+# prefix of every sequence is its tokens/s over the whole layer.
+REF_TOKENS = {"long_d128": 2048, "llm_d64": 1024, "momentum_d128": 256, "tiny_f32": 256}
+CPU_TOKENS = {"long_d128": 16384, "llm_d64": 4096, "momentum_d128": 2048, "tiny_f32": 256}
+
+
+def oracle_sample(c, tokens, x=None):
+    """Runs the float64 oracle on the first `tokens` tokens of every (b, h)
+    sequence of the workload's inputs `x` (make_case(c) when None); returns
+    (wall seconds, process CPU seconds, o [B*H, tokens, d_v])."""
     import oracle
     x = make_case(c) if x is None else x
-    f = lambda t: t.float().double().reshape(-1, *t.shape[2:])[:heads].numpy()  # noqa: E731
+    tokens = min(tokens, c.T)
+    f = lambda t: t[:, :, :tokens].float().double().reshape(-1, tokens, *t.shape[3:]).numpy()  # noqa: E731
     eta = f(x["eta"]) if x["eta"] is not None else x["eta_const"]
-    t0 = time.perf_counter()
-    o, _, _ = oracle.ttt_recurrence_f64(f(x["q"]), f(x["k"]), f(x["v"]), eta, beta=c.beta)
-    dt = time.perf_counter() - t0
-    return dt, heads * c.T, o
+    q, k, v = f(x["q"]), f(x["k"]), f(x["v"])
+    t0, c0 = time.perf_counter(), time.process_time()
+    o, _, _ = oracle.ttt_recurrence_f64(q, k, v, eta, beta=c.beta)
+    return time.perf_counter() - t0, time.process_time() - c0, o
 
 
 def parity(o_gpu, o_ref, tol=2e-2):
-    """Worst relative Frobenius error over the sampled (b, h) sequences of the
-    GPU output against the oracle's."""
+    """Worst relative Frobenius error over the (b, h) sequences of the GPU
+    output's first o_ref.shape[1] tokens against the oracle's."""
     import numpy as np
-    g = o_gpu.float().double().reshape(-1, *o_gpu.shape[2:])[:o_ref.shape[0]].numpy()
+    n = o_ref.shape[1]
+    g = o_gpu[:, :, :n].float().double().reshape(-1, n, o_gpu.shape[-1]).numpy()
     err = np.linalg.norm(g - o_ref, axis=(1, 2)) / np.maximum(np.linalg.norm(o_ref, axis=(1, 2)), 1e-30)
     worst = float(err.max())
-    return {"sequences": int(o_ref.shape[0]), "rel_frobenius_max": worst, "tolerance": tol, "pass": worst <= tol}
+    return {"sequences": int(o_ref.shape[0]), "tokens_each": int(n), "rel_frobenius_max": worst, "tolerance": tol,
+            "pass": worst <= tol}
 
 
-def cpu_baseline(c, heads, x=None):
-    """The oracle timed on `heads` sequences of the workload's inputs; also
+def cpu_line(c, tokens, wall, cpu, what):
+    """cpu_baseline object: tokens/s of the layer (B sequences x `tokens`
+    tokens, all heads) over the oracle's wall time; `cores` is the number of
+    threads the oracle kept busy (process CPU time / wall time)."""
+    n = min(tokens, c.T)
+    return {"value": c.B * n / wall, "unit": "tokens/s", "cores": max(1, round(cpu / wall)),
+            "host_cpu_count": os.cpu_count(), "kind": "oracle",
+            "sample": f"{what}: the first {n} of {c.T} tokens of all {c.B * c.H} (b,h) sequences of the benchmark's "
+                      f"own inputs ({wall:.1f} s of float64 numpy, {c.B * n} layer tokens; the oracle's per-token "
+                      "cost does not depend on the position, so this is its rate on the whole layer)"}
+
+
+def cpu_baseline(c, tokens, x=None):
+    """The oracle timed on a bounded sample of the workload's inputs; also
     returns its outputs, for the parity check of the GPU result."""
-    dt, head_tokens, o_ref = oracle_sample(c, heads, x)
-    total_head_tokens = c.B * c.H * c.T
-    t_full = dt * total_head_tokens / head_tokens
-    return {"value": c.B * c.T / t_full, "unit": "tokens/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{heads} of {c.B * c.H} (b,h) sequences of the benchmark's own inputs at full length "
-                      f"T={c.T} ({dt:.1f} s of single-threaded float64 numpy), scaled to the whole layer"}, o_ref
+    wall, cpu, o_ref = oracle_sample(c, tokens, x)
+    return cpu_line(c, tokens, wall, cpu, "one run"), o_ref
 
 
 def run_reference(args, c, ws, rank, info):
     if rank != 0:
         return
-    heads = max(1, min(c.B * c.H, args.ref_heads))
+    tokens = min(c.T, args.ref_tokens or REF_TOKENS.get(c.name, 1024))
     x = make_case(c)
     for _ in range(args.warmup):
-        oracle_sample(c, heads, x)
-    times = []
+        oracle_sample(c, tokens, x)
+    walls, cpus = [], []
     for _ in range(args.steps):
-        dt, _, _ = oracle_sample(c, heads, x)
-        times.append(dt * (c.B * c.H) / heads)
-    t = sum(times) / len(times)
-    val = c.B * c.T / t
+        wall, cpu, _ = oracle_sample(c, tokens, x)
+        walls.append(wall)
+        cpus.append(cpu)
+    t = sum(walls) / len(walls)
+    line_cpu = cpu_line(c, tokens, t, sum(cpus) / len(cpus), f"each of {args.steps} steps")
+    val = line_cpu["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(c, args),
-        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: the first {heads} of {c.B * c.H} (b,h) sequences of the "
-                                   "workload at full length, scaled to the whole layer"},
+        "config": dict(workload_config(c, args), step_tokens=c.B * tokens),
+        "cpu_baseline": line_cpu,
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def graph_time_us(fns, reps_min=20, min_ms=300.0, sampler=None):
+    """Device time per call of `fns` (a list of callables, one per rotating
+    input set): one CUDA graph holds a call on every set; it is replayed for
+    about a second untimed, then at least `reps_min` times and `min_ms`
+    milliseconds between CUDA events on the launching stream."""
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    stream = torch.cuda.current_stream()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    per_replay_ms = max(e0.elapsed_time(e1), 1e-3)
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        for _ in range(max(1, int(50.0 / per_replay_ms))):
+            g.replay()
+        torch.cuda.synchronize()
+    reps = max(reps_min, int(min_ms / per_replay_ms))
+    if sampler is not None:
+        sampler.mark_start()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.mark_end()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * len(fns))
+
+
+def forward_measure(ttt, dev, c, chunk, peaks, sets=4, segments=0):
+    """One workload's chunked forward: device time per call over `sets`
+    rotating input sets (together larger than L2), algorithmic bytes, the HBM
+    and executed-tensor-flop fractions of the measured peaks, the launch plan
+    and the clocks seen meanwhile."""
+    x = make_case(c)
+    bufs = []
+    for _ in range(sets):
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        eta = x["eta"].to(dev) if x["eta"] is not None else None
+        o = torch.empty_like(v)
+        S = torch.empty(c.B, c.H, c.d_v, c.d_k, device=dev, dtype=torch.float32)
+        M = torch.empty_like(S) if c.beta else None
+        bufs.append((q, k, v, eta, o, S, M))
+    wsb = ttt.workspace_bytes(bufs[0][0], bufs[0][2], chunk=chunk, beta=c.beta, segments=segments)
+    work = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+
+    def call(i):
+        q, k, v, eta, o, S, M = bufs[i]
+        return lambda: ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=chunk,
+                                           segments=segments, out=o, state_out=S, mom_out=M, workspace=work)
+    sampler = ClockSampler(dev.index or 0)
+    sampler.start()
+    us = graph_time_us([call(i) for i in range(sets)], sampler=sampler)
+    clocks = sampler.stop()
+    if ttt.device_status() != 0:
+        raise SystemExit(f"device status reports a timed-out wait ({c.name}, chunk {chunk})")
+    nbytes = algorithmic_bytes(c, c.B, c.H, c.T)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    flops = executed_flops(c, c.B, c.H, c.T, chunk)
+    tf = flops / (us * 1e-6) / 1e12
+    plan = ttt.chunked_plan(c.B, c.H, c.T, c.d_k, c.d_v, chunk=chunk, beta=c.beta, segments=segments,
+                            eta=c.eta_mode == "token")
+    del bufs, work
+    torch.cuda.empty_cache()
+    return {"workload": c.name, "chunk": chunk, "us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6),
+            "algorithmic_bytes": nbytes, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+            "executed_tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"],
+            "traffic": read_traffic(c.name, chunk), "plan": plan, "clocks": clocks,
+            "gpu_launches_per_call": 1}
 
 
 def decode_measure(ttt, dev, peaks):
@@ -333,32 +436,49 @@ def phi_measure(ttt, dev, peaks, reps=100):
             "gpu_launches_per_step": 2}
 
 
-def backward_measure(ttt, dev, reps=5):
-    """The layer's backward (ttt_la_backward_recurrent) on the llm_d64 inputs
-    (B4 H16 T4096 d64, per-token eta) with a seeded upstream gradient: dq,
-    dk, dv, per-token deta and dW0.  CUDA events over `reps` calls after one
-    warm-up call."""
+def backward_measure(ttt, dev, peaks, reps=5):
+    """The layer's backward on the llm_d64 inputs (B4 H16 T4096 d64, per-token
+    eta) with a seeded upstream gradient dL/do and dL/dW_T: dq, dk, dv,
+    per-token deta and dW0, in both forms -- the recurrent kernel (one block
+    per head) and the chunk-parallel one (three chunked forward runs).  CUDA
+    events over `reps` calls after one warm-up call of each."""
     c = CONFIGS["llm_d64"]
     x = make_case(c)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
     eta = x["eta"].to(dev)
     g = torch.Generator(device=dev).manual_seed(11)
     dO = torch.randn(v.shape, generator=g, device=dev).to(v.dtype)
-    out = ttt.backward_recurrent(q, k, v, dO, eta, eta_const=x["eta_const"])
-    torch.cuda.synchronize()
+    dW = torch.randn(c.B, c.H, c.d_v, c.d_k, generator=g, device=dev)
     stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        out = ttt.backward_recurrent(q, k, v, dO, eta, eta_const=x["eta_const"])
-    e1.record(stream)
-    torch.cuda.synchronize()
-    del out
-    if ttt.device_status() != 0:
-        raise SystemExit("device status reports a timed-out wait")
-    us = e0.elapsed_time(e1) * 1e3 / reps
-    return {"workload": "llm_d64 backward (recurrent form, one block per head)", "us_per_call": us,
-            "tokens_per_s": c.B * c.T / (us * 1e-6), "gpu_launches_per_call": 1}
+    # bytes a backward must move: q, k, v, dO read, dq, dk, dv written (bf16),
+    # eta read and deta written (fp32), dL/dW_T read and dL/dW_0 written
+    nbytes = c.B * c.H * (c.T * (2 * (2 * c.d_k + 2 * c.d_v) + 2 * (2 * c.d_k + c.d_v) + 8) + 2 * 4 * c.d_v * c.d_k)
+    out = {"workload": "llm_d64 backward (dq, dk, dv, deta, dW0 from dL/do and dL/dW_T)",
+           "algorithmic_bytes": nbytes}
+    ws = {}
+    for name, fn, n in (("recurrent", ttt.backward_recurrent, reps), ("chunked", ttt.backward_chunked, 20 * reps)):
+        def call():
+            return fn(q, k, v, dO, eta, eta_const=x["eta_const"], grad_state=dW, workspace=ws.get(name))
+        r = call()
+        del r
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            r = call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        del r
+        if ttt.device_status() != 0:
+            raise SystemExit("device status reports a timed-out wait")
+        us = e0.elapsed_time(e1) * 1e3 / n
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6), "hbm_gbs": gbs,
+                     "hbm_frac": gbs / peaks["hbm_gbs"],
+                     "gpu_launches_per_call": 1 if name == "recurrent" else 7}
+    out["chunked_speedup_over_recurrent"] = out["recurrent"]["us_per_call"] / out["chunked"]["us_per_call"]
+    torch.cuda.empty_cache()
+    return out
 
 
 def workload_config(c, args):
@@ -373,6 +493,7 @@ def run_ours(args, c, ws, rank, local, info):
     import test_layers_causal_b200 as ttt
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    peaks, src = load_peaks()
     chunk = args.chunk or c.chunk
     x = make_case(c)
     qh, kh, vh = x["q"], x["k"], x["v"]
@@ -454,6 +575,9 @@ def run_ours(args, c, ws, rank, local, info):
     value = ranks.weak_scaling_tokens_per_s(tokens_per_step, ws, ms_per_step)
     if ttt.device_status() != 0:
         raise RuntimeError("device status reports a timed-out wait")
+    del graphs, big
+    plan = ttt.chunked_plan(c.B, c.H, c.T, c.d_k, c.d_v, chunk=chunk, beta=c.beta, segments=args.segments,
+                            eta=c.eta_mode == "token")
 
     # ---- end to end: pinned host buffers in, o (and final state) back out
     qp, kp, vp = (t.pin_memory() for t in (qh, kh, vh))
@@ -462,8 +586,8 @@ def run_ours(args, c, ws, rank, local, info):
     Sh = torch.empty(c.B, c.H, c.d_v, c.d_k, dtype=torch.float32, pin_memory=True)
     bufs = ttt.host.HostStaging()
     kw = dict(eta_const=x["eta_const"], beta=c.beta, chunk=chunk, segments=args.segments)
-    e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(3):
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
         ttt.forward_chunked_host(qp, kp, vp, ep, o_host=oh, bufs=bufs, state_host=Sh, **kw)
     torch.cuda.synchronize()
     barrier(info)
@@ -475,43 +599,56 @@ def run_ours(args, c, ws, rank, local, info):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), info) / e2e_steps
     e2e_val = tokens_per_step * ws / (e2e_ms * 1e-3)
+    del bufs
 
-    # ---- roofline of the forward call
-    peaks, src = load_peaks()
+    # ---- roofline of the forward call (one kernel launch after a flag memset)
     nbytes = algorithmic_bytes(c, c.B, c.H, c.T)
     achieved = nbytes / (ms_per_step * 1e-3) / 1e9
     flops = executed_flops(c, c.B, c.H, c.T, chunk)
     tflops = flops / (ms_per_step * 1e-3) / 1e12
     traffic = read_traffic(c.name, chunk)
+    kname = ("chunked_tc_mom_kernel" if c.beta else f"chunked_tc_kernel<{chunk},{c.d_k}>")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if c.dtype == "bf16" else "f32", "data": "synthetic",
         "config": workload_config(c, args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "kernel": ("chunked_tc_mom_kernel" if c.beta else "chunked_tc_kernel")
-                               + (" (phase A, start states, phase B: one launch)" if wsb > 0
-                                  else " (one segment per sequence: phase B only)"),
-                     "algorithmic_bytes": nbytes, "peak_source": f"{src} (copy bandwidth)"},
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": kname,
+                     "algorithmic_bytes": nbytes, "peak_source": f"{src} copy bandwidth (of {src})",
+                     "timed_unit": "one forward call per step: the flag memset and one kernel launch"},
         "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                   "frac": tflops / peaks["bf16_tflops"], "executed_flops": flops},
+                   "frac": tflops / peaks["bf16_tflops"], "executed_flops": flops,
+                   "peak_source": f"{src} cuBLAS bf16 burst (of {src})"},
+        "plan": plan,
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,  # one kernel per step (plus a flag memset when segmented)
         "clocks": clocks,
     }
-    if not args.no_decode:
-        del sets, graphs
-        torch.cuda.empty_cache()
+    del sets, work
+    torch.cuda.empty_cache()
+    if ws == 1 and not args.no_extra:
+        # chunk sweep of the headline workload, then the other layer workloads
+        sweep = {}
+        for C in (64, 128):
+            if C != chunk and c.beta == 0:
+                sweep[str(C)] = forward_measure(ttt, dev, c, C, peaks)
+        if sweep:
+            line["chunk_sweep"] = sweep
+        others = {}
+        for name in ("llm_d64", "momentum_d128", "long_d128"):
+            if name != c.name:
+                oc = CONFIGS[name]
+                others[name] = forward_measure(ttt, dev, oc, oc.chunk, peaks)
+        line["workloads"] = others
         line["decode"] = decode_measure(ttt, dev, peaks)
-    if not args.no_phi:
         torch.cuda.empty_cache()
         line["phi_layer"] = phi_measure(ttt, dev, peaks)
-    if not args.no_backward:
         torch.cuda.empty_cache()
-        line["backward"] = backward_measure(ttt, dev)
+        line["backward"] = backward_measure(ttt, dev, peaks)
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"], o_ref = cpu_baseline(c, c.B * c.H if args.cpu_heads == 0 else args.cpu_heads, x)
+        tokens = args.cpu_tokens or CPU_TOKENS.get(c.name, c.T)
+        line["cpu_baseline"], o_ref = cpu_baseline(c, tokens, x)
         # the end-to-end run's output (public host-buffer API) against the oracle on the same inputs
         line["parity"] = parity(oh, o_ref)
     if rank == 0:
@@ -560,16 +697,17 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llm_d64", choices=sorted(CONFIGS) + ["decode", "phi"])
+    ap.add_argument("--workload", default="long_d128", choices=sorted(CONFIGS) + ["decode", "phi"])
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--sets", type=int, default=4)
-    ap.add_argument("--ref-heads", type=int, default=8, help="(b,h) sequences per reference-arm step")
-    ap.add_argument("--cpu-heads", type=int, default=0, help="cpu_baseline sample; 0 = the whole layer")
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="tokens of every sequence per reference-arm step (0: the workload's default sample)")
+    ap.add_argument("--cpu-tokens", type=int, default=0,
+                    help="tokens of every sequence in the cpu_baseline sample (0: the workload's default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--no-phi", action="store_true", help="skip the feature-map layer measurement")
-    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="headline only: no chunk sweep, other workloads, decode, feature map or backward")
     ap.add_argument("--profile-run", action="store_true",
                     help="plain launches for a profiler: no graphs, timing, decode or CPU baseline")
     args = ap.parse_args()

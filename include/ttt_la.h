@@ -45,11 +45,15 @@
  *    drains its own copies, frees its tensor memory and returns;
  *    ttt_la_get_last_device_status reads (and clears) that word.
  *  - The chunked forward splits long sequences into segments whose blocks
- *    exchange segment states through the workspace.  When the grid fits in
- *    one wave of resident blocks, the blocks of a head can wait for one
- *    another: other work running at the same time on the device delays them,
- *    and a delay beyond the wait limit (ttt_la_set_wait_limit_ns, default
- *    1 s) ends the call with TTT_LA_ERR_TIMEOUT rather than a hang.
+ *    exchange segment states through the workspace.  Where the blocks of a
+ *    head wait for one another (ttt_la_chunked_plan reports it as
+ *    `cooperative`), the kernel is launched cooperatively: every block of the
+ *    grid is then resident at once, or the launch fails with
+ *    TTT_LA_ERR_CUDA.  Elsewhere a block only waits for blocks that started
+ *    before it.  Every wait is still bounded (ttt_la_set_wait_limit_ns,
+ *    default 1 s); a wait that runs out is reported through the device status
+ *    word, not by the call's return value, so callers that must know check
+ *    ttt_la_get_last_device_status after the work.
  *  - o must not alias q, k, v, eta or the states.  state_out may equal
  *    state_in (in place), and mom_out may equal mom_in.
  */
@@ -116,6 +120,23 @@ TTT_LA_API size_t ttt_la_workspace_size(const ttt_la_args *args);
  * chunk in {64, 128}.  fp32 inputs run in fp32 FMA: d_k, d_v multiples of 4
  * up to 128, chunk in {16, 32, 64}.  Other combinations: UNSUPPORTED. */
 TTT_LA_API ttt_la_status ttt_la_forward_chunked(const ttt_la_args *args, void *stream);
+
+/* How ttt_la_forward_chunked would run these arguments on the current
+ * device (no launch; pointers are not read; without a device the figures are
+ * those of a 148-SM B200).  Fills *plan and returns TTT_LA_OK, or the status
+ * the forward would return for unusable arguments. */
+typedef struct ttt_la_plan {
+  int32_t path;             /* 0: tensor cores, no momentum; 1: tensor cores with momentum; 2: fp32 FMA */
+  int32_t tile;             /* tokens per tensor-core tile (the chunk; 64 with momentum) */
+  int32_t segments;         /* blocks per (b,h) sequence (one for the fp32 path) */
+  int32_t chunks_per_segment;
+  int32_t cooperative;      /* 1: blocks of a head wait for one another: launched cooperatively */
+  int32_t blocks;           /* grid size of the forward kernel */
+  int32_t resident;         /* blocks of that kernel resident at once on the device */
+  int32_t reserved;
+  size_t workspace_bytes;   /* = ttt_la_workspace_size(args) */
+} ttt_la_plan;
+TTT_LA_API ttt_la_status ttt_la_chunked_plan(const ttt_la_args *args, ttt_la_plan *plan);
 
 /* Token-by-token forward (the recurrence itself): fp32 or bf16 inputs,
  * d_k in {32, 64, 128}, d_v <= 1024; chunk and workspace are ignored. */

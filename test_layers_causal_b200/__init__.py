@@ -12,7 +12,7 @@ timing) and ``forward_sequence_sharded`` (one sequence split over ranks along
 T, see ``seqshard``).
 """
 from ._abi import (  # noqa: F401
-    TttError, backward_chunked, backward_recurrent, compose_maps, decode_step, device_status, feature_map, forward_chunked,
+    TttError, backward_chunked, backward_recurrent, chunked_plan, compose_maps, decode_step, device_status, feature_map, forward_chunked,
     forward_chunked_phi,
     forward_recurrent, lib, segment_map,
     selftest_wait_timeout, set_wait_limit_ns, status_string, version, workspace_bytes,

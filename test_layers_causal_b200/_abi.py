@@ -66,10 +66,20 @@ class TttGradArgs(ctypes.Structure):
     ]
 
 
+class TttPlan(ctypes.Structure):
+    """Mirror of ``ttt_la_plan``."""
+    _fields_ = [
+        ("path", _c_i32), ("tile", _c_i32), ("segments", _c_i32), ("chunks_per_segment", _c_i32),
+        ("cooperative", _c_i32), ("blocks", _c_i32), ("resident", _c_i32), ("reserved", _c_i32),
+        ("workspace_bytes", _c_sz),
+    ]
+
+
 # (name, restype, argtypes) for every symbol of include/ttt_la.h
 SIGNATURES = [
     ("ttt_la_workspace_size", _c_sz, [ctypes.POINTER(TttArgs)]),
     ("ttt_la_forward_chunked", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
+    ("ttt_la_chunked_plan", ctypes.c_int, [ctypes.POINTER(TttArgs), ctypes.POINTER(TttPlan)]),
     ("ttt_la_forward_chunked_noalloc", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp]),
     ("ttt_la_host_staging_size", _c_sz, [ctypes.POINTER(TttArgs)]),
     ("ttt_la_forward_chunked_host", ctypes.c_int, [ctypes.POINTER(TttArgs), _c_vp, _c_sz, _c_vp]),
@@ -432,6 +442,21 @@ def workspace_bytes(q, v, chunk=64, beta=0.0, segments=0):
     a.q, a.k, a.v, a.o = 16, 32, 48, 64  # never dereferenced by the size query
     a.beta, a.chunk, a.segments = float(beta), int(chunk), int(segments)
     return int(lib().ttt_la_workspace_size(ctypes.byref(a)))
+
+
+def chunked_plan(B, H, T, d_k, d_v, dtype="bf16", chunk=64, beta=0.0, segments=0, eta=False):
+    """How ttt_la_forward_chunked would run these shapes on the current device
+    (ttt_la_chunked_plan; no launch, no tensors): a dict of the plan's fields."""
+    a = TttArgs()
+    a.B, a.H, a.T, a.d_k, a.d_v = B, H, T, d_k, d_v
+    a.dtype = BF16 if dtype == "bf16" else F32
+    a.q, a.k, a.v, a.o = 16, 32, 48, 64  # never dereferenced by the query
+    a.eta = 80 if eta else None
+    a.eta_const = 1.0 / math.sqrt(d_k)
+    a.beta, a.chunk, a.segments = float(beta), int(chunk), int(segments)
+    p = TttPlan()
+    _check("ttt_la_chunked_plan", lib().ttt_la_chunked_plan(ctypes.byref(a), ctypes.byref(p)))
+    return {name: getattr(p, name) for name, _ in TttPlan._fields_ if name != "reserved"}
 
 
 def forward_recurrent(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, state_in=None, mom_in=None,

@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/ttt_la.h"
 #include "backward.cuh"
@@ -35,6 +37,75 @@ int sm_count() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
   return n;
+}
+
+// Raises `fn`'s dynamic shared-memory limit to `bytes` on the current device.
+// The attribute belongs to each device's context, so the grant is recorded
+// per (kernel, device), under a lock: host threads may launch concurrently,
+// and one process may drive several devices.
+bool grant_smem(const void* fn, int bytes) {
+  if (bytes <= 48 * 1024) return true;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  struct Grant {
+    const void* fn;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Grant> granted;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Grant& g : granted)
+    if (g.fn == fn && g.dev == dev && g.bytes >= bytes) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  for (Grant& g : granted)
+    if (g.fn == fn && g.dev == dev) {
+      g.bytes = bytes;
+      return true;
+    }
+  granted.push_back({fn, dev, bytes});
+  return true;
+}
+
+// Blocks of `fn` (threads, dynamic shared memory) that one SM holds at once on
+// the current device, from the occupancy calculator, at most `cap` (tensor
+// memory, which the calculator does not count, caps some kernels).  Without a
+// device (size queries on a host with no GPU) the answer is `cap`.
+int resident_per_sm(const void* fn, int threads, int smem, int cap) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return cap;
+  }
+  int n = 0;
+  if (!grant_smem(fn, smem) || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    return cap;
+  }
+  return std::min(n, cap);
+}
+
+// Launches `kern` on `st`; `coop` makes it a cooperative launch, which
+// guarantees that every block of the grid is resident at once (or fails to
+// launch), as kernels whose blocks wait for one another need.
+template <typename... P, typename... A>
+ttt_la_status launch_kernel(void (*kern)(P...), int grid, int threads, int smem, cudaStream_t st, bool coop,
+                            A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = coop ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return TTT_LA_ERR_CUDA;
+  }
+  return TTT_LA_OK;
 }
 
 // ------------------------------------------------------------ TMA maps ----
@@ -137,14 +208,32 @@ ttt_la_status recurrent_dk(const ttt_la_args* a, cudaStream_t st) {
 // --------------------------------------------------------------- chunked ----
 struct SegPlan {
   int nchunks, cps, nseg;
-  bool coop = false;  // plain kernel: cooperative prefix instead of decoupled look-back
+  int resident = 0;   // blocks of the selected kernel resident at once on the device
+  bool coop = false;  // cooperative start states (the head's blocks wait for one another)
 };
-
-int tc_ctas_per_sm(int C, int D) { return (C == 64 && D == 64) ? 2 : 1; }
 
 // Tokens per tensor-core tile: the requested chunk, except with momentum, whose
 // kernel always runs 64-token tiles (a 128-token chunk is the same layer).
 int tc_tile(const ttt_la_args* a) { return a->beta != 0.f ? 64 : a->chunk; }
+
+// Resident blocks per SM of the tensor-core kernel that these arguments
+// select (1 for every tile but 64 x 64, whose 256 tensor-memory columns let
+// two blocks share an SM).
+template <int C, int D>
+int tc_per_sm() {
+  using Cfg = ttt::TcCfg<C, D>;
+  return resident_per_sm(reinterpret_cast<const void*>(ttt::chunked_tc_kernel<C, D>), 256, Cfg::SMEM, Cfg::MINB);
+}
+template <int D>
+int tcm_per_sm() {
+  using Cfg = ttt::TcMomCfg<D>;
+  return resident_per_sm(reinterpret_cast<const void*>(ttt::chunked_tc_mom_kernel<D>), Cfg::THREADS, Cfg::SMEM, 1);
+}
+int tc_resident_per_sm(const ttt_la_args* a) {
+  if (a->beta != 0.f) return a->d_k == 64 ? tcm_per_sm<64>() : tcm_per_sm<128>();
+  if (a->d_k == 64) return a->chunk == 64 ? tc_per_sm<64, 64>() : tc_per_sm<128, 64>();
+  return a->chunk == 64 ? tc_per_sm<64, 128>() : tc_per_sm<128, 128>();
+}
 
 SegPlan plan_segments(const ttt_la_args* a) {
   SegPlan s;
@@ -153,18 +242,18 @@ SegPlan plan_segments(const ttt_la_args* a) {
   const int bh = a->B * a->H;
   // Automatic: as many segments as fit in one wave of resident blocks (never
   // a partial second wave), at least one per sequence.
-  const int per_sm = a->beta != 0.f ? 1 : tc_ctas_per_sm(C, a->d_k);
-  const int resident = sm_count() * per_sm;
-  int nseg = a->segments > 0 ? a->segments : std::max(1, resident / bh);
+  s.resident = sm_count() * tc_resident_per_sm(a);
+  int nseg = a->segments > 0 ? a->segments : std::max(1, s.resident / bh);
   nseg = std::max(1, std::min(nseg, s.nchunks));
   s.cps = (s.nchunks + nseg - 1) / nseg;
   s.nseg = (s.nchunks + s.cps - 1) / s.cps;
-  // Start states by a cooperative prefix (blocks of a head wait for one
-  // another: only when the whole grid is resident at once) when a decoupled
-  // look-back would have the last segment read more than 192 KB of totals.
+  // Cooperative start states (blocks of a head wait for one another, so the
+  // grid must be one wave and is launched cooperatively): with momentum
+  // whenever the grid is one wave; without, when a decoupled look-back would
+  // also have the last segment read more than 192 KB of totals.
+  const bool one_wave = s.nseg > 1 && static_cast<long long>(bh) * s.nseg <= s.resident;
   const size_t lookback_bytes = static_cast<size_t>(s.nseg - 1) * a->d_k * a->d_v * sizeof(float);
-  s.coop = a->beta == 0.f && s.nseg > 1 && static_cast<long long>(bh) * s.nseg <= resident &&
-           lookback_bytes > 192 * 1024;
+  s.coop = one_wave && (a->beta != 0.f || lookback_bytes > 192 * 1024);
   return s;
 }
 
@@ -200,13 +289,7 @@ size_t tc_ws_bytes(int bh, int nseg, int D) {
 template <int C, int D>
 ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
   using Cfg = ttt::TcCfg<C, D>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(ttt::chunked_tc_kernel<C, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
-        cudaSuccess)
-      return TTT_LA_ERR_CUDA;
-    attr_done = true;
-  }
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_tc_kernel<C, D>), Cfg::SMEM)) return TTT_LA_ERR_CUDA;
   const int bh = a->B * a->H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
@@ -233,20 +316,14 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
-  ttt::chunked_tc_kernel<C, D><<<bh * sp.nseg, 256, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
-  return launched();
+  return launch_kernel(ttt::chunked_tc_kernel<C, D>, bh * sp.nseg, 256, Cfg::SMEM, st, sp.coop, mq, mk, mv, mo, p);
 }
 
 template <bool MOM>
 ttt_la_status launch_simt(const ttt_la_args* a, const ttt::SimtShape& sh, cudaStream_t st) {
-  static size_t attr_bytes = 0;
   const size_t bytes = sh.bytes();
-  if (bytes > 48 * 1024 && bytes > attr_bytes) {
-    if (cudaFuncSetAttribute(ttt::chunked_simt_f32_kernel<MOM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bytes)) != cudaSuccess)
-      return TTT_LA_ERR_CUDA;
-    attr_bytes = bytes;
-  }
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_simt_f32_kernel<MOM>), static_cast<int>(bytes)))
+    return TTT_LA_ERR_CUDA;
   ttt::chunked_simt_f32_kernel<MOM><<<a->B * a->H, 256, bytes, st>>>(seq_params(a), sh);
   return launched();
 }
@@ -270,13 +347,7 @@ template <int D>
 ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
   using Cfg = ttt::TcMomCfg<D>;
   constexpr int C = Cfg::C;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(ttt::chunked_tc_mom_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM) != cudaSuccess)
-      return TTT_LA_ERR_CUDA;
-    attr_done = true;
-  }
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_tc_mom_kernel<D>), Cfg::SMEM)) return TTT_LA_ERR_CUDA;
   const int bh = a->B * a->H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
@@ -300,8 +371,7 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
   p.S_out = a->state_out;
   p.M_out = a->mom_out;
   p.limit_ns = g_limit_ns;
-  // cooperative start states whenever the whole grid is one wave (one block per SM)
-  p.coop = (sp.nseg > 1 && static_cast<long long>(bh) * sp.nseg <= sm_count()) ? 1 : 0;
+  p.coop = sp.coop ? 1 : 0;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
     p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;
@@ -309,8 +379,8 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
-  ttt::chunked_tc_mom_kernel<D><<<bh * sp.nseg, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, mv, mo, p);
-  return launched();
+  return launch_kernel(ttt::chunked_tc_mom_kernel<D>, bh * sp.nseg, Cfg::THREADS, Cfg::SMEM, st, sp.coop, mq, mk, mv,
+                       mo, p);
 }
 
 // ---------------------------------------------------------------- decode ----
@@ -382,13 +452,8 @@ ttt_la_status check_feature(const ttt_la_feature_args* a) {
 template <int DIN, int DOUT>
 ttt_la_status launch_feature(const ttt_la_feature_args* a, cudaStream_t st) {
   using Cfg = ttt::FmapCfg<DIN, DOUT>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(ttt::feature_map_kernel<DIN, DOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM) != cudaSuccess)
-      return TTT_LA_ERR_CUDA;
-    attr_done = true;
-  }
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::feature_map_kernel<DIN, DOUT>), Cfg::SMEM))
+    return TTT_LA_ERR_CUDA;
   const int bh = a->B * a->H;
   CUtensorMap mx[2], my[2], m1, m3;
   for (int i = 0; i < 2; ++i) {
@@ -466,13 +531,8 @@ template <int DK, typename T, bool MOM>
 ttt_la_status launch_backward(const ttt_la_grad_args* a, cudaStream_t st) {
   using Sh = ttt::BwdShape<DK>;
   const size_t smem = ttt::bwd_smem_floats(DK, a->d_v, Sh::CK) * sizeof(float);
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(ttt::backward_recurrent_kernel<DK, T, MOM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             232448) != cudaSuccess)
-      return TTT_LA_ERR_CUDA;
-    attr_done = true;
-  }
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::backward_recurrent_kernel<DK, T, MOM>), 232448))
+    return TTT_LA_ERR_CUDA;
   ttt::BwdParams p;
   p.BH = a->B * a->H;
   p.T = a->T;
@@ -598,6 +658,35 @@ ttt_la_status ttt_la_forward_chunked(const ttt_la_args* a, void* stream) {
   if (mom) return a->d_k == 64 ? launch_tc_mom<64>(a, sp, st) : launch_tc_mom<128>(a, sp, st);
   if (a->d_k == 64) return a->chunk == 64 ? launch_tc<64, 64>(a, sp, st) : launch_tc<128, 64>(a, sp, st);
   return a->chunk == 64 ? launch_tc<64, 128>(a, sp, st) : launch_tc<128, 128>(a, sp, st);
+}
+
+ttt_la_status ttt_la_chunked_plan(const ttt_la_args* a, ttt_la_plan* out) {
+  if (!out) return TTT_LA_ERR_INVALID_ARG;
+  std::memset(out, 0, sizeof *out);
+  const ttt_la_status s = check_seq(a);
+  if (s != TTT_LA_OK) return s;
+  if (a->dtype == TTT_LA_F32) {
+    ttt::SimtShape sh;
+    if (!simt_supported(a, &sh)) return TTT_LA_ERR_UNSUPPORTED;
+    out->path = 2;
+    out->tile = a->chunk;
+    out->segments = 1;
+    out->chunks_per_segment = (a->T + a->chunk - 1) / a->chunk;
+    out->blocks = a->B * a->H;
+    out->resident = out->blocks;
+    return TTT_LA_OK;
+  }
+  if (!tc_supported(a)) return TTT_LA_ERR_UNSUPPORTED;
+  const SegPlan sp = plan_segments(a);
+  out->path = a->beta != 0.f ? 1 : 0;
+  out->tile = tc_tile(a);
+  out->segments = sp.nseg;
+  out->chunks_per_segment = sp.cps;
+  out->cooperative = sp.coop ? 1 : 0;
+  out->blocks = a->B * a->H * sp.nseg;
+  out->resident = sp.resident;
+  out->workspace_bytes = workspace_for(a);
+  return TTT_LA_OK;
 }
 
 ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args* a, void* stream) {

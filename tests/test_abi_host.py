@@ -65,6 +65,8 @@ int main(void) {
   P(ttt_la_grad_args, q); P(ttt_la_grad_args, eta_const); P(ttt_la_grad_args, state_in);
   P(ttt_la_grad_args, grad_o); P(ttt_la_grad_args, grad_q); P(ttt_la_grad_args, grad_eta);
   P(ttt_la_grad_args, grad_mom_in); P(ttt_la_grad_args, workspace_bytes);
+  printf("ttt_la_plan %zu\n", sizeof(ttt_la_plan));
+  P(ttt_la_plan, cooperative); P(ttt_la_plan, resident); P(ttt_la_plan, workspace_bytes);
   return 0;
 }
 """
@@ -79,8 +81,10 @@ int main(void) {
     assert int(vals["ttt_la_decode_args"]) == ctypes.sizeof(abi.TttDecodeArgs)
     assert int(vals["ttt_la_feature_args"]) == ctypes.sizeof(abi.TttFeatureArgs)
     assert int(vals["ttt_la_grad_args"]) == ctypes.sizeof(abi.TttGradArgs)
+    assert int(vals["ttt_la_plan"]) == ctypes.sizeof(abi.TttPlan)
     classes = {"ttt_la_args": abi.TttArgs, "ttt_la_decode_args": abi.TttDecodeArgs,
-               "ttt_la_feature_args": abi.TttFeatureArgs, "ttt_la_grad_args": abi.TttGradArgs}
+               "ttt_la_feature_args": abi.TttFeatureArgs, "ttt_la_grad_args": abi.TttGradArgs,
+               "ttt_la_plan": abi.TttPlan}
     for key, v in vals.items():
         if "." in key:
             struct, field = key.split(".")
@@ -251,6 +255,30 @@ def test_workspace_query(abi):
     assert L.ttt_la_forward_chunked(ctypes.byref(fixed), None) == abi.ERR_INVALID_ARG
     assert L.ttt_la_set_wait_limit_ns(10) == abi.ERR_INVALID_ARG
     assert L.ttt_la_selftest_wait_timeout(10, None) == abi.ERR_INVALID_ARG
+
+
+def test_chunked_plan_launch_modes(abi):
+    """Blocks of a head that wait for one another (cooperative start states)
+    are launched cooperatively, which guarantees they are resident together;
+    the plan the launch uses is the one the query reports.  Without a GPU the
+    plan is that of a 148-SM B200 (one 128-wide tile per SM, two 64 x 64)."""
+    long_ctx = abi.chunked_plan(1, 8, 65536, 128, 128, chunk=128)
+    assert long_ctx["path"] == 0 and long_ctx["cooperative"] == 1
+    assert long_ctx["segments"] == 18 and long_ctx["blocks"] == 144 <= long_ctx["resident"] == 148
+    mom = abi.chunked_plan(2, 16, 8192, 128, 128, chunk=128, beta=0.9, eta=True)
+    assert mom["path"] == 1 and mom["tile"] == 64 and mom["cooperative"] == 1 and mom["blocks"] <= mom["resident"]
+    llm = abi.chunked_plan(4, 16, 4096, 64, 64, chunk=64, eta=True)  # short look-back: no waiting on peers
+    assert llm["path"] == 0 and llm["cooperative"] == 0 and llm["segments"] == 4 and llm["resident"] == 296
+    # a grid beyond one wave never waits on peers
+    wide = abi.chunked_plan(1, 8, 65536, 128, 128, chunk=128, segments=40)
+    assert wide["cooperative"] == 0 and wide["blocks"] == 320
+    # one segment per sequence: no scratch, nothing to wait for
+    many = abi.chunked_plan(64, 16, 256, 64, 64, chunk=64)
+    assert many["segments"] == 1 and many["cooperative"] == 0 and many["workspace_bytes"] == 0
+    f32 = abi.chunked_plan(1, 2, 256, 32, 32, dtype="f32", chunk=64)
+    assert f32["path"] == 2 and f32["blocks"] == 2
+    with pytest.raises(abi.TttError):
+        abi.chunked_plan(1, 8, 1024, 96, 96, chunk=64)
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -15,17 +15,21 @@ from synth import CONFIGS  # noqa: E402
 
 
 def test_reference_arm_line():
-    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
-                        "--ref-heads", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2", "--warmup", "0",
+                        "--ref-tokens", "64"], cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     line = json.loads(r.stdout.strip().splitlines()[-1])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in line, key
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
-    assert line["config"]["workload"] == "llm_d64"
+    assert line["config"]["workload"] == "long_d128" and line["config"]["step_tokens"] == 64
     assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert cb["host_cpu_count"] == os.cpu_count()
+    # the value is the measured rate of the sampled step itself: no scaling factor
+    assert abs(line["value"] - 64 / (line["ms_per_step"] * 1e-3)) < 1e-6 * line["value"]
 
 
 def test_algorithmic_bytes_and_flops():
@@ -57,22 +61,27 @@ def test_hashed_sources_exist(name):
 
 def test_parity_helper_against_the_oracle_samples():
     """The bench's parity figure: fp32 rounding for the oracle's own output,
-    the relative error of a known perturbation otherwise."""
+    the relative error of a known perturbation otherwise; a prefix of every
+    sequence is compared with the oracle run on that prefix (causality)."""
     import torch
     c = CONFIGS["tiny_f32"]
     x = bench.make_case(c)
-    _, _, o_ref = bench.oracle_sample(c, 2, x)
-    o = torch.from_numpy(o_ref).reshape(c.B, c.H, c.T, c.d_v)
-    p = bench.parity(o, o_ref)
+    _, _, o_full = bench.oracle_sample(c, c.T, x)
+    o = torch.from_numpy(o_full).reshape(c.B, c.H, c.T, c.d_v)
+    p = bench.parity(o, o_full)
     assert p["sequences"] == 2 and p["rel_frobenius_max"] < 1e-7 and p["pass"]  # fp32 rounding only
-    p = bench.parity(1.03 * o, o_ref)
+    p = bench.parity(1.03 * o, o_full)
     assert abs(p["rel_frobenius_max"] - 0.03) < 1e-6 and not p["pass"]
+    _, _, o_pre = bench.oracle_sample(c, 100, x)
+    p = bench.parity(o, o_pre)
+    assert p["tokens_each"] == 100 and p["rel_frobenius_max"] < 1e-7
 
 
 def test_cpu_baseline_returns_the_line_object_and_its_outputs():
     c = CONFIGS["tiny_f32"]
     x = bench.make_case(c)
-    line, o_ref = bench.cpu_baseline(c, 2, x)
-    assert line["kind"] == "oracle" and line["cores"] == 1 and line["unit"] == "tokens/s" and line["value"] > 0
-    assert "2 of 2" in line["sample"]
-    assert o_ref.shape == (2, c.T, c.d_v)
+    line, o_ref = bench.cpu_baseline(c, 128, x)
+    assert line["kind"] == "oracle" and line["cores"] >= 1 and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["host_cpu_count"] == os.cpu_count()
+    assert "first 128 of 256 tokens of all 2" in line["sample"]
+    assert o_ref.shape == (2, 128, c.d_v)

@@ -2,10 +2,6 @@
 (ttt_la_backward_chunked: three runs of the chunked forward) against the
 float64 gradient oracle and against the recurrent backward.
 
-Skipped until these have run on a B200.  Its orchestration (which pass reads
-which tensors, the reversals, transposes and the final scaling) was checked
-on CPU with the forward oracle in place of the chunked kernel.
-
 Tolerances: bf16 inputs, relative Frobenius error <= 2e-2 per (b, h) slice
 and overall; fp32 inputs (the fp32 chunked forward), max-rel <= 1e-4.
 """
@@ -18,7 +14,7 @@ import oracle
 from synth import make_qkv
 from tests.gpu_util import assert_bf16, assert_f32, f64
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="not yet run on a B200")]
+pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     from test_layers_causal_b200 import _abi
