@@ -79,7 +79,8 @@ typedef enum {
   TTT_LA_ERR_UNSUPPORTED = 2,  /* valid but not built: (d_k, d_v, chunk, dtype) combination */
   TTT_LA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   TTT_LA_ERR_TIMEOUT = 4,      /* a bounded in-kernel wait ran out (device status word) */
-  TTT_LA_ERR_SCRATCH_LIMIT = 5 /* ttt_la_forward_chunked_noalloc: scratch need exceeds its fixed array */
+  TTT_LA_ERR_SCRATCH_LIMIT = 5, /* ttt_la_forward_chunked_noalloc: scratch need exceeds its fixed array */
+  TTT_LA_ERR_DEVICE_CHECK = 6   /* debug builds: a device-side bounds check failed (device status word) */
 } ttt_la_status;
 
 typedef enum { TTT_LA_F32 = 0, TTT_LA_BF16 = 1 } ttt_la_dtype;
@@ -133,7 +134,10 @@ typedef struct ttt_la_plan {
   int32_t cooperative;      /* 1: blocks of a head wait for one another: launched cooperatively */
   int32_t blocks;           /* grid size of the forward kernel */
   int32_t resident;         /* blocks of that kernel resident at once on the device */
-  int32_t reserved;
+  int32_t waves;            /* cooperative schedule without momentum: the sequence is cut into
+                               `waves` waves of `segments` runs, and phase B of each wave re-reads
+                               K and V from L2 (about 512 tokens per run; the environment variable
+                               TTT_LA_WAVE_TOKENS overrides that, for tuning); 1 otherwise */
   size_t workspace_bytes;   /* = ttt_la_workspace_size(args) */
 } ttt_la_plan;
 TTT_LA_API ttt_la_status ttt_la_chunked_plan(const ttt_la_args *args, ttt_la_plan *plan);
@@ -341,9 +345,20 @@ TTT_LA_API ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args *args,
 TTT_LA_API size_t ttt_la_backward_chunked_workspace_size(const ttt_la_grad_args *args);
 TTT_LA_API ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args *args, void *stream);
 
-/* Synchronises `stream`, returns the device status word (TTT_LA_OK or
- * TTT_LA_ERR_TIMEOUT) of the current device and clears it. */
+/* Synchronises `stream`, returns the device status word (TTT_LA_OK,
+ * TTT_LA_ERR_TIMEOUT, or in debug builds TTT_LA_ERR_DEVICE_CHECK, which wins
+ * over a timeout) of the current device and clears it. */
 TTT_LA_API ttt_la_status ttt_la_get_last_device_status(void *stream);
+
+/* Debug builds (the library compiled with -DTTT_LA_DEBUG, libttt_la_debug.so):
+ * the chunked kernels check every hand-indexed access to the workspace, the
+ * flags and the states against the sizes of this call; a failed check
+ * records TTT_LA_ERR_DEVICE_CHECK and the source line, and the access goes to
+ * a private sink instead (nothing faults or traps).  Synchronises `stream`,
+ * returns the line of the first failed check since the last query (0: none)
+ * and clears it; -1 in release builds (no checks compiled), -2 if CUDA
+ * failed. */
+TTT_LA_API int32_t ttt_la_debug_check_line(void *stream);
 
 /* Sets the time limit of every in-kernel wait (nanoseconds, >= 1000);
  * default 1e9 (one second).  Affects launches made after the call. */

@@ -15,8 +15,9 @@ import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libttt_la.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libttt_la_debug.so")  # built with -DTTT_LA_DEBUG (device-side bounds checks)
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = 0, 1, 2, 3, 4, 5
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT, ERR_DEVICE_CHECK = 0, 1, 2, 3, 4, 5, 6
 STATIC_SCRATCH_BYTES = 8 << 20  # TTT_LA_STATIC_SCRATCH_BYTES
 F32, BF16 = 0, 1
 
@@ -70,7 +71,7 @@ class TttPlan(ctypes.Structure):
     """Mirror of ``ttt_la_plan``."""
     _fields_ = [
         ("path", _c_i32), ("tile", _c_i32), ("segments", _c_i32), ("chunks_per_segment", _c_i32),
-        ("cooperative", _c_i32), ("blocks", _c_i32), ("resident", _c_i32), ("reserved", _c_i32),
+        ("cooperative", _c_i32), ("blocks", _c_i32), ("resident", _c_i32), ("waves", _c_i32),
         ("workspace_bytes", _c_sz),
     ]
 
@@ -93,6 +94,7 @@ SIGNATURES = [
     ("ttt_la_backward_chunked_workspace_size", _c_sz, [ctypes.POINTER(TttGradArgs)]),
     ("ttt_la_backward_chunked", ctypes.c_int, [ctypes.POINTER(TttGradArgs), _c_vp]),
     ("ttt_la_get_last_device_status", ctypes.c_int, [_c_vp]),
+    ("ttt_la_debug_check_line", _c_i32, [_c_vp]),
     ("ttt_la_set_wait_limit_ns", ctypes.c_int, [ctypes.c_int64]),
     ("ttt_la_selftest_wait_timeout", ctypes.c_int, [ctypes.c_int64, _c_vp]),
     ("ttt_la_status_string", ctypes.c_char_p, [ctypes.c_int]),
@@ -109,19 +111,35 @@ class TttError(RuntimeError):
         super().__init__(f"{fn} failed: {msg} (status {code})")
 
 
+def _load(path):
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m test_layers_causal_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, res, args in SIGNATURES:
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
 def lib():
     """Loads the shared library (once).  Raises if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m test_layers_causal_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, res, args in SIGNATURES:
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _lib = L
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+_debug_lib = None
+
+
+def debug_lib():
+    """The debug build of the library (device-side bounds checks), loaded once
+    beside the release one; the binding's functions keep using lib()."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(DEBUG_LIB_PATH)
+    return _debug_lib
 
 
 def status_string(code: int) -> str:
@@ -456,7 +474,7 @@ def chunked_plan(B, H, T, d_k, d_v, dtype="bf16", chunk=64, beta=0.0, segments=0
     a.beta, a.chunk, a.segments = float(beta), int(chunk), int(segments)
     p = TttPlan()
     _check("ttt_la_chunked_plan", lib().ttt_la_chunked_plan(ctypes.byref(a), ctypes.byref(p)))
-    return {name: getattr(p, name) for name, _ in TttPlan._fields_ if name != "reserved"}
+    return {name: getattr(p, name) for name, _ in TttPlan._fields_}
 
 
 def forward_recurrent(q, k, v, eta=None, eta_const=None, beta=0.0, ascent=False, state_in=None, mom_in=None,

@@ -67,11 +67,11 @@ __global__ void __launch_bounds__(256) transpose_states_kernel(const TransposePa
 }
 
 // dv_t = sigma eta_t u_t, dk_t = sigma eta_t r_t, deta_t = sigma v_t . u_t,
-// with u and r stored in reversed token order.  One warp per (b, h, t).
+// with u and r stored in fp32 in reversed token order.  One warp per (b, h, t).
 struct FinishParams {
   int BH, T, dk, dv;
-  const void* u_rev;  // [BH][T][dv]
-  const void* r_rev;  // [BH][T][dk]
+  const float* u_rev; // [BH][T][dv]
+  const float* r_rev; // [BH][T][dk]
   const void* v;      // [BH][T][dv]
   const float* eta;   // [BH][T] or nullptr
   float eta_const, sigma;
@@ -89,18 +89,18 @@ __global__ void __launch_bounds__(256) backward_finish_kernel(const FinishParams
   const int t = static_cast<int>(warp - bh * p.T);
   const long long fwd = warp, rev = bh * p.T + (p.T - 1 - t);
   const float s = p.sigma * (p.eta ? p.eta[fwd] : p.eta_const);
-  const T* u = static_cast<const T*>(p.u_rev) + rev * p.dv;
-  const T* r = static_cast<const T*>(p.r_rev) + rev * p.dk;
+  const float* u = p.u_rev + rev * p.dv;
+  const float* r = p.r_rev + rev * p.dk;
   const T* v = static_cast<const T*>(p.v) + fwd * p.dv;
   T* dv = static_cast<T*>(p.dv_out) + fwd * p.dv;
   T* dk = static_cast<T*>(p.dk_out) + fwd * p.dk;
   float vu = 0.f;
   for (int c = lane; c < p.dv; c += 32) {
-    const float uc = to_f(u[c]);
+    const float uc = u[c];
     vu = fmaf(to_f(v[c]), uc, vu);
     dv[c] = from_f<T>(s * uc);
   }
-  for (int c = lane; c < p.dk; c += 32) dk[c] = from_f<T>(s * to_f(r[c]));
+  for (int c = lane; c < p.dk; c += 32) dk[c] = from_f<T>(s * r[c]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) vu += __shfl_xor_sync(0xffffffffu, vu, off);
   if (lane == 0 && p.deta) p.deta[fwd] = p.sigma * vu;

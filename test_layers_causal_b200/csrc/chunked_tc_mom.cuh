@@ -49,6 +49,8 @@ struct TcMomParams {
   float* S_out;
   float* M_out;
   uint64_t limit_ns;
+  size_t ws_floats;    // floats of scratch before the flags (bounds of the debug checks)
+  unsigned flag_words; // words of flags and counters
 };
 
 template <int D>
@@ -487,8 +489,9 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
 
     // ---- phase A result and look-back
     {
-      float* me = p.ws ? p.ws + (static_cast<size_t>(bh) * p.nseg + seg) * 4 * DD : nullptr;
-      unsigned* flag_me = p.flags ? p.flags + bh * p.nseg + seg : nullptr;
+      float* me = p.ws ? TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + seg) * 4 * DD, 4 * DD, p.ws_floats)
+                       : nullptr;
+      unsigned* flag_me = p.flags ? TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + seg, 1, p.flag_words) : nullptr;
       if (nA > 0) {
         if (!dead) dead = !mbar_wait(sdone, 0, lim);
         if (!dead) dead = !mbar_wait(seg_ready, 0, lim);
@@ -512,8 +515,10 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           }
         }
         if (et == 0) {
-          p.wsc[(static_cast<size_t>(bh) * p.nseg + seg) * 2 + 0] = segsc[0];
-          p.wsc[(static_cast<size_t>(bh) * p.nseg + seg) * 2 + 1] = segsc[1];
+          float* sc = TTT_AT(p.wsc, (static_cast<size_t>(bh) * p.nseg + seg) * 2, 2,
+                             p.ws_floats - static_cast<size_t>(p.BH) * p.nseg * 4 * DD);
+          sc[0] = segsc[0];
+          sc[1] = segsc[1];
         }
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -530,17 +535,25 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         // slots 2 and 3; the blocks meet at the head's counter and each then
         // reads its own start state.
         for (int j = et; j < p.nseg - 1; j += 128)
-          if (!dead && wait_geq(p.flags + bh * p.nseg + j, 1u, lim) == 0) dead = true;
+          if (!dead && wait_geq(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + j, 1, p.flag_words), 1u, lim) == 0)
+            dead = true;
         asm volatile("bar.sync 1, 128;" ::: "memory");
         const int DDi = D * D;
         const int SL = ((DDi + p.nseg - 1) / p.nseg + 31) / 32 * 32;  // slice, a multiple of 32
         const int v1 = min(DDi, (seg + 1) * SL) / 4;
         const int nagg = p.nseg - 1;
-        float4* w4 = reinterpret_cast<float4*>(p.ws + static_cast<size_t>(bh) * p.nseg * 4 * DD);
-        const size_t SEG4 = DD, Q4 = DD / 4;  // float4 strides: between segments, between a segment's matrices
-        const float* maps = p.wsc + static_cast<size_t>(bh) * p.nseg * 2;
-        const float4* sw4 = p.S_in ? reinterpret_cast<const float4*>(p.S_in + static_cast<size_t>(bh) * DD) : nullptr;
-        const float4* sm4 = p.M_in ? reinterpret_cast<const float4*>(p.M_in + static_cast<size_t>(bh) * DD) : nullptr;
+        // segment j's four matrices (dW, dM, then W and M at its start)
+        auto seg4 = [&](int j) {
+          return reinterpret_cast<float4*>(
+              TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + j) * 4 * DD, 4 * DD, p.ws_floats));
+        };
+        const size_t Q4 = DD / 4;  // float4 stride between a segment's matrices
+        const float* maps = TTT_AT(p.wsc, static_cast<size_t>(bh) * p.nseg * 2, 2 * p.nseg,
+                                   p.ws_floats - static_cast<size_t>(p.BH) * p.nseg * 4 * DD);
+        const size_t nst = static_cast<size_t>(p.BH) * DD;
+        const float4* sw4 = p.S_in ? reinterpret_cast<const float4*>(TTT_AT(p.S_in, bh * DD, DD, nst)) : nullptr;
+        const float4* sm4 = p.M_in ? reinterpret_cast<const float4*>(TTT_AT(p.M_in, bh * DD, DD, nst)) : nullptr;
+        TTT_EXPECT(v1 <= static_cast<int>(DD / 4));
         const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
         // two positions per thread per round, four maps per round
         for (int v0 = seg * SL / 4 + et; v0 < v1; v0 += 256) {
@@ -563,8 +576,8 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                   if (ok[e]) {
-                    dw[e][u] = __ldcg(w4 + (j + u) * SEG4 + vv[e]);
-                    dm[e][u] = __ldcg(w4 + (j + u) * SEG4 + Q4 + vv[e]);
+                    dw[e][u] = __ldcg(seg4(j + u) + vv[e]);
+                    dm[e][u] = __ldcg(seg4(j + u) + Q4 + vv[e]);
                   }
                 }
               }
@@ -575,8 +588,8 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                   if (!ok[e]) continue;
-                  __stcg(w4 + (j + u) * SEG4 + 2 * Q4 + vv[e], w[e]);
-                  __stcg(w4 + (j + u) * SEG4 + 3 * Q4 + vv[e], m[e]);
+                  __stcg(seg4(j + u) + 2 * Q4 + vv[e], w[e]);
+                  __stcg(seg4(j + u) + 3 * Q4 + vv[e], m[e]);
                   // (W, M) -> (W - G M + dW, B M + dM)
                   const float4 a = w[e], b = m[e], x = dw[e][u], y = dm[e][u];
                   w[e] = make_float4(fmaf(-G[u], b.x, a.x) + x.x, fmaf(-G[u], b.y, a.y) + x.y,
@@ -590,20 +603,20 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             if (!ok[e]) continue;
-            __stcg(w4 + nagg * SEG4 + 2 * Q4 + vv[e], w[e]);
-            __stcg(w4 + nagg * SEG4 + 3 * Q4 + vv[e], m[e]);
+            __stcg(seg4(nagg) + 2 * Q4 + vv[e], w[e]);
+            __stcg(seg4(nagg) + 3 * Q4 + vv[e], m[e]);
           }
         }
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        unsigned* cnt = p.flags + p.BH * p.nseg + 1 + bh;
+        unsigned* cnt = TTT_AT(p.flags, static_cast<size_t>(p.BH) * p.nseg + 1 + bh, 1, p.flag_words);
         if (et == 0) {
           atomicAdd(cnt, 1u);
           if (!dead && wait_geq(cnt, static_cast<unsigned>(p.nseg), lim) == 0) dead = true;
           __threadfence();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + seg) * 4 + 2) * DD;
+        bw = TTT_AT(p.ws, ((static_cast<size_t>(bh) * p.nseg + seg) * 4 + 2) * DD, 2 * DD, p.ws_floats);
         bm = bw + DD;
         base_qm = true;
         first = seg;
@@ -614,7 +627,8 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         if (et == 0) sh_lb[1] = -1;
         asm volatile("bar.sync 1, 128;" ::: "memory");
         for (int j = et; j < seg; j += 128) {
-          const unsigned f = dead ? 1u : wait_geq(p.flags + bh * p.nseg + j, 1u, lim);
+          const unsigned f =
+              dead ? 1u : wait_geq(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + j, 1, p.flag_words), 1u, lim);
           if (f == 0) dead = true;
           if (f >= 2) atomicMax(&sh_lb[1], j);
         }
@@ -622,12 +636,12 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         const int incl = sh_lb[1];
         first = incl + 1;
         if (incl >= 0) {
-          bw = p.ws + ((static_cast<size_t>(bh) * p.nseg + incl) * 4 + 2) * DD;
+          bw = TTT_AT(p.ws, ((static_cast<size_t>(bh) * p.nseg + incl) * 4 + 2) * DD, 2 * DD, p.ws_floats);
           bm = bw + DD;
           base_qm = true;
         } else {
-          if (p.S_in) bw = p.S_in + static_cast<size_t>(bh) * DD;
-          if (p.M_in) bm = p.M_in + static_cast<size_t>(bh) * DD;
+          if (p.S_in) bw = TTT_AT(p.S_in, bh * DD, DD, static_cast<size_t>(p.BH) * DD);
+          if (p.M_in) bm = TTT_AT(p.M_in, bh * DD, DD, static_cast<size_t>(p.BH) * DD);
         }
       }
       const float Gme = (nA > 0) ? segsc[0] : 0.f, Bme = (nA > 0) ? segsc[1] : 1.f;
@@ -660,10 +674,11 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           }
           // apply the published segment maps in order
           for (int jj = first; jj < seg; ++jj) {
-            const float* dw = p.ws + (static_cast<size_t>(bh) * p.nseg + jj) * 4 * DD;
+            const float* dw = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + jj) * 4 * DD, 2 * DD, p.ws_floats);
             const float* dm = dw + DD;
-            const float G = __ldcg(p.wsc + (static_cast<size_t>(bh) * p.nseg + jj) * 2);
-            const float B = __ldcg(p.wsc + (static_cast<size_t>(bh) * p.nseg + jj) * 2 + 1);
+            const float* gb = TTT_AT(p.wsc, (static_cast<size_t>(bh) * p.nseg + jj) * 2, 2,
+                                     p.ws_floats - static_cast<size_t>(p.BH) * p.nseg * 4 * DD);
+            const float G = __ldcg(gb), B = __ldcg(gb + 1);
             float8 xw[4], xm[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -715,6 +730,13 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) st_release(flag_me, 2u);
+      }
+      // look-back: count the blocks that are done reading W_0 and M_0, which
+      // the last segment's W_T and M_T may overwrite (in place)
+      if (!p.coop && p.nseg > 1 && seg < p.nseg - 1) {
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) atomicAdd(TTT_AT(p.flags, static_cast<size_t>(p.BH) * p.nseg + 1 + bh, 1, p.flag_words), 1u);
       }
     }
 
@@ -839,6 +861,14 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
 
     // final state (last segment)
     if (seg == p.nseg - 1 && (p.S_out != nullptr || p.M_out != nullptr)) {
+      // look-back: W_T, M_T may overwrite W_0, M_0 (in place) once every
+      // other block has its start state (the cooperative prefix has already
+      // met at the same counter)
+      if (!p.coop && p.nseg > 1 && et == 0 && !dead &&
+          wait_geq(TTT_AT(p.flags, static_cast<size_t>(p.BH) * p.nseg + 1 + bh, 1, p.flag_words),
+                   static_cast<unsigned>(p.nseg - 1), lim) == 0)
+        dead = true;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       if (!dead) dead = !mbar_wait(sdone, ((nA > 0 ? 1 : 0) + nB - 1) & 1, lim);
       tc_fence_after();
 #pragma unroll
@@ -851,7 +881,8 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
           tmem_ld32(tq + lane_off + cb * 32, r);
           tmem_ld_wait();
           if (dst && wrow_ok) {
-            float4* d4 = reinterpret_cast<float4*>(dst + static_cast<size_t>(bh) * DD + static_cast<size_t>(wrow) * D + cb * 32);
+            float4* d4 = reinterpret_cast<float4*>(TTT_AT(dst, bh * DD, DD, static_cast<size_t>(p.BH) * DD) +
+                                                   static_cast<size_t>(wrow) * D + cb * 32);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),

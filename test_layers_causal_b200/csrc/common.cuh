@@ -15,12 +15,56 @@
 namespace ttt {
 
 // Device status word (one per device, per loaded library): 0 = OK,
-// 4 = an in-kernel wait ran out (TTT_LA_ERR_TIMEOUT).
+// 4 = an in-kernel wait ran out (TTT_LA_ERR_TIMEOUT), 6 = a device-side
+// bounds check failed (debug builds, TTT_LA_ERR_DEVICE_CHECK).  The larger
+// code wins when both happen.
 __device__ int g_status;
+// Source line of the first failed bounds check (debug builds; 0 = none).
+__device__ int g_check_line;
 
 constexpr int kStatusTimeout = 4;
+constexpr int kStatusDeviceCheck = 6;
 
-__device__ __forceinline__ void record_timeout() { atomicExch(&g_status, kStatusTimeout); }
+__device__ __forceinline__ void record_timeout() { atomicMax(&g_status, kStatusTimeout); }
+
+// ------------------------------------------------------- debug checks ----
+// Built with -DTTT_LA_DEBUG, the kernels check every hand-indexed access to
+// the caller's scratch and to the states against the sizes the host passed:
+// a failed check records its source line and TTT_LA_ERR_DEVICE_CHECK, and the
+// access goes to a private sink array instead, so nothing faults or traps.
+// Release builds compile the checks away.
+#ifdef TTT_LA_DEBUG
+constexpr bool kDebugChecks = true;
+constexpr size_t kSinkFloats = 4 * 128 * 128 + 64;  // the largest span addressed from one checked base
+__device__ __align__(16) float g_check_sink[kSinkFloats];
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+__device__ __noinline__ void record_check(int line) {
+  atomicCAS(&g_check_line, 0, line);
+  atomicMax(&g_status, kStatusDeviceCheck);
+}
+
+// base + off, where [off, off + count) must lie within [0, limit).
+template <typename T>
+__device__ __forceinline__ T* checked(T* base, size_t off, size_t count, size_t limit, int line) {
+#ifdef TTT_LA_DEBUG
+  if (base == nullptr || off + count > limit || count * sizeof(T) > kSinkFloats * sizeof(float)) {
+    record_check(line);
+    return reinterpret_cast<T*>(g_check_sink);
+  }
+#endif
+  return base + off;
+}
+// A condition that must hold (debug builds record the line when it does not).
+__device__ __forceinline__ void check_that(bool ok, int line) {
+#ifdef TTT_LA_DEBUG
+  if (!ok) record_check(line);
+#endif
+}
+#define TTT_AT(base, off, count, limit) ::ttt::checked((base), (off), (count), (limit), __LINE__)
+#define TTT_EXPECT(cond) ::ttt::check_that((cond), __LINE__)
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -101,6 +145,12 @@ __device__ __forceinline__ void tma_load_3d_hint(const CUtensorMap* m, uint64_t*
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// For tiles read again soon by the same block: kept ahead of normal lines.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int x, int y, int z) {

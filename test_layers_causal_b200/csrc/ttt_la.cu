@@ -8,11 +8,14 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 #include <utility>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/ttt_la.h"
 #include "backward.cuh"
@@ -29,6 +32,27 @@
 namespace {
 
 uint64_t g_limit_ns = 1000000000ull;
+
+// NVTX range around each entry point, in the "ttt_la" domain: a profiler
+// (nsys, ncu --nvtx) shows which call launched what.  NVTX v3 is header-only;
+// with no tool attached each push and pop is a call through a no-op pointer.
+nvtxDomainHandle_t nvtx_domain() {
+  static const nvtxDomainHandle_t d = nvtxDomainCreateA("ttt_la");
+  return d;
+}
+struct NvtxRange {
+  explicit NvtxRange(const char* name) {
+    nvtxEventAttributes_t e = {};
+    e.version = NVTX_VERSION;
+    e.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    e.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    e.message.ascii = name;
+    nvtxDomainRangePushEx(nvtx_domain(), &e);
+  }
+  ~NvtxRange() { nvtxDomainRangePop(nvtx_domain()); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -56,7 +80,12 @@ bool grant_smem(const void* fn, int bytes) {
   std::lock_guard<std::mutex> lock(mu);
   for (const Grant& g : granted)
     if (g.fn == fn && g.dev == dev && g.bytes >= bytes) return true;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  // the largest shared-memory carveout, so that the occupancy calculator and
+  // the launch both see the whole 228 KB of an SM
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+      cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+          cudaSuccess)
+    return false;
   for (Grant& g : granted)
     if (g.fn == fn && g.dev == dev) {
       g.bytes = bytes;
@@ -208,9 +237,33 @@ ttt_la_status recurrent_dk(const ttt_la_args* a, cudaStream_t st) {
 // --------------------------------------------------------------- chunked ----
 struct SegPlan {
   int nchunks, cps, nseg;
+  int nwave = 1;      // waves of the cooperative schedule without momentum (1 otherwise)
+  int keep = 0;       // phase-A chunks per run whose K and V are loaded evict-last
   int resident = 0;   // blocks of the selected kernel resident at once on the device
   bool coop = false;  // cooperative start states (the head's blocks wait for one another)
 };
+
+// Tokens each block handles per wave in the cooperative schedule without
+// momentum.  More waves keep K and V in L2 for phase B (two waves live, about
+// 150 KB per 512 tokens per block at d = 128), but every wave costs one
+// in-place scan of the blocks' d x d totals and a meeting of the head's
+// blocks; measured on the long-context layer (B1 H8 T65536 d128) the
+// meetings cost more than the re-read saves at every length tried (256 to
+// 1024 tokens), so by default the schedule is a single wave (phase A over a
+// block's whole run, one scan, phase B).  TTT_LA_WAVE_TOKENS sets the length
+// (tuning and tests).
+// MB of phase-A K and V loaded evict-last (TTT_LA_L2_KEEP_MB, tuning).
+int l2_keep_mb() {
+  const char* e = std::getenv("TTT_LA_L2_KEEP_MB");
+  const int v = e ? std::atoi(e) : -1;
+  return v >= 0 ? v : 64;
+}
+
+int wave_tokens() {
+  const char* e = std::getenv("TTT_LA_WAVE_TOKENS");
+  const int v = e ? std::atoi(e) : 0;
+  return v > 0 ? v : (1 << 30);
+}
 
 // Tokens per tensor-core tile: the requested chunk, except with momentum, whose
 // kernel always runs 64-token tiles (a 128-token chunk is the same layer).
@@ -240,10 +293,14 @@ SegPlan plan_segments(const ttt_la_args* a) {
   const int C = tc_tile(a);
   s.nchunks = (a->T + C - 1) / C;
   const int bh = a->B * a->H;
-  // Automatic: as many segments as fit in one wave of resident blocks (never
-  // a partial second wave), at least one per sequence.
+  // Automatic: as many segments as the tile's design places on the SMs at
+  // once (two 64 x 64 blocks per SM, one otherwise; never a partial second
+  // wave), at least one per sequence.  Whether the grid is really resident as
+  // a whole, which the cooperative schedules need, is the occupancy
+  // calculator's answer (`resident`).
   s.resident = sm_count() * tc_resident_per_sm(a);
-  int nseg = a->segments > 0 ? a->segments : std::max(1, s.resident / bh);
+  const int design_per_sm = (a->beta == 0.f && C == 64 && a->d_k == 64) ? 2 : 1;
+  int nseg = a->segments > 0 ? a->segments : std::max(1, sm_count() * design_per_sm / bh);
   nseg = std::max(1, std::min(nseg, s.nchunks));
   s.cps = (s.nchunks + nseg - 1) / nseg;
   s.nseg = (s.nchunks + s.cps - 1) / s.cps;
@@ -253,7 +310,22 @@ SegPlan plan_segments(const ttt_la_args* a) {
   // also have the last segment read more than 192 KB of totals.
   const bool one_wave = s.nseg > 1 && static_cast<long long>(bh) * s.nseg <= s.resident;
   const size_t lookback_bytes = static_cast<size_t>(s.nseg - 1) * a->d_k * a->d_v * sizeof(float);
-  s.coop = one_wave && (a->beta != 0.f || lookback_bytes > 192 * 1024);
+  // (the 64 x 64 tile without momentum runs the look-back only: see chunked_tc.cuh)
+  const bool tile64 = a->beta == 0.f && C == 64 && a->d_k == 64;
+  s.coop = one_wave && (a->beta != 0.f || (lookback_bytes > 192 * 1024 && !tile64));
+  if (s.coop && a->beta == 0.f) {
+    // every run of every wave holds at least one chunk: nwave <= nchunks / nseg
+    const int per_run = std::max(1, wave_tokens() / C);
+    s.nwave = std::max(1, std::min(s.nchunks / (s.nseg * per_run), s.nchunks / s.nseg));
+  }
+  if (a->beta == 0.f && s.nseg > 1) {
+    // K and V phase B reads first, kept in L2 from phase A: about l2_keep_mb
+    // MB over the whole grid (beside the Q, O and scratch streams)
+    const size_t chunk_kv = static_cast<size_t>(C) * (a->d_k + a->d_v) * 2;
+    const size_t blocks = static_cast<size_t>(bh) * s.nseg;
+    s.keep = static_cast<int>(std::min<size_t>(static_cast<size_t>(l2_keep_mb()) << 20, size_t(1) << 40) /
+                              (blocks * chunk_kv));
+  }
   return s;
 }
 
@@ -279,21 +351,29 @@ bool simt_supported(const ttt_la_args* a, ttt::SimtShape* sh) {
 // (segment totals, segment start states), then nseg*BH publication flags, one
 // tile counter and BH per-head counters (uint32), which every call clears
 // before its launch.
-size_t tc_ws_floats(int bh, int nseg, int D) { return static_cast<size_t>(bh) * nseg * 2 * D * D; }
+// The wave schedule uses fp32 [BH][2][nseg][d_v][d_k] (run totals, scanned in
+// place into start states, slot = wave parity) plus [BH][d_v][d_k] (state at
+// the wave's end): (2 nseg + 1) matrices per head instead of 2 nseg.
+size_t tc_ws_floats(int bh, int nseg, int D, bool waves = false) {
+  return static_cast<size_t>(bh) * (2 * nseg + (waves ? 1 : 0)) * D * D;
+}
 size_t tc_flag_words(int bh, int nseg) { return static_cast<size_t>(bh) * nseg + 1 + bh; }
-size_t tc_ws_bytes(int bh, int nseg, int D) {
-  const size_t b = tc_ws_floats(bh, nseg, D) * sizeof(float) + tc_flag_words(bh, nseg) * sizeof(unsigned);
+size_t tc_ws_bytes(int bh, int nseg, int D, bool waves = false) {
+  const size_t b = tc_ws_floats(bh, nseg, D, waves) * sizeof(float) + tc_flag_words(bh, nseg) * sizeof(unsigned);
   return (b + 15) & ~static_cast<size_t>(15);
 }
 
-template <int C, int D>
-ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st) {
-  using Cfg = ttt::TcCfg<C, D>;
-  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_tc_kernel<C, D>), Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+// SPLIT: the split state readout with fp32 output to o32 (the backward's
+// passes; the bf16 O map is then never used and is built over q).
+template <int C, int D, bool SPLIT = false>
+ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st, float* o32 = nullptr) {
+  using Cfg = ttt::TcCfg<C, D, SPLIT>;
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_tc_kernel<C, D, SPLIT>), Cfg::SMEM))
+    return TTT_LA_ERR_CUDA;
   const int bh = a->B * a->H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
-      !make_map(&mv, a->v, bh, a->T, D, C) || !make_map(&mo, a->o, bh, a->T, D, C))
+      !make_map(&mv, a->v, bh, a->T, D, C) || !make_map(&mo, SPLIT ? a->q : a->o, bh, a->T, D, C))
     return TTT_LA_ERR_CUDA;
   ttt::TcParams p;
   p.BH = bh;
@@ -308,15 +388,47 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
   p.ws = nullptr;
   p.flags = nullptr;
   p.coop = sp.coop ? 1 : 0;
+  p.nwave = sp.coop ? sp.nwave : 1;
+  p.keep = sp.keep;
   p.S_out = a->state_out;
+  p.o32 = o32;
   p.limit_ns = g_limit_ns;
+  p.ws_floats = 0;
+  p.flag_words = 0;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
-    p.flags = reinterpret_cast<unsigned*>(p.ws + tc_ws_floats(bh, sp.nseg, D));
+    p.ws_floats = tc_ws_floats(bh, sp.nseg, D, sp.coop);
+    p.flag_words = static_cast<unsigned>(tc_flag_words(bh, sp.nseg));
+    p.flags = reinterpret_cast<unsigned*>(p.ws + p.ws_floats);
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
-  return launch_kernel(ttt::chunked_tc_kernel<C, D>, bh * sp.nseg, 256, Cfg::SMEM, st, sp.coop, mq, mk, mv, mo, p);
+  return launch_kernel(ttt::chunked_tc_kernel<C, D, SPLIT>, bh * sp.nseg, 256, Cfg::SMEM, st, sp.coop, mq, mk, mv, mo,
+                       p);
+}
+
+// The chunked forward of the backward's passes (bf16, no momentum): the
+// state read out as bf16(W) + bf16(W - bf16(W)) and O written in fp32 to
+// o32 [B,H,T,d_v] (a->o is ignored), so that the products the backward forms
+// from O (dv, dk and the per-token deta, a d-term dot product that can
+// cancel) keep fp32 precision.  Tiles: d = 64 with 128 tokens, d = 128 with
+// 64 (the two whose shared memory holds the second bf16 copy of W).
+size_t workspace_for(const ttt_la_args* a);
+ttt_la_status forward_chunked_split(const ttt_la_args* a0, float* o32, cudaStream_t st) {
+  if (!a0 || !o32 || !aligned16(o32)) return TTT_LA_ERR_INVALID_ARG;
+  ttt_la_args a = *a0;
+  a.o = o32;
+  const ttt_la_status s = check_seq(&a);
+  if (s != TTT_LA_OK) return s;
+  if (a.dtype != TTT_LA_BF16 || a.beta != 0.f || a.d_k != a.d_v ||
+      !((a.d_k == 64 && a.chunk == 128) || (a.d_k == 128 && a.chunk == 64)))
+    return TTT_LA_ERR_UNSUPPORTED;
+  const SegPlan sp = plan_segments(&a);
+  if (sp.nseg > 1) {
+    const size_t need = workspace_for(&a);
+    if (!a.workspace || a.workspace_bytes < need || !aligned16(a.workspace)) return TTT_LA_ERR_INVALID_ARG;
+  }
+  return a.d_k == 64 ? launch_tc<128, 64, true>(&a, sp, st, o32) : launch_tc<64, 128, true>(&a, sp, st, o32);
 }
 
 template <bool MOM>
@@ -340,7 +452,8 @@ size_t workspace_for(const ttt_la_args* a) {
   if (!tc_supported(a)) return 0;
   const SegPlan sp = plan_segments(a);
   if (sp.nseg <= 1) return 0;
-  return a->beta != 0.f ? tcm_ws_bytes(a->B * a->H, sp.nseg, a->d_k) : tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k);
+  return a->beta != 0.f ? tcm_ws_bytes(a->B * a->H, sp.nseg, a->d_k)
+                        : tc_ws_bytes(a->B * a->H, sp.nseg, a->d_k, sp.coop);
 }
 
 template <int D>
@@ -372,8 +485,12 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
   p.M_out = a->mom_out;
   p.limit_ns = g_limit_ns;
   p.coop = sp.coop ? 1 : 0;
+  p.ws_floats = 0;
+  p.flag_words = 0;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
+    p.ws_floats = tcm_ws_floats(bh, sp.nseg, D);
+    p.flag_words = static_cast<unsigned>(tc_flag_words(bh, sp.nseg));
     p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;
     p.flags = reinterpret_cast<unsigned*>(p.ws + tcm_ws_floats(bh, sp.nseg, D));
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
@@ -621,11 +738,12 @@ const char* ttt_la_status_string(ttt_la_status s) {
     case TTT_LA_ERR_CUDA: return "CUDA error";
     case TTT_LA_ERR_TIMEOUT: return "in-kernel wait timed out";
     case TTT_LA_ERR_SCRATCH_LIMIT: return "scratch need exceeds the fixed no-alloc array";
+    case TTT_LA_ERR_DEVICE_CHECK: return "device-side bounds check failed (debug build)";
   }
   return "unknown status";
 }
 
-const char* ttt_la_version(void) { return "ttt_la 0.1 (sm_100a)"; }
+const char* ttt_la_version(void) { return ttt::kDebugChecks ? "ttt_la 0.2 (sm_100a, debug checks)" : "ttt_la 0.2 (sm_100a)"; }
 
 ttt_la_status ttt_la_set_wait_limit_ns(int64_t limit_ns) {
   if (limit_ns < 1000) return TTT_LA_ERR_INVALID_ARG;
@@ -639,6 +757,7 @@ size_t ttt_la_workspace_size(const ttt_la_args* a) {
 }
 
 ttt_la_status ttt_la_forward_chunked(const ttt_la_args* a, void* stream) {
+  NvtxRange range("ttt_la_forward_chunked");
   ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -683,6 +802,7 @@ ttt_la_status ttt_la_chunked_plan(const ttt_la_args* a, ttt_la_plan* out) {
   out->segments = sp.nseg;
   out->chunks_per_segment = sp.cps;
   out->cooperative = sp.coop ? 1 : 0;
+  out->waves = sp.nwave;
   out->blocks = a->B * a->H * sp.nseg;
   out->resident = sp.resident;
   out->workspace_bytes = workspace_for(a);
@@ -690,6 +810,7 @@ ttt_la_status ttt_la_chunked_plan(const ttt_la_args* a, ttt_la_plan* out) {
 }
 
 ttt_la_status ttt_la_forward_chunked_noalloc(const ttt_la_args* a, void* stream) {
+  NvtxRange range("ttt_la_forward_chunked_noalloc");
   ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
   const size_t need = workspace_for(a);
@@ -713,6 +834,7 @@ size_t ttt_la_host_staging_size(const ttt_la_args* a) {
 
 ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args* a, void* device_buf, size_t device_bytes,
                                           void* stream) {
+  NvtxRange range("ttt_la_forward_chunked_host");
   ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
   if (a->dtype == TTT_LA_F32) {
@@ -782,6 +904,7 @@ ttt_la_status ttt_la_forward_chunked_host(const ttt_la_args* a, void* device_buf
 }
 
 ttt_la_status ttt_la_segment_map(const ttt_la_args* a, float* dW, float* dM, float* GB, void* stream) {
+  NvtxRange range("ttt_la_segment_map");
   ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
   const bool mom = a->beta != 0.f;
@@ -809,6 +932,7 @@ ttt_la_status ttt_la_segment_map(const ttt_la_args* a, float* dW, float* dM, flo
 ttt_la_status ttt_la_compose_maps(int32_t nmaps, int32_t BH, int32_t d_v, int32_t d_k, const float* dW,
                                   const float* dM, const float* GB, const float* W0, const float* M0, float* W_out,
                                   float* M_out, void* stream) {
+  NvtxRange range("ttt_la_compose_maps");
   if (nmaps < 0 || BH < 1 || d_v < 1 || d_k < 1 || !W_out || (nmaps > 0 && !dW)) return TTT_LA_ERR_INVALID_ARG;
   if ((dM == nullptr) != (GB == nullptr)) return TTT_LA_ERR_INVALID_ARG;
   if (static_cast<long long>(BH) * d_v * d_k >= (1ll << 40)) return TTT_LA_ERR_INVALID_ARG;
@@ -830,6 +954,7 @@ ttt_la_status ttt_la_compose_maps(int32_t nmaps, int32_t BH, int32_t d_v, int32_
 }
 
 ttt_la_status ttt_la_feature_map(const ttt_la_feature_args* a, void* stream) {
+  NvtxRange range("ttt_la_feature_map");
   const ttt_la_status s = check_feature(a);
   if (s != TTT_LA_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -843,6 +968,7 @@ size_t ttt_la_backward_workspace_size(const ttt_la_grad_args* a) {
 }
 
 ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args* a, void* stream) {
+  NvtxRange range("ttt_la_backward_recurrent");
   const ttt_la_status s = check_grad(a);
   if (s != TTT_LA_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -852,6 +978,7 @@ ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args* a, void* stream)
 }
 
 ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {
+  NvtxRange range("ttt_la_forward_recurrent");
   ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
   if (a->d_v > 1024) return TTT_LA_ERR_UNSUPPORTED;
@@ -863,6 +990,7 @@ ttt_la_status ttt_la_forward_recurrent(const ttt_la_args* a, void* stream) {
 }
 
 ttt_la_status ttt_la_decode_step(const ttt_la_decode_args* a, void* stream) {
+  NvtxRange range("ttt_la_decode_step");
   if (!a) return TTT_LA_ERR_INVALID_ARG;
   if (a->N < 1 || a->H < 1 || a->d_k < 1 || a->d_v < 1) return TTT_LA_ERR_INVALID_ARG;
   if (a->dtype != TTT_LA_F32 && a->dtype != TTT_LA_BF16) return TTT_LA_ERR_INVALID_ARG;
@@ -885,7 +1013,19 @@ ttt_la_status ttt_la_get_last_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, ttt::g_status, sizeof(int)) != cudaSuccess) return TTT_LA_ERR_CUDA;
   const int zero = 0;
   if (cudaMemcpyToSymbol(ttt::g_status, &zero, sizeof(int)) != cudaSuccess) return TTT_LA_ERR_CUDA;
-  return v == 0 ? TTT_LA_OK : TTT_LA_ERR_TIMEOUT;
+  if (v == 0) return TTT_LA_OK;
+  return v == ttt::kStatusDeviceCheck ? TTT_LA_ERR_DEVICE_CHECK : TTT_LA_ERR_TIMEOUT;
+}
+
+int32_t ttt_la_debug_check_line(void* stream) {
+  if (!ttt::kDebugChecks) return -1;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return -2;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, ttt::g_check_line, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(ttt::g_check_line, &zero, sizeof(int)) != cudaSuccess)
+    return -2;
+  return v;
 }
 
 ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void* stream) {
@@ -903,7 +1043,12 @@ struct BwdChunkedLayout {
   size_t rev[4], u, r, w0t, dwt, fwd, total, fwd_bytes;
 };
 
-int bwdc_chunk(const ttt_la_grad_args* a) { return (a->dtype == TTT_LA_BF16 && a->d_k == 128) ? 128 : 64; }
+// bf16: the tiles of the split readout (d = 64: 128 tokens, d = 128: 64);
+// fp32: the fp32 chunked path's 64.
+int bwdc_chunk(const ttt_la_grad_args* a) {
+  if (a->dtype != TTT_LA_BF16) return 64;
+  return a->d_k == 128 ? 64 : 128;
+}
 
 // Arguments of forward pass p: 0 gives dq, 1 gives u = G k (reversed order)
 // and dL/dW_0, 2 gives r = G^T v (reversed order).  rev[] are q, k, v, dO
@@ -963,10 +1108,11 @@ BwdChunkedLayout bwdc_layout(const ttt_la_grad_args* a) {
     L.rev[i] = off;
     off += sizes[i];
   }
+  // u and r in fp32 whatever the dtype
   L.u = off;
-  off += nv;
+  off += align256(bh * a->T * a->d_v * 4);
   L.r = off;
-  off += nk;
+  off += align256(bh * a->T * a->d_k * 4);
   L.w0t = off;
   off += a->state_in ? ns : 0;
   L.dwt = off;
@@ -1003,6 +1149,7 @@ size_t ttt_la_backward_chunked_workspace_size(const ttt_la_grad_args* a) {
 }
 
 ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
+  NvtxRange range("ttt_la_backward_chunked");
   ttt_la_status s = check_grad_chunked(a);
   if (s != TTT_LA_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1054,7 +1201,11 @@ ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
     ttt_la_args f = bwdc_pass(a, p, rev, u, r, w0t, dwt);
     f.workspace = L.fwd_bytes ? ws + L.fwd : nullptr;
     f.workspace_bytes = L.fwd_bytes;
-    if ((s = ttt_la_forward_chunked(&f, stream)) != TTT_LA_OK) return s;
+    if (p > 0 && a->dtype == TTT_LA_BF16)  // u and r: split readout, fp32 out
+      s = forward_chunked_split(&f, static_cast<float*>(p == 1 ? u : r), st);
+    else
+      s = ttt_la_forward_chunked(&f, stream);
+    if (s != TTT_LA_OK) return s;
   }
   // dv, dk, deta
   ttt::FinishParams fp;
@@ -1062,8 +1213,8 @@ ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
   fp.T = a->T;
   fp.dk = a->d_k;
   fp.dv = a->d_v;
-  fp.u_rev = u;
-  fp.r_rev = r;
+  fp.u_rev = static_cast<const float*>(u);
+  fp.r_rev = static_cast<const float*>(r);
   fp.v = a->v;
   fp.eta = a->eta;
   fp.eta_const = a->eta_const;

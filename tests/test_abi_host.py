@@ -257,7 +257,7 @@ def test_workspace_query(abi):
     assert L.ttt_la_selftest_wait_timeout(10, None) == abi.ERR_INVALID_ARG
 
 
-def test_chunked_plan_launch_modes(abi):
+def test_chunked_plan_launch_modes(abi, monkeypatch):
     """Blocks of a head that wait for one another (cooperative start states)
     are launched cooperatively, which guarantees they are resident together;
     the plan the launch uses is the one the query reports.  Without a GPU the
@@ -265,8 +265,19 @@ def test_chunked_plan_launch_modes(abi):
     long_ctx = abi.chunked_plan(1, 8, 65536, 128, 128, chunk=128)
     assert long_ctx["path"] == 0 and long_ctx["cooperative"] == 1
     assert long_ctx["segments"] == 18 and long_ctx["blocks"] == 144 <= long_ctx["resident"] == 148
+    # by default a single wave; runs of about 512 tokens: 512 chunks / (18 x 4) -> 7 waves
+    assert long_ctx["waves"] == 1
+    monkeypatch.setenv("TTT_LA_WAVE_TOKENS", "512")
+    assert abi.chunked_plan(1, 8, 65536, 128, 128, chunk=128)["waves"] == 7
+    long64 = abi.chunked_plan(1, 8, 65536, 128, 128, chunk=64)
+    assert long64["cooperative"] == 1 and long64["waves"] == 1024 // (18 * 8)
+    monkeypatch.delenv("TTT_LA_WAVE_TOKENS")
+    # the merged 64 x 64 tile keeps the decoupled look-back even for one long sequence
+    d64 = abi.chunked_plan(1, 1, 64 * 400, 64, 64, chunk=64)
+    assert d64["cooperative"] == 0 and d64["waves"] == 1
     mom = abi.chunked_plan(2, 16, 8192, 128, 128, chunk=128, beta=0.9, eta=True)
     assert mom["path"] == 1 and mom["tile"] == 64 and mom["cooperative"] == 1 and mom["blocks"] <= mom["resident"]
+    assert mom["waves"] == 1
     llm = abi.chunked_plan(4, 16, 4096, 64, 64, chunk=64, eta=True)  # short look-back: no waiting on peers
     assert llm["path"] == 0 and llm["cooperative"] == 0 and llm["segments"] == 4 and llm["resident"] == 296
     # a grid beyond one wave never waits on peers
@@ -279,6 +290,20 @@ def test_chunked_plan_launch_modes(abi):
     assert f32["path"] == 2 and f32["blocks"] == 2
     with pytest.raises(abi.TttError):
         abi.chunked_plan(1, 8, 1024, 96, 96, chunk=64)
+
+
+def test_debug_build_exports_the_same_abi(abi):
+    """The debug build (-DTTT_LA_DEBUG) exports every declared symbol and says
+    it checks; the release build compiles the checks away (line query -1)."""
+    from test_layers_causal_b200.build import DEBUG_OUT, build
+    build(out=DEBUG_OUT, debug=True)
+    D = abi.debug_lib()
+    for n in declared_functions():
+        assert hasattr(D, n), n
+    assert b"debug checks" in D.ttt_la_version() and b"debug" not in abi.lib().ttt_la_version()
+    assert abi.lib().ttt_la_debug_check_line(None) == -1
+    assert D.ttt_la_status_string(abi.ERR_DEVICE_CHECK) == abi.lib().ttt_la_status_string(6)
+    assert b"bounds check" in D.ttt_la_status_string(6)
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -1,0 +1,69 @@
+"""The debug build (libttt_la_debug.so, compiled with -DTTT_LA_DEBUG) on tiny,
+ragged shapes through the C ABI: every hand-indexed access of the chunked
+kernels to the workspace, flags and states is checked against the sizes of
+the call, and a failed check would record TTT_LA_ERR_DEVICE_CHECK and its
+source line instead of touching memory.  Each case covers one scratch
+layout -- one segment (none), the decoupled look-back, the wave schedule,
+and momentum with its look-back and its cooperative prefix -- and must leave
+a clean status word, a clean check line and outputs within the bf16
+tolerance of the float64 oracle."""
+import ctypes
+import math
+
+import pytest
+import torch
+
+from synth import make_qkv
+from tests.gpu_util import assert_bf16, oracle_forward
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, H, T, d, seed):
+    q, k, v, z = make_qkv((B, H), T, d, d, seed)
+    eta = (torch.sigmoid(z) / math.sqrt(d)).float()
+    return [x.cuda().contiguous() for x in (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), eta)]
+
+
+# (d, chunk, B, H, T, segments, beta, wave tokens): ragged T everywhere
+CASES = [
+    (64, 64, 1, 2, 100, 1, 0.0, 0),           # one segment: no scratch
+    (64, 64, 2, 3, 64 * 9 + 5, 3, 0.0, 0),    # look-back, merged 64 x 64 tiles
+    (128, 128, 1, 2, 128 * 7 + 9, 4, 0.0, 0), # look-back, 128-wide tiles
+    (128, 128, 1, 2, 128 * 36 - 1, 6, 0.0, 128),  # wave schedule, six waves
+    (128, 64, 1, 2, 64 * 30 + 3, 6, 0.0, 64),     # wave schedule, 64-token tiles
+    (64, 128, 1, 3, 128 * 45 - 7, 14, 0.0, 128),  # wave schedule, d = 64
+    (128, 64, 1, 2, 64 * 9 + 1, 3, 0.9, 0),   # momentum, cooperative prefix
+    (64, 64, 16, 16, 64 * 3 + 2, 2, 0.9, 0),  # momentum, look-back (grid beyond one wave)
+]
+
+
+@pytest.mark.parametrize("d,chunk,B,H,T,segments,beta,wave_tokens", CASES)
+def test_debug_build_checks_stay_clean(d, chunk, B, H, T, segments, beta, wave_tokens, monkeypatch):
+    from test_layers_causal_b200 import _abi
+    if wave_tokens:
+        monkeypatch.setenv("TTT_LA_WAVE_TOKENS", str(wave_tokens))
+    L = _abi.debug_lib()
+    assert b"debug checks" in L.ttt_la_version()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    L.ttt_la_debug_check_line(st)  # clear whatever an earlier call left
+    L.ttt_la_get_last_device_status(st)
+    q, k, v, eta = _inputs(B, H, T, d, 300 + d + T)
+    S0 = 0.1 * torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(5)).cuda()
+    M0 = 0.1 * torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(6)).cuda() if beta else None
+    o = torch.empty_like(v)
+    S = S0.clone()  # in place: state_out == state_in
+    M = M0.clone() if beta else None
+    a = _abi._seq_args(q, k, v, eta, None, beta, False, chunk, segments, S, M, o, S, M)
+    need = int(L.ttt_la_workspace_size(ctypes.byref(a)))
+    ws = torch.full((max(need, 16),), 0x7F, dtype=torch.uint8, device="cuda")  # stale-looking scratch
+    a.workspace, a.workspace_bytes = ws.data_ptr(), need
+    code = L.ttt_la_forward_chunked(ctypes.byref(a), st)
+    assert code == 0, _abi.status_string(code)
+    assert L.ttt_la_get_last_device_status(st) == _abi.OK
+    assert L.ttt_la_debug_check_line(st) == 0
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, 1.0 / math.sqrt(d), beta, False, S0, M0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+    if beta:
+        assert_bf16(M, M_ref, "momentum")

@@ -145,6 +145,70 @@ def test_chunked_tc_many_segments(d, chunk, segments, with_state):
     assert_bf16(S, S_ref, "state")
 
 
+@pytest.mark.parametrize("d,chunk,segments", [(128, 128, 6), (128, 64, 6), (64, 128, 14)])
+@pytest.mark.parametrize("runs_of", [1, 2])
+@pytest.mark.parametrize("token_eta", [True, False])
+def test_chunked_tc_waves(d, chunk, segments, runs_of, token_eta, monkeypatch):
+    """The wave schedule: several waves of `segments` runs of one or two chunks
+    (ragged splits, a ragged last chunk), starting from W_0, including the
+    wave-end state carried between waves and the final state of the last
+    scan."""
+    monkeypatch.setenv("TTT_LA_WAVE_TOKENS", str(runs_of * chunk))
+    B, H, T = 1, 3, segments * 7 * chunk - 29
+    plan = ttt.chunked_plan(B, H, T, d, d, chunk=chunk, segments=segments, eta=token_eta)
+    assert plan["cooperative"] == 1 and plan["waves"] >= (3 if runs_of == 1 else 2), plan
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 140 + d + chunk + runs_of, token_eta)
+    S0 = _state(B, H, d, d, 15, scale=0.1)
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, eta_const=ec, chunk=chunk, segments=segments, state_in=S0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec, 0.0, False, S0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+
+
+@pytest.mark.parametrize("d,chunk,segments,waves", [(128, 128, 6, True), (128, 128, 3, False), (64, 64, 4, False)])
+def test_chunked_tc_state_in_place(d, chunk, segments, waves, monkeypatch):
+    """state_out may be state_in: W_T overwrites W_0 only after every block has
+    read it (wave schedule over five waves, and decoupled look-back)."""
+    monkeypatch.setenv("TTT_LA_WAVE_TOKENS", str(chunk))
+    B, H, T = 1, 2, segments * 5 * chunk - 3
+    plan = ttt.chunked_plan(B, H, T, d, d, chunk=chunk, segments=segments, eta=True)
+    assert plan["cooperative"] == int(waves) and plan["waves"] == (5 if waves else 1)
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 160 + d + segments)
+    S0 = _state(B, H, d, d, 16, scale=0.1)
+    Sx = S0.clone()
+    o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=chunk, segments=segments, state_in=Sx, state_out=Sx)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0 and S.data_ptr() == Sx.data_ptr()
+    o_ref, S_ref, _ = oracle_forward(q, k, v, eta, ec, 0.0, False, S0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(Sx, S_ref, "state")
+
+
+@pytest.mark.parametrize("H,segments", [(2, 3), (40, 2)])
+def test_chunked_tc_momentum_state_in_place(H, segments):
+    """With momentum, W_T and M_T may overwrite W_0 and M_0: cooperative
+    prefix (H = 2, one wave) and decoupled look-back (H = 40: 80 blocks of
+    one per SM would fit, so force a grid beyond one wave with d = 128 and
+    B = 2)."""
+    B, d, T = 2, 128, 64 * 7 + 5
+    plan = ttt.chunked_plan(B, H, T, d, d, chunk=64, beta=0.9, segments=segments, eta=True)
+    assert plan["cooperative"] == (1 if plan["blocks"] <= plan["resident"] else 0)
+    q, k, v, eta, ec = _case(B, H, T, d, d, "bf16", 170 + H)
+    S0 = _state(B, H, d, d, 17, scale=0.1)
+    M0 = _state(B, H, d, d, 18, scale=0.1)
+    Sx, Mx = S0.clone(), M0.clone()
+    o, _, _ = ttt.forward_chunked(q, k, v, eta, beta=0.9, chunk=64, segments=segments, state_in=Sx, mom_in=Mx,
+                                  state_out=Sx, mom_out=Mx)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, M_ref = oracle_forward(q, k, v, eta, ec, 0.9, False, S0, M0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(Sx, S_ref, "state")
+    assert_bf16(Mx, M_ref, "momentum")
+
+
 @pytest.mark.parametrize("d,chunk", [(64, 64), (128, 128)])
 def test_chunked_tc_ascent_zero_state_and_exact_multiple(d, chunk):
     B, H, T = 1, 2, 4 * chunk
@@ -267,11 +331,16 @@ def _full_case(name, heads):
     return c, x, q, k, v, eta, heads
 
 
-@pytest.mark.parametrize("name,heads", [("llm_d64", [(0, 0), (3, 15), (1, 7)]), ("long_d128", [(0, 0), (0, 5)]),
-                                        ("momentum_d128", [(0, 0), (1, 9)])])
-def test_full_size_sampled_heads(name, heads):
+@pytest.mark.parametrize("name,chunk,heads", [("llm_d64", 64, [(0, 0), (3, 15), (1, 7)]),
+                                              ("long_d128", 128, [(0, 0), (0, 5)]),
+                                              ("long_d128", 64, [(0, 2), (0, 7)]),
+                                              ("momentum_d128", 128, [(0, 0), (1, 9)])])
+def test_full_size_sampled_heads(name, chunk, heads):
+    """The workloads at full size, in the launch configuration the benchmark
+    times (automatic segments and schedule), on sampled heads against the
+    oracle over the whole sequence."""
     c, x, q, k, v, eta, heads = _full_case(name, heads)
-    o, S, M = ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=c.chunk)
+    o, S, M = ttt.forward_chunked(q, k, v, eta, eta_const=x["eta_const"], beta=c.beta, chunk=chunk)
     torch.cuda.synchronize()
     assert ttt.device_status() == 0
     for b, h in heads:
@@ -285,11 +354,15 @@ def test_full_size_sampled_heads(name, heads):
 
 
 @pytest.mark.parametrize("chunk", [64, 128])
-def test_long_context_chunk_sweep_consistent(chunk):
-    """The long-context workload at every swept chunk size gives the same layer."""
+def test_long_context_schedules_agree(chunk):
+    """Property at full size (all 8 heads): the benchmark's cooperative
+    schedule and a single sequential pass per head (one segment) give the
+    same layer."""
     c, x, q, k, v, eta, _ = _full_case("long_d128", [])
+    plan = ttt.chunked_plan(c.B, c.H, c.T, c.d_k, c.d_v, chunk=chunk)
+    assert plan["cooperative"] == 1
     o, S, _ = ttt.forward_chunked(q, k, v, None, eta_const=x["eta_const"], chunk=chunk)
-    o_ref, S_ref, _ = ttt.forward_chunked(q, k, v, None, eta_const=x["eta_const"], chunk=128, segments=1)
+    o_ref, S_ref, _ = ttt.forward_chunked(q, k, v, None, eta_const=x["eta_const"], chunk=chunk, segments=1)
     assert (o.float() - o_ref.float()).norm() / o_ref.float().norm() < 1e-2
     assert (S - S_ref).norm() / S_ref.norm() < 1e-2
 
