@@ -101,7 +101,11 @@ struct TcCfg {
   static constexpr int PBUF = PSEP ? C * C * 2 : 0;
   static constexpr int SBF_LO = SPLIT ? D * D * 2 : 0;       // bf16 residual of W (split readout)
   static constexpr int BIG = NST * STAGE + SBF + PBUF + SBF_LO;
-  static constexpr int NBAR = 4 * NST + 12;
+  // The 128 x 128 tile streams phase A through three K/V slots (A3): the two
+  // stages' K and V regions and a third made of their Q regions, which phase
+  // A leaves idle; they have barriers of their own.
+  static constexpr bool A3 = (C == 128 && D == 128);
+  static constexpr int NBAR = 4 * NST + 12 + (A3 ? 9 : 0);
   static constexpr int SMALL = NBAR * 8 + NST * C * 4 + 32;
   static constexpr int SMEM = BIG + SMALL + 1024;            // + alignment slack
   // W, O x 2 and the scores, which phase A's D-column total shares: C + 3D
@@ -291,6 +295,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
   uint64_t* drain = sc_full + 8;        // final MMA drain
   uint64_t* adone = sc_full + 9;        // a run's phase-A total complete in TMEM
   uint64_t* a_read = sc_full + 10;      // that total read out of TMEM (its columns free again)
+  uint64_t* fullA = sc_full + 11;       // [3] phase-A slot landed (A3)
+  uint64_t* kreadyA = sc_full + 14;     // [3] its K scaled
+  uint64_t* emptyA = sc_full + 17;      // [3] slot free
   float* es = reinterpret_cast<float*>(smem + Cfg::BIG + Cfg::NBAR * 8);  // [NST][C] sigma*eta
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(es + NST * C);
   int* sh_tile = reinterpret_cast<int*>(tmem_holder + 1);
@@ -317,6 +324,12 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
     mbar_init(drain, 1);
     mbar_init(adone, 1);
     mbar_init(a_read, 128);
+    if constexpr (Cfg::A3)
+      for (int x = 0; x < 3; ++x) {
+        mbar_init(&fullA[x], 1);
+        mbar_init(&kreadyA[x], 1);
+        mbar_init(&emptyA[x], 1);
+      }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -358,6 +371,15 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
   auto t_o_of = [&](int b) -> uint32_t {  // O[b]: D columns, M = C
     return Cfg::MRG ? (b ? tmem + D : tmem + 2 * D + C) : SC_LAST ? tmem + D + b * D : tmem + D + C + b * D;
   };
+  // Three phase-A slots (A3 tile, when every phase-A chunk of the block comes
+  // before its phase-B ones: a single wave).  Phase-A chunk ia goes to slot
+  // ia % 3: slot x < 2 is stage x's K and V regions, slot 2 keeps K in stage
+  // 0's Q region and V in stage 1's.  Phase-B chunk itb then uses stage
+  // itb % NST, whose first use waits for the phase-A slots it overlaps.
+  const bool a3 = Cfg::A3 && p.nwave == 1;
+  const int nA0 = tc_span_a(p, seg, 0).n;  // the block's phase-A chunks (a single wave)
+  auto a_koff = [](int x) { return x == 2 ? 0 : x * STAGE + Cfg::OK; };
+  auto a_voff = [](int x) { return x == 2 ? STAGE : x * STAGE + Cfg::OV; };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -370,15 +392,36 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       // beside the streams), the rest evict-first.
       const uint64_t pol_once = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
-      int g = 0, itb = 0;
+      int g = 0, itb = 0, ia = 0;
       TcCursor cur;
       for (cur.init(p, seg); cur.valid(p); cur.next(p, seg), ++g) {
-        const int s = g % NST;
-        if (g >= NST && !dead) dead = !mbar_wait(&empty[s], ((g / NST) - 1) & 1, lim);
         const bool pb = cur.is_b();
         const int t0 = cur.chunk() * C;
         TTT_EXPECT(cur.chunk() >= 0 && cur.chunk() < p.nchunks);
         const uint64_t pol_kv = (!pb && cur.chunk() - cur.A.c0 < p.keep) ? pol_keep : pol_once;
+        if (a3 && !pb) {
+          const int x = ia % 3, u = ia / 3;
+          if (u > 0 && !dead) dead = !mbar_wait(&emptyA[x], (u - 1) & 1, lim);
+          mbar_arrive_expect_tx(&fullA[x], 2 * TILE);
+#pragma unroll
+          for (int kb = 0; kb < D / 64; ++kb) {
+            tma_load_3d_hint(&tmK, &fullA[x], smem + a_koff(x) + kb * C * 128, kb * 64, t0, bh, pol_kv);
+            tma_load_3d_hint(&tmV, &fullA[x], smem + a_voff(x) + kb * C * 128, kb * 64, t0, bh, pol_kv);
+          }
+          ++ia;
+          continue;
+        }
+        const int s = (a3 ? itb : g) % NST, u = (a3 ? itb : g) / NST;
+        if (a3 && u == 0) {
+          // first use of stage s: the phase-A slots on it (slot s; slot 2 in the Q regions) are free
+          const int on_stage[2] = {s, 2};
+          for (int i = 0; i < 2; ++i) {
+            const int x = on_stage[i], uses = nA0 / 3 + (x < nA0 % 3 ? 1 : 0);
+            if (uses > 0 && !dead) dead = !mbar_wait(&emptyA[x], (uses - 1) & 1, lim);
+          }
+        } else if (u > 0 && !dead) {
+          dead = !mbar_wait(&empty[s], (u - 1) & 1, lim);
+        }
         mbar_arrive_expect_tx(&full[s], pb ? 3 * TILE : 2 * TILE);
         uint8_t* st = smem + s * STAGE;
 #pragma unroll
@@ -391,7 +434,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         }
         if (pb) ++itb;
       }
-      for (int j = max(0, g - NST); j < g; ++j) mbar_wait(&full[j % NST], (j / NST) & 1, lim);
+      const int nst_items = a3 ? itb : g;  // loads on the stage barriers
+      for (int j = max(0, nst_items - NST); j < nst_items; ++j) mbar_wait(&full[j % NST], (j / NST) & 1, lim);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
@@ -406,7 +450,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       const uint64_t d_wbf = sdesc_sw128(sbase + NST * STAGE, 16, 1024);
       const uint64_t d_pbuf = sdesc_sw128(sbase + NST * STAGE + Cfg::SBF, 16, 1024);
       const uint64_t d_wlo = sdesc_sw128(sbase + NST * STAGE + Cfg::SBF + Cfg::PBUF, 16, 1024);
-      int g = 0, itb = 0, nread = 0;
+      int g = 0, itb = 0, nread = 0, ia = 0;
       bool pending_read = false;  // a phase-A total sits in the score columns, not yet read out
       auto free_scores = [&]() {
         if (pending_read) {
@@ -417,18 +461,20 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       };
       TcCursor cur;
       for (cur.init(p, seg); cur.valid(p); cur.next(p, seg), ++g) {
-        const int s = g % NST;
         if (!cur.is_b()) {
           // phase A: T (+)= V^T K~ into the score columns
-          const uint32_t stk = sbase + s * STAGE + Cfg::OK, stv = sbase + s * STAGE + Cfg::OV;
+          const int x = ia % 3, s = g % NST;
+          const uint32_t stk = a3 ? sbase + a_koff(x) : sbase + s * STAGE + Cfg::OK;
+          const uint32_t stv = a3 ? sbase + a_voff(x) : sbase + s * STAGE + Cfg::OV;
           const uint64_t dkm = sdesc_sw128(stk, Cfg::KWR * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
           if (cur.k == 0) free_scores();
-          if (!dead) dead = !mbar_wait(&kready[s], (g / NST) & 1, lim);
+          if (!dead) dead = !mbar_wait(a3 ? &kreadyA[x] : &kready[s], ((a3 ? ia / 3 : g / NST)) & 1, lim);
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk)
             mma_bf16_ss(t_a, dvm + mn_step(kk), dkm + mn_step(kk), ID_W, (cur.k > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&empty[s]);
+          tc_commit(a3 ? &emptyA[x] : &empty[s]);
+          ++ia;
           if (cur.k == cur.A.n - 1) {
             tc_commit(adone);
             pending_read = true;
@@ -436,14 +482,14 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
           continue;
         }
         // phase B
-        const int b = itb & 1;
+        const int b = itb & 1, s = (a3 ? itb : g) % NST, u = (a3 ? itb : g) / NST;
         const uint32_t stq = sbase + s * STAGE, stk = stq + Cfg::OK, stv = stq + Cfg::OV;
         const uint64_t dq = sdesc_sw128(stq, 16, 1024), dkk = sdesc_sw128(stk, 16, 1024);
         const uint64_t dkm = sdesc_sw128(stk + krow_of(true, itb) * 128, Cfg::KWR * 128, 1024);
         const uint64_t dvm = sdesc_sw128(stv, C * 128, 1024);
         const uint64_t dp = Cfg::PSEP ? d_pbuf : dq;
         const uint32_t t_o = t_o_of(b);
-        if (!dead) dead = !mbar_wait(&kready[s], (g / NST) & 1, lim);
+        if (!dead) dead = !mbar_wait(&kready[s], u & 1, lim);
         free_scores();
         if (Cfg::MRG) {
           // [Sc | O] in one N = C + D MMA: needs this chunk's Wbf and a free O[b]
@@ -494,7 +540,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       TcCursor cur;
       for (cur.init(p, seg); cur.valid(p); cur.next(p, seg), ++g) {
         if (!cur.is_b()) continue;
-        const int s = g % NST;
+        const int s = (a3 ? itb : g) % NST;
         if (!dead) dead = !mbar_wait(&staged[itb % NST], (itb / NST) & 1, lim);
         if constexpr (!SPLIT) {  // the split readout's epilogue wrote O itself
           const uint8_t* sv = smem + s * STAGE + Cfg::OV;
@@ -535,10 +581,15 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
     if (ahead.valid(p)) ahead.next(p, seg);
     constexpr int PER_LANE = C * (D / 8) / 32;  // 16-byte units of the K tile per lane
     constexpr int BATCH = 8;
-    int g = 0, itb = 0;
+    int g = 0, itb = 0, ia = 0;
     for (; cur.valid(p); cur.next(p, seg), ++g) {
-      const int s = g % NST;
       const bool pb = cur.is_b();
+      const bool slotA = a3 && !pb;  // a three-slot phase-A chunk
+      const int x = ia % 3;
+      const int s = slotA ? x % NST : (a3 ? itb : g) % NST;
+      const int u = slotA ? ia / 3 : (a3 ? itb : g) / NST;
+      uint64_t* fb = slotA ? &fullA[x] : &full[s];
+      uint64_t* kb_ready = slotA ? &kreadyA[x] : &kready[s];
       float* ess = es + s * C;
 #pragma unroll
       for (int j = 0; j < RPL; ++j) ess[lane + 32 * j] = p.sigma * er[j];
@@ -547,8 +598,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       fetch(ahead, en);
       if (ahead.valid(p)) ahead.next(p, seg);
       __syncwarp();
-      if (!dead) dead = !mbar_wait(&full[s], (g / NST) & 1, lim);
-      uint8_t* sk = smem + s * STAGE + Cfg::OK + krow_of(pb, itb) * 128;
+      if (!dead) dead = !mbar_wait(fb, u & 1, lim);
+      uint8_t* sk = slotA ? smem + a_koff(x) : smem + s * STAGE + Cfg::OK + krow_of(pb, itb) * 128;
 #pragma unroll 1
       for (int b0 = 0; b0 < PER_LANE; b0 += BATCH) {
         uint4 u[BATCH];
@@ -576,8 +627,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&kready[s]);
+      if (lane == 0) mbar_arrive(kb_ready);
       if (pb) ++itb;
+      if (slotA) ++ia;
     }
   } else {
     // --------------------------------------------------------- epilogue --
@@ -896,7 +948,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
 
       // ---------------------------------------------------------- phase B
       for (int j = 0; j < Bs.n; ++j, ++itb) {
-        const int g = gb0 + j, s = g % NST, b = itb & 1;
+        const int g = gb0 + j, s = (a3 ? itb : g) % NST, b = itb & 1;
         uint8_t* st = smem + s * STAGE;
         // P = bf16(tril(scores)) into the Q (and K) slots
         {

@@ -318,9 +318,11 @@ SegPlan plan_segments(const ttt_la_args* a) {
     const int per_run = std::max(1, wave_tokens() / C);
     s.nwave = std::max(1, std::min(s.nchunks / (s.nseg * per_run), s.nchunks / s.nseg));
   }
-  if (a->beta == 0.f && s.nseg > 1) {
+  if (a->beta == 0.f && s.nseg > 1 && !tile64) {
     // K and V phase B reads first, kept in L2 from phase A: about l2_keep_mb
-    // MB over the whole grid (beside the Q, O and scratch streams)
+    // MB over the whole grid (beside the Q, O and scratch streams).  Measured
+    // on the 128-wide tiles only: on 64 x 64 tiles, whose K and V of a whole
+    // call already fit in L2 at the LLM shape, the hint was slower.
     const size_t chunk_kv = static_cast<size_t>(C) * (a->d_k + a->d_v) * 2;
     const size_t blocks = static_cast<size_t>(bh) * s.nseg;
     s.keep = static_cast<int>(std::min<size_t>(static_cast<size_t>(l2_keep_mb()) << 20, size_t(1) << 40) /
