@@ -75,8 +75,13 @@ struct TcParams {
   float* S_out;                   // [BH, dv, dk] final state or nullptr
   float* o32;                     // split readout: O in fp32 [BH, T, dv] (the bf16 O map is unused)
   uint64_t limit_ns;
-  size_t ws_floats;               // floats of scratch before the flags (bounds of the debug checks)
-  unsigned flag_words;            // words of flags and counters
+  // Scratch bounds of the debug checks, from the sizes above (kept out of the
+  // parameter struct, which a few bytes more made measurably slower in the
+  // momentum kernel).
+  __device__ __forceinline__ size_t ws_floats_of(int D) const {
+    return static_cast<size_t>(BH) * (2 * nseg + (coop ? 1 : 0)) * static_cast<size_t>(D) * D;
+  }
+  __device__ __forceinline__ size_t flag_words_of() const { return static_cast<size_t>(BH) * nseg + 1 + BH; }
 };
 
 // SPLIT (the backward's passes): the state is read out as bf16(W) +
@@ -537,6 +542,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
     if (lane == 0) {
       bool dead = false;
       int g = 0, itb = 0;
+      const uint64_t pol_out = l2_policy_evict_first();
       TcCursor cur;
       for (cur.init(p, seg); cur.valid(p); cur.next(p, seg), ++g) {
         if (!cur.is_b()) continue;
@@ -545,8 +551,10 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         if constexpr (!SPLIT) {  // the split readout's epilogue wrote O itself
           const uint8_t* sv = smem + s * STAGE + Cfg::OV;
           const int t0 = cur.chunk() * C;
+          // O is not read again: evict-first, so that it does not push out
+          // the K and V phase B still reads from L2
 #pragma unroll
-          for (int kb = 0; kb < D / 64; ++kb) tma_store_3d(&tmO, sv + kb * C * 128, kb * 64, t0, bh);
+          for (int kb = 0; kb < D / 64; ++kb) tma_store_3d_hint(&tmO, sv + kb * C * 128, kb * 64, t0, bh, pol_out);
           bulk_commit();
           bulk_wait_read0();
         }
@@ -718,7 +726,11 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       tmem_st_wait();
     };
 
-    for (int it = 0; it <= p.nwave; ++it) {
+    // (the merged 64 x 64 tile always runs one wave: a constant trip count
+    // lets the compiler lay its two iterations out straight)
+    const int nwave = Cfg::MRG ? 1 : p.nwave;
+#pragma unroll(Cfg::MRG ? 2 : 1)
+    for (int it = 0; it <= nwave; ++it) {
       const TcSpan A = tc_span_a(p, seg, it), Bs = tc_span_b(p, seg, it);
       const int gb0 = g0 + A.n;  // tile index of the first phase-B chunk
       g0 += A.n + Bs.n;
@@ -726,9 +738,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         // ================================================ wave schedule ==
         const int P = p.nseg;
         float4* ws4 = reinterpret_cast<float4*>(p.ws);
-        const size_t DD4 = DD / 4, ws4n = p.ws_floats / 4;
-        unsigned* wflag = TTT_AT(p.flags, static_cast<size_t>(bh) * P, P, p.flag_words);  // [P] published-wave counts
-        unsigned* cnt = TTT_AT(p.flags, static_cast<size_t>(p.BH) * P + 1 + bh, 1, p.flag_words);
+        const size_t DD4 = DD / 4, ws4n = p.ws_floats_of(D) / 4;
+        unsigned* wflag = TTT_AT(p.flags, static_cast<size_t>(bh) * P, P, p.flag_words_of());  // [P] published-wave counts
+        unsigned* cnt = TTT_AT(p.flags, static_cast<size_t>(p.BH) * P + 1 + bh, 1, p.flag_words_of());
         auto tot4 = [&](int slot, int j) {
           return TTT_AT(ws4, ((static_cast<size_t>(bh) * 2 + slot) * P + j) * DD4, DD4, ws4n);
         };
@@ -826,18 +838,18 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         // publish this segment's total (its state leaves t_a only once the
         // inclusive state is out, in iteration 1)
         if (A.n > 0) {
-          float* agg_me = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + seg) * 2 * DD, DD, p.ws_floats);
+          float* agg_me = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + seg) * 2 * DD, DD, p.ws_floats_of(D));
           publish_total(agg_me, false);
           __threadfence();
           asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (et == 0) st_release(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + seg, 1, p.flag_words), 1u);
+          if (et == 0) st_release(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + seg, 1, p.flag_words_of()), 1u);
         }
       } else {
         // W_start = W_0 + the totals of the segments after the nearest
         // predecessor that has published its inclusive state (start + total).
         // One thread per predecessor reads the flags.
         const bool hasA = tc_span_a(p, seg, 0).n > 0;
-        float* agg_me = hasA ? TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + seg) * 2 * DD, 2 * DD, p.ws_floats)
+        float* agg_me = hasA ? TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + seg) * 2 * DD, 2 * DD, p.ws_floats_of(D))
                              : nullptr;
         const float* base = p.S_in ? TTT_AT(p.S_in, bh * DD, DD, static_cast<size_t>(p.BH) * DD) : nullptr;
         int first = 0;
@@ -847,14 +859,14 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
           asm volatile("bar.sync 1, 128;" ::: "memory");
           for (int j = et; j < seg; j += 128) {
             const unsigned f =
-                dead ? 1u : wait_geq(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + j, 1, p.flag_words), 1u, lim);
+                dead ? 1u : wait_geq(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + j, 1, p.flag_words_of()), 1u, lim);
             if (f == 0) dead = true;
             if (f >= 2) atomicMax(&sh_lb[1], j);
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
           const int incl = sh_lb[1];
           if (incl >= 0) {
-            base = TTT_AT(p.ws, ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD, DD, p.ws_floats);
+            base = TTT_AT(p.ws, ((static_cast<size_t>(bh) * p.nseg + incl) * 2 + 1) * DD, DD, p.ws_floats_of(D));
             base_qm = true;
           }
           first = incl + 1;
@@ -882,7 +894,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
               float8 x[NR][4];
 #pragma unroll
               for (int u = 0; u < NR; ++u) {
-                const float* ag = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD, DD, p.ws_floats);
+                const float* ag = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + jj + u) * 2 * DD, DD, p.ws_floats_of(D));
 #pragma unroll
                 for (int j = 0; j < 4; ++j) x[u][j] = ld_cg_f8_qm<D>(ag, wrow, cb * 8 + 2 * j);
               }
@@ -894,7 +906,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
                   for (int e = 0; e < 8; ++e) acc[8 * j + e] += x[u][j].v[e];
             }
             for (; jj < seg; ++jj) {
-              const float* ag = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD, DD, p.ws_floats);
+              const float* ag = TTT_AT(p.ws, (static_cast<size_t>(bh) * p.nseg + jj) * 2 * DD, DD, p.ws_floats_of(D));
               float8 x[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) x[j] = ld_cg_f8_qm<D>(ag, wrow, cb * 8 + 2 * j);
@@ -939,7 +951,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
           mbar_arrive(a_read);  // the score columns are free for phase B
           __threadfence();
           asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (et == 0) st_release(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + seg, 1, p.flag_words), 2u);
+          if (et == 0) st_release(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + seg, 1, p.flag_words_of()), 2u);
         }
         fence_async_smem();
         tc_fence_before();
@@ -1115,7 +1127,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       // W_T may overwrite W_0 (in place): first every predecessor must have
       // read W_0, which it has once its inclusive state is out (flag 2)
       for (int j = et; j < seg; j += 128)
-        if (!dead && wait_geq(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + j, 1, p.flag_words), 2u, lim) == 0)
+        if (!dead && wait_geq(TTT_AT(p.flags, static_cast<size_t>(bh) * p.nseg + j, 1, p.flag_words_of()), 2u, lim) == 0)
           dead = true;
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (!dead) dead = !mbar_wait(sdone, (itb - 1) & 1, lim);

@@ -395,13 +395,9 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
   p.S_out = a->state_out;
   p.o32 = o32;
   p.limit_ns = g_limit_ns;
-  p.ws_floats = 0;
-  p.flag_words = 0;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
-    p.ws_floats = tc_ws_floats(bh, sp.nseg, D, sp.coop);
-    p.flag_words = static_cast<unsigned>(tc_flag_words(bh, sp.nseg));
-    p.flags = reinterpret_cast<unsigned*>(p.ws + p.ws_floats);
+    p.flags = reinterpret_cast<unsigned*>(p.ws + tc_ws_floats(bh, sp.nseg, D, sp.coop));
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
@@ -487,12 +483,8 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
   p.M_out = a->mom_out;
   p.limit_ns = g_limit_ns;
   p.coop = sp.coop ? 1 : 0;
-  p.ws_floats = 0;
-  p.flag_words = 0;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
-    p.ws_floats = tcm_ws_floats(bh, sp.nseg, D);
-    p.flag_words = static_cast<unsigned>(tc_flag_words(bh, sp.nseg));
     p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;
     p.flags = reinterpret_cast<unsigned*>(p.ws + tcm_ws_floats(bh, sp.nseg, D));
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
