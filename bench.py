@@ -440,8 +440,10 @@ def backward_measure(ttt, dev, peaks, reps=5):
     """The layer's backward on the llm_d64 inputs (B4 H16 T4096 d64, per-token
     eta) with a seeded upstream gradient dL/do and dL/dW_T: dq, dk, dv,
     per-token deta and dW0, in both forms -- the recurrent kernel (one block
-    per head) and the chunk-parallel one (three chunked forward runs).  CUDA
-    events over `reps` calls after one warm-up call of each."""
+    per head) and the chunk-parallel one (a transpose of dL/dW_T and three
+    chunked forward runs, the two reverse-time ones writing dv, deta and dk
+    themselves: four launches).  CUDA events over `reps` calls after one
+    warm-up call of each."""
     c = CONFIGS["llm_d64"]
     x = make_case(c)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
@@ -475,7 +477,7 @@ def backward_measure(ttt, dev, peaks, reps=5):
         gbs = nbytes / (us * 1e-6) / 1e9
         out[name] = {"us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6), "hbm_gbs": gbs,
                      "hbm_frac": gbs / peaks["hbm_gbs"],
-                     "gpu_launches_per_call": 1 if name == "recurrent" else 7}
+                     "gpu_launches_per_call": 1 if name == "recurrent" else 4}
     out["chunked_speedup_over_recurrent"] = out["recurrent"]["us_per_call"] / out["chunked"]["us_per_call"]
     torch.cuda.empty_cache()
     return out

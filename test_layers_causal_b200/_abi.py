@@ -419,11 +419,9 @@ def backward_recurrent(q, k, v, grad_o, eta=None, eta_const=None, beta=0.0, asce
     return out
 
 
-def backward_chunked(q, k, v, grad_o, eta=None, eta_const=None, ascent=False, state_in=None, grad_state=None,
-                     workspace=None, stream=None):
-    """Gradients of the layer without momentum from three chunked forward runs
-    (ttt_la_backward_chunked): returns a dict with dq, dk, dv (dtype of q),
-    deta [B,H,T] fp32 (per token) and dW0 [B,H,d_v,d_k] fp32."""
+def _chunked_grad_args(q, k, v, grad_o, eta, eta_const, ascent, state_in, grad_state):
+    """The TttGradArgs of ttt_la_backward_chunked and the output tensors it
+    points at (no workspace yet)."""
     _check_shapes(q, k, v, eta, state_in, None)
     if grad_o.shape != v.shape or grad_o.dtype != v.dtype:
         raise ValueError("grad_o must match v")
@@ -431,7 +429,7 @@ def backward_chunked(q, k, v, grad_o, eta=None, eta_const=None, ascent=False, st
     dv = v.shape[-1]
     if grad_state is not None and (grad_state.shape != (B, H, dv, dk) or grad_state.dtype != torch.float32):
         raise ValueError("grad_state must be fp32 [B,H,d_v,d_k]")
-    _need_cuda(q, k, v, grad_o, eta, state_in, grad_state, workspace)
+    _need_cuda(q, k, v, grad_o, eta, state_in, grad_state)
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                deta=torch.empty(B, H, T, device=q.device, dtype=torch.float32),
                dW0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32))
@@ -443,6 +441,16 @@ def backward_chunked(q, k, v, grad_o, eta=None, eta_const=None, ascent=False, st
     a.state_in, a.grad_o, a.grad_state = _ptr(state_in), grad_o.data_ptr(), _ptr(grad_state)
     a.grad_q, a.grad_k, a.grad_v = out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr()
     a.grad_eta, a.grad_state_in = out["deta"].data_ptr(), out["dW0"].data_ptr()
+    return a, out
+
+
+def backward_chunked(q, k, v, grad_o, eta=None, eta_const=None, ascent=False, state_in=None, grad_state=None,
+                     workspace=None, stream=None):
+    """Gradients of the layer without momentum from three chunked forward runs
+    (ttt_la_backward_chunked): returns a dict with dq, dk, dv (dtype of q),
+    deta [B,H,T] fp32 (per token) and dW0 [B,H,d_v,d_k] fp32."""
+    _need_cuda(workspace)
+    a, out = _chunked_grad_args(q, k, v, grad_o, eta, eta_const, ascent, state_in, grad_state)
     L = lib()
     need = L.ttt_la_backward_chunked_workspace_size(ctypes.byref(a))
     if workspace is None or workspace.numel() * workspace.element_size() < need:

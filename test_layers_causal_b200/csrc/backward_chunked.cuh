@@ -3,7 +3,7 @@
 //
 // The gradient of the plain layer (update, then read; W_t = W_{t-1} +
 // sigma eta_t v_t k_t^T, o_t = W_t q_t) is three runs of the forward layer
-// itself, each computed by the chunked forward on the tensor cores:
+// itself, each computed by the chunked forward:
 //   dq_t = W_t^T do_t       the forward on (q, k, v) := (do, v, k) from W_0^T,
 //                           same eta and sigma;
 //   u_t  = G_t k_t          the forward on the time-reversed sequence of
@@ -12,9 +12,12 @@
 //   r_t  = G_t^T v_t        the same on (v, do, q) from (dL/dW_T)^T;
 // with G_t = dL/dW_T + sum_{t' >= t} do_t' q_t'^T.  Then
 //   dv_t = sigma eta_t u_t,  dk_t = sigma eta_t r_t,  deta_t = sigma v_t . u_t.
-// The kernels here reverse sequences along T, transpose states and apply
-// that last step.  (The gradient of "Test-Time Training with KV Binding Is
-// Secretly Linear Attention"'s layer, needed for the training of its
+// In bf16 the two reverse-time passes run on the tensor cores straight over
+// the inputs, chunks last to first with the anti-causal mask (chunked_tc.cuh,
+// BWD), and their epilogues apply that last step.  The fp32 path runs them
+// on copies reversed along T and applies it in a finishing kernel.  Both
+// transpose W_0 and dL/dW_T with the kernel here.  (The gradient of "Test-Time Training with KV Binding
+// Is Secretly Linear Attention"'s layer, needed for the training of its
 // Figure 4, thelatestinai.com listing.)
 #pragma once
 #include "common.cuh"
@@ -67,20 +70,20 @@ __global__ void __launch_bounds__(256) transpose_states_kernel(const TransposePa
 }
 
 // dv_t = sigma eta_t u_t, dk_t = sigma eta_t r_t, deta_t = sigma v_t . u_t,
-// with u and r stored in fp32 in reversed token order.  One warp per (b, h, t).
+// with u and r stored in fp32 in reversed token order (the fp32 path).  One
+// warp per (b, h, t).
 struct FinishParams {
   int BH, T, dk, dv;
   const float* u_rev; // [BH][T][dv]
   const float* r_rev; // [BH][T][dk]
-  const void* v;      // [BH][T][dv]
+  const float* v;     // [BH][T][dv]
   const float* eta;   // [BH][T] or nullptr
   float eta_const, sigma;
-  void* dk_out;       // [BH][T][dk]
-  void* dv_out;       // [BH][T][dv]
+  float* dk_out;      // [BH][T][dk]
+  float* dv_out;      // [BH][T][dv]
   float* deta;        // [BH][T] or nullptr
 };
 
-template <typename T>
 __global__ void __launch_bounds__(256) backward_finish_kernel(const FinishParams p) {
   const long long warp = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -91,16 +94,16 @@ __global__ void __launch_bounds__(256) backward_finish_kernel(const FinishParams
   const float s = p.sigma * (p.eta ? p.eta[fwd] : p.eta_const);
   const float* u = p.u_rev + rev * p.dv;
   const float* r = p.r_rev + rev * p.dk;
-  const T* v = static_cast<const T*>(p.v) + fwd * p.dv;
-  T* dv = static_cast<T*>(p.dv_out) + fwd * p.dv;
-  T* dk = static_cast<T*>(p.dk_out) + fwd * p.dk;
+  const float* v = p.v + fwd * p.dv;
+  float* dv = p.dv_out + fwd * p.dv;
+  float* dk = p.dk_out + fwd * p.dk;
   float vu = 0.f;
   for (int c = lane; c < p.dv; c += 32) {
     const float uc = u[c];
-    vu = fmaf(to_f(v[c]), uc, vu);
-    dv[c] = from_f<T>(s * uc);
+    vu = fmaf(v[c], uc, vu);
+    dv[c] = s * uc;
   }
-  for (int c = lane; c < p.dk; c += 32) dk[c] = from_f<T>(s * r[c]);
+  for (int c = lane; c < p.dk; c += 32) dk[c] = s * r[c];
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) vu += __shfl_xor_sync(0xffffffffu, vu, off);
   if (lane == 0 && p.deta) p.deta[fwd] = p.sigma * vu;

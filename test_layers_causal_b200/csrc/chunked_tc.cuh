@@ -73,7 +73,10 @@ struct TcParams {
   int keep;                       // phase A: K, V of a run's first `keep` chunks loaded evict-last (phase B reads
                                   // them first), the rest evict-first
   float* S_out;                   // [BH, dv, dk] final state or nullptr
-  float* o32;                     // split readout: O in fp32 [BH, T, dv] (the bf16 O map is unused)
+  // BWD only: rows [BH, T, dv] (bf16) dotted with O for the per-token
+  // learning-rate gradient deta [BH, T] (both nullptr: no deta)
+  const void* vdot;
+  float* deta;
   uint64_t limit_ns;
   // Scratch bounds of the debug checks, from the sizes above (kept out of the
   // parameter struct, which a few bytes more made measurably slower in the
@@ -84,10 +87,16 @@ struct TcParams {
   __device__ __forceinline__ size_t flag_words_of() const { return static_cast<size_t>(BH) * nseg + 1 + BH; }
 };
 
-// SPLIT (the backward's passes): the state is read out as bf16(W) +
-// bf16(W - bf16(W)), two MMAs whose sum carries W to about 2^-17, and O is
-// written in fp32 straight from TMEM to `o32` instead of through TMA.
-template <int C, int D, bool SPLIT = false>
+// BWD (the backward's two reverse-time passes, see backward_chunked.cuh):
+// the chunks are walked last to first (logical chunk c is chunk N-1-c of the
+// sequence) with the anti-causal mask j >= i inside a chunk, so the state
+// carried in is the sum over the later tokens; K is used unscaled (the pass
+// runs with eta = 1, sigma = +1, so `eta`, `eta_const` and `sigma` carry
+// the layer's own); the state is read out as bf16(W) + bf16(W - bf16(W)),
+// two MMAs whose sum carries W to about 2^-17; and the epilogue writes
+// sigma * eta_t * O_t (dv or dk, bf16, through the O map) and, when `deta`
+// is set, deta_t = sigma * vdot_t . O_t from O in fp32.
+template <int C, int D, bool BWD = false>
 struct TcCfg {
   static constexpr int TILE = C * D * 2;                     // bytes of one bf16 C x D tile
   // 64 x 64 tiles fuse (1) and (2) into one N = C + D MMA, [Sc | O] = Q [K~; Wbf]^T:
@@ -104,7 +113,7 @@ struct TcCfg {
   // 128 x 128 tile, where it reuses the Q/K slots once (1)-(3) have read them.
   static constexpr bool PSEP = !(C == 128 && D == 128);
   static constexpr int PBUF = PSEP ? C * C * 2 : 0;
-  static constexpr int SBF_LO = SPLIT ? D * D * 2 : 0;       // bf16 residual of W (split readout)
+  static constexpr int SBF_LO = BWD ? D * D * 2 : 0;         // bf16 residual of W (split readout)
   static constexpr int BIG = NST * STAGE + SBF + PBUF + SBF_LO;
   // The 128 x 128 tile streams phase A through three K/V slots (A3): the two
   // stages' K and V regions and a third made of their Q regions, which phase
@@ -123,7 +132,8 @@ struct TcCfg {
   static_assert(C <= 2 * D, "P must fit in the Q and K slots");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(TCOLS_USED <= 512, "tensor memory");
-  static_assert(!(SPLIT && MRG), "the split readout needs the separate Wbf buffer");
+  static_assert(!BWD || (C == 128 && D == 64) || (C == 64 && D == 128),
+                "the reverse passes' epilogue handles 64 values of a row per thread");
 };
 
 // K-major operand (rows x 64-element k-blocks, SW128): descriptor of the
@@ -274,12 +284,12 @@ __device__ __forceinline__ void to_residual(uint32_t (&r)[N]) {
   }
 }
 
-template <int C, int D, bool SPLIT = false>
-__global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
+template <int C, int D, bool BWD = false>
+__global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
     chunked_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                       const TcParams p) {
-  using Cfg = TcCfg<C, D, SPLIT>;
+  using Cfg = TcCfg<C, D, BWD>;
   constexpr int NST = Cfg::NST, TILE = Cfg::TILE, STAGE = Cfg::STAGE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -361,6 +371,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
   const int tile = *sh_tile;
   const int seg = tile / p.BH, bh = tile % p.BH;  // segment-major: predecessors have smaller tiles
   TTT_EXPECT(tile >= 0 && tile < p.BH * p.nseg);
+  // Chunk of the sequence that logical chunk c is (reverse time for BWD).
+  auto phys = [&](int c) { return BWD ? p.nchunks - 1 - c : c; };
   // Row offsets inside the K region (merged tiles): even phase-B chunks hold
   // [K~ ; Wbf], odd ones [Wbf ; K~], so that the fused MMA writes [Sc | O0] or
   // [O1 | Sc] and O stays double-buffered around one score region in TMEM.
@@ -401,7 +413,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       TcCursor cur;
       for (cur.init(p, seg); cur.valid(p); cur.next(p, seg), ++g) {
         const bool pb = cur.is_b();
-        const int t0 = cur.chunk() * C;
+        const int t0 = phys(cur.chunk()) * C;
         TTT_EXPECT(cur.chunk() >= 0 && cur.chunk() < p.nchunks);
         const uint64_t pol_kv = (!pb && cur.chunk() - cur.A.c0 < p.keep) ? pol_keep : pol_once;
         if (a3 && !pb) {
@@ -473,7 +485,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
           const uint32_t stv = a3 ? sbase + a_voff(x) : sbase + s * STAGE + Cfg::OV;
           const uint64_t dkm = sdesc_sw128(stk, Cfg::KWR * 128, 1024), dvm = sdesc_sw128(stv, C * 128, 1024);
           if (cur.k == 0) free_scores();
-          if (!dead) dead = !mbar_wait(a3 ? &kreadyA[x] : &kready[s], ((a3 ? ia / 3 : g / NST)) & 1, lim);
+          // (BWD: K is used as loaded and the scaler warp sits out)
+          if (!dead) dead = !mbar_wait(a3 ? &kreadyA[x] : BWD ? &full[s] : &kready[s], ((a3 ? ia / 3 : g / NST)) & 1, lim);
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk)
@@ -494,7 +507,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         const uint64_t dvm = sdesc_sw128(stv, C * 128, 1024);
         const uint64_t dp = Cfg::PSEP ? d_pbuf : dq;
         const uint32_t t_o = t_o_of(b);
-        if (!dead) dead = !mbar_wait(&kready[s], u & 1, lim);
+        if (!dead) dead = !mbar_wait(BWD ? &full[s] : &kready[s], u & 1, lim);
         free_scores();
         if (Cfg::MRG) {
           // [Sc | O] in one N = C + D MMA: needs this chunk's Wbf and a free O[b]
@@ -518,7 +531,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_QW, kk > 0);
-          if constexpr (SPLIT) {
+          if constexpr (BWD) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_o, dq + k_step(C, kk), d_wlo + k_step(D, kk), ID_O_QW, 1);
           }
@@ -548,9 +561,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         if (!cur.is_b()) continue;
         const int s = (a3 ? itb : g) % NST;
         if (!dead) dead = !mbar_wait(&staged[itb % NST], (itb / NST) & 1, lim);
-        if constexpr (!SPLIT) {  // the split readout's epilogue wrote O itself
+        {
           const uint8_t* sv = smem + s * STAGE + Cfg::OV;
-          const int t0 = cur.chunk() * C;
+          const int t0 = phys(cur.chunk()) * C;
           // O is not read again: evict-first, so that it does not push out
           // the K and V phase B still reads from L2
 #pragma unroll
@@ -566,78 +579,81 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
   } else if (warp == 7) {
     // ------------------------------------------------------- K scaler --
     // K~ = diag(sigma * eta) K for every tile as it lands (phase A and B),
-    // in place, swizzle-aware; eta is fetched two tiles ahead.
-    bool dead = false;
-    constexpr int RPL = C / 32;  // rows of a chunk whose eta this lane fetches
-    const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
-    auto fetch = [&](const TcCursor& c, float (&dst)[RPL]) {
-      const bool ok = c.valid(p);
-      const int c0 = ok ? c.chunk() * C : 0;
+    // in place, swizzle-aware; eta is fetched two tiles ahead.  (BWD: no
+    // scaling.)
+    if constexpr (!BWD) {
+      bool dead = false;
+      constexpr int RPL = C / 32;  // rows of a chunk whose eta this lane fetches
+      const float* eg = p.eta ? p.eta + static_cast<size_t>(bh) * p.T : nullptr;
+      auto fetch = [&](const TcCursor& c, float (&dst)[RPL]) {
+        const bool ok = c.valid(p);
+        const int c0 = ok ? c.chunk() * C : 0;
 #pragma unroll
-      for (int j = 0; j < RPL; ++j) {
-        const int t = c0 + lane + 32 * j;
-        dst[j] = (ok && t < p.T) ? (eg ? __ldg(eg + t) : p.eta_const) : 0.f;
-      }
-    };
-    TcCursor cur, ahead;
-    cur.init(p, seg);
-    ahead = cur;
-    float er[RPL], en[RPL];
-    fetch(ahead, er);
-    if (ahead.valid(p)) ahead.next(p, seg);
-    fetch(ahead, en);
-    if (ahead.valid(p)) ahead.next(p, seg);
-    constexpr int PER_LANE = C * (D / 8) / 32;  // 16-byte units of the K tile per lane
-    constexpr int BATCH = 8;
-    int g = 0, itb = 0, ia = 0;
-    for (; cur.valid(p); cur.next(p, seg), ++g) {
-      const bool pb = cur.is_b();
-      const bool slotA = a3 && !pb;  // a three-slot phase-A chunk
-      const int x = ia % 3;
-      const int s = slotA ? x % NST : (a3 ? itb : g) % NST;
-      const int u = slotA ? ia / 3 : (a3 ? itb : g) / NST;
-      uint64_t* fb = slotA ? &fullA[x] : &full[s];
-      uint64_t* kb_ready = slotA ? &kreadyA[x] : &kready[s];
-      float* ess = es + s * C;
-#pragma unroll
-      for (int j = 0; j < RPL; ++j) ess[lane + 32 * j] = p.sigma * er[j];
-#pragma unroll
-      for (int j = 0; j < RPL; ++j) er[j] = en[j];
+        for (int j = 0; j < RPL; ++j) {
+          const int t = c0 + lane + 32 * j;
+          dst[j] = (ok && t < p.T) ? (eg ? __ldg(eg + t) : p.eta_const) : 0.f;
+        }
+      };
+      TcCursor cur, ahead;
+      cur.init(p, seg);
+      ahead = cur;
+      float er[RPL], en[RPL];
+      fetch(ahead, er);
+      if (ahead.valid(p)) ahead.next(p, seg);
       fetch(ahead, en);
       if (ahead.valid(p)) ahead.next(p, seg);
-      __syncwarp();
-      if (!dead) dead = !mbar_wait(fb, u & 1, lim);
-      uint8_t* sk = slotA ? smem + a_koff(x) : smem + s * STAGE + Cfg::OK + krow_of(pb, itb) * 128;
+      constexpr int PER_LANE = C * (D / 8) / 32;  // 16-byte units of the K tile per lane
+      constexpr int BATCH = 8;
+      int g = 0, itb = 0, ia = 0;
+      for (; cur.valid(p); cur.next(p, seg), ++g) {
+        const bool pb = cur.is_b();
+        const bool slotA = a3 && !pb;  // a three-slot phase-A chunk
+        const int x = ia % 3;
+        const int s = slotA ? x % NST : (a3 ? itb : g) % NST;
+        const int u = slotA ? ia / 3 : (a3 ? itb : g) / NST;
+        uint64_t* fb = slotA ? &fullA[x] : &full[s];
+        uint64_t* kb_ready = slotA ? &kreadyA[x] : &kready[s];
+        float* ess = es + s * C;
+#pragma unroll
+        for (int j = 0; j < RPL; ++j) ess[lane + 32 * j] = p.sigma * er[j];
+#pragma unroll
+        for (int j = 0; j < RPL; ++j) er[j] = en[j];
+        fetch(ahead, en);
+        if (ahead.valid(p)) ahead.next(p, seg);
+        __syncwarp();
+        if (!dead) dead = !mbar_wait(fb, u & 1, lim);
+        uint8_t* sk = slotA ? smem + a_koff(x) : smem + s * STAGE + Cfg::OK + krow_of(pb, itb) * 128;
 #pragma unroll 1
-      for (int b0 = 0; b0 < PER_LANE; b0 += BATCH) {
-        uint4 u[BATCH];
-        uint32_t off[BATCH];
-        float e[BATCH];
+        for (int b0 = 0; b0 < PER_LANE; b0 += BATCH) {
+          uint4 u[BATCH];
+          uint32_t off[BATCH];
+          float e[BATCH];
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-          const int idx = lane + 32 * (b0 + i);
-          const int r = idx / (D / 8), cc = idx % (D / 8);
-          off[i] = (cc >> 3) * Cfg::KWR * 128 + sw128_off(r, cc & 7);
-          e[i] = ess[r];
-          u[i] = *reinterpret_cast<const uint4*>(sk + off[i]);
-        }
+          for (int i = 0; i < BATCH; ++i) {
+            const int idx = lane + 32 * (b0 + i);
+            const int r = idx / (D / 8), cc = idx % (D / 8);
+            off[i] = (cc >> 3) * Cfg::KWR * 128 + sw128_off(r, cc & 7);
+            e[i] = ess[r];
+            u[i] = *reinterpret_cast<const uint4*>(sk + off[i]);
+          }
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-          // packed bf16 multiply: eta_r is rounded to bf16 once, then each
-          // product is rounded to bf16 as the operand itself would be
-          const uint32_t e2 = pack_bf16x2(e[i], e[i]);
-          u[i].x = mul_bf16x2(u[i].x, e2);
-          u[i].y = mul_bf16x2(u[i].y, e2);
-          u[i].z = mul_bf16x2(u[i].z, e2);
-          u[i].w = mul_bf16x2(u[i].w, e2);
-          *reinterpret_cast<uint4*>(sk + off[i]) = u[i];
+          for (int i = 0; i < BATCH; ++i) {
+            // packed bf16 multiply: eta_r is rounded to bf16 once, then each
+            // product is rounded to bf16 as the operand itself would be
+            const uint32_t e2 = pack_bf16x2(e[i], e[i]);
+            u[i].x = mul_bf16x2(u[i].x, e2);
+            u[i].y = mul_bf16x2(u[i].y, e2);
+            u[i].z = mul_bf16x2(u[i].z, e2);
+            u[i].w = mul_bf16x2(u[i].w, e2);
+            *reinterpret_cast<uint4*>(sk + off[i]) = u[i];
+          }
         }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(kb_ready);
+        if (pb) ++itb;
+        if (slotA) ++ia;
       }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(kb_ready);
-      if (pb) ++itb;
-      if (slotA) ++ia;
     }
   } else {
     // --------------------------------------------------------- epilogue --
@@ -716,7 +732,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
                                (cb0 + cb) * 32, r);
             else
               store_row32_bf16(sbase + NST * STAGE, D * 128, wrow, (cb0 + cb) * 32, r);
-            if constexpr (SPLIT) {
+            if constexpr (BWD) {
               to_residual(r);
               store_row32_bf16(sbase + NST * STAGE + Cfg::SBF + Cfg::PBUF, D * 128, wrow, (cb0 + cb) * 32, r);
             }
@@ -939,7 +955,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
                                cb * 32, r);
             else
               store_row32_bf16(sbase + NST * STAGE, D * 128, wrow, cb * 32, r);
-            if constexpr (SPLIT) {
+            if constexpr (BWD) {
               to_residual(r);
               store_row32_bf16(sbase + NST * STAGE + Cfg::SBF + Cfg::PBUF, D * 128, wrow, cb * 32, r);
             }
@@ -962,7 +978,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
       for (int j = 0; j < Bs.n; ++j, ++itb) {
         const int g = gb0 + j, s = (a3 ? itb : g) % NST, b = itb & 1;
         uint8_t* st = smem + s * STAGE;
-        // P = bf16(tril(scores)) into the Q (and K) slots
+        // P = bf16(tril(scores)) into the Q (and K) slots (BWD: triu, j >= i)
         {
           if (!dead) dead = !mbar_wait(sc_full, itb & 1, lim);
           tc_fence_after();
@@ -975,15 +991,16 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
             tmem_ld_half32(t_sc + lane_off, r);
             tmem_ld_wait();
             const uint32_t pdst = sbase + NST * STAGE + Cfg::SBF;
-            const int jmax = row64h - 32 * half;  // last unmasked column of this half
+            const int jd = row64h - 32 * half;  // the diagonal's column in this half
+            auto keep = [&](int jj) { return BWD ? jj >= jd : jj <= jd; };
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int jj = 8 * i + 2 * e;
-                w[e] = pack_bf16x2((jj <= jmax) ? __uint_as_float(r[jj]) : 0.f,
-                                   (jj + 1 <= jmax) ? __uint_as_float(r[jj + 1]) : 0.f);
+                w[e] = pack_bf16x2(keep(jj) ? __uint_as_float(r[jj]) : 0.f,
+                                   keep(jj + 1) ? __uint_as_float(r[jj + 1]) : 0.f);
               }
               st_shared_v4(pdst + sw128_off(row64h, 4 * half + i), w[0], w[1], w[2], w[3]);
             }
@@ -997,8 +1014,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
 #pragma unroll
               for (int jj = 0; jj < 64; jj += 2) {
                 const int col = cb * 64 + jj;
-                const float a0 = (col <= qrow) ? __uint_as_float(r[jj]) : 0.f;
-                const float a1 = (col + 1 <= qrow) ? __uint_as_float(r[jj + 1]) : 0.f;
+                const bool k0 = BWD ? col >= qrow : col <= qrow, k1 = BWD ? col + 1 >= qrow : col + 1 <= qrow;
+                const float a0 = k0 ? __uint_as_float(r[jj]) : 0.f;
+                const float a1 = k1 ? __uint_as_float(r[jj + 1]) : 0.f;
                 pk[col >> 1] = pack_bf16x2(a0, a1);
               }
             }
@@ -1032,7 +1050,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
             tmem_ld_half32(t_w + lane_off, r);
             tmem_ld_wait();
             store_row32_bf16(wdst, wblk, row64h, 32 * half, r);
-            if constexpr (SPLIT) {
+            if constexpr (BWD) {
               to_residual(r);
               store_row32_bf16(wlo, wblk, row64h, 32 * half, r);
             }
@@ -1043,7 +1061,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
               tmem_ld64(t_w + lane_off + cb * 64, r);
               tmem_ld_wait();
               store_row64_bf16(wdst, wblk, wrow, cb * 64, r);
-              if constexpr (SPLIT) {
+              if constexpr (BWD) {
                 to_residual(r);
                 store_row64_bf16(wlo, wblk, wrow, cb * 64, r);
               }
@@ -1056,44 +1074,56 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, SPLIT>::MINB)
         // O[b]: TMEM -> bf16 -> V slot, then the store warp takes it
         {
           const uint32_t sv = sbase + s * STAGE + Cfg::OV;
+          // BWD: this thread's token (row crow of the chunk, 64 columns from
+          // c0), its sigma * eta and its 64 values of vdot, fetched before
+          // the wait (rows past T give zeros, which the TMA store drops)
+          [[maybe_unused]] const int crow = (C == 128) ? qrow : row64h;
+          [[maybe_unused]] const int c0 = (C == 128) ? 0 : 64 * half;
+          [[maybe_unused]] size_t rowi = 0;
+          [[maybe_unused]] bool live = false;
+          [[maybe_unused]] float es_t = 0.f;
+          [[maybe_unused]] uint4 vv[8];
+          if constexpr (BWD) {
+            const int tok = phys(Bs.c0 + j) * C + crow;
+            const size_t ntok = static_cast<size_t>(p.BH) * p.T;
+            live = tok < p.T;
+            rowi = static_cast<size_t>(bh) * p.T + tok;
+            es_t = live ? p.sigma * (p.eta ? __ldg(TTT_AT(p.eta, rowi, 1, ntok)) : p.eta_const) : 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) vv[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (p.deta && live) {
+              const uint4* src = TTT_AT(static_cast<const uint4*>(p.vdot), (rowi * D + c0) / 8, 8, ntok * D / 8);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) vv[i] = __ldg(src + i);
+            }
+          }
           if (!dead) dead = !mbar_wait(&o_full[b], (itb >> 1) & 1, lim);
           tc_fence_after();
           const uint32_t t_o = t_o_of(b);
-          if constexpr (SPLIT) {
-            // fp32 rows straight to global (ragged tail: rows past T are not written)
-            const int crow = (C == 128) ? qrow : row64h;
-            const bool crow_ok = (C == 128) ? qrow_ok : true;
-            const int tok = (Bs.c0 + j) * C + crow;
-            if constexpr (C == 64) {
-              uint32_t r[64];
+          if constexpr (BWD) {
+            uint32_t r[64];
+            if constexpr (C == 64)
               tmem_ld_half64(t_o + lane_off, r);
-              tmem_ld_wait();
-              if (tok < p.T) {
-                float4* d4 = reinterpret_cast<float4*>(
-                    TTT_AT(p.o32, (static_cast<size_t>(bh) * p.T + tok) * D + 64 * half, 64,
-                           static_cast<size_t>(p.BH) * p.T * D));
+            else
+              tmem_ld64(t_o + lane_off, r);
+            tmem_ld_wait();
+            if (p.deta) {
+              float dot = 0.f;
 #pragma unroll
-                for (int q4 = 0; q4 < 16; ++q4)
-                  d4[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
-                                       __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
-              }
-            } else {
+              for (int i = 0; i < 8; ++i) {
+                const uint32_t w[4] = {vv[i].x, vv[i].y, vv[i].z, vv[i].w};
 #pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) {
-                uint32_t r[64];
-                tmem_ld64(t_o + lane_off + cb * 64, r);
-                tmem_ld_wait();
-                if (crow_ok && tok < p.T) {
-                  float4* d4 = reinterpret_cast<float4*>(
-                      TTT_AT(p.o32, (static_cast<size_t>(bh) * p.T + tok) * D + cb * 64, 64,
-                             static_cast<size_t>(p.BH) * p.T * D));
-#pragma unroll
-                  for (int q4 = 0; q4 < 16; ++q4)
-                    d4[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
-                                         __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
+                for (int e = 0; e < 4; ++e) {
+                  dot = fmaf(__uint_as_float(w[e] << 16), __uint_as_float(r[8 * i + 2 * e]), dot);
+                  dot = fmaf(__uint_as_float(w[e] & 0xffff0000u), __uint_as_float(r[8 * i + 2 * e + 1]), dot);
                 }
               }
+              if constexpr (C == 64) dot += __shfl_xor_sync(0xffffffffu, dot, 16);  // the row's other half
+              if (live && (C == 128 || half == 0)) *TTT_AT(p.deta, rowi, 1, static_cast<size_t>(p.BH) * p.T) = p.sigma * dot;
             }
+#pragma unroll
+            for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(es_t * __uint_as_float(r[i]));
+            store_row64_bf16(sv, C * 128, crow, c0, r);
           } else if constexpr (C == 64 && D == 64) {
             uint32_t r[32];
             tmem_ld_half32(t_o + lane_off, r);

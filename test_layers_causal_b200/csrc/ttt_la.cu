@@ -365,17 +365,18 @@ size_t tc_ws_bytes(int bh, int nseg, int D, bool waves = false) {
   return (b + 15) & ~static_cast<size_t>(15);
 }
 
-// SPLIT: the split state readout with fp32 output to o32 (the backward's
-// passes; the bf16 O map is then never used and is built over q).
-template <int C, int D, bool SPLIT = false>
-ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st, float* o32 = nullptr) {
-  using Cfg = ttt::TcCfg<C, D, SPLIT>;
-  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_tc_kernel<C, D, SPLIT>), Cfg::SMEM))
+// BWD: one of the backward's reverse-time passes (see chunked_tc.cuh), with
+// vdot/deta for the per-token learning-rate gradient.
+template <int C, int D, bool BWD = false>
+ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st, const void* vdot = nullptr,
+                        float* deta = nullptr) {
+  using Cfg = ttt::TcCfg<C, D, BWD>;
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::chunked_tc_kernel<C, D, BWD>), Cfg::SMEM))
     return TTT_LA_ERR_CUDA;
   const int bh = a->B * a->H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a->q, bh, a->T, D, C) || !make_map(&mk, a->k, bh, a->T, D, C) ||
-      !make_map(&mv, a->v, bh, a->T, D, C) || !make_map(&mo, SPLIT ? a->q : a->o, bh, a->T, D, C))
+      !make_map(&mv, a->v, bh, a->T, D, C) || !make_map(&mo, a->o, bh, a->T, D, C))
     return TTT_LA_ERR_CUDA;
   ttt::TcParams p;
   p.BH = bh;
@@ -393,7 +394,8 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
   p.nwave = sp.coop ? sp.nwave : 1;
   p.keep = sp.keep;
   p.S_out = a->state_out;
-  p.o32 = o32;
+  p.vdot = vdot;
+  p.deta = deta;
   p.limit_ns = g_limit_ns;
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
@@ -401,32 +403,33 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
     if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
       return TTT_LA_ERR_CUDA;
   }
-  return launch_kernel(ttt::chunked_tc_kernel<C, D, SPLIT>, bh * sp.nseg, 256, Cfg::SMEM, st, sp.coop, mq, mk, mv, mo,
+  return launch_kernel(ttt::chunked_tc_kernel<C, D, BWD>, bh * sp.nseg, 256, Cfg::SMEM, st, sp.coop, mq, mk, mv, mo,
                        p);
 }
 
-// The chunked forward of the backward's passes (bf16, no momentum): the
-// state read out as bf16(W) + bf16(W - bf16(W)) and O written in fp32 to
-// o32 [B,H,T,d_v] (a->o is ignored), so that the products the backward forms
-// from O (dv, dk and the per-token deta, a d-term dot product that can
-// cancel) keep fp32 precision.  Tiles: d = 64 with 128 tokens, d = 128 with
-// 64 (the two whose shared memory holds the second bf16 copy of W).
+// One of the backward's two reverse-time passes (bf16, no momentum): the
+// chunked forward over the chunks last to first with the anti-causal mask,
+// K unscaled, the state read out as bf16(W) + bf16(W - bf16(W)), and the
+// epilogue writing o_t := sigma eta_t O_t in bf16 (dv or dk; a->eta,
+// a->eta_const and a->ascent are the layer's) plus, when deta is given,
+// deta_t = sigma vdot_t . O_t from O in fp32.  Tiles: d = 64 with 128
+// tokens, d = 128 with 64 (the two whose shared memory holds the second bf16
+// copy of W).
 size_t workspace_for(const ttt_la_args* a);
-ttt_la_status forward_chunked_split(const ttt_la_args* a0, float* o32, cudaStream_t st) {
-  if (!a0 || !o32 || !aligned16(o32)) return TTT_LA_ERR_INVALID_ARG;
-  ttt_la_args a = *a0;
-  a.o = o32;
-  const ttt_la_status s = check_seq(&a);
+ttt_la_status backward_pass_tc(const ttt_la_args* a, const void* vdot, float* deta, cudaStream_t st) {
+  if (!a || (deta && (!vdot || !aligned16(vdot)))) return TTT_LA_ERR_INVALID_ARG;
+  const ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
-  if (a.dtype != TTT_LA_BF16 || a.beta != 0.f || a.d_k != a.d_v ||
-      !((a.d_k == 64 && a.chunk == 128) || (a.d_k == 128 && a.chunk == 64)))
+  if (a->dtype != TTT_LA_BF16 || a->beta != 0.f || a->d_k != a->d_v ||
+      !((a->d_k == 64 && a->chunk == 128) || (a->d_k == 128 && a->chunk == 64)))
     return TTT_LA_ERR_UNSUPPORTED;
-  const SegPlan sp = plan_segments(&a);
+  const SegPlan sp = plan_segments(a);
   if (sp.nseg > 1) {
-    const size_t need = workspace_for(&a);
-    if (!a.workspace || a.workspace_bytes < need || !aligned16(a.workspace)) return TTT_LA_ERR_INVALID_ARG;
+    const size_t need = workspace_for(a);
+    if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace)) return TTT_LA_ERR_INVALID_ARG;
   }
-  return a.d_k == 64 ? launch_tc<128, 64, true>(&a, sp, st, o32) : launch_tc<64, 128, true>(&a, sp, st, o32);
+  return a->d_k == 64 ? launch_tc<128, 64, true>(a, sp, st, vdot, deta)
+                      : launch_tc<64, 128, true>(a, sp, st, vdot, deta);
 }
 
 template <bool MOM>
@@ -1032,21 +1035,26 @@ ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 
 // Chunk-parallel backward without momentum: three runs of the chunked forward
 // (see backward_chunked.cuh) over scratch carved from the caller's workspace.
+// bf16: the two reverse-time passes run on the tensor cores in reverse chunk
+// order and write dv (with deta) and dk themselves; fp32: they run on copies
+// of the inputs reversed along T and a finishing kernel forms dv, dk, deta.
 namespace {
 struct BwdChunkedLayout {
   size_t rev[4], u, r, w0t, dwt, fwd, total, fwd_bytes;
 };
 
-// bf16: the tiles of the split readout (d = 64: 128 tokens, d = 128: 64);
+bool bwdc_fused(const ttt_la_grad_args* a) { return a->dtype == TTT_LA_BF16; }
+
+// bf16: the tiles of the reverse passes (d = 64: 128 tokens, d = 128: 64);
 // fp32: the fp32 chunked path's 64.
 int bwdc_chunk(const ttt_la_grad_args* a) {
   if (a->dtype != TTT_LA_BF16) return 64;
   return a->d_k == 128 ? 64 : 128;
 }
 
-// Arguments of forward pass p: 0 gives dq, 1 gives u = G k (reversed order)
-// and dL/dW_0, 2 gives r = G^T v (reversed order).  rev[] are q, k, v, dO
-// reversed along T.
+// Arguments of forward pass p: 0 gives dq, 1 gives u = G k (bf16: dv) and
+// dL/dW_0, 2 gives r = G^T v (bf16: dk).  fp32: rev[] are q, k, v, dO
+// reversed along T, and u, r come out in reversed order.
 ttt_la_args bwdc_pass(const ttt_la_grad_args* a, int p, void* const* rev, void* u, void* r, const float* w0t,
                       const float* dwt) {
   ttt_la_args f;
@@ -1057,6 +1065,14 @@ ttt_la_args bwdc_pass(const ttt_la_grad_args* a, int p, void* const* rev, void* 
   f.dtype = a->dtype;
   f.chunk = bwdc_chunk(a);
   f.beta = 0.f;
+  const bool fused = bwdc_fused(a);
+  // the reverse passes: the layer's eta and sigma for the fused epilogue, or
+  // eta = 1, sigma = +1 for a plain run on reversed copies
+  if (p > 0) {
+    f.eta = fused ? a->eta : nullptr;
+    f.eta_const = fused ? a->eta_const : 1.f;
+    f.ascent = fused ? a->ascent : 0;
+  }
   if (p == 0) {  // W_t^T do_t: keys v, values k, from W_0^T, the layer's eta and sigma
     f.d_k = a->d_v;
     f.d_v = a->d_k;
@@ -1068,45 +1084,46 @@ ttt_la_args bwdc_pass(const ttt_la_grad_args* a, int p, void* const* rev, void* 
     f.ascent = a->ascent;
     f.state_in = w0t;
     f.o = a->grad_q;
-  } else if (p == 1) {  // G_t k_t: reversed (q, k, v) := (k, q, dO), eta = 1, from dL/dW_T
+  } else if (p == 1) {  // G_t k_t: reverse time, (q, k, v) := (k, q, dO), from dL/dW_T
     f.d_k = a->d_k;
     f.d_v = a->d_v;
-    f.q = rev[1];
-    f.k = rev[0];
-    f.v = rev[3];
-    f.eta_const = 1.f;
+    f.q = fused ? a->k : rev[1];
+    f.k = fused ? a->q : rev[0];
+    f.v = fused ? a->grad_o : rev[3];
     f.state_in = a->grad_state;
     f.state_out = a->grad_state_in;
-    f.o = u;
-  } else {  // G_t^T v_t: reversed (q, k, v) := (v, dO, q), eta = 1, from (dL/dW_T)^T
+    f.o = fused ? a->grad_v : u;
+  } else {  // G_t^T v_t: reverse time, (q, k, v) := (v, dO, q), from (dL/dW_T)^T
     f.d_k = a->d_v;
     f.d_v = a->d_k;
-    f.q = rev[2];
-    f.k = rev[3];
-    f.v = rev[0];
-    f.eta_const = 1.f;
+    f.q = fused ? a->v : rev[2];
+    f.k = fused ? a->grad_o : rev[3];
+    f.v = fused ? a->q : rev[0];
     f.state_in = dwt;
-    f.o = r;
+    f.o = fused ? a->grad_k : r;
   }
   return f;
 }
 
 BwdChunkedLayout bwdc_layout(const ttt_la_grad_args* a) {
   BwdChunkedLayout L;
+  std::memset(&L, 0, sizeof L);
   const size_t el = a->dtype == TTT_LA_F32 ? 4 : 2, bh = static_cast<size_t>(a->B) * a->H;
-  const size_t nk = align256(bh * a->T * a->d_k * el), nv = align256(bh * a->T * a->d_v * el);
   const size_t ns = align256(bh * a->d_k * a->d_v * 4);
   size_t off = 0;
-  const size_t sizes[4] = {nk, nk, nv, nv};
-  for (int i = 0; i < 4; ++i) {
-    L.rev[i] = off;
-    off += sizes[i];
+  if (!bwdc_fused(a)) {
+    // q, k, v, dO reversed, then u and r (fp32)
+    const size_t nk = align256(bh * a->T * a->d_k * el), nv = align256(bh * a->T * a->d_v * el);
+    const size_t sizes[4] = {nk, nk, nv, nv};
+    for (int i = 0; i < 4; ++i) {
+      L.rev[i] = off;
+      off += sizes[i];
+    }
+    L.u = off;
+    off += align256(bh * a->T * a->d_v * 4);
+    L.r = off;
+    off += align256(bh * a->T * a->d_k * 4);
   }
-  // u and r in fp32 whatever the dtype
-  L.u = off;
-  off += align256(bh * a->T * a->d_v * 4);
-  L.r = off;
-  off += align256(bh * a->T * a->d_k * 4);
   L.w0t = off;
   off += a->state_in ? ns : 0;
   L.dwt = off;
@@ -1148,6 +1165,7 @@ ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
   if (s != TTT_LA_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const BwdChunkedLayout L = bwdc_layout(a);
+  const bool fused = bwdc_fused(a);
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   void* rev[4] = {ws + L.rev[0], ws + L.rev[1], ws + L.rev[2], ws + L.rev[3]};
   float* w0t = a->state_in ? reinterpret_cast<float*>(ws + L.w0t) : nullptr;
@@ -1155,8 +1173,8 @@ ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
   const int BH = a->B * a->H, el = a->dtype == TTT_LA_F32 ? 4 : 2;
   const int grid = sm_count() * 4;
 
-  // q, k (rows of d_k) and v, dO (rows of d_v) reversed along T
-  for (int g = 0; g < 2; ++g) {
+  // fp32: q, k (rows of d_k) and v, dO (rows of d_v) reversed along T
+  for (int g = 0; g < 2 && !fused; ++g) {
     ttt::ReverseParams rp;
     std::memset(&rp, 0, sizeof rp);
     rp.n = 2;
@@ -1195,34 +1213,33 @@ ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
     ttt_la_args f = bwdc_pass(a, p, rev, u, r, w0t, dwt);
     f.workspace = L.fwd_bytes ? ws + L.fwd : nullptr;
     f.workspace_bytes = L.fwd_bytes;
-    if (p > 0 && a->dtype == TTT_LA_BF16)  // u and r: split readout, fp32 out
-      s = forward_chunked_split(&f, static_cast<float*>(p == 1 ? u : r), st);
+    if (p > 0 && fused)  // dv with deta (the layer's v dotted with u), then dk
+      s = backward_pass_tc(&f, p == 1 ? a->v : nullptr, p == 1 ? a->grad_eta : nullptr, st);
     else
       s = ttt_la_forward_chunked(&f, stream);
     if (s != TTT_LA_OK) return s;
   }
-  // dv, dk, deta
-  ttt::FinishParams fp;
-  fp.BH = BH;
-  fp.T = a->T;
-  fp.dk = a->d_k;
-  fp.dv = a->d_v;
-  fp.u_rev = static_cast<const float*>(u);
-  fp.r_rev = static_cast<const float*>(r);
-  fp.v = a->v;
-  fp.eta = a->eta;
-  fp.eta_const = a->eta_const;
-  fp.sigma = a->ascent ? -1.f : 1.f;
-  fp.dk_out = a->grad_k;
-  fp.dv_out = a->grad_v;
-  fp.deta = a->grad_eta;
-  const long long warps = static_cast<long long>(BH) * a->T;
-  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
-  if (a->dtype == TTT_LA_F32)
-    ttt::backward_finish_kernel<float><<<blocks, 256, 0, st>>>(fp);
-  else
-    ttt::backward_finish_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(fp);
-  if ((s = launched()) != TTT_LA_OK) return s;
+  if (!fused) {
+    // dv, dk, deta
+    ttt::FinishParams fp;
+    fp.BH = BH;
+    fp.T = a->T;
+    fp.dk = a->d_k;
+    fp.dv = a->d_v;
+    fp.u_rev = static_cast<const float*>(u);
+    fp.r_rev = static_cast<const float*>(r);
+    fp.v = static_cast<const float*>(a->v);
+    fp.eta = a->eta;
+    fp.eta_const = a->eta_const;
+    fp.sigma = a->ascent ? -1.f : 1.f;
+    fp.dk_out = static_cast<float*>(a->grad_k);
+    fp.dv_out = static_cast<float*>(a->grad_v);
+    fp.deta = a->grad_eta;
+    const long long warps = static_cast<long long>(BH) * a->T;
+    const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+    ttt::backward_finish_kernel<<<blocks, 256, 0, st>>>(fp);
+    if ((s = launched()) != TTT_LA_OK) return s;
+  }
   if (a->grad_mom_in &&
       cudaMemsetAsync(a->grad_mom_in, 0, static_cast<size_t>(BH) * a->d_v * a->d_k * sizeof(float), st) !=
           cudaSuccess)

@@ -360,11 +360,17 @@ def test_backward_chunked_workspace_and_validation(abi):
     L = abi.lib()
     call = lambda g: L.ttt_la_backward_chunked(ctypes.byref(g), None)  # noqa: E731
     size = lambda g: L.ttt_la_backward_chunked_workspace_size(ctypes.byref(g))  # noqa: E731
+    # bf16: the reverse passes read the inputs in place and write dv, dk
+    # themselves; the scratch holds the two transposed states (and whatever
+    # the chunked forward's own plan needs)
     g = _grad_args(abi, T=100)
-    seq = 2 * 2 * 100 * 64 * 2  # one reversed bf16 tensor
-    assert size(g) >= 6 * seq  # four reversed inputs and the two passes' outputs
     g.state_in, g.grad_state = 0x8000000, 0x9000000
-    assert size(g) >= 6 * seq + 2 * 2 * 2 * 64 * 64 * 4  # plus the two transposed states
+    states = 2 * 2 * 2 * 64 * 64 * 4
+    assert states <= size(g) < states + 2 * 2 * 100 * 64 * 2
+    # fp32: plus four inputs reversed along T and the passes' fp32 outputs
+    f = _grad_args(abi, T=100)
+    f.dtype = abi.F32
+    assert size(f) >= 6 * (2 * 2 * 100 * 64 * 4)
     assert L.ttt_la_backward_chunked_workspace_size(None) == 0
     assert L.ttt_la_backward_chunked(None, None) == abi.ERR_INVALID_ARG
     # momentum is the recurrent form's
@@ -377,5 +383,6 @@ def test_backward_chunked_workspace_and_validation(abi):
     g.workspace_bytes = 1 << 40
     assert call(g) == abi.ERR_UNSUPPORTED
     g = _grad_args(abi)
+    g.state_in, g.grad_state = 0x8000000, 0x9000000
     g.workspace_bytes = size(g) - 256
     assert call(g) == abi.ERR_INVALID_ARG

@@ -46,7 +46,8 @@ def _ref(x, ascent):
 
 
 @pytest.mark.parametrize("d,T,token_eta,ascent,states", [(64, 300, True, False, True), (128, 257, False, True, True),
-                                                         (64, 64, True, False, False), (128, 1, True, False, True)])
+                                                         (64, 64, True, False, False), (128, 1, True, False, True),
+                                                         (64, 100, True, True, True), (128, 33, True, False, False)])
 def test_backward_chunked_bf16_matches_oracle(d, T, token_eta, ascent, states):
     x = _case(2, 3, T, d, d, "bf16", 90 + d + T, token_eta, states)
     g = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], eta_const=x["ec"], ascent=ascent,
@@ -73,6 +74,24 @@ def test_backward_chunked_agrees_with_recurrent_at_llm_shape():
     x = _case(4, 16, 4096, 64, 64, "bf16", 140)
     a = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], state_in=x["S0"], grad_state=x["dW"])
     b = _abi.backward_recurrent(x["q"], x["k"], x["v"], x["dO"], x["eta"], state_in=x["S0"], grad_state=x["dW"])
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dW0"):
+        assert_bf16(a[n], f64(b[n]), n)
+
+
+@pytest.mark.parametrize("d,T,wave_tokens", [(128, 64 * 400 + 5, 0), (128, 64 * 400 + 5, 128),
+                                             (64, 128 * 150 + 3, 0), (64, 128 * 150 + 3, 256)])
+def test_backward_chunked_long_sequence_schedules(d, T, wave_tokens, monkeypatch):
+    """Two heads of a long ragged sequence: the reverse passes run tens of
+    segments per head with the cooperative start states, in one wave or
+    (TTT_LA_WAVE_TOKENS) in several, and agree with the recurrent backward."""
+    if wave_tokens:
+        monkeypatch.setenv("TTT_LA_WAVE_TOKENS", str(wave_tokens))
+    x = _case(1, 2, T, d, d, "bf16", 170 + d)
+    a = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], ascent=True, state_in=x["S0"],
+                              grad_state=x["dW"])
+    b = _abi.backward_recurrent(x["q"], x["k"], x["v"], x["dO"], x["eta"], ascent=True, state_in=x["S0"],
+                                grad_state=x["dW"])
     torch.cuda.synchronize()
     for n in ("dq", "dk", "dv", "deta", "dW0"):
         assert_bf16(a[n], f64(b[n]), n)

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from synth import make_qkv
-from tests.gpu_util import assert_bf16, oracle_forward
+from tests.gpu_util import assert_bf16, f64, oracle_forward
 
 pytestmark = pytest.mark.gpu
 
@@ -67,3 +67,39 @@ def test_debug_build_checks_stay_clean(d, chunk, B, H, T, segments, beta, wave_t
     assert_bf16(S, S_ref, "state")
     if beta:
         assert_bf16(M, M_ref, "momentum")
+
+
+# (d, B, H, T, wave tokens): the backward's reverse passes (chunk 128 for d = 64, 64 for d = 128)
+BWD_CASES = [
+    (64, 2, 3, 128 * 3 + 5, 0),    # look-back, a few segments per head
+    (64, 1, 2, 128 * 20 + 3, 0),   # cooperative start states, one wave
+    (128, 1, 2, 64 * 160 + 3, 64), # wave schedule, two waves
+]
+
+
+@pytest.mark.parametrize("d,B,H,T,wave_tokens", BWD_CASES)
+def test_debug_build_backward_checks_stay_clean(d, B, H, T, wave_tokens, monkeypatch):
+    from test_layers_causal_b200 import _abi
+    if wave_tokens:
+        monkeypatch.setenv("TTT_LA_WAVE_TOKENS", str(wave_tokens))
+    L = _abi.debug_lib()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    L.ttt_la_debug_check_line(st)
+    L.ttt_la_get_last_device_status(st)
+    q, k, v, eta = _inputs(B, H, T, d, 400 + d + T)
+    g = torch.Generator().manual_seed(7)
+    dO = torch.randn(v.shape, generator=g).to(torch.bfloat16).cuda()
+    S0 = 0.1 * torch.randn(B, H, d, d, generator=g).cuda()
+    dW = torch.randn(B, H, d, d, generator=g).cuda()
+    a, out = _abi._chunked_grad_args(q, k, v, dO, eta, None, False, S0, dW)
+    need = int(L.ttt_la_backward_chunked_workspace_size(ctypes.byref(a)))
+    ws = torch.full((max(need, 16),), 0x7F, dtype=torch.uint8, device="cuda")
+    a.workspace, a.workspace_bytes = ws.data_ptr(), need
+    code = L.ttt_la_backward_chunked(ctypes.byref(a), st)
+    assert code == 0, _abi.status_string(code)
+    assert L.ttt_la_get_last_device_status(st) == _abi.OK
+    assert L.ttt_la_debug_check_line(st) == 0
+    ref = _abi.backward_recurrent(q, k, v, dO, eta, state_in=S0, grad_state=dW)
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dW0"):
+        assert_bf16(out[n], f64(ref[n]), n)
