@@ -326,22 +326,30 @@ typedef struct ttt_la_grad_args {
 TTT_LA_API size_t ttt_la_backward_workspace_size(const ttt_la_grad_args *args);
 TTT_LA_API ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args *args, void *stream);
 
-/* Chunk-parallel backward of the layer without momentum (beta == 0): the
- * same gradients as ttt_la_backward_recurrent, from three runs of the chunked
- * forward on the tensor cores.  With G_t = dL/dW_T + sum_{t' >= t} do_t' q_t'^T:
- *   dq_t = W_t^T do_t   the forward on (q, k, v) := (do, v, k) from W_0^T;
- *   G_t k_t, G_t^T v_t  the forward on the time-reversed sequences of
- *                       (k, q, do) and (v, do, q), learning rate 1, from
+/* Chunk-parallel backward of the layer: the same gradients as
+ * ttt_la_backward_recurrent ("Test-Time Training with KV Binding Is Secretly
+ * Linear Attention", thelatestinai.com listing, Figure 4: training with the
+ * parallel form), from chunked runs on the tensor cores.
+ * Without momentum (beta == 0), with G_t = dL/dW_T + sum_{t' >= t} do_t' q_t'^T:
+ *   dq_t = W_t^T do_t   the chunked forward on (q, k, v) := (do, v, k) from W_0^T;
+ *   G_t k_t, G_t^T v_t  the chunked forward over the chunks last to first
+ *                       (anti-causal mask) on (k, q, do) and (v, do, q), from
  *                       dL/dW_T and its transpose (the first run's final
- *                       state is dL/dW_0);
- *   dv_t = sigma eta_t G_t k_t, dk_t = sigma eta_t G_t^T v_t,
+ *                       state is dL/dW_0), whose epilogues write
+ *   dv_t = sigma eta_t G_t k_t, dk_t = sigma eta_t G_t^T v_t and
  *   deta_t = sigma v_t . G_t k_t.
- * bf16: d_k == d_v in {64, 128}; fp32: d_k, d_v multiples of 4 up to 128.
- * beta != 0, mom_in or grad_mom: TTT_LA_ERR_UNSUPPORTED; grad_mom_in, if
- * given, is zeroed.  The workspace (ttt_la_backward_chunked_workspace_size
- * bytes) holds reversed copies of q, k, v and grad_o, the passes' outputs,
- * the transposed states and one forward workspace.  Errors as
- * ttt_la_backward_recurrent. */
+ * With momentum (beta != 0; bf16 only): dq is the momentum forward on
+ * (do, v, k) from W_0^T and M_0^T; dv, dk, dL/dW_0 and dL/dM_0 come from a
+ * reverse chunkwise kernel carrying (dL/dW, beta dL/dM), deta from a
+ * forward-order one carrying (M, dL/dW); grad_mom (dL/dM_T) and mom_in (M_0)
+ * are optional (zero).
+ * bf16: d_k == d_v in {64, 128}; fp32 (no momentum): d_k, d_v multiples of 4
+ * up to 128; momentum in fp32, or mom_in / grad_mom without momentum:
+ * TTT_LA_ERR_UNSUPPORTED.  Without momentum, grad_mom_in, if given, is zeroed.
+ * The workspace (ttt_la_backward_chunked_workspace_size bytes) holds the
+ * transposed states and one forward workspace (fp32 also: reversed copies of
+ * q, k, v, grad_o and the reverse runs' outputs; momentum also: dL/dW_0 when
+ * grad_state_in is NULL).  Errors as ttt_la_backward_recurrent. */
 TTT_LA_API size_t ttt_la_backward_chunked_workspace_size(const ttt_la_grad_args *args);
 TTT_LA_API ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args *args, void *stream);
 

@@ -419,38 +419,45 @@ def backward_recurrent(q, k, v, grad_o, eta=None, eta_const=None, beta=0.0, asce
     return out
 
 
-def _chunked_grad_args(q, k, v, grad_o, eta, eta_const, ascent, state_in, grad_state):
+def _chunked_grad_args(q, k, v, grad_o, eta, eta_const, ascent, state_in, grad_state, beta=0.0, mom_in=None,
+                       grad_mom=None):
     """The TttGradArgs of ttt_la_backward_chunked and the output tensors it
     points at (no workspace yet)."""
-    _check_shapes(q, k, v, eta, state_in, None)
+    _check_shapes(q, k, v, eta, state_in, mom_in)
     if grad_o.shape != v.shape or grad_o.dtype != v.dtype:
         raise ValueError("grad_o must match v")
     B, H, T, dk = q.shape
     dv = v.shape[-1]
-    if grad_state is not None and (grad_state.shape != (B, H, dv, dk) or grad_state.dtype != torch.float32):
-        raise ValueError("grad_state must be fp32 [B,H,d_v,d_k]")
-    _need_cuda(q, k, v, grad_o, eta, state_in, grad_state)
+    for t in (grad_state, grad_mom):
+        if t is not None and (t.shape != (B, H, dv, dk) or t.dtype != torch.float32):
+            raise ValueError("grad_state / grad_mom must be fp32 [B,H,d_v,d_k]")
+    _need_cuda(q, k, v, grad_o, eta, state_in, grad_state, mom_in, grad_mom)
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                deta=torch.empty(B, H, T, device=q.device, dtype=torch.float32),
-               dW0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32))
+               dW0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32),
+               dM0=torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32) if beta else None)
     a = TttGradArgs()
     a.B, a.H, a.T, a.d_k, a.d_v, a.dtype = B, H, T, dk, dv, _dtype_code(q)
     a.q, a.k, a.v, a.eta = q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(eta)
     a.eta_const = (1.0 / math.sqrt(dk)) if eta_const is None else float(eta_const)
-    a.beta, a.ascent = 0.0, int(bool(ascent))
+    a.beta, a.ascent = float(beta), int(bool(ascent))
     a.state_in, a.grad_o, a.grad_state = _ptr(state_in), grad_o.data_ptr(), _ptr(grad_state)
+    a.mom_in, a.grad_mom = _ptr(mom_in), _ptr(grad_mom)
     a.grad_q, a.grad_k, a.grad_v = out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr()
     a.grad_eta, a.grad_state_in = out["deta"].data_ptr(), out["dW0"].data_ptr()
+    a.grad_mom_in = _ptr(out["dM0"])
     return a, out
 
 
 def backward_chunked(q, k, v, grad_o, eta=None, eta_const=None, ascent=False, state_in=None, grad_state=None,
-                     workspace=None, stream=None):
-    """Gradients of the layer without momentum from three chunked forward runs
+                     workspace=None, stream=None, beta=0.0, mom_in=None, grad_mom=None):
+    """Gradients of the layer from its chunk-parallel form
     (ttt_la_backward_chunked): returns a dict with dq, dk, dv (dtype of q),
-    deta [B,H,T] fp32 (per token) and dW0 [B,H,d_v,d_k] fp32."""
+    deta [B,H,T] fp32 (per token), dW0 [B,H,d_v,d_k] fp32 and, with momentum
+    (beta != 0: bf16, d_k == d_v in {64, 128}), dM0 (else None)."""
     _need_cuda(workspace)
-    a, out = _chunked_grad_args(q, k, v, grad_o, eta, eta_const, ascent, state_in, grad_state)
+    a, out = _chunked_grad_args(q, k, v, grad_o, eta, eta_const, ascent, state_in, grad_state, beta, mom_in,
+                                grad_mom)
     L = lib()
     need = L.ttt_la_backward_chunked_workspace_size(ctypes.byref(a))
     if workspace is None or workspace.numel() * workspace.element_size() < need:

@@ -48,11 +48,11 @@ __global__ void __launch_bounds__(256) reverse_tokens_kernel(const ReverseParams
   }
 }
 
-// Up to two [BH][R][C] fp32 matrices transposed to [BH][C][R].
+// Up to four [BH][R][C] fp32 matrices transposed to [BH][C][R].
 struct TransposeParams {
   int n, BH, R, C;
-  const float* src[2];
-  float* dst[2];
+  const float* src[4];
+  float* dst[4];
 };
 
 __global__ void __launch_bounds__(256) transpose_states_kernel(const TransposeParams p) {
@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(256) transpose_states_kernel(const TransposePa
     const int r = rc / p.C, c = rc % p.C;
     const long long o = bh * p.R * p.C + static_cast<long long>(c) * p.R + r;
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < 4; ++j)
       if (j < p.n) p.dst[j][o] = p.src[j][i];
   }
 }

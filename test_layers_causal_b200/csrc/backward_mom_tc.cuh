@@ -1,0 +1,869 @@
+// backward_mom_tc.cuh -- chunkwise backward of the layer with SGD momentum on
+// the sm_100a tensor cores (Variant 3 of Table 2 in the thelatestinai.com
+// listing of "Test-Time Training with KV Binding Is Secretly Linear
+// Attention": per-token learning rate, momentum in SGD; its Figure 4 trains
+// with the parallel form, which needs this gradient).
+//
+// Forward (update, then read): M_t = beta M_{t-1} - sigma v_t k_t^T,
+// W_t = W_{t-1} - eta_t M_t, o_t = W_t q_t.  Reverse mode, with G_t = dL/dW_t
+// and H_t = dL/dM_t (dL/dW_T, dL/dM_T given):
+//   G_t = G_{t+1} + do_t q_t^T              (G_T := dL/dW_T)
+//   H_t = beta H_{t+1} - eta_t G_t          (beta H_T := dL/dM_T)
+//   dv_t = -sigma H_t k_t,   dk_t = -sigma H_t^T v_t,
+//   deta_t = -<G_t, M_t>,    dq_t = W_t^T do_t,
+//   dL/dW_0 = G_0,           dL/dM_0 = beta H_0.
+// dq is the momentum forward itself on (q, k, v) := (do, v, k) from W_0^T,
+// M_0^T (chunked_tc_mom.cuh).  The rest regroups over chunks of C tokens
+// (local i, j, n valid) exactly:
+//
+// Reverse kernel (chunks last to first; carried state G and X = beta H at
+// the chunk's end), with e_i = sum_{r=i}^{n-1} beta^(r-i) eta_r and
+// w_ij = sum_{r=i}^{j} beta^(r-i) eta_r = e_i - beta^(j+1-i) e_{j+1} (j >= i;
+// no division, so no cancellation that grows like beta^-C):
+//   dv_i = -sigma beta^(n-1-i) X k_i + sigma e_i G k_i
+//          + sigma sum_{j>=i} w_ij (k_i . q_j) do_j
+//   X   <- beta^n X - beta e_0 G - sum_j beta w_0j do_j q_j^T
+//   G   <- G + sum_j do_j q_j^T
+// and dk is the same kernel on (k, q, do) := (v, do, q) from the transposed
+// states.  deta kernel (chunks first to last; carried state M and
+// P = -G = sum of do q^T so far - dL/dW_0, G at the chunk's start):
+//   <G_t, M_t> = beta^(i+1) (<G, M> - sum_{j<i} y_j) - sigma sum_{s<=i} beta^(i-s) z_s
+//                + sigma sum_{s<=i} beta^(i-s) F_is,
+//   y_j = do_j . (M q_j),  z_s = v_s . (G k_s),
+//   F = Lstrict (Q K^T o dO V^T)   (Lstrict: ones strictly below the diagonal)
+//   M <- beta^n M - sigma sum_s beta^(n-1-s) v_s k_s^T,  P <- P + sum_j do_j q_j^T.
+// y and z read M and G through two bf16 MMAs each (bf16(x) + bf16(x -
+// bf16(x))), which carries them to about 2^-17: deta is a d^2-term inner
+// product that can cancel.
+//
+// One block per (b, h, 64 rows of the state) walks its chunks in order (no
+// segment scan): every term above is linear in the rows of the states (and of
+// dv, dk), so a block owns rows [r0, r0 + 64) of G, X (or M, P) and the
+// matching 64 columns of the output, with its own copy of the scores; the
+// deta blocks of one head add their partial sums into a zeroed deta.  Warp 0
+// loads tiles with TMA, warp 1 owns TMEM and issues the MMAs, warps 2-5 (one
+// TMEM lane each) run the epilogue, and the rest scale operand copies (and,
+// in the reverse kernel, store the output rows).  Every wait is bounded
+// (common.cuh); a thread whose wait runs out stops waiting but keeps
+// arriving, so the block drains and exits.
+#pragma once
+#include "chunked_tc.cuh"
+#include "common.cuh"
+
+namespace ttt {
+
+struct MomBwdParams {
+  int BH, T, nchunks;
+  const float* eta;    // [BH, T] or nullptr (reverse kernel)
+  float eta_const, sigma, beta;
+  const float* G_in;   // [BH, D, D] row-major: reverse: dL/dW_T (or its transpose), deta: dL/dW_0; or nullptr
+  const float* X_in;   // reverse: dL/dM_T (or its transpose); deta: M_0; or nullptr (zero)
+  float* G_out;        // reverse: dL/dW_0 or nullptr
+  float* X_out;        // reverse: dL/dM_0 or nullptr
+  float* deta;         // deta kernel: [BH, T]
+  uint64_t limit_ns;
+};
+
+// x * s for both bf16 halves of `u`, in fp32 with one rounding.
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t u, float s) {
+  const float2 f = unpack_bf16x2(u);
+  return pack_bf16x2(f.x * s, f.y * s);
+}
+
+// fp32 row values (raw bits) split into bf16(x) and bf16(x - bf16(x)), written
+// as row `row`, columns [col0, col0 + 32) of two 64-row K-major SW128 tiles.
+__device__ __forceinline__ void store_row32_split(uint32_t hi, uint32_t lo, int row, int col0, uint32_t (&r)[32]) {
+  store_row32_bf16(hi, 64 * 128, row, col0, r);
+  to_residual(r);
+  store_row32_bf16(lo, 64 * 128, row, col0, r);
+}
+
+// A block's share of the state rows (one M = 64 accumulator).
+constexpr int kMomRows = 64;
+
+template <int D>
+struct MomRevCfg {
+  static constexpr int C = 64, RS = kMomRows;
+  static constexpr int TILE = C * D * 2;          // bf16 C x D
+  static constexpr int SQ = RS * D * 2;           // bf16 RS x D
+  static constexpr int NST = 2;
+  static constexpr int STAGE = 3 * TILE;          // K, Q, dO roles
+  static constexpr int OFF_XBF = NST * STAGE;     // bf16 rows of X (B operand)
+  static constexpr int OFF_GBF = OFF_XBF + SQ;
+  static constexpr int OFF_QW = OFF_GBF + SQ;     // [2] diag(-beta w_0j) Q (chunk parity)
+  static constexpr int OFF_P = OFF_QW + 2 * TILE; // C x C weights
+  static constexpr int BIG = OFF_P + C * C * 2;
+  static constexpr int NE = 3;                    // coefficient slots
+  static constexpr int NBAR = 3 * NST + 13;
+  static constexpr int SMALL = NBAR * 8 + (NE * (C + 1) + (C + 1) + 4) * 4 + 16;
+  static constexpr int SMEM = BIG + SMALL + 1024;
+  static constexpr int TCOLS_USED = 2 * D + C + 3 * RS;  // G, X, scores, U1, U2, U3
+  static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
+  static constexpr int THREADS = 288;             // 9 warps
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+template <int D>
+struct MomDetaCfg {
+  static constexpr int C = 64, RS = kMomRows;
+  static constexpr int TILE = C * D * 2;
+  static constexpr int NST = 2;
+  static constexpr int STAGE = 4 * TILE;          // Q, K, V, dO
+  static constexpr int SQ = RS * D * 2;
+  static constexpr int OFF_MBF = NST * STAGE;     // bf16 rows of M, their residual, the same of G
+  static constexpr int OFF_MLO = OFF_MBF + SQ;
+  static constexpr int OFF_GBF = OFF_MLO + SQ;
+  static constexpr int OFF_GLO = OFF_GBF + SQ;
+  static constexpr int OFF_KB = OFF_GLO + SQ;     // diag(-sigma beta^(n-1-s)) K
+  static constexpr int OFF_A = OFF_KB + TILE;     // bf16(Q K^T o dO V^T), token-major
+  static constexpr int OFF_L = OFF_A + C * C * 2; // strictly lower ones
+  static constexpr int BIG = OFF_L + C * C * 2;
+  static constexpr int NBAR = 2 * NST + 11;
+  static constexpr int SMALL = NBAR * 8 + ((C + 1) + 4 * C + 8) * 4 + 16;
+  static constexpr int SMEM = BIG + SMALL + 1024;
+  static constexpr int TCOLS_USED = 2 * D + 3 * C + RS;  // M, P, S1, S2, F, Y / Z
+  static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
+  static constexpr int THREADS = 224;             // 7 warps
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(TCOLS_USED <= 512, "tensor memory");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+// Reverse kernel: tmK, tmQ, tmD are the K, Q and dO roles (dv: k, q, do;
+// dk: v, do, q), tmO the output rows; block (bh, r0) owns state rows
+// [r0, r0 + 64) and output columns [r0, r0 + 64) (dO_r: those columns of dO).
+// Per chunk the MMA thread issues
+//   (1) S  = K Q^T                            [TMEM, M=C, N=C]
+//   (2) U1 = K Xbf^T,  U2 = K Gbf^T           [TMEM, M=C, N=64 each]
+//   (3) G += dO_r^T Q,  (4) X += dO_r^T Qw    [TMEM, M=64, N=D]
+//   (5) U3 = P dO_r                           P = bf16(sigma w o triu(S))
+// after the epilogue has taken Xbf, Gbf and replaced X by beta^n X - beta e_0 G;
+// the output row is -sigma beta^(n-1-i) U1 + sigma e_i U2 + U3, formed in fp32.
+// The coefficients e and the copy Qw of a chunk are made while the previous
+// chunk's MMAs run (three coefficient slots, two Qw buffers).
+template <int D>
+__global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
+    mom_bwd_rev_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmO,
+                       const MomBwdParams p) {
+  using Cfg = MomRevCfg<D>;
+  constexpr int C = Cfg::C, RS = Cfg::RS, NST = Cfg::NST, TILE = Cfg::TILE, STAGE = Cfg::STAGE;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BIG);
+  uint64_t* full = bars;                // [NST] tiles landed
+  uint64_t* empty = bars + NST;         // [NST] output rows stored: stage free
+  uint64_t* staged = bars + 2 * NST;    // [NST] output rows written into the stage's K slot
+  // Barriers the coefficient warps fill run one per slot, so that none of
+  // them can complete two phases ahead of a waiter.
+  uint64_t* e_ready = bars + 3 * NST;   // [3] e of the chunks of slot c % 3 written
+  uint64_t* qw_ready = e_ready + 3;     // [2] Qw of the chunks of parity c & 1 written
+  uint64_t* ks_free = qw_ready + 2;     // [2] (2)-(4) of the chunks of parity c & 1 done: Qw buffer free
+  uint64_t* wbf_ready = ks_free + 2;    // Xbf, Gbf written, X rewritten
+  uint64_t* sc_full = wbf_ready + 1;    // (1) done
+  uint64_t* sdone = wbf_ready + 2;      // (2)-(4) done
+  uint64_t* p_ready = wbf_ready + 3;    // P written
+  uint64_t* o_full = wbf_ready + 4;     // (5) done
+  uint64_t* drain = wbf_ready + 5;
+  float* ebuf = reinterpret_cast<float*>(bars + Cfg::NBAR);  // [NE][C + 1] e_i of the chunk (e_C = 0)
+  float* bpow = ebuf + Cfg::NE * (C + 1);                     // [C + 1] beta^k
+  float* xw = bpow + C + 1;                                   // [4] cross-warp carry of the e scan
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xw + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.limit_ns;
+  const int bh = blockIdx.x / (D / RS), r0 = (blockIdx.x % (D / RS)) * RS, rb = r0 / 64;
+  const int nch = p.nchunks;
+  // logical chunk c is chunk nch - 1 - c of the sequence, with n valid tokens
+  auto phys = [&](int c) { return nch - 1 - c; };
+  auto nvalid = [&](int c) { return min(C, p.T - phys(c) * C); };
+
+  if (threadIdx.x <= C) {
+    float b = 1.f;
+    for (int k = 0; k < static_cast<int>(threadIdx.x); ++k) b *= p.beta;
+    bpow[threadIdx.x] = b;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&staged[s], 128);
+    }
+    for (int x = 0; x < 3; ++x) mbar_init(&e_ready[x], 64);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&qw_ready[x], 64);
+      mbar_init(&ks_free[x], 1);
+    }
+    mbar_init(wbf_ready, 128);
+    mbar_init(sc_full, 1);
+    mbar_init(sdone, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::TCOLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmD);
+    prefetch_tmap(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t t_g = tmem, t_x = tmem + D, t_s = tmem + 2 * D;
+  const uint32_t t_u1 = t_s + C, t_u2 = t_u1 + RS, t_u3 = t_u2 + RS;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      bool dead = false;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NST, u = c / NST;
+        if (u > 0 && !dead) dead = !mbar_wait(&empty[s], (u - 1) & 1, lim);
+        mbar_arrive_expect_tx(&full[s], 3 * TILE);
+        uint8_t* st = smem + s * STAGE;
+        const int t0 = phys(c) * C;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_load_3d(&tmK, &full[s], st + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmQ, &full[s], st + TILE + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmD, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, t0, bh);
+        }
+      }
+      for (int j = max(0, nch - NST); j < nch; ++j) mbar_wait(&full[j % NST], (j / NST) & 1, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      bool dead = false;
+      constexpr uint32_t ID_S = idesc_bf16_f32(C, C, false, false);
+      constexpr uint32_t ID_U = idesc_bf16_f32(C, RS, false, false);
+      constexpr uint32_t ID_ST = idesc_bf16_f32(RS, D, true, true);
+      constexpr uint32_t ID_PU = idesc_bf16_f32(C, RS, false, true);
+      const uint64_t d_xbf = sdesc_sw128(sbase + Cfg::OFF_XBF, 16, 1024);
+      const uint64_t d_gbf = sdesc_sw128(sbase + Cfg::OFF_GBF, 16, 1024);
+      const uint64_t d_p = sdesc_sw128(sbase + Cfg::OFF_P, 16, 1024);
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NST, u = c / NST;
+        const uint32_t st = sbase + s * STAGE;
+        const uint64_t d_k = sdesc_sw128(st, 16, 1024), d_q = sdesc_sw128(st + TILE, 16, 1024);
+        const uint64_t d_qm = sdesc_sw128(st + TILE, C * 128, 1024);
+        const uint64_t d_dm = sdesc_sw128(st + 2 * TILE + rb * C * 128, C * 128, 1024);  // this block's dO columns
+        const uint64_t d_qw = sdesc_sw128(sbase + Cfg::OFF_QW + (c & 1) * TILE, C * 128, 1024);  // MN-major
+        if (!dead) dead = !mbar_wait(&full[s], u & 1, lim);
+        tc_fence_after();
+        // (1); the scores of chunk c-1 were read before p_ready(c-1), waited below
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_s, d_k + k_step(C, kk), d_q + k_step(C, kk), ID_S, kk > 0);
+        tc_commit(sc_full);
+        if (!dead) dead = !mbar_wait(&qw_ready[c & 1], (c >> 1) & 1, lim);
+        if (!dead) dead = !mbar_wait(wbf_ready, c & 1, lim);
+        tc_fence_after();
+        // (2); U1-U3 of chunk c-1 were read before wbf_ready(c)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          mma_bf16_ss(t_u1, d_k + k_step(C, kk), d_xbf + k_step(RS, kk), ID_U, kk > 0);
+          mma_bf16_ss(t_u2, d_k + k_step(C, kk), d_gbf + k_step(RS, kk), ID_U, kk > 0);
+        }
+        // (3), (4)
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_g, d_dm + mn_step(kk), d_qm + mn_step(kk), ID_ST, 1);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_x, d_dm + mn_step(kk), d_qw + mn_step(kk), ID_ST, 1);
+        tc_commit(sdone);
+        tc_commit(&ks_free[c & 1]);
+        if (!dead) dead = !mbar_wait(p_ready, c & 1, lim);
+        tc_fence_after();
+        // (5)
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_u3, d_p + k_step(C, kk), d_dm + mn_step(kk), ID_PU, kk > 0);
+        tc_commit(o_full);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, lim);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------ output store warp --
+    if (lane == 0) {
+      bool dead = false;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NST;
+        if (!dead) dead = !mbar_wait(&staged[s], (c / NST) & 1, lim);
+        tma_store_3d(&tmO, smem + s * STAGE, r0, phys(c) * C, bh);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait0();
+    }
+  } else if (warp >= 7) {
+    // ------------------------------------------------ coefficient warps --
+    // e_i of chunk c (one token per thread: a shuffle scan within each warp
+    // and one carry across), then Qw into the buffer of c's parity.  Both wait
+    // only for (2)-(4) of chunk c - 2: slot c % 3 of e was last read by the
+    // epilogue's P of chunk c - 3, which precedes its Xbf of chunk c - 2.
+    const int tid = threadIdx.x - 224;  // 0..63: warp 7 tokens 0-31, warp 8 tokens 32-63
+    bool dead = false;
+    auto eta_of = [&](int c) {
+      const int t = phys(c) * C + tid;
+      return (tid < nvalid(c)) ? (p.eta ? __ldg(p.eta + static_cast<size_t>(bh) * p.T + t) : p.eta_const) : 0.f;
+    };
+    float eta_next = eta_of(0);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NST;
+      float* e = ebuf + (c % Cfg::NE) * (C + 1);
+      float v = eta_next;
+      if (c + 1 < nch) eta_next = eta_of(c + 1);
+      if (c >= 2 && !dead) dead = !mbar_wait(&ks_free[c & 1], ((c >> 1) - 1) & 1, lim);
+      // v_i = sum_{r=i}^{end of the warp's 32 tokens} beta^(r-i) eta_r
+#pragma unroll
+      for (int k = 1; k < 32; k <<= 1) {
+        const float u = __shfl_down_sync(0xffffffffu, v, k);
+        if (lane + k < 32) v = fmaf(bpow[k], u, v);
+      }
+      if (warp == 8 && lane == 0) xw[0] = v;  // e_32
+      asm volatile("bar.sync 2, 64;" ::: "memory");
+      if (warp == 7) v = fmaf(bpow[32 - lane], xw[0], v);
+      e[tid] = v;
+      if (tid == 0) e[C] = 0.f;
+      asm volatile("bar.sync 2, 64;" ::: "memory");
+      mbar_arrive(&e_ready[c % 3]);
+      if (!dead) dead = !mbar_wait(&full[s], (c / NST) & 1, lim);
+      const uint8_t* qr = smem + s * STAGE + TILE;
+      uint8_t* qw = smem + Cfg::OFF_QW + (c & 1) * TILE;
+      const float e0 = e[0];
+#pragma unroll 4
+      for (int k = 0; k < D / 8; ++k) {
+        const int idx = tid + 64 * k;
+        const int r = idx / (D / 8), cc = idx % (D / 8);
+        const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
+        const float cw = -p.beta * (e0 - bpow[r + 1] * e[r + 1]);
+        const uint4 b = *reinterpret_cast<const uint4*>(qr + off);
+        *reinterpret_cast<uint4*>(qw + off) =
+            make_uint4(scale_bf16x2(b.x, cw), scale_bf16x2(b.y, cw), scale_bf16x2(b.z, cw), scale_bf16x2(b.w, cw));
+      }
+      fence_async_smem();
+      mbar_arrive(&qw_ready[c & 1]);
+    }
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int g4 = warp & 3;  // TMEM lane quadrant of this warp
+    const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
+    // M = 64 accumulators: lanes 0-15 of each quadrant hold rows 16 g4 + lane
+    const int wrow = 16 * g4 + lane;
+    const bool wrow_ok = lane < 16;
+    // read with the whole warp: row 16 g4 + lane % 16, column half lane / 16
+    const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
+    const size_t DD = static_cast<size_t>(D) * D, nst = static_cast<size_t>(p.BH) * DD;
+    const size_t grow = bh * DD + static_cast<size_t>(r0 + wrow) * D;  // this thread's state row in global
+    bool dead = false;
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NST, n = nvalid(c);
+      const float* e = ebuf + (c % Cfg::NE) * (C + 1);
+      // (b) Xbf, Gbf from the chunk-end states; X <- beta^n X - beta e_0 G
+      if (c >= 1 && !dead) dead = !mbar_wait(sdone, (c - 1) & 1, lim);
+      if (!dead) dead = !mbar_wait(&e_ready[c % 3], (c / 3) & 1, lim);
+      tc_fence_after();
+      const float xs = bpow[n], gs = -p.beta * e[0];
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t g[32], x[32];
+        if (c == 0) {
+          const float* gi = (p.G_in && wrow_ok) ? TTT_AT(p.G_in, grow + cb * 32, 32, nst) : nullptr;
+          const float* xi = (p.X_in && wrow_ok) ? TTT_AT(p.X_in, grow + cb * 32, 32, nst) : nullptr;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            g[j] = __float_as_uint(gi ? __ldg(gi + j) : 0.f);
+            x[j] = __float_as_uint(xi ? __ldg(xi + j) : 0.f);
+          }
+          tmem_st32(t_g + lane_off + cb * 32, g);  // G accumulator := dL/dW_T (rows)
+        } else {
+          tmem_ld32(t_g + lane_off + cb * 32, g);
+          tmem_ld32(t_x + lane_off + cb * 32, x);
+          tmem_ld_wait();
+        }
+        if (wrow_ok) {
+          store_row32_bf16(sbase + Cfg::OFF_GBF, RS * 128, wrow, cb * 32, g);
+          store_row32_bf16(sbase + Cfg::OFF_XBF, RS * 128, wrow, cb * 32, x);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = __float_as_uint(fmaf(xs, __uint_as_float(x[j]), gs * __uint_as_float(g[j])));
+        tmem_st32(t_x + lane_off + cb * 32, x);
+      }
+      tmem_st_wait();
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(wbf_ready);
+      // (d) P_ij = sigma w_ij S_ij for j >= i
+      if (!dead) dead = !mbar_wait(sc_full, c & 1, lim);
+      tc_fence_after();
+      {
+        uint32_t r[32];
+        tmem_ld_half32(t_s + lane_off, r);
+        tmem_ld_wait();
+        const int i = row64h;
+        const float ei = e[i];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int j0 = 32 * half + 8 * q + 2 * h;
+            // w_ij = e_i - beta^(j+1-i) e_{j+1}  (j >= i; the index is clamped for j < i)
+            const float w0 = ei - bpow[max(j0 + 1 - i, 0)] * e[j0 + 1];
+            const float w1 = ei - bpow[max(j0 + 2 - i, 0)] * e[j0 + 2];
+            const float a0 = (j0 >= i) ? p.sigma * w0 * __uint_as_float(r[8 * q + 2 * h]) : 0.f;
+            const float a1 = (j0 + 1 >= i) ? p.sigma * w1 * __uint_as_float(r[8 * q + 2 * h + 1]) : 0.f;
+            w[h] = pack_bf16x2(a0, a1);
+          }
+          st_shared_v4(sbase + Cfg::OFF_P + sw128_off(i, 4 * half + q), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      // (f) row i = -sigma beta^(n-1-i) U1 + sigma e_i U2 + U3 -> bf16 -> the stage's K slot
+      // (every MMA of the chunk is done), then the store warp
+      if (!dead) dead = !mbar_wait(o_full, c & 1, lim);
+      tc_fence_after();
+      {
+        uint32_t u1[32], u2[32], r[32];
+        tmem_ld_half32(t_u1 + lane_off, u1);
+        tmem_ld_half32(t_u2 + lane_off, u2);
+        tmem_ld_half32(t_u3 + lane_off, r);
+        tmem_ld_wait();
+        const int i = row64h;
+        const float a1 = (i < n) ? -p.sigma * bpow[max(n - 1 - i, 0)] : 0.f, a2 = p.sigma * e[i];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          r[j] = __float_as_uint(fmaf(a1, __uint_as_float(u1[j]), fmaf(a2, __uint_as_float(u2[j]), __uint_as_float(r[j]))));
+        store_row32_bf16(sbase + s * STAGE, C * 128, row64h, 32 * half, r);
+      }
+      tc_fence_before();
+      fence_async_smem();
+      mbar_arrive(&staged[s]);
+    }
+    // final states: G = dL/dW_0, X = beta H_0 = dL/dM_0 (this block's rows)
+    if (!dead) dead = !mbar_wait(sdone, (nch - 1) & 1, lim);
+    tc_fence_after();
+#pragma unroll 1
+    for (int cb = 0; cb < D / 32; ++cb) {
+      uint32_t g[32], x[32];
+      tmem_ld32(t_g + lane_off + cb * 32, g);
+      tmem_ld32(t_x + lane_off + cb * 32, x);
+      tmem_ld_wait();
+      if (wrow_ok) {
+        if (p.G_out) {
+          float4* d4 = reinterpret_cast<float4*>(TTT_AT(p.G_out, grow + cb * 32, 32, nst));
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            d4[j] = make_float4(__uint_as_float(g[4 * j]), __uint_as_float(g[4 * j + 1]), __uint_as_float(g[4 * j + 2]),
+                                __uint_as_float(g[4 * j + 3]));
+        }
+        if (p.X_out) {
+          float4* d4 = reinterpret_cast<float4*>(TTT_AT(p.X_out, grow + cb * 32, 32, nst));
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            d4[j] = make_float4(__uint_as_float(x[4 * j]), __uint_as_float(x[4 * j + 1]), __uint_as_float(x[4 * j + 2]),
+                                __uint_as_float(x[4 * j + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::TCOLS);
+}
+
+// deta kernel: tmQ, tmK, tmV, tmD over q, k, v, do; G_in = dL/dW_0, X_in =
+// M_0; block (bh, r0) owns rows [r0, r0 + 64) of M and P (V_r, dO_r: those
+// columns of V and dO) and adds its partial deta.  Per chunk the MMA thread
+// issues
+//   (1) S1 = Q K^T,  S2 = dO_r V_r^T            [TMEM, M=C, N=C each]
+//   (2) Y  = Q Mbf^T + Q Mlo^T                  [TMEM, M=C, N=64]
+//   (2') Z = K Gbf^T + K Glo^T                  (Y's columns, once y is read)
+//   (4) M += V_r^T Kb,  P += dO_r^T Q           [TMEM, M=64, N=D]
+//   (3) F  = Lstrict A,  A = bf16(S1 o S2)      [TMEM, M=C, N=C]
+// after the epilogue has taken the bf16 pairs of M and G = -P and replaced M
+// by beta^n M.  The epilogue takes chunk c+1's states as soon as it has read
+// z of chunk c, so that chunk c+1's scores and Y overlap its F and prefix sums.
+template <int D>
+__global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
+    mom_bwd_deta_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmD,
+                        const MomBwdParams p) {
+  using Cfg = MomDetaCfg<D>;
+  constexpr int C = Cfg::C, RS = Cfg::RS, NST = Cfg::NST, TILE = Cfg::TILE, STAGE = Cfg::STAGE;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BIG);
+  uint64_t* full = bars;                 // [NST] tiles landed
+  uint64_t* empty = bars + NST;          // [NST] stage free: (3) issued after (1)-(4), and the epilogue read V, dO
+  uint64_t* mbf_ready = bars + 2 * NST;  // bf16 pairs written, M rewritten
+  uint64_t* sc_full = mbf_ready + 1;
+  uint64_t* y_full = mbf_ready + 2;
+  uint64_t* y_free = mbf_ready + 3;
+  uint64_t* z_full = mbf_ready + 4;
+  uint64_t* kb_ready = mbf_ready + 5;
+  uint64_t* sdone = mbf_ready + 6;       // (2)-(4) done
+  uint64_t* a_ready = mbf_ready + 7;
+  uint64_t* f_full = mbf_ready + 8;
+  uint64_t* drain = mbf_ready + 9;
+  uint64_t* f_free = mbf_ready + 10;     // F read out of TMEM
+  float* bpow = reinterpret_cast<float*>(bars + Cfg::NBAR);  // [C + 1] beta^k
+  float* ys = bpow + C + 1;                                   // [C]
+  float* zs = ys + C;                                         // [C]
+  float* red = zs + 3 * C;                                    // [8]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(red + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.limit_ns;
+  const int bh = blockIdx.x / (D / RS), r0 = (blockIdx.x % (D / RS)) * RS, rb = r0 / 64;
+  const int nch = p.nchunks;
+  auto nvalid = [&](int c) { return min(C, p.T - c * C); };
+
+  if (threadIdx.x <= C) {
+    float b = 1.f;
+    for (int k = 0; k < static_cast<int>(threadIdx.x); ++k) b *= p.beta;
+    bpow[threadIdx.x] = b;
+  }
+  // Lstrict (K-major, one 64-column block): 1 where column < row
+  for (int u = threadIdx.x; u < C * 8; u += blockDim.x) {
+    const int r = u >> 3, c16 = u & 7;
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) w[h] = pack_bf16x2(8 * c16 + 2 * h < r ? 1.f : 0.f, 8 * c16 + 2 * h + 1 < r ? 1.f : 0.f);
+    st_shared_v4(sbase + Cfg::OFF_L + sw128_off(r, c16), w[0], w[1], w[2], w[3]);
+  }
+  fence_async_smem();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 129);
+    }
+    mbar_init(mbf_ready, 128);
+    mbar_init(sc_full, 1);
+    mbar_init(y_full, 1);
+    mbar_init(y_free, 128);
+    mbar_init(z_full, 1);
+    mbar_init(kb_ready, 1);
+    mbar_init(sdone, 1);
+    mbar_init(a_ready, 128);
+    mbar_init(f_full, 1);
+    mbar_init(drain, 1);
+    mbar_init(f_free, 128);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::TCOLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmD);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t t_m = tmem, t_p = tmem + D, t_s1 = tmem + 2 * D, t_s2 = t_s1 + C, t_f = t_s2 + C, t_yz = t_f + C;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      bool dead = false;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NST, u = c / NST;
+        if (u > 0 && !dead) dead = !mbar_wait(&empty[s], (u - 1) & 1, lim);
+        mbar_arrive_expect_tx(&full[s], 4 * TILE);
+        uint8_t* st = smem + s * STAGE;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, c * C, bh);
+          tma_load_3d(&tmK, &full[s], st + TILE + kb * C * 128, kb * 64, c * C, bh);
+          tma_load_3d(&tmV, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, c * C, bh);
+          tma_load_3d(&tmD, &full[s], st + 3 * TILE + kb * C * 128, kb * 64, c * C, bh);
+        }
+      }
+      for (int j = max(0, nch - NST); j < nch; ++j) mbar_wait(&full[j % NST], (j / NST) & 1, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      bool dead = false;
+      constexpr uint32_t ID_S = idesc_bf16_f32(C, C, false, false);
+      constexpr uint32_t ID_Y = idesc_bf16_f32(C, RS, false, false);
+      constexpr uint32_t ID_ST = idesc_bf16_f32(RS, D, true, true);
+      constexpr uint32_t ID_F = idesc_bf16_f32(C, C, false, true);
+      const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
+      const uint64_t d_mlo = sdesc_sw128(sbase + Cfg::OFF_MLO, 16, 1024);
+      const uint64_t d_gbf = sdesc_sw128(sbase + Cfg::OFF_GBF, 16, 1024);
+      const uint64_t d_glo = sdesc_sw128(sbase + Cfg::OFF_GLO, 16, 1024);
+      const uint64_t d_kbm = sdesc_sw128(sbase + Cfg::OFF_KB, C * 128, 1024);  // MN-major
+      const uint64_t d_am = sdesc_sw128(sbase + Cfg::OFF_A, C * 128, 1024);    // MN-major
+      const uint64_t d_l = sdesc_sw128(sbase + Cfg::OFF_L, 16, 1024);
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NST, u = c / NST;
+        const uint32_t st = sbase + s * STAGE;
+        const uint32_t vr = st + 2 * TILE + rb * C * 128, dr = st + 3 * TILE + rb * C * 128;  // this block's columns
+        const uint64_t d_q = sdesc_sw128(st, 16, 1024), d_k = sdesc_sw128(st + TILE, 16, 1024);
+        const uint64_t d_vr = sdesc_sw128(vr, 16, 1024), d_dr = sdesc_sw128(dr, 16, 1024);
+        const uint64_t d_qm = sdesc_sw128(st, C * 128, 1024);
+        const uint64_t d_vrm = sdesc_sw128(vr, C * 128, 1024), d_drm = sdesc_sw128(dr, C * 128, 1024);
+        if (!dead) dead = !mbar_wait(&full[s], u & 1, lim);
+        // the epilogue has read S1, S2, Z of chunk c-1 before taking chunk c's bf16 pairs
+        if (!dead) dead = !mbar_wait(mbf_ready, c & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_s1, d_q + k_step(C, kk), d_k + k_step(C, kk), ID_S, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(t_s2, d_dr + k_step(C, kk), d_vr + k_step(C, kk), ID_S, kk > 0);
+        tc_commit(sc_full);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_q + k_step(C, kk), d_mbf + k_step(RS, kk), ID_Y, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_q + k_step(C, kk), d_mlo + k_step(RS, kk), ID_Y, 1);
+        tc_commit(y_full);
+        if (!dead) dead = !mbar_wait(y_free, c & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_k + k_step(C, kk), d_gbf + k_step(RS, kk), ID_Y, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_k + k_step(C, kk), d_glo + k_step(RS, kk), ID_Y, 1);
+        tc_commit(z_full);
+        if (!dead) dead = !mbar_wait(kb_ready, c & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16_ss(t_m, d_vrm + mn_step(kk), d_kbm + mn_step(kk), ID_ST, 1);
+          mma_bf16_ss(t_p, d_drm + mn_step(kk), d_qm + mn_step(kk), ID_ST, 1);
+        }
+        tc_commit(sdone);
+        if (!dead) dead = !mbar_wait(a_ready, c & 1, lim);
+        if (c >= 1 && !dead) dead = !mbar_wait(f_free, (c - 1) & 1, lim);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_f, d_l + k_step(C, kk), d_am + mn_step(kk), ID_F, kk > 0);
+        tc_commit(f_full);
+        tc_commit(&empty[s]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, lim);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------- K scaler --
+    // Kb = diag(-sigma beta^(n-1-s)) K, once (4) of the previous chunk is done
+    bool dead = false;
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NST, n = nvalid(c);
+      if (!dead) dead = !mbar_wait(&full[s], (c / NST) & 1, lim);
+      if (c >= 1 && !dead) dead = !mbar_wait(sdone, (c - 1) & 1, lim);
+      const uint8_t* kt = smem + s * STAGE + TILE;
+#pragma unroll 4
+      for (int k = 0; k < D / 4; ++k) {
+        const int idx = lane + 32 * k;
+        const int r = idx / (D / 8), cc = idx % (D / 8);
+        const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
+        const float cb = (r < n) ? -p.sigma * bpow[n - 1 - r] : 0.f;
+        const uint4 a = *reinterpret_cast<const uint4*>(kt + off);
+        *reinterpret_cast<uint4*>(smem + Cfg::OFF_KB + off) =
+            make_uint4(scale_bf16x2(a.x, cb), scale_bf16x2(a.y, cb), scale_bf16x2(a.z, cb), scale_bf16x2(a.w, cb));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(kb_ready);
+    }
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int g4 = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
+    const int wrow = 16 * g4 + lane;  // M = 64 state rows: lanes 0-15 of each quadrant
+    const bool wrow_ok = lane < 16;
+    const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
+    const size_t DD = static_cast<size_t>(D) * D, nst = static_cast<size_t>(p.BH) * DD;
+    const size_t grow = bh * DD + static_cast<size_t>(r0 + wrow) * D;
+    bool dead = false;
+    // this thread's half (32 columns) of row row64h of Y or Z, dotted with the
+    // same columns of this block's 64 columns of a token tile
+    auto row_dot = [&](const uint8_t* tile, const uint32_t (&r)[32]) {
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 x = *reinterpret_cast<const uint4*>(tile + sw128_off(row64h, 4 * half + q));
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          acc = fmaf(__uint_as_float(w[h] << 16), __uint_as_float(r[8 * q + 2 * h]), acc);
+          acc = fmaf(__uint_as_float(w[h] & 0xffff0000u), __uint_as_float(r[8 * q + 2 * h + 1]), acc);
+        }
+      }
+      return acc + __shfl_xor_sync(0xffffffffu, acc, 16);  // the row's other half
+    };
+    // (b) of chunk c: bf16 pairs of M and G = -P, this block's part of <G, M>
+    // (returned), M <- beta^n M
+    auto take_states = [&](int c) {
+      if (c >= 1 && !dead) dead = !mbar_wait(sdone, (c - 1) & 1, lim);
+      tc_fence_after();
+      const float bn = bpow[nvalid(c)];
+      float part = 0.f;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t m[32], g[32], mm[32];
+        if (c == 0) {
+          const float* mi = (p.X_in && wrow_ok) ? TTT_AT(p.X_in, grow + cb * 32, 32, nst) : nullptr;
+          const float* gi = wrow_ok ? TTT_AT(p.G_in, grow + cb * 32, 32, nst) : nullptr;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            m[j] = __float_as_uint(mi ? __ldg(mi + j) : 0.f);
+            g[j] = __float_as_uint(gi ? -__ldg(gi + j) : 0.f);  // P := -dL/dW_0
+          }
+          tmem_st32(t_p + lane_off + cb * 32, g);
+        } else {
+          tmem_ld32(t_m + lane_off + cb * 32, m);
+          tmem_ld32(t_p + lane_off + cb * 32, g);
+          tmem_ld_wait();
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float gj = -__uint_as_float(g[j]);  // G = -P
+          g[j] = __float_as_uint(gj);
+          part = fmaf(gj, __uint_as_float(m[j]), part);
+          mm[j] = __float_as_uint(bn * __uint_as_float(m[j]));
+        }
+        tmem_st32(t_m + lane_off + cb * 32, mm);
+        if (wrow_ok) {
+          store_row32_split(sbase + Cfg::OFF_MBF, sbase + Cfg::OFF_MLO, wrow, cb * 32, m);
+          store_row32_split(sbase + Cfg::OFF_GBF, sbase + Cfg::OFF_GLO, wrow, cb * 32, g);
+        }
+      }
+      tmem_st_wait();
+      if (!wrow_ok) part = 0.f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      // by chunk parity: the barrier of chunk c+1's call orders chunk c+2's writes after these reads
+      float* rd = red + (c & 1) * 4;
+      if (lane == 0) rd[warp - 2] = part;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const float g0 = rd[0] + rd[1] + rd[2] + rd[3];
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(mbf_ready);
+      return g0;
+    };
+    float g0 = take_states(0);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NST, n = nvalid(c);
+      const uint8_t* st = smem + s * STAGE;
+      // (d) A = bf16(S1 o S2), token-major (rows j, columns s)
+      if (!dead) dead = !mbar_wait(sc_full, c & 1, lim);
+      tc_fence_after();
+      {
+        uint32_t a[32], b[32];
+        tmem_ld_half32(t_s1 + lane_off, a);
+        tmem_ld_half32(t_s2 + lane_off, b);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int x = 8 * q + 2 * h;
+            w[h] = pack_bf16x2(__uint_as_float(a[x]) * __uint_as_float(b[x]),
+                               __uint_as_float(a[x + 1]) * __uint_as_float(b[x + 1]));
+          }
+          st_shared_v4(sbase + Cfg::OFF_A + sw128_off(row64h, 4 * half + q), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(a_ready);
+      // (e) y_j = do_j . (M q_j) over this block's rows of M
+      if (!dead) dead = !mbar_wait(y_full, c & 1, lim);
+      tc_fence_after();
+      float y, z;
+      {
+        uint32_t r[32];
+        tmem_ld_half32(t_yz + lane_off, r);
+        tmem_ld_wait();
+        y = row_dot(st + 3 * TILE + rb * C * 128, r);
+      }
+      tc_fence_before();
+      mbar_arrive(y_free);
+      // (f) z_s = v_s . (G k_s)
+      if (!dead) dead = !mbar_wait(z_full, c & 1, lim);
+      tc_fence_after();
+      {
+        uint32_t r[32];
+        tmem_ld_half32(t_yz + lane_off, r);
+        tmem_ld_wait();
+        z = row_dot(st + 2 * TILE + rb * C * 128, r);
+      }
+      tc_fence_before();
+      mbar_arrive(&empty[s]);  // done with this stage's V and dO rows
+      const float g0_next = (c + 1 < nch) ? take_states(c + 1) : 0.f;
+      // (g) rf_i = sum_{s<=i} beta^(i-s) F_is
+      if (!dead) dead = !mbar_wait(f_full, c & 1, lim);
+      tc_fence_after();
+      float rf = 0.f;
+      {
+        uint32_t r[32];
+        tmem_ld_half32(t_f + lane_off, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int sc = 32 * half + jj;
+          rf += (sc <= row64h) ? bpow[max(row64h - sc, 0)] * __uint_as_float(r[jj]) : 0.f;
+        }
+        rf += __shfl_xor_sync(0xffffffffu, rf, 16);
+      }
+      tc_fence_before();
+      mbar_arrive(f_free);
+      // (h) prefix sums of y (half 0) and of beta-weighted z (half 1) over the
+      // chunk, then this block's part of deta
+      if (half == 0) {
+        ys[row64h] = y;
+        zs[row64h] = z;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      {
+        const int i = row64h;
+        float acc = 0.f;
+        if (half == 0) {
+          for (int j = 0; j < i; ++j) acc += ys[j];
+        } else {
+          for (int j = 0; j <= i; ++j) acc = fmaf(bpow[i - j], zs[j], acc);
+        }
+        const float other = __shfl_xor_sync(0xffffffffu, acc, 16);
+        if (half == 0 && i < n) {
+          const float ypre = acc, zpre = other;
+          const float val = bpow[i + 1] * (g0 - ypre) - p.sigma * zpre + p.sigma * rf;
+          atomicAdd(TTT_AT(p.deta, static_cast<size_t>(bh) * p.T + c * C + i, 1, static_cast<size_t>(p.BH) * p.T), -val);
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      g0 = g0_next;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::TCOLS);
+}
+
+}  // namespace ttt

@@ -20,6 +20,7 @@
 #include "../../include/ttt_la.h"
 #include "backward.cuh"
 #include "backward_chunked.cuh"
+#include "backward_mom_tc.cuh"
 #include "chunked_simt.cuh"
 #include "chunked_tc.cuh"
 #include "chunked_tc_mom.cuh"
@@ -447,6 +448,67 @@ size_t tcm_ws_floats(int bh, int nseg, int D) { return static_cast<size_t>(bh) *
 size_t tcm_ws_bytes(int bh, int nseg, int D) {
   const size_t b = tcm_ws_floats(bh, nseg, D) * sizeof(float) + tc_flag_words(bh, nseg) * sizeof(unsigned);
   return (b + 15) & ~static_cast<size_t>(15);
+}
+
+// Chunkwise momentum backward (backward_mom_tc.cuh): one block per (b, h)
+// and 64 rows of the state.
+// Reverse kernel: rows of `kr` (the K role) get the output rows `out`; qr,
+// dr are the Q and dO roles; G_in/X_in the chunk-end states of the sequence
+// (nullptr: zero); G_out/X_out its chunk-start states (nullptr: not written).
+template <int D>
+ttt_la_status launch_mom_rev(int BH, int T, const void* kr, const void* qr, const void* dr, void* out,
+                             const float* eta, float eta_const, float sigma, float beta, const float* G_in,
+                             const float* X_in, float* G_out, float* X_out, cudaStream_t st) {
+  using Cfg = ttt::MomRevCfg<D>;
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::mom_bwd_rev_kernel<D>), Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+  CUtensorMap mk, mq, md, mo;
+  if (!make_map(&mk, kr, BH, T, D, Cfg::C) || !make_map(&mq, qr, BH, T, D, Cfg::C) ||
+      !make_map(&md, dr, BH, T, D, Cfg::C) || !make_map(&mo, out, BH, T, D, Cfg::C))
+    return TTT_LA_ERR_CUDA;
+  ttt::MomBwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.BH = BH;
+  p.T = T;
+  p.nchunks = (T + Cfg::C - 1) / Cfg::C;
+  p.eta = eta;
+  p.eta_const = eta_const;
+  p.sigma = sigma;
+  p.beta = beta;
+  p.G_in = G_in;
+  p.X_in = X_in;
+  p.G_out = G_out;
+  p.X_out = X_out;
+  p.limit_ns = g_limit_ns;
+  return launch_kernel(ttt::mom_bwd_rev_kernel<D>, BH * (D / Cfg::RS), Cfg::THREADS, Cfg::SMEM, st, false, mk, mq, md,
+                       mo, p);
+}
+
+// deta kernel: G_in = dL/dW_0 (required), X_in = M_0 (nullptr: zero).
+template <int D>
+ttt_la_status launch_mom_deta(int BH, int T, const void* q, const void* k, const void* v, const void* dO,
+                              float sigma, float beta, const float* G_in, const float* X_in, float* deta,
+                              cudaStream_t st) {
+  using Cfg = ttt::MomDetaCfg<D>;
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::mom_bwd_deta_kernel<D>), Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+  CUtensorMap mq, mk, mv, md;
+  if (!make_map(&mq, q, BH, T, D, Cfg::C) || !make_map(&mk, k, BH, T, D, Cfg::C) ||
+      !make_map(&mv, v, BH, T, D, Cfg::C) || !make_map(&md, dO, BH, T, D, Cfg::C))
+    return TTT_LA_ERR_CUDA;
+  ttt::MomBwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.BH = BH;
+  p.T = T;
+  p.nchunks = (T + Cfg::C - 1) / Cfg::C;
+  p.sigma = sigma;
+  p.beta = beta;
+  p.G_in = G_in;
+  p.X_in = X_in;
+  p.deta = deta;
+  p.limit_ns = g_limit_ns;
+  // the blocks of a head add their rows' parts
+  if (cudaMemsetAsync(deta, 0, static_cast<size_t>(BH) * T * sizeof(float), st) != cudaSuccess) return TTT_LA_ERR_CUDA;
+  return launch_kernel(ttt::mom_bwd_deta_kernel<D>, BH * (D / Cfg::RS), Cfg::THREADS, Cfg::SMEM, st, false, mq, mk, mv,
+                       md, p);
 }
 
 size_t workspace_for(const ttt_la_args* a) {
@@ -1040,10 +1102,36 @@ ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 // of the inputs reversed along T and a finishing kernel forms dv, dk, deta.
 namespace {
 struct BwdChunkedLayout {
-  size_t rev[4], u, r, w0t, dwt, fwd, total, fwd_bytes;
+  size_t rev[4], u, r, w0t, dwt, m0t, dmt, dw0, fwd, total, fwd_bytes;
 };
 
 bool bwdc_fused(const ttt_la_grad_args* a) { return a->dtype == TTT_LA_BF16; }
+bool bwdc_mom(const ttt_la_grad_args* a) { return a->beta != 0.f; }
+
+// Momentum: the dq pass, the momentum forward on (q, k, v) := (do, v, k)
+// from W_0^T and M_0^T (64-token tiles).
+ttt_la_args bwdc_mom_dq(const ttt_la_grad_args* a, const float* w0t, const float* m0t) {
+  ttt_la_args f;
+  std::memset(&f, 0, sizeof f);
+  f.B = a->B;
+  f.H = a->H;
+  f.T = a->T;
+  f.d_k = a->d_v;
+  f.d_v = a->d_k;
+  f.dtype = a->dtype;
+  f.chunk = 64;
+  f.beta = a->beta;
+  f.q = a->grad_o;
+  f.k = a->v;
+  f.v = a->k;
+  f.eta = a->eta;
+  f.eta_const = a->eta_const;
+  f.ascent = a->ascent;
+  f.state_in = w0t;
+  f.mom_in = m0t;
+  f.o = a->grad_q;
+  return f;
+}
 
 // bf16: the tiles of the reverse passes (d = 64: 128 tokens, d = 128: 64);
 // fp32: the fp32 chunked path's 64.
@@ -1128,12 +1216,24 @@ BwdChunkedLayout bwdc_layout(const ttt_la_grad_args* a) {
   off += a->state_in ? ns : 0;
   L.dwt = off;
   off += a->grad_state ? ns : 0;
+  const bool mom = bwdc_mom(a);
+  L.m0t = off;  // momentum: M_0^T, (dL/dM_T)^T, and dL/dW_0 when the caller does not take it
+  off += (mom && a->mom_in) ? ns : 0;
+  L.dmt = off;
+  off += (mom && a->grad_mom) ? ns : 0;
+  L.dw0 = off;
+  off += (mom && !a->grad_state_in) ? ns : 0;
   L.fwd = off;
   L.fwd_bytes = 0;
-  void* none[4] = {nullptr, nullptr, nullptr, nullptr};
-  for (int p = 0; p < 3; ++p) {
-    ttt_la_args f = bwdc_pass(a, p, none, nullptr, nullptr, nullptr, nullptr);
-    L.fwd_bytes = std::max(L.fwd_bytes, ttt_la_workspace_size(&f));
+  if (mom) {
+    ttt_la_args f = bwdc_mom_dq(a, nullptr, nullptr);
+    L.fwd_bytes = ttt_la_workspace_size(&f);
+  } else {
+    void* none[4] = {nullptr, nullptr, nullptr, nullptr};
+    for (int p = 0; p < 3; ++p) {
+      ttt_la_args f = bwdc_pass(a, p, none, nullptr, nullptr, nullptr, nullptr);
+      L.fwd_bytes = std::max(L.fwd_bytes, ttt_la_workspace_size(&f));
+    }
   }
   L.total = off + align256(L.fwd_bytes);
   return L;
@@ -1142,12 +1242,60 @@ BwdChunkedLayout bwdc_layout(const ttt_la_grad_args* a) {
 ttt_la_status check_grad_chunked(const ttt_la_grad_args* a) {
   const ttt_la_status s = check_grad_common(a);
   if (s != TTT_LA_OK) return s;
-  if (a->beta != 0.f || a->mom_in || a->grad_mom) return TTT_LA_ERR_UNSUPPORTED;
+  if (a->beta == 0.f && (a->mom_in || a->grad_mom)) return TTT_LA_ERR_UNSUPPORTED;
+  if (a->beta != 0.f && a->dtype != TTT_LA_BF16) return TTT_LA_ERR_UNSUPPORTED;  // momentum: bf16 tensor cores
   if (a->dtype == TTT_LA_BF16 && !(a->d_k == a->d_v && (a->d_k == 64 || a->d_k == 128)))
     return TTT_LA_ERR_UNSUPPORTED;
   if (a->dtype == TTT_LA_F32 && (a->d_k % 4 || a->d_v % 4 || a->d_k > 128 || a->d_v > 128))
     return TTT_LA_ERR_UNSUPPORTED;
   if (!a->workspace || a->workspace_bytes < bwdc_layout(a).total) return TTT_LA_ERR_INVALID_ARG;
+  return TTT_LA_OK;
+}
+
+// Momentum (bf16): transposes of W_0, M_0, dL/dW_T, dL/dM_T; dq from the
+// momentum forward; dv, dL/dW_0, dL/dM_0 from the reverse kernel on (k, q,
+// do); dk from it on (v, do, q) with the transposed states; deta from the
+// forward-order kernel (backward_mom_tc.cuh).
+template <int D>
+ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLayout& L, cudaStream_t st) {
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  auto at = [&](bool present, size_t off) { return present ? reinterpret_cast<float*>(ws + off) : nullptr; };
+  float* w0t = at(a->state_in != nullptr, L.w0t);
+  float* dwt = at(a->grad_state != nullptr, L.dwt);
+  float* m0t = at(a->mom_in != nullptr, L.m0t);
+  float* dmt = at(a->grad_mom != nullptr, L.dmt);
+  float* dw0 = a->grad_state_in ? a->grad_state_in : reinterpret_cast<float*>(ws + L.dw0);
+  const int BH = a->B * a->H;
+  ttt_la_status s;
+  ttt::TransposeParams tp;
+  std::memset(&tp, 0, sizeof tp);
+  tp.BH = BH;
+  tp.R = D;
+  tp.C = D;
+  const float* src[4] = {a->state_in, a->mom_in, a->grad_state, a->grad_mom};
+  float* dst[4] = {w0t, m0t, dwt, dmt};
+  for (int i = 0; i < 4; ++i)
+    if (src[i]) {
+      tp.src[tp.n] = src[i];
+      tp.dst[tp.n++] = dst[i];
+    }
+  if (tp.n > 0) {
+    ttt::transpose_states_kernel<<<sm_count() * 4, 256, 0, st>>>(tp);
+    if ((s = launched()) != TTT_LA_OK) return s;
+  }
+  ttt_la_args f = bwdc_mom_dq(a, w0t, m0t);
+  f.workspace = L.fwd_bytes ? ws + L.fwd : nullptr;
+  f.workspace_bytes = L.fwd_bytes;
+  if ((s = ttt_la_forward_chunked(&f, st)) != TTT_LA_OK) return s;
+  const float sigma = a->ascent ? -1.f : 1.f;
+  if ((s = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma, a->beta,
+                             a->grad_state, a->grad_mom, dw0, a->grad_mom_in, st)) != TTT_LA_OK)
+    return s;
+  if ((s = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma, a->beta, dwt,
+                             dmt, nullptr, nullptr, st)) != TTT_LA_OK)
+    return s;
+  if (a->grad_eta)
+    return launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, st);
   return TTT_LA_OK;
 }
 }  // namespace
@@ -1165,6 +1313,8 @@ ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args* a, void* stream) {
   if (s != TTT_LA_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const BwdChunkedLayout L = bwdc_layout(a);
+  if (bwdc_mom(a))
+    return a->d_k == 64 ? backward_chunked_mom<64>(a, L, st) : backward_chunked_mom<128>(a, L, st);
   const bool fused = bwdc_fused(a);
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   void* rev[4] = {ws + L.rev[0], ws + L.rev[1], ws + L.rev[2], ws + L.rev[3]};

@@ -373,12 +373,26 @@ def test_backward_chunked_workspace_and_validation(abi):
     assert size(f) >= 6 * (2 * 2 * 100 * 64 * 4)
     assert L.ttt_la_backward_chunked_workspace_size(None) == 0
     assert L.ttt_la_backward_chunked(None, None) == abi.ERR_INVALID_ARG
-    # momentum is the recurrent form's
-    for field, val in [("beta", 0.9), ("mom_in", 0xA000000), ("grad_mom", 0xB000000)]:
+    # momentum states without momentum, and momentum in fp32 (the recurrent form's)
+    for field, val in [("mom_in", 0xA000000), ("grad_mom", 0xB000000)]:
         g = _grad_args(abi)
         setattr(g, field, val)
         g.workspace_bytes = 1 << 40
         assert call(g) == abi.ERR_UNSUPPORTED, field
+    g = _grad_args(abi, beta=0.9)
+    g.dtype = abi.F32
+    g.workspace_bytes = 1 << 40
+    assert call(g) == abi.ERR_UNSUPPORTED
+    g = _grad_args(abi, dk=64, dv=128, beta=0.9)
+    g.workspace_bytes = 1 << 40
+    assert call(g) == abi.ERR_UNSUPPORTED
+    # momentum scratch: the four transposed states, and dL/dW_0 when the caller does not take it
+    g = _grad_args(abi, T=100, beta=0.9)
+    base = size(g)
+    g.state_in, g.mom_in, g.grad_state, g.grad_mom = 0x8000000, 0xA000000, 0x9000000, 0xB000000
+    assert size(g) == base + 4 * 2 * 2 * 64 * 64 * 4
+    g.grad_state_in = 0xC000000
+    assert size(g) == base + 3 * 2 * 2 * 64 * 64 * 4
     g = _grad_args(abi, dk=64, dv=128)  # the bf16 tensor-core forward wants d_k == d_v
     g.workspace_bytes = 1 << 40
     assert call(g) == abi.ERR_UNSUPPORTED

@@ -95,3 +95,41 @@ def test_backward_chunked_long_sequence_schedules(d, T, wave_tokens, monkeypatch
     torch.cuda.synchronize()
     for n in ("dq", "dk", "dv", "deta", "dW0"):
         assert_bf16(a[n], f64(b[n]), n)
+
+
+def _mom_case(B, H, T, d, seed, token_eta=True, states=True):
+    x = _case(B, H, T, d, d, "bf16", seed, token_eta, states)
+    g = torch.Generator().manual_seed(seed + 3000)
+    x["M0"] = (0.3 * torch.randn(B, H, d, d, generator=g)).cuda() if states else None
+    x["dM"] = torch.randn(B, H, d, d, generator=g).cuda() if states else None
+    return x
+
+
+@pytest.mark.parametrize("d,T,token_eta,ascent,states", [(64, 300, True, False, True), (128, 257, True, True, True),
+                                                         (64, 1, True, True, True), (128, 64, False, False, False),
+                                                         (128, 1, True, False, True), (64, 129, False, True, True)])
+def test_backward_chunked_momentum_matches_oracle(d, T, token_eta, ascent, states):
+    """beta = 0.9: dq from the momentum forward, dv / dk / dW0 / dM0 from the
+    reverse chunkwise kernel, deta from the forward-order one."""
+    x = _mom_case(2, 3, T, d, 210 + d + T, token_eta, states)
+    g = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], eta_const=x["ec"], ascent=ascent,
+                              state_in=x["S0"], grad_state=x["dW"], beta=0.9, mom_in=x["M0"], grad_mom=x["dM"])
+    torch.cuda.synchronize()
+    e = f64(x["eta"]) if x["eta"] is not None else x["ec"]
+    ref = oracle.ttt_backward_f64(f64(x["q"]), f64(x["k"]), f64(x["v"]), e, f64(x["dO"]), f64(x["dW"]),
+                                  f64(x["dM"]), beta=0.9, ascent=ascent, S0=f64(x["S0"]), M0=f64(x["M0"]))
+    for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
+        assert_bf16(g[n], ref[n], n)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_chunked_momentum_agrees_with_recurrent(d):
+    """Four heads of a long ragged sequence (dozens of chunks carried by one
+    block each): the chunkwise and recurrent momentum backwards agree."""
+    x = _mom_case(1, 4, 64 * 60 + 7, d, 260 + d)
+    kw = dict(state_in=x["S0"], grad_state=x["dW"], beta=0.9, mom_in=x["M0"], grad_mom=x["dM"], ascent=True)
+    a = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], **kw)
+    b = _abi.backward_recurrent(x["q"], x["k"], x["v"], x["dO"], x["eta"], **kw)
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
+        assert_bf16(a[n], f64(b[n]), n)

@@ -103,3 +103,31 @@ def test_debug_build_backward_checks_stay_clean(d, B, H, T, wave_tokens, monkeyp
     torch.cuda.synchronize()
     for n in ("dq", "dk", "dv", "deta", "dW0"):
         assert_bf16(out[n], f64(ref[n]), n)
+
+
+@pytest.mark.parametrize("d,T", [(64, 64 * 5 + 3), (128, 64 * 3 + 1)])
+def test_debug_build_momentum_backward_checks_stay_clean(d, T):
+    """The chunkwise momentum backward (reverse and deta kernels) with every
+    state given, ragged T, through the debug build."""
+    from test_layers_causal_b200 import _abi
+    L = _abi.debug_lib()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    L.ttt_la_debug_check_line(st)
+    L.ttt_la_get_last_device_status(st)
+    q, k, v, eta = _inputs(2, 2, T, d, 500 + d + T)
+    g = torch.Generator().manual_seed(9)
+    dO = torch.randn(v.shape, generator=g).to(torch.bfloat16).cuda()
+    S0, M0, dW, dM = (0.2 * torch.randn(2, 2, d, d, generator=g)).cuda(), (0.2 * torch.randn(2, 2, d, d, generator=g)).cuda(), \
+        torch.randn(2, 2, d, d, generator=g).cuda(), torch.randn(2, 2, d, d, generator=g).cuda()
+    a, out = _abi._chunked_grad_args(q, k, v, dO, eta, None, False, S0, dW, 0.9, M0, dM)
+    need = int(L.ttt_la_backward_chunked_workspace_size(ctypes.byref(a)))
+    ws = torch.full((max(need, 16),), 0x7F, dtype=torch.uint8, device="cuda")
+    a.workspace, a.workspace_bytes = ws.data_ptr(), need
+    code = L.ttt_la_backward_chunked(ctypes.byref(a), st)
+    assert code == 0, _abi.status_string(code)
+    assert L.ttt_la_get_last_device_status(st) == _abi.OK
+    assert L.ttt_la_debug_check_line(st) == 0
+    ref = _abi.backward_recurrent(q, k, v, dO, eta, beta=0.9, state_in=S0, mom_in=M0, grad_state=dW, grad_mom=dM)
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
+        assert_bf16(out[n], f64(ref[n]), n)
