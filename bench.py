@@ -436,31 +436,44 @@ def phi_measure(ttt, dev, peaks, reps=100):
             "gpu_launches_per_step": 2}
 
 
-def backward_measure(ttt, dev, peaks, reps=5):
-    """The layer's backward on the llm_d64 inputs (B4 H16 T4096 d64, per-token
-    eta) with a seeded upstream gradient dL/do and dL/dW_T: dq, dk, dv,
-    per-token deta and dW0, in both forms -- the recurrent kernel (one block
-    per head) and the chunk-parallel one (a transpose of dL/dW_T and three
-    chunked forward runs, the two reverse-time ones writing dv, deta and dk
-    themselves: four launches).  CUDA events over `reps` calls after one
-    warm-up call of each."""
-    c = CONFIGS["llm_d64"]
+def backward_measure(ttt, dev, peaks, name="llm_d64", reps=5):
+    """The layer's backward on a workload's inputs with a seeded upstream
+    gradient dL/do, dL/dW_T (and dL/dM_T with momentum): dq, dk, dv, per-token
+    deta, dW0 (and dM0), in both forms -- the recurrent kernel (one block per
+    head) and the chunk-parallel one.  Without momentum that is a transpose of
+    dL/dW_T and three chunked forward runs, the two reverse-time ones writing
+    dv, deta and dk themselves (four launches); with momentum, one transpose
+    launch, the momentum forward for dq, the reverse chunkwise kernel twice
+    and the deta kernel (five).  Workspaces are allocated once; CUDA events
+    over `reps` calls (the chunked form 20x as many) after one warm-up call of
+    each."""
+    c = CONFIGS[name]
     x = make_case(c)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
     eta = x["eta"].to(dev)
     g = torch.Generator(device=dev).manual_seed(11)
     dO = torch.randn(v.shape, generator=g, device=dev).to(v.dtype)
     dW = torch.randn(c.B, c.H, c.d_v, c.d_k, generator=g, device=dev)
+    dM = torch.randn(c.B, c.H, c.d_v, c.d_k, generator=g, device=dev) if c.beta else None
     stream = torch.cuda.current_stream()
     # bytes a backward must move: q, k, v, dO read, dq, dk, dv written (bf16),
-    # eta read and deta written (fp32), dL/dW_T read and dL/dW_0 written
-    nbytes = c.B * c.H * (c.T * (2 * (2 * c.d_k + 2 * c.d_v) + 2 * (2 * c.d_k + c.d_v) + 8) + 2 * 4 * c.d_v * c.d_k)
-    out = {"workload": "llm_d64 backward (dq, dk, dv, deta, dW0 from dL/do and dL/dW_T)",
-           "algorithmic_bytes": nbytes}
-    ws = {}
-    for name, fn, n in (("recurrent", ttt.backward_recurrent, reps), ("chunked", ttt.backward_chunked, 20 * reps)):
+    # eta read and deta written (fp32), dL/dW_T read and dL/dW_0 written (and
+    # the same pair for M with momentum)
+    nstates = 4 if c.beta else 2
+    nbytes = c.B * c.H * (c.T * (2 * (2 * c.d_k + 2 * c.d_v) + 2 * (2 * c.d_k + c.d_v) + 8)
+                          + nstates * 4 * c.d_v * c.d_k)
+    what = "dq, dk, dv, deta, dW0, dM0 from dL/do, dL/dW_T and dL/dM_T" if c.beta else \
+        "dq, dk, dv, deta, dW0 from dL/do and dL/dW_T"
+    out = {"workload": f"{name} backward ({what})", "algorithmic_bytes": nbytes}
+    # generous preallocated scratch (the recurrent form keeps checkpoints of W and M)
+    ws = {"recurrent": torch.empty(3 << 30, dtype=torch.uint8, device=dev),
+          "chunked": torch.empty(256 << 20, dtype=torch.uint8, device=dev)}
+    kw = dict(eta_const=x["eta_const"], grad_state=dW)
+    if c.beta:
+        kw.update(beta=c.beta, grad_mom=dM)
+    for form, fn, n in (("recurrent", ttt.backward_recurrent, reps), ("chunked", ttt.backward_chunked, 20 * reps)):
         def call():
-            return fn(q, k, v, dO, eta, eta_const=x["eta_const"], grad_state=dW, workspace=ws.get(name))
+            return fn(q, k, v, dO, eta, workspace=ws[form], **kw)
         r = call()
         del r
         torch.cuda.synchronize()
@@ -475,10 +488,11 @@ def backward_measure(ttt, dev, peaks, reps=5):
             raise SystemExit("device status reports a timed-out wait")
         us = e0.elapsed_time(e1) * 1e3 / n
         gbs = nbytes / (us * 1e-6) / 1e9
-        out[name] = {"us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6), "hbm_gbs": gbs,
+        out[form] = {"us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6), "hbm_gbs": gbs,
                      "hbm_frac": gbs / peaks["hbm_gbs"],
-                     "gpu_launches_per_call": 1 if name == "recurrent" else 4}
+                     "gpu_launches_per_call": 1 if form == "recurrent" else (5 if c.beta else 4)}
     out["chunked_speedup_over_recurrent"] = out["recurrent"]["us_per_call"] / out["chunked"]["us_per_call"]
+    del ws
     torch.cuda.empty_cache()
     return out
 
@@ -648,6 +662,7 @@ def run_ours(args, c, ws, rank, local, info):
         line["phi_layer"] = phi_measure(ttt, dev, peaks)
         torch.cuda.empty_cache()
         line["backward"] = backward_measure(ttt, dev, peaks)
+        line["backward_momentum"] = backward_measure(ttt, dev, peaks, "momentum_d128", reps=2)
     if rank == 0 and not args.no_cpu_baseline:
         tokens = args.cpu_tokens or CPU_TOKENS.get(c.name, c.T)
         line["cpu_baseline"], o_ref = cpu_baseline(c, tokens, x)
@@ -660,7 +675,9 @@ def run_ours(args, c, ws, rank, local, info):
 def profile_run(args):
     """Plain launches (no graphs, no timing) for ncu: --warmup + --steps calls
     of the workload's forward, of the decode step on a random 256 MiB state,
-    or (phi) of the feature map plus chunked forward on the llm_d64 shape."""
+    (phi) of the feature map plus chunked forward on the llm_d64 shape, or of
+    the chunk-parallel backward on the llm_d64 (backward) or momentum_d128
+    (backward_momentum) inputs."""
     import test_layers_causal_b200 as ttt
     dev = torch.device("cuda", 0)
     if args.workload == "decode":
@@ -679,6 +696,18 @@ def profile_run(args):
         W1, W3 = (w.to(dev) for w in make_feature_weights(c.H, c.d_k, c.d_k, 7))
         for _ in range(args.warmup + args.steps):
             ttt.forward_chunked_phi(q, k, v, W1, W3, x["eta"].to(dev), eta_const=x["eta_const"], chunk=c.chunk)
+    elif args.workload in ("backward", "backward_momentum"):
+        c = CONFIGS["llm_d64" if args.workload == "backward" else "momentum_d128"]
+        x = make_case(c)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        g = torch.Generator(device=dev).manual_seed(11)
+        dO = torch.randn(v.shape, generator=g, device=dev).to(v.dtype)
+        kw = dict(eta_const=x["eta_const"], grad_state=torch.randn(c.B, c.H, c.d_v, c.d_k, generator=g, device=dev),
+                  workspace=torch.empty(256 << 20, dtype=torch.uint8, device=dev))
+        if c.beta:
+            kw.update(beta=c.beta, grad_mom=torch.randn(c.B, c.H, c.d_v, c.d_k, generator=g, device=dev))
+        for _ in range(args.warmup + args.steps):
+            ttt.backward_chunked(q, k, v, dO, x["eta"].to(dev), **kw)
     else:
         c = CONFIGS[args.workload]
         x = make_case(c)
@@ -699,7 +728,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="long_d128", choices=sorted(CONFIGS) + ["decode", "phi"])
+    ap.add_argument("--workload", default="long_d128",
+                    choices=sorted(CONFIGS) + ["decode", "phi", "backward", "backward_momentum"])
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--sets", type=int, default=4)
@@ -716,7 +746,7 @@ def main():
     if args.profile_run:
         profile_run(args)
         return
-    if args.workload in ("decode", "phi"):
+    if args.workload in ("decode", "phi", "backward", "backward_momentum"):
         raise SystemExit(f"{args.workload} is measured inside every chunked run (its own object in the line)")
     c = CONFIGS[args.workload]
     if c.dtype != "bf16":

@@ -1162,6 +1162,8 @@ ttt_la_args bwdc_pass(const ttt_la_grad_args* a, int p, void* const* rev, void* 
     f.ascent = fused ? a->ascent : 0;
   }
   if (p == 0) {  // W_t^T do_t: keys v, values k, from W_0^T, the layer's eta and sigma
+    // (a plain forward: bf16 takes the forward's own best tile, 64 tokens at d = 64, 128 at d = 128)
+    if (a->dtype == TTT_LA_BF16) f.chunk = a->d_k == 64 ? 64 : 128;
     f.d_k = a->d_v;
     f.d_v = a->d_k;
     f.q = a->grad_o;
