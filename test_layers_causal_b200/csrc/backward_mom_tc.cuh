@@ -32,9 +32,10 @@
 //   y_j = do_j . (M q_j),  z_s = v_s . (G k_s),
 //   F = Lstrict (Q K^T o dO V^T)   (Lstrict: ones strictly below the diagonal)
 //   M <- beta^n M - sigma sum_s beta^(n-1-s) v_s k_s^T,  P <- P + sum_j do_j q_j^T.
-// y and z read M and G through two bf16 MMAs each (bf16(x) + bf16(x -
-// bf16(x))), which carries them to about 2^-17: deta is a d^2-term inner
-// product that can cancel.
+// z reads G through two bf16 MMAs (bf16(x) + bf16(x - bf16(x)), which carries
+// it to about 2^-17): deta is a d^2-term inner product that can cancel, and
+// G holds dL/dW_T.  y reads M in bf16 alone (its rounding measured no larger
+// than the rest at the test scales).
 //
 // One block per (b, h, 64 rows of the state) walks its chunks in order (no
 // segment scan): every term above is linear in the rows of the states (and of
@@ -78,6 +79,20 @@ __device__ __forceinline__ void store_row32_split(uint32_t hi, uint32_t lo, int 
   store_row32_bf16(lo, 64 * 128, row, col0, r);
 }
 
+// Store counterpart of tmem_ld_half32 (common.cuh): threads 0-15 write lanes
+// 0-15 of the warp's quadrant at columns [c, c + 32), threads 16-31 the same
+// lanes at [c + 32, c + 64).
+__device__ __forceinline__ void tmem_st_half32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
 // A block's share of the state rows (one M = 64 accumulator).
 constexpr int kMomRows = 64;
 
@@ -111,9 +126,8 @@ struct MomDetaCfg {
   static constexpr int NST = 2;
   static constexpr int STAGE = 4 * TILE;          // Q, K, V, dO
   static constexpr int SQ = RS * D * 2;
-  static constexpr int OFF_MBF = NST * STAGE;     // bf16 rows of M, their residual, the same of G
-  static constexpr int OFF_MLO = OFF_MBF + SQ;
-  static constexpr int OFF_GBF = OFF_MLO + SQ;
+  static constexpr int OFF_MBF = NST * STAGE;     // bf16 rows of M; bf16 rows of G and their residual
+  static constexpr int OFF_GBF = OFF_MBF + SQ;
   static constexpr int OFF_GLO = OFF_GBF + SQ;
   static constexpr int OFF_KB = OFF_GLO + SQ;     // diag(-sigma beta^(n-1-s)) K
   static constexpr int OFF_A = OFF_KB + TILE;     // bf16(Q K^T o dO V^T), token-major
@@ -359,13 +373,11 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
     // --------------------------------------------------------- epilogue --
     const int g4 = warp & 3;  // TMEM lane quadrant of this warp
     const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
-    // M = 64 accumulators: lanes 0-15 of each quadrant hold rows 16 g4 + lane
-    const int wrow = 16 * g4 + lane;
-    const bool wrow_ok = lane < 16;
-    // read with the whole warp: row 16 g4 + lane % 16, column half lane / 16
+    // M = 64 accumulators fill lanes 0-15 of each quadrant; the whole warp
+    // reads them: row 16 g4 + lane % 16, column half lane / 16
     const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
     const size_t DD = static_cast<size_t>(D) * D, nst = static_cast<size_t>(p.BH) * DD;
-    const size_t grow = bh * DD + static_cast<size_t>(r0 + wrow) * D;  // this thread's state row in global
+    const size_t grow = bh * DD + static_cast<size_t>(r0 + row64h) * D;  // this thread's state row in global
     bool dead = false;
     for (int c = 0; c < nch; ++c) {
       const int s = c % NST, n = nvalid(c);
@@ -376,29 +388,28 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
       tc_fence_after();
       const float xs = bpow[n], gs = -p.beta * e[0];
 #pragma unroll 1
-      for (int cb = 0; cb < D / 32; ++cb) {
+      for (int cb = 0; cb < D; cb += 64) {
+        const int col = cb + 32 * half;
         uint32_t g[32], x[32];
         if (c == 0) {
-          const float* gi = (p.G_in && wrow_ok) ? TTT_AT(p.G_in, grow + cb * 32, 32, nst) : nullptr;
-          const float* xi = (p.X_in && wrow_ok) ? TTT_AT(p.X_in, grow + cb * 32, 32, nst) : nullptr;
+          const float* gi = p.G_in ? TTT_AT(p.G_in, grow + col, 32, nst) : nullptr;
+          const float* xi = p.X_in ? TTT_AT(p.X_in, grow + col, 32, nst) : nullptr;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             g[j] = __float_as_uint(gi ? __ldg(gi + j) : 0.f);
             x[j] = __float_as_uint(xi ? __ldg(xi + j) : 0.f);
           }
-          tmem_st32(t_g + lane_off + cb * 32, g);  // G accumulator := dL/dW_T (rows)
+          tmem_st_half32(t_g + lane_off + cb, g);  // G accumulator := dL/dW_T (rows)
         } else {
-          tmem_ld32(t_g + lane_off + cb * 32, g);
-          tmem_ld32(t_x + lane_off + cb * 32, x);
+          tmem_ld_half32(t_g + lane_off + cb, g);
+          tmem_ld_half32(t_x + lane_off + cb, x);
           tmem_ld_wait();
         }
-        if (wrow_ok) {
-          store_row32_bf16(sbase + Cfg::OFF_GBF, RS * 128, wrow, cb * 32, g);
-          store_row32_bf16(sbase + Cfg::OFF_XBF, RS * 128, wrow, cb * 32, x);
-        }
+        store_row32_bf16(sbase + Cfg::OFF_GBF, RS * 128, row64h, col, g);
+        store_row32_bf16(sbase + Cfg::OFF_XBF, RS * 128, row64h, col, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = __float_as_uint(fmaf(xs, __uint_as_float(x[j]), gs * __uint_as_float(g[j])));
-        tmem_st32(t_x + lane_off + cb * 32, x);
+        tmem_st_half32(t_x + lane_off + cb, x);
       }
       tmem_st_wait();
       fence_async_smem();
@@ -457,26 +468,25 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
     if (!dead) dead = !mbar_wait(sdone, (nch - 1) & 1, lim);
     tc_fence_after();
 #pragma unroll 1
-    for (int cb = 0; cb < D / 32; ++cb) {
+    for (int cb = 0; cb < D; cb += 64) {
+      const int col = cb + 32 * half;
       uint32_t g[32], x[32];
-      tmem_ld32(t_g + lane_off + cb * 32, g);
-      tmem_ld32(t_x + lane_off + cb * 32, x);
+      tmem_ld_half32(t_g + lane_off + cb, g);
+      tmem_ld_half32(t_x + lane_off + cb, x);
       tmem_ld_wait();
-      if (wrow_ok) {
-        if (p.G_out) {
-          float4* d4 = reinterpret_cast<float4*>(TTT_AT(p.G_out, grow + cb * 32, 32, nst));
+      if (p.G_out) {
+        float4* d4 = reinterpret_cast<float4*>(TTT_AT(p.G_out, grow + col, 32, nst));
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            d4[j] = make_float4(__uint_as_float(g[4 * j]), __uint_as_float(g[4 * j + 1]), __uint_as_float(g[4 * j + 2]),
-                                __uint_as_float(g[4 * j + 3]));
-        }
-        if (p.X_out) {
-          float4* d4 = reinterpret_cast<float4*>(TTT_AT(p.X_out, grow + cb * 32, 32, nst));
+        for (int j = 0; j < 8; ++j)
+          d4[j] = make_float4(__uint_as_float(g[4 * j]), __uint_as_float(g[4 * j + 1]), __uint_as_float(g[4 * j + 2]),
+                              __uint_as_float(g[4 * j + 3]));
+      }
+      if (p.X_out) {
+        float4* d4 = reinterpret_cast<float4*>(TTT_AT(p.X_out, grow + col, 32, nst));
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            d4[j] = make_float4(__uint_as_float(x[4 * j]), __uint_as_float(x[4 * j + 1]), __uint_as_float(x[4 * j + 2]),
-                                __uint_as_float(x[4 * j + 3]));
-        }
+        for (int j = 0; j < 8; ++j)
+          d4[j] = make_float4(__uint_as_float(x[4 * j]), __uint_as_float(x[4 * j + 1]), __uint_as_float(x[4 * j + 2]),
+                              __uint_as_float(x[4 * j + 3]));
       }
     }
   }
@@ -491,7 +501,7 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
 // columns of V and dO) and adds its partial deta.  Per chunk the MMA thread
 // issues
 //   (1) S1 = Q K^T,  S2 = dO_r V_r^T            [TMEM, M=C, N=C each]
-//   (2) Y  = Q Mbf^T + Q Mlo^T                  [TMEM, M=C, N=64]
+//   (2) Y  = Q Mbf^T                            [TMEM, M=C, N=64]
 //   (2') Z = K Gbf^T + K Glo^T                  (Y's columns, once y is read)
 //   (4) M += V_r^T Kb,  P += dO_r^T Q           [TMEM, M=64, N=D]
 //   (3) F  = Lstrict A,  A = bf16(S1 o S2)      [TMEM, M=C, N=C]
@@ -612,7 +622,6 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       constexpr uint32_t ID_ST = idesc_bf16_f32(RS, D, true, true);
       constexpr uint32_t ID_F = idesc_bf16_f32(C, C, false, true);
       const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
-      const uint64_t d_mlo = sdesc_sw128(sbase + Cfg::OFF_MLO, 16, 1024);
       const uint64_t d_gbf = sdesc_sw128(sbase + Cfg::OFF_GBF, 16, 1024);
       const uint64_t d_glo = sdesc_sw128(sbase + Cfg::OFF_GLO, 16, 1024);
       const uint64_t d_kbm = sdesc_sw128(sbase + Cfg::OFF_KB, C * 128, 1024);  // MN-major
@@ -637,8 +646,6 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
         tc_commit(sc_full);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_q + k_step(C, kk), d_mbf + k_step(RS, kk), ID_Y, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_q + k_step(C, kk), d_mlo + k_step(RS, kk), ID_Y, 1);
         tc_commit(y_full);
         if (!dead) dead = !mbar_wait(y_free, c & 1, lim);
         tc_fence_after();
@@ -693,11 +700,10 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
     // --------------------------------------------------------- epilogue --
     const int g4 = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
-    const int wrow = 16 * g4 + lane;  // M = 64 state rows: lanes 0-15 of each quadrant
-    const bool wrow_ok = lane < 16;
+    // M = 64 accumulators fill lanes 0-15 of each quadrant; the whole warp
+    // reads them: row 16 g4 + lane % 16, column half lane / 16
     const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
     const size_t DD = static_cast<size_t>(D) * D, nst = static_cast<size_t>(p.BH) * DD;
-    const size_t grow = bh * DD + static_cast<size_t>(r0 + wrow) * D;
     bool dead = false;
     // this thread's half (32 columns) of row row64h of Y or Z, dotted with the
     // same columns of this block's 64 columns of a token tile
@@ -722,21 +728,24 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       tc_fence_after();
       const float bn = bpow[nvalid(c)];
       float part = 0.f;
+      // the whole warp: row row64h, columns [cb + 32 half, cb + 32 half + 32)
 #pragma unroll 1
-      for (int cb = 0; cb < D / 32; ++cb) {
-        uint32_t m[32], g[32], mm[32];
+      for (int cb = 0; cb < D; cb += 64) {
+        const int col = cb + 32 * half;
+        uint32_t m[32], g[32];
         if (c == 0) {
-          const float* mi = (p.X_in && wrow_ok) ? TTT_AT(p.X_in, grow + cb * 32, 32, nst) : nullptr;
-          const float* gi = wrow_ok ? TTT_AT(p.G_in, grow + cb * 32, 32, nst) : nullptr;
+          const size_t row = bh * DD + static_cast<size_t>(r0 + row64h) * D + col;
+          const float* mi = p.X_in ? TTT_AT(p.X_in, row, 32, nst) : nullptr;
+          const float* gi = TTT_AT(p.G_in, row, 32, nst);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             m[j] = __float_as_uint(mi ? __ldg(mi + j) : 0.f);
-            g[j] = __float_as_uint(gi ? -__ldg(gi + j) : 0.f);  // P := -dL/dW_0
+            g[j] = __float_as_uint(-__ldg(gi + j));  // P := -dL/dW_0
           }
-          tmem_st32(t_p + lane_off + cb * 32, g);
+          tmem_st_half32(t_p + lane_off + cb, g);
         } else {
-          tmem_ld32(t_m + lane_off + cb * 32, m);
-          tmem_ld32(t_p + lane_off + cb * 32, g);
+          tmem_ld_half32(t_m + lane_off + cb, m);
+          tmem_ld_half32(t_p + lane_off + cb, g);
           tmem_ld_wait();
         }
 #pragma unroll
@@ -744,16 +753,14 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
           const float gj = -__uint_as_float(g[j]);  // G = -P
           g[j] = __float_as_uint(gj);
           part = fmaf(gj, __uint_as_float(m[j]), part);
-          mm[j] = __float_as_uint(bn * __uint_as_float(m[j]));
         }
-        tmem_st32(t_m + lane_off + cb * 32, mm);
-        if (wrow_ok) {
-          store_row32_split(sbase + Cfg::OFF_MBF, sbase + Cfg::OFF_MLO, wrow, cb * 32, m);
-          store_row32_split(sbase + Cfg::OFF_GBF, sbase + Cfg::OFF_GLO, wrow, cb * 32, g);
-        }
+        store_row32_bf16(sbase + Cfg::OFF_MBF, RS * 128, row64h, col, m);
+        store_row32_split(sbase + Cfg::OFF_GBF, sbase + Cfg::OFF_GLO, row64h, col, g);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m[j] = __float_as_uint(bn * __uint_as_float(m[j]));
+        tmem_st_half32(t_m + lane_off + cb, m);
       }
       tmem_st_wait();
-      if (!wrow_ok) part = 0.f;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
       // by chunk parity: the barrier of chunk c+1's call orders chunk c+2's writes after these reads
