@@ -103,9 +103,10 @@ struct MomRevCfg {
   static constexpr int SQ = RS * D * 2;           // bf16 RS x D
   static constexpr int NST = 2;
   static constexpr int STAGE = 3 * TILE;          // K, Q, dO roles
-  static constexpr int OFF_XBF = NST * STAGE;     // bf16 rows of X (B operand)
-  static constexpr int OFF_GBF = OFF_XBF + SQ;
-  static constexpr int OFF_QW = OFF_GBF + SQ;     // [2] diag(-beta w_0j) Q (chunk parity)
+  // bf16 rows of X and of G stacked as one B operand of 128 rows per
+  // 64-column block (X rows 0-63, G rows 64-127), so (2) is one N = 128 MMA
+  static constexpr int OFF_XG = NST * STAGE;
+  static constexpr int OFF_QW = OFF_XG + 2 * SQ;  // [2] diag(-beta w_0j) Q (chunk parity)
   static constexpr int OFF_P = OFF_QW + 2 * TILE; // C x C weights
   static constexpr int BIG = OFF_P + C * C * 2;
   static constexpr int NE = 3;                    // coefficient slots
@@ -124,10 +125,13 @@ struct MomDetaCfg {
   static constexpr int C = 64, RS = kMomRows;
   static constexpr int TILE = C * D * 2;
   static constexpr int NST = 2;
-  static constexpr int STAGE = 4 * TILE;          // Q, K, V, dO
+  // Q, then K with the chunk's bf16 rows of M stacked below it (one B
+  // operand of 128 rows per 64-column block: K rows 0-63, M rows 64-127),
+  // then V and dO
+  static constexpr int OFF_SK = TILE, OFF_SV = 3 * TILE, OFF_SD = 4 * TILE;
+  static constexpr int STAGE = 5 * TILE;
   static constexpr int SQ = RS * D * 2;
-  static constexpr int OFF_MBF = NST * STAGE;     // bf16 rows of M; bf16 rows of G and their residual
-  static constexpr int OFF_GBF = OFF_MBF + SQ;
+  static constexpr int OFF_GBF = NST * STAGE;     // bf16 rows of G and their residual
   static constexpr int OFF_GLO = OFF_GBF + SQ;
   static constexpr int OFF_KB = OFF_GLO + SQ;     // diag(-sigma beta^(n-1-s)) K
   static constexpr int OFF_A = OFF_KB + TILE;     // bf16(Q K^T o dO V^T), token-major
@@ -149,7 +153,7 @@ struct MomDetaCfg {
 // [r0, r0 + 64) and output columns [r0, r0 + 64) (dO_r: those columns of dO).
 // Per chunk the MMA thread issues
 //   (1) S  = K Q^T                            [TMEM, M=C, N=C]
-//   (2) U1 = K Xbf^T,  U2 = K Gbf^T           [TMEM, M=C, N=64 each]
+//   (2) [U1 | U2] = K [Xbf ; Gbf]^T           [TMEM, M=C, N=128]
 //   (3) G += dO_r^T Q,  (4) X += dO_r^T Qw    [TMEM, M=64, N=D]
 //   (5) U3 = P dO_r                           P = bf16(sigma w o triu(S))
 // after the epilogue has taken Xbf, Gbf and replaced X by beta^n X - beta e_0 G;
@@ -261,11 +265,10 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
     if (lane == 0) {
       bool dead = false;
       constexpr uint32_t ID_S = idesc_bf16_f32(C, C, false, false);
-      constexpr uint32_t ID_U = idesc_bf16_f32(C, RS, false, false);
+      constexpr uint32_t ID_U = idesc_bf16_f32(C, 2 * RS, false, false);
       constexpr uint32_t ID_ST = idesc_bf16_f32(RS, D, true, true);
       constexpr uint32_t ID_PU = idesc_bf16_f32(C, RS, false, true);
-      const uint64_t d_xbf = sdesc_sw128(sbase + Cfg::OFF_XBF, 16, 1024);
-      const uint64_t d_gbf = sdesc_sw128(sbase + Cfg::OFF_GBF, 16, 1024);
+      const uint64_t d_xg = sdesc_sw128(sbase + Cfg::OFF_XG, 16, 1024);
       const uint64_t d_p = sdesc_sw128(sbase + Cfg::OFF_P, 16, 1024);
       for (int c = 0; c < nch; ++c) {
         const int s = c % NST, u = c / NST;
@@ -283,12 +286,10 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
         if (!dead) dead = !mbar_wait(&qw_ready[c & 1], (c >> 1) & 1, lim);
         if (!dead) dead = !mbar_wait(wbf_ready, c & 1, lim);
         tc_fence_after();
-        // (2); U1-U3 of chunk c-1 were read before wbf_ready(c)
+        // (2) into U1 and U2 (adjacent columns); U1-U3 of chunk c-1 were read before wbf_ready(c)
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          mma_bf16_ss(t_u1, d_k + k_step(C, kk), d_xbf + k_step(RS, kk), ID_U, kk > 0);
-          mma_bf16_ss(t_u2, d_k + k_step(C, kk), d_gbf + k_step(RS, kk), ID_U, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(t_u1, d_k + k_step(C, kk), d_xg + k_step(2 * RS, kk), ID_U, kk > 0);
         // (3), (4)
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_g, d_dm + mn_step(kk), d_qm + mn_step(kk), ID_ST, 1);
@@ -405,8 +406,8 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
           tmem_ld_half32(t_x + lane_off + cb, x);
           tmem_ld_wait();
         }
-        store_row32_bf16(sbase + Cfg::OFF_GBF, RS * 128, row64h, col, g);
-        store_row32_bf16(sbase + Cfg::OFF_XBF, RS * 128, row64h, col, x);
+        store_row32_bf16(sbase + Cfg::OFF_XG, 2 * RS * 128, row64h, col, x);
+        store_row32_bf16(sbase + Cfg::OFF_XG, 2 * RS * 128, RS + row64h, col, g);
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = __float_as_uint(fmaf(xs, __uint_as_float(x[j]), gs * __uint_as_float(g[j])));
         tmem_st_half32(t_x + lane_off + cb, x);
@@ -500,12 +501,11 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
 // M_0; block (bh, r0) owns rows [r0, r0 + 64) of M and P (V_r, dO_r: those
 // columns of V and dO) and adds its partial deta.  Per chunk the MMA thread
 // issues
-//   (1) S1 = Q K^T,  S2 = dO_r V_r^T            [TMEM, M=C, N=C each]
-//   (2) Y  = Q Mbf^T                            [TMEM, M=C, N=64]
+//   (1) [S1 | Y] = Q [K ; Mbf]^T,  S2 = dO_r V_r^T   [TMEM, M=C, N=128 and 64]
 //   (2') Z = K Gbf^T + K Glo^T                  (Y's columns, once y is read)
 //   (4) M += V_r^T Kb,  P += dO_r^T Q           [TMEM, M=64, N=D]
 //   (3) F  = Lstrict A,  A = bf16(S1 o S2)      [TMEM, M=C, N=C]
-// after the epilogue has taken the bf16 pairs of M and G = -P and replaced M
+// after the epilogue has taken the bf16 copies of M and G = -P and replaced M
 // by beta^n M.  The epilogue takes chunk c+1's states as soon as it has read
 // z of chunk c, so that chunk c+1's scores and Y overlap its F and prefix sums.
 template <int D>
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
   uint64_t* empty = bars + NST;          // [NST] stage free: (3) issued after (1)-(4), and the epilogue read V, dO
   uint64_t* mbf_ready = bars + 2 * NST;  // bf16 pairs written, M rewritten
   uint64_t* sc_full = mbf_ready + 1;
-  uint64_t* y_full = mbf_ready + 2;
+  // (mbf_ready + 2 unused: Y lands with S1, on sc_full)
   uint64_t* y_free = mbf_ready + 3;
   uint64_t* z_full = mbf_ready + 4;
   uint64_t* kb_ready = mbf_ready + 5;
@@ -567,7 +567,6 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
     }
     mbar_init(mbf_ready, 128);
     mbar_init(sc_full, 1);
-    mbar_init(y_full, 1);
     mbar_init(y_free, 128);
     mbar_init(z_full, 1);
     mbar_init(kb_ready, 1);
@@ -592,7 +591,8 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t t_m = tmem, t_p = tmem + D, t_s1 = tmem + 2 * D, t_s2 = t_s1 + C, t_f = t_s2 + C, t_yz = t_f + C;
+  // S1 and Y adjacent: (1) writes both
+  const uint32_t t_m = tmem, t_p = tmem + D, t_s1 = tmem + 2 * D, t_yz = t_s1 + C, t_s2 = t_yz + RS, t_f = t_s2 + C;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -606,9 +606,9 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
           tma_load_3d(&tmQ, &full[s], st + kb * C * 128, kb * 64, c * C, bh);
-          tma_load_3d(&tmK, &full[s], st + TILE + kb * C * 128, kb * 64, c * C, bh);
-          tma_load_3d(&tmV, &full[s], st + 2 * TILE + kb * C * 128, kb * 64, c * C, bh);
-          tma_load_3d(&tmD, &full[s], st + 3 * TILE + kb * C * 128, kb * 64, c * C, bh);
+          tma_load_3d(&tmK, &full[s], st + Cfg::OFF_SK + kb * 2 * C * 128, kb * 64, c * C, bh);  // rows 0-63
+          tma_load_3d(&tmV, &full[s], st + Cfg::OFF_SV + kb * C * 128, kb * 64, c * C, bh);
+          tma_load_3d(&tmD, &full[s], st + Cfg::OFF_SD + kb * C * 128, kb * 64, c * C, bh);
         }
       }
       for (int j = max(0, nch - NST); j < nch; ++j) mbar_wait(&full[j % NST], (j / NST) & 1, lim);
@@ -618,10 +618,10 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
     if (lane == 0) {
       bool dead = false;
       constexpr uint32_t ID_S = idesc_bf16_f32(C, C, false, false);
+      constexpr uint32_t ID_SY = idesc_bf16_f32(C, C + RS, false, false);
       constexpr uint32_t ID_Y = idesc_bf16_f32(C, RS, false, false);
       constexpr uint32_t ID_ST = idesc_bf16_f32(RS, D, true, true);
       constexpr uint32_t ID_F = idesc_bf16_f32(C, C, false, true);
-      const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
       const uint64_t d_gbf = sdesc_sw128(sbase + Cfg::OFF_GBF, 16, 1024);
       const uint64_t d_glo = sdesc_sw128(sbase + Cfg::OFF_GLO, 16, 1024);
       const uint64_t d_kbm = sdesc_sw128(sbase + Cfg::OFF_KB, C * 128, 1024);  // MN-major
@@ -630,8 +630,9 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       for (int c = 0; c < nch; ++c) {
         const int s = c % NST, u = c / NST;
         const uint32_t st = sbase + s * STAGE;
-        const uint32_t vr = st + 2 * TILE + rb * C * 128, dr = st + 3 * TILE + rb * C * 128;  // this block's columns
-        const uint64_t d_q = sdesc_sw128(st, 16, 1024), d_k = sdesc_sw128(st + TILE, 16, 1024);
+        const uint32_t vr = st + Cfg::OFF_SV + rb * C * 128, dr = st + Cfg::OFF_SD + rb * C * 128;  // this block's columns
+        // K and [K ; Mbf]: 128-row blocks (k_step over 2C rows); K as an A operand reads rows 0-63
+        const uint64_t d_q = sdesc_sw128(st, 16, 1024), d_k = sdesc_sw128(st + Cfg::OFF_SK, 16, 1024);
         const uint64_t d_vr = sdesc_sw128(vr, 16, 1024), d_dr = sdesc_sw128(dr, 16, 1024);
         const uint64_t d_qm = sdesc_sw128(st, C * 128, 1024);
         const uint64_t d_vrm = sdesc_sw128(vr, C * 128, 1024), d_drm = sdesc_sw128(dr, C * 128, 1024);
@@ -640,19 +641,17 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
         if (!dead) dead = !mbar_wait(mbf_ready, c & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_s1, d_q + k_step(C, kk), d_k + k_step(C, kk), ID_S, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(t_s1, d_q + k_step(C, kk), d_k + k_step(2 * C, kk), ID_SY, kk > 0);  // [S1 | Y]
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(t_s2, d_dr + k_step(C, kk), d_vr + k_step(C, kk), ID_S, kk > 0);
         tc_commit(sc_full);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_q + k_step(C, kk), d_mbf + k_step(RS, kk), ID_Y, kk > 0);
-        tc_commit(y_full);
         if (!dead) dead = !mbar_wait(y_free, c & 1, lim);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_k + k_step(C, kk), d_gbf + k_step(RS, kk), ID_Y, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_k + k_step(2 * C, kk), d_gbf + k_step(RS, kk), ID_Y, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_k + k_step(C, kk), d_glo + k_step(RS, kk), ID_Y, 1);
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16_ss(t_yz, d_k + k_step(2 * C, kk), d_glo + k_step(RS, kk), ID_Y, 1);
         tc_commit(z_full);
         if (!dead) dead = !mbar_wait(kb_ready, c & 1, lim);
         tc_fence_after();
@@ -681,14 +680,15 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       const int s = c % NST, n = nvalid(c);
       if (!dead) dead = !mbar_wait(&full[s], (c / NST) & 1, lim);
       if (c >= 1 && !dead) dead = !mbar_wait(sdone, (c - 1) & 1, lim);
-      const uint8_t* kt = smem + s * STAGE + TILE;
+      const uint8_t* kt = smem + s * STAGE + Cfg::OFF_SK;
 #pragma unroll 4
       for (int k = 0; k < D / 4; ++k) {
         const int idx = lane + 32 * k;
         const int r = idx / (D / 8), cc = idx % (D / 8);
-        const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
+        const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);  // Kb: 64-row blocks
+        const uint32_t koff = (cc >> 3) * 2 * C * 128 + sw128_off(r, cc & 7);  // K: rows 0-63 of 128-row blocks
         const float cb = (r < n) ? -p.sigma * bpow[n - 1 - r] : 0.f;
-        const uint4 a = *reinterpret_cast<const uint4*>(kt + off);
+        const uint4 a = *reinterpret_cast<const uint4*>(kt + koff);
         *reinterpret_cast<uint4*>(smem + Cfg::OFF_KB + off) =
             make_uint4(scale_bf16x2(a.x, cb), scale_bf16x2(a.y, cb), scale_bf16x2(a.z, cb), scale_bf16x2(a.w, cb));
       }
@@ -754,7 +754,7 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
           g[j] = __float_as_uint(gj);
           part = fmaf(gj, __uint_as_float(m[j]), part);
         }
-        store_row32_bf16(sbase + Cfg::OFF_MBF, RS * 128, row64h, col, m);
+        store_row32_bf16(sbase + (c % NST) * STAGE + Cfg::OFF_SK, 2 * C * 128, C + row64h, col, m);  // rows 64-127
         store_row32_split(sbase + Cfg::OFF_GBF, sbase + Cfg::OFF_GLO, row64h, col, g);
 #pragma unroll
         for (int j = 0; j < 32; ++j) m[j] = __float_as_uint(bn * __uint_as_float(m[j]));
@@ -800,15 +800,13 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(a_ready);
-      // (e) y_j = do_j . (M q_j) over this block's rows of M
-      if (!dead) dead = !mbar_wait(y_full, c & 1, lim);
-      tc_fence_after();
+      // (e) y_j = do_j . (M q_j) over this block's rows of M (Y landed with S1)
       float y, z;
       {
         uint32_t r[32];
         tmem_ld_half32(t_yz + lane_off, r);
         tmem_ld_wait();
-        y = row_dot(st + 3 * TILE + rb * C * 128, r);
+        y = row_dot(st + Cfg::OFF_SD + rb * C * 128, r);
       }
       tc_fence_before();
       mbar_arrive(y_free);
@@ -819,7 +817,7 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
         uint32_t r[32];
         tmem_ld_half32(t_yz + lane_off, r);
         tmem_ld_wait();
-        z = row_dot(st + 2 * TILE + rb * C * 128, r);
+        z = row_dot(st + Cfg::OFF_SV + rb * C * 128, r);
       }
       tc_fence_before();
       mbar_arrive(&empty[s]);  // done with this stage's V and dO rows
@@ -841,29 +839,42 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(f_free);
-      // (h) prefix sums of y (half 0) and of beta-weighted z (half 1) over the
-      // chunk, then this block's part of deta
+      // (h) the chunk's prefix sums, ypre_i = sum_{j<i} y_j and
+      // zpre_i = sum_{s<=i} beta^(i-s) z_s, by two warps (two tokens a lane,
+      // shuffle scans), then this block's part of deta.  (No barrier after:
+      // the scans of the next chunk write only after its first barrier.)
+      float* ypre = zs + C;
+      float* zpre = zs + 2 * C;
       if (half == 0) {
         ys[row64h] = y;
         zs[row64h] = z;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      {
-        const int i = row64h;
-        float acc = 0.f;
-        if (half == 0) {
-          for (int j = 0; j < i; ++j) acc += ys[j];
-        } else {
-          for (int j = 0; j <= i; ++j) acc = fmaf(bpow[i - j], zs[j], acc);
+      if (g4 < 2) {
+        const float a0 = (g4 == 0 ? ys : zs)[2 * lane], a1 = (g4 == 0 ? ys : zs)[2 * lane + 1];
+        // pair sum (y) or pair value beta a0 + a1 (z), then an inclusive scan over the lanes
+        float pr = (g4 == 0) ? a0 + a1 : fmaf(p.beta, a0, a1);
+#pragma unroll
+        for (int k = 1; k < 32; k <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, pr, k);
+          if (lane >= k) pr = fmaf(g4 == 0 ? 1.f : bpow[2 * k], u, pr);
         }
-        const float other = __shfl_xor_sync(0xffffffffu, acc, 16);
-        if (half == 0 && i < n) {
-          const float ypre = acc, zpre = other;
-          const float val = bpow[i + 1] * (g0 - ypre) - p.sigma * zpre + p.sigma * rf;
-          atomicAdd(TTT_AT(p.deta, static_cast<size_t>(bh) * p.T + c * C + i, 1, static_cast<size_t>(p.BH) * p.T), -val);
+        const float prev = __shfl_up_sync(0xffffffffu, pr, 1);  // through token 2 lane - 1
+        const float pv = lane > 0 ? prev : 0.f;
+        if (g4 == 0) {
+          ypre[2 * lane] = pv;
+          ypre[2 * lane + 1] = pv + a0;
+        } else {
+          zpre[2 * lane] = fmaf(p.beta, pv, a0);
+          zpre[2 * lane + 1] = pr;
         }
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (half == 0 && row64h < n) {
+        const int i = row64h;
+        const float val = bpow[i + 1] * (g0 - ypre[i]) - p.sigma * zpre[i] + p.sigma * rf;
+        atomicAdd(TTT_AT(p.deta, static_cast<size_t>(bh) * p.T + c * C + i, 1, static_cast<size_t>(p.BH) * p.T), -val);
+      }
       g0 = g0_next;
     }
   }
