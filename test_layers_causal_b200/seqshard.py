@@ -58,11 +58,29 @@ class Backend:
     backward: object = None
 
 
+def chunked_backward_supported(q, v, beta):
+    """Whether ttt_la_backward_chunked takes these shapes: bf16 with d_k == d_v
+    in {64, 128} (with or without momentum), fp32 without momentum with d_k,
+    d_v multiples of 4 up to 128."""
+    dk, dv = q.shape[-1], v.shape[-1]
+    if q.dtype == torch.bfloat16:
+        return dk == dv and dk in (64, 128)
+    return not beta and dk % 4 == 0 and dv % 4 == 0 and dk <= 128 and dv <= 128
+
+
+def _library_backward(q, k, v, dO, eta, **kw):
+    """A run's backward: the chunk-parallel form where the library has it,
+    else the recurrent one."""
+    if chunked_backward_supported(q, v, kw.get("beta", 0.0)):
+        return _abi.backward_chunked(q, k, v, dO, eta, **kw)
+    return _abi.backward_recurrent(q, k, v, dO, eta, **kw)
+
+
 LIBRARY = Backend(
     segment_map=_abi.segment_map,
     compose_maps=_abi.compose_maps,
     forward=lambda q, k, v, eta, **kw: _abi.forward_chunked(q, k, v, eta, **kw),
-    backward=lambda q, k, v, dO, eta, **kw: _abi.backward_recurrent(q, k, v, dO, eta, **kw),
+    backward=_library_backward,
 )
 
 

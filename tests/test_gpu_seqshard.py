@@ -80,13 +80,15 @@ def test_compose_is_exact_elementwise_and_module_world_one():
     assert_bf16(W_T, W_ref, "W_T")
 
 
+@pytest.mark.parametrize("form", ["recurrent", "chunked"])
 @pytest.mark.parametrize("world", [1, 2, 3])
-def test_backward_runs_compose_to_the_whole_sequence(world):
+def test_backward_runs_compose_to_the_whole_sequence(world, form):
     """The backward split without momentum, ranks one after another: each run's
     start state from the forward maps, its own do q^T sum from a backward with
     no final-state gradient, the later runs' sums added onto dL/dW_T, then the
     run's backward; dq, dk, dv, deta of every run and dL/dW_0 against the
-    whole-sequence gradient oracle."""
+    whole-sequence gradient oracle, with the runs' backward in either form."""
+    bwd = _abi.backward_recurrent if form == "recurrent" else _abi.backward_chunked
     B, H, T, d = 2, 2, 3 * 32 + 17, 64
     x = _inputs(B, H, T, d, "bf16", 210 + world)
     q, k, v, eta = x
@@ -100,20 +102,20 @@ def test_backward_runs_compose_to_the_whole_sequence(world):
     maps = torch.stack([_abi.segment_map(run(q, s), run(k, s), run(v, s), run(eta, s), eta_const=ec, chunk=64)[0]
                         for s in sl])
     starts = [_abi.compose_maps(maps[:r], None, None, S0, None)[0] for r in range(world)]
-    own = torch.stack([_abi.backward_recurrent(run(q, s), run(k, s), run(v, s), run(dO, s), run(eta, s),
-                                               eta_const=ec, state_in=starts[r])["dW0"] for r, s in enumerate(sl)])
+    own = torch.stack([bwd(run(q, s), run(k, s), run(v, s), run(dO, s), run(eta, s), eta_const=ec,
+                           state_in=starts[r])["dW0"] for r, s in enumerate(sl)])
     parts = []
     for r, s in enumerate(sl):
         G_end, _ = _abi.compose_maps(own[r + 1:], None, None, dW_T, None)
-        parts.append(_abi.backward_recurrent(run(q, s), run(k, s), run(v, s), run(dO, s), run(eta, s),
-                                             eta_const=ec, state_in=starts[r], grad_state=G_end))
+        parts.append(bwd(run(q, s), run(k, s), run(v, s), run(dO, s), run(eta, s), eta_const=ec,
+                         state_in=starts[r], grad_state=G_end))
     dW0, _ = _abi.compose_maps(own, None, None, dW_T, None)
     torch.cuda.synchronize()
     ref = oracle.ttt_backward_f64(f64(q), f64(k), f64(v), f64(eta), f64(dO), f64(dW_T), S0=f64(S0))
     for n in ("dq", "dk", "dv", "deta"):
         assert_bf16(torch.cat([p[n] for p in parts], dim=2), ref[n], n)
     assert_bf16(dW0, ref["dW0"], "dW0")
-    if world == 1:  # the module itself, no exchange
+    if world == 1 and form == "chunked":  # the module itself (its runs take the chunked form), no exchange
         dq, dk, dv, deta, dW0m, dM0m = seqshard.backward_sequence_sharded(q, k, v, dO, eta, eta_const=ec,
                                                                           state_in=S0, grad_state=dW_T)
         assert dM0m is None

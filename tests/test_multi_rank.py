@@ -257,3 +257,16 @@ def test_backward_sequence_split_over_ranks_matches_the_whole_sequence(world):
     for key, (err, covered) in res.items():
         assert covered == [1] * 47, key
         assert err < 1e-11, (key, err)
+
+
+def test_library_backward_takes_the_chunked_form_where_it_exists():
+    """seqshard.LIBRARY runs a run's backward chunk-parallel for the shapes
+    ttt_la_backward_chunked takes, and recurrent otherwise (host logic only)."""
+    import torch
+    from test_layers_causal_b200.seqshard import chunked_backward_supported as ok
+    bf, f32 = torch.bfloat16, torch.float32
+    t = lambda d, dt: torch.empty(1, 1, 4, d, dtype=dt)  # noqa: E731
+    assert ok(t(64, bf), t(64, bf), 0.0) and ok(t(128, bf), t(128, bf), 0.9)
+    assert not ok(t(32, bf), t(32, bf), 0.0) and not ok(t(64, bf), t(128, bf), 0.0)
+    assert ok(t(48, f32), t(64, f32), 0.0) and not ok(t(48, f32), t(64, f32), 0.9)
+    assert not ok(t(130, f32), t(64, f32), 0.0) and not ok(t(30, f32), t(64, f32), 0.0)
