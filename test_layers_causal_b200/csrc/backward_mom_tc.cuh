@@ -101,7 +101,7 @@ struct MomRevCfg {
   static constexpr int C = 64, RS = kMomRows;
   static constexpr int TILE = C * D * 2;          // bf16 C x D
   static constexpr int SQ = RS * D * 2;           // bf16 RS x D
-  static constexpr int NST = 2;
+  static constexpr int NST = 3;
   static constexpr int STAGE = 3 * TILE;          // K, Q, dO roles
   // bf16 rows of X and of G stacked as one B operand of 128 rows per
   // 64-column block (X rows 0-63, G rows 64-127), so (2) is one N = 128 MMA
@@ -110,12 +110,14 @@ struct MomRevCfg {
   static constexpr int OFF_P = OFF_QW + 2 * TILE; // C x C weights
   static constexpr int BIG = OFF_P + C * C * 2;
   static constexpr int NE = 3;                    // coefficient slots
+  static constexpr int ES = C + 4;                // slot stride (floats): e_1 .. e_C 16-byte aligned
   static constexpr int NBAR = 3 * NST + 13;
-  static constexpr int SMALL = NBAR * 8 + (NE * (C + 1) + (C + 1) + 4) * 4 + 16;
+  static_assert(NBAR % 2 == 0, "coefficient slots start 16-byte aligned");
+  static constexpr int SMALL = NBAR * 8 + (NE * ES + (C + 1) + 4) * 4 + 16;
   static constexpr int SMEM = BIG + SMALL + 1024;
   static constexpr int TCOLS_USED = 2 * D + C + 3 * RS;  // G, X, scores, U1, U2, U3
   static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
-  static constexpr int THREADS = 288;             // 9 warps
+  static constexpr int THREADS = 352;             // 11 warps
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(SMEM <= 232448, "shared memory");
 };
@@ -155,9 +157,11 @@ struct MomDetaCfg {
 //   (1) S  = K Q^T                            [TMEM, M=C, N=C]
 //   (2) [U1 | U2] = K [Xbf ; Gbf]^T           [TMEM, M=C, N=128]
 //   (3) G += dO_r^T Q,  (4) X += dO_r^T Qw    [TMEM, M=64, N=D]
-//   (5) U3 = P dO_r                           P = bf16(sigma w o triu(S))
-// after the epilogue has taken Xbf, Gbf and replaced X by beta^n X - beta e_0 G;
-// the output row is -sigma beta^(n-1-i) U1 + sigma e_i U2 + U3, formed in fp32.
+//   (5) U3 += P dO_r                          P = bf16(sigma w o triu(S))
+// after the epilogue has taken Xbf, Gbf and replaced X by beta^n X - beta e_0 G,
+// and, before (5), set U3 to the rows' fp32 combination -sigma beta^(n-1-i) U1
+// + sigma e_i U2; U3 is then the output row.  The epilogue takes the next
+// chunk's Xbf, Gbf while (5) runs.
 // The coefficients e and the copy Qw of a chunk are made while the previous
 // chunk's MMAs run (three coefficient slots, two Qw buffers).
 template <int D>
@@ -184,11 +188,12 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
   uint64_t* wbf_ready = ks_free + 2;    // Xbf, Gbf written, X rewritten
   uint64_t* sc_full = wbf_ready + 1;    // (1) done
   uint64_t* sdone = wbf_ready + 2;      // (2)-(4) done
-  uint64_t* p_ready = wbf_ready + 3;    // P written
+  uint64_t* p_ready = wbf_ready + 3;    // P written and U3 set
   uint64_t* o_full = wbf_ready + 4;     // (5) done
   uint64_t* drain = wbf_ready + 5;
-  float* ebuf = reinterpret_cast<float*>(bars + Cfg::NBAR);  // [NE][C + 1] e_i of the chunk (e_C = 0)
-  float* bpow = ebuf + Cfg::NE * (C + 1);                     // [C + 1] beta^k
+  // [NE][ES]: slot x holds e_0 .. e_C (e_C = 0) from float 3, so that e_1 .. e_C are 16-byte aligned
+  float* ebuf = reinterpret_cast<float*>(bars + Cfg::NBAR);
+  float* bpow = ebuf + Cfg::NE * Cfg::ES;                     // [C + 1] beta^k
   float* xw = bpow + C + 1;                                   // [4] cross-warp carry of the e scan
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xw + 4);
 
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
     }
     for (int x = 0; x < 3; ++x) mbar_init(&e_ready[x], 64);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&qw_ready[x], 64);
+      mbar_init(&qw_ready[x], 128);
       mbar_init(&ks_free[x], 1);
     }
     mbar_init(wbf_ready, 128);
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
         if (!dead) dead = !mbar_wait(&qw_ready[c & 1], (c >> 1) & 1, lim);
         if (!dead) dead = !mbar_wait(wbf_ready, c & 1, lim);
         tc_fence_after();
-        // (2) into U1 and U2 (adjacent columns); U1-U3 of chunk c-1 were read before wbf_ready(c)
+        // (2) into U1 and U2 (adjacent columns); the epilogue read U1, U2 of chunk c-1 before wbf_ready(c)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_bf16_ss(t_u1, d_k + k_step(C, kk), d_xg + k_step(2 * RS, kk), ID_U, kk > 0);
@@ -299,9 +304,9 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
         tc_commit(&ks_free[c & 1]);
         if (!dead) dead = !mbar_wait(p_ready, c & 1, lim);
         tc_fence_after();
-        // (5)
+        // (5) onto U3, which the epilogue has set to the rows' combination of U1 and U2 (p_ready)
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_u3, d_p + k_step(C, kk), d_dm + mn_step(kk), ID_PU, kk > 0);
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_u3, d_p + k_step(C, kk), d_dm + mn_step(kk), ID_PU, 1);
         tc_commit(o_full);
       }
       tc_commit(drain);
@@ -323,43 +328,48 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
     }
   } else if (warp >= 7) {
     // ------------------------------------------------ coefficient warps --
-    // e_i of chunk c (one token per thread: a shuffle scan within each warp
-    // and one carry across), then Qw into the buffer of c's parity.  Both wait
+    // e_i of chunk c (warps 7-8, one token per thread: a shuffle scan within
+    // each warp and one carry across), then Qw into the buffer of c's parity
+    // (warps 7-10).  Both wait
     // only for (2)-(4) of chunk c - 2: slot c % 3 of e was last read by the
     // epilogue's P of chunk c - 3, which precedes its Xbf of chunk c - 2.
-    const int tid = threadIdx.x - 224;  // 0..63: warp 7 tokens 0-31, warp 8 tokens 32-63
+    const int tid = threadIdx.x - 224;  // 0..127; 0..63 (warps 7-8) also one token each
+    const bool scan = tid < 64;
     bool dead = false;
     auto eta_of = [&](int c) {
       const int t = phys(c) * C + tid;
       return (tid < nvalid(c)) ? (p.eta ? __ldg(p.eta + static_cast<size_t>(bh) * p.T + t) : p.eta_const) : 0.f;
     };
-    float eta_next = eta_of(0);
+    float eta_next = scan ? eta_of(0) : 0.f;
     for (int c = 0; c < nch; ++c) {
       const int s = c % NST;
-      float* e = ebuf + (c % Cfg::NE) * (C + 1);
+      float* e = ebuf + (c % Cfg::NE) * Cfg::ES + 3;
       float v = eta_next;
-      if (c + 1 < nch) eta_next = eta_of(c + 1);
+      if (scan && c + 1 < nch) eta_next = eta_of(c + 1);
       if (c >= 2 && !dead) dead = !mbar_wait(&ks_free[c & 1], ((c >> 1) - 1) & 1, lim);
       // v_i = sum_{r=i}^{end of the warp's 32 tokens} beta^(r-i) eta_r
+      if (scan) {
 #pragma unroll
-      for (int k = 1; k < 32; k <<= 1) {
-        const float u = __shfl_down_sync(0xffffffffu, v, k);
-        if (lane + k < 32) v = fmaf(bpow[k], u, v);
+        for (int k = 1; k < 32; k <<= 1) {
+          const float u = __shfl_down_sync(0xffffffffu, v, k);
+          if (lane + k < 32) v = fmaf(bpow[k], u, v);
+        }
+        if (warp == 8 && lane == 0) xw[0] = v;  // e_32
+        asm volatile("bar.sync 2, 64;" ::: "memory");
+        if (warp == 7) v = fmaf(bpow[32 - lane], xw[0], v);
+        e[tid] = v;
+        if (tid == 0) e[C] = 0.f;
+        asm volatile("bar.sync 2, 64;" ::: "memory");
+        mbar_arrive(&e_ready[c % 3]);
       }
-      if (warp == 8 && lane == 0) xw[0] = v;  // e_32
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (warp == 7) v = fmaf(bpow[32 - lane], xw[0], v);
-      e[tid] = v;
-      if (tid == 0) e[C] = 0.f;
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      mbar_arrive(&e_ready[c % 3]);
+      asm volatile("bar.sync 3, 128;" ::: "memory");  // e of chunk c written
       if (!dead) dead = !mbar_wait(&full[s], (c / NST) & 1, lim);
       const uint8_t* qr = smem + s * STAGE + TILE;
       uint8_t* qw = smem + Cfg::OFF_QW + (c & 1) * TILE;
       const float e0 = e[0];
 #pragma unroll 4
-      for (int k = 0; k < D / 8; ++k) {
-        const int idx = tid + 64 * k;
+      for (int k = 0; k < D / 16; ++k) {
+        const int idx = tid + 128 * k;
         const int r = idx / (D / 8), cc = idx % (D / 8);
         const uint32_t off = (cc >> 3) * C * 128 + sw128_off(r, cc & 7);
         const float cw = -p.beta * (e0 - bpow[r + 1] * e[r + 1]);
@@ -380,10 +390,10 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
     const size_t DD = static_cast<size_t>(D) * D, nst = static_cast<size_t>(p.BH) * DD;
     const size_t grow = bh * DD + static_cast<size_t>(r0 + row64h) * D;  // this thread's state row in global
     bool dead = false;
-    for (int c = 0; c < nch; ++c) {
-      const int s = c % NST, n = nvalid(c);
-      const float* e = ebuf + (c % Cfg::NE) * (C + 1);
-      // (b) Xbf, Gbf from the chunk-end states; X <- beta^n X - beta e_0 G
+    // (b) of chunk c: Xbf, Gbf from the chunk-end states; X <- beta^n X - beta e_0 G
+    auto take = [&](int c) {
+      const int n = nvalid(c);
+      const float* e = ebuf + (c % Cfg::NE) * Cfg::ES + 3;
       if (c >= 1 && !dead) dead = !mbar_wait(sdone, (c - 1) & 1, lim);
       if (!dead) dead = !mbar_wait(&e_ready[c % 3], (c / 3) & 1, lim);
       tc_fence_after();
@@ -416,49 +426,71 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(wbf_ready);
-      // (d) P_ij = sigma w_ij S_ij for j >= i
+    };
+    // Per chunk: P (the scores land early), U3 := -sigma beta^(n-1-i) U1 +
+    // sigma e_i U2 once (2) is done, then (b) of the next chunk while (5) adds
+    // P dO onto U3, then U3 out.
+    take(0);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NST, n = nvalid(c);
+      const float* e = ebuf + (c % Cfg::NE) * Cfg::ES + 3;
+      const int i = row64h;
+      // (d) P_ij = sigma w_ij S_ij for j >= i, w_ij = e_i - beta^(j+1-i) e_{j+1}; the
+      // power of beta runs along the row from the first unmasked column
       if (!dead) dead = !mbar_wait(sc_full, c & 1, lim);
       tc_fence_after();
       {
         uint32_t r[32];
         tmem_ld_half32(t_s + lane_off, r);
         tmem_ld_wait();
-        const int i = row64h;
         const float ei = e[i];
+        const int jlo = 32 * half;
+        float pw = bpow[max(jlo, i) + 1 - i];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
+          const float4 e0 = *reinterpret_cast<const float4*>(e + jlo + 8 * q + 1);
+          const float4 e1 = *reinterpret_cast<const float4*>(e + jlo + 8 * q + 5);
+          const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+          float a[8];
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int j0 = 32 * half + 8 * q + 2 * h;
-            // w_ij = e_i - beta^(j+1-i) e_{j+1}  (j >= i; the index is clamped for j < i)
-            const float w0 = ei - bpow[max(j0 + 1 - i, 0)] * e[j0 + 1];
-            const float w1 = ei - bpow[max(j0 + 2 - i, 0)] * e[j0 + 2];
-            const float a0 = (j0 >= i) ? p.sigma * w0 * __uint_as_float(r[8 * q + 2 * h]) : 0.f;
-            const float a1 = (j0 + 1 >= i) ? p.sigma * w1 * __uint_as_float(r[8 * q + 2 * h + 1]) : 0.f;
-            w[h] = pack_bf16x2(a0, a1);
+          for (int h = 0; h < 8; ++h) {
+            const int j = jlo + 8 * q + h;
+            a[h] = 0.f;
+            if (j >= i) {
+              a[h] = p.sigma * (ei - pw * ev[h]) * __uint_as_float(r[8 * q + h]);
+              pw *= p.beta;
+            }
           }
-          st_shared_v4(sbase + Cfg::OFF_P + sw128_off(i, 4 * half + q), w[0], w[1], w[2], w[3]);
+          st_shared_v4(sbase + Cfg::OFF_P + sw128_off(i, 4 * half + q), pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                       pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
         }
       }
       fence_async_smem();
+      // (u) U1, U2 are complete with (2)-(4): their rows' combination goes into U3
+      if (!dead) dead = !mbar_wait(sdone, c & 1, lim);
+      tc_fence_after();
+      {
+        uint32_t u1[32], u2[32];
+        tmem_ld_half32(t_u1 + lane_off, u1);
+        tmem_ld_half32(t_u2 + lane_off, u2);
+        tmem_ld_wait();
+        const float a1 = (i < n) ? -p.sigma * bpow[max(n - 1 - i, 0)] : 0.f, a2 = p.sigma * e[i];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) u1[j] = __float_as_uint(fmaf(a1, __uint_as_float(u1[j]), a2 * __uint_as_float(u2[j])));
+        tmem_st_half32(t_u3 + lane_off, u1);
+        tmem_st_wait();
+      }
       tc_fence_before();
       mbar_arrive(p_ready);
-      // (f) row i = -sigma beta^(n-1-i) U1 + sigma e_i U2 + U3 -> bf16 -> the stage's K slot
-      // (every MMA of the chunk is done), then the store warp
+      // (b) of the next chunk while (5) runs (U1, U2 of this chunk are read)
+      if (c + 1 < nch) take(c + 1);
+      // (f) U3 -> bf16 -> the stage's K slot (every MMA of the chunk is done), then the store warp
       if (!dead) dead = !mbar_wait(o_full, c & 1, lim);
       tc_fence_after();
       {
-        uint32_t u1[32], u2[32], r[32];
-        tmem_ld_half32(t_u1 + lane_off, u1);
-        tmem_ld_half32(t_u2 + lane_off, u2);
+        uint32_t r[32];
         tmem_ld_half32(t_u3 + lane_off, r);
         tmem_ld_wait();
-        const int i = row64h;
-        const float a1 = (i < n) ? -p.sigma * bpow[max(n - 1 - i, 0)] : 0.f, a2 = p.sigma * e[i];
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          r[j] = __float_as_uint(fmaf(a1, __uint_as_float(u1[j]), fmaf(a2, __uint_as_float(u2[j]), __uint_as_float(r[j]))));
         store_row32_bf16(sbase + s * STAGE, C * 128, row64h, 32 * half, r);
       }
       tc_fence_before();
