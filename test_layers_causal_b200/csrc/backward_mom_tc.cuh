@@ -139,12 +139,12 @@ struct MomDetaCfg {
   static constexpr int OFF_A = OFF_KB + TILE;     // bf16(Q K^T o dO V^T), token-major
   static constexpr int OFF_L = OFF_A + C * C * 2; // strictly lower ones
   static constexpr int BIG = OFF_L + C * C * 2;
-  static constexpr int NBAR = 2 * NST + 11;
-  static constexpr int SMALL = NBAR * 8 + ((C + 1) + 4 * C + 8) * 4 + 16;
+  static constexpr int NBAR = 2 * NST + 15;
+  static constexpr int SMALL = NBAR * 8 + ((C + 1) + 6 * C + 10) * 4 + 16;
   static constexpr int SMEM = BIG + SMALL + 1024;
   static constexpr int TCOLS_USED = 2 * D + 3 * C + RS;  // M, P, S1, S2, F, Y / Z
   static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
-  static constexpr int THREADS = 224;             // 7 warps
+  static constexpr int THREADS = 352;             // 11 warps
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(TCOLS_USED <= 512, "tensor memory");
   static_assert(SMEM <= 232448, "shared memory");
@@ -538,8 +538,9 @@ __global__ void __launch_bounds__(MomRevCfg<D>::THREADS, 1)
 //   (4) M += V_r^T Kb,  P += dO_r^T Q           [TMEM, M=64, N=D]
 //   (3) F  = Lstrict A,  A = bf16(S1 o S2)      [TMEM, M=C, N=C]
 // after the epilogue has taken the bf16 copies of M and G = -P and replaced M
-// by beta^n M.  The epilogue takes chunk c+1's states as soon as it has read
-// z of chunk c, so that chunk c+1's scores and Y overlap its F and prefix sums.
+// by beta^n M.  The epilogue (warps 2-5) takes chunk c+1's states as soon as it
+// has read z of chunk c and handed y, z over; warps 7-10 read F and finish the
+// chunk's deta meanwhile.
 template <int D>
 __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
     mom_bwd_deta_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -566,10 +567,15 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
   uint64_t* f_full = mbf_ready + 8;
   uint64_t* drain = mbf_ready + 9;
   uint64_t* f_free = mbf_ready + 10;     // F read out of TMEM
+  uint64_t* yz_ready = mbf_ready + 11;   // [2] y, z, <G, M> of the chunks of parity c & 1 handed over
+  uint64_t* yz_free = mbf_ready + 13;    // [2] that slot read
   float* bpow = reinterpret_cast<float*>(bars + Cfg::NBAR);  // [C + 1] beta^k
-  float* ys = bpow + C + 1;                                   // [C]
-  float* zs = ys + C;                                         // [C]
-  float* red = zs + 3 * C;                                    // [8]
+  float* ybuf = bpow + C + 1;                                 // [2][C] y of the chunk (slot c & 1)
+  float* zbuf = ybuf + 2 * C;                                 // [2][C] z
+  float* ypre = zbuf + 2 * C;                                 // [C] prefix sums of y
+  float* zpre = ypre + C;                                     // [C] beta-weighted prefix sums of z
+  float* g0buf = zpre + C;                                    // [2] <G, M> at the chunk's start
+  float* red = g0buf + 2;                                     // [8]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(red + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -607,6 +613,10 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
     mbar_init(f_full, 1);
     mbar_init(drain, 1);
     mbar_init(f_free, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&yz_ready[x], 128);
+      mbar_init(&yz_free[x], 128);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -728,8 +738,66 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(kb_ready);
     }
+  } else if (warp >= 7) {
+    // ------------------------------------------------ deta warps (7-10) --
+    // Per chunk: rf_i = sum_{s<=i} beta^(i-s) F_is, the chunk's prefix sums
+    // ypre_i = sum_{j<i} y_j and zpre_i = sum_{s<=i} beta^(i-s) z_s (two warps,
+    // two tokens a lane, shuffle scans), then this block's part of deta.
+    const int g4 = warp & 3;  // TMEM lane quadrant (warps 7-10 cover all four)
+    const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
+    const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
+    bool dead = false;
+    for (int c = 0; c < nch; ++c) {
+      const int n = nvalid(c);
+      const float* ys = ybuf + (c & 1) * C;
+      const float* zs = zbuf + (c & 1) * C;
+      if (!dead) dead = !mbar_wait(&yz_ready[c & 1], (c >> 1) & 1, lim);
+      if (!dead) dead = !mbar_wait(f_full, c & 1, lim);
+      tc_fence_after();
+      float rf = 0.f;
+      {
+        uint32_t r[32];
+        tmem_ld_half32(t_f + lane_off, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int sc = 32 * half + jj;
+          rf += (sc <= row64h) ? bpow[max(row64h - sc, 0)] * __uint_as_float(r[jj]) : 0.f;
+        }
+        rf += __shfl_xor_sync(0xffffffffu, rf, 16);
+      }
+      tc_fence_before();
+      mbar_arrive(f_free);
+      if (g4 < 2) {
+        const float a0 = (g4 == 0 ? ys : zs)[2 * lane], a1 = (g4 == 0 ? ys : zs)[2 * lane + 1];
+        // pair sum (y) or pair value beta a0 + a1 (z), then an inclusive scan over the lanes
+        float pr = (g4 == 0) ? a0 + a1 : fmaf(p.beta, a0, a1);
+#pragma unroll
+        for (int k = 1; k < 32; k <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, pr, k);
+          if (lane >= k) pr = fmaf(g4 == 0 ? 1.f : bpow[2 * k], u, pr);
+        }
+        const float prev = __shfl_up_sync(0xffffffffu, pr, 1);  // through token 2 lane - 1
+        const float pv = lane > 0 ? prev : 0.f;
+        if (g4 == 0) {
+          ypre[2 * lane] = pv;
+          ypre[2 * lane + 1] = pv + a0;
+        } else {
+          zpre[2 * lane] = fmaf(p.beta, pv, a0);
+          zpre[2 * lane + 1] = pr;
+        }
+      }
+      asm volatile("bar.sync 4, 128;" ::: "memory");
+      if (half == 0 && row64h < n) {
+        const int i = row64h;
+        const float val = bpow[i + 1] * (g0buf[c & 1] - ypre[i]) - p.sigma * zpre[i] + p.sigma * rf;
+        atomicAdd(TTT_AT(p.deta, static_cast<size_t>(bh) * p.T + c * C + i, 1, static_cast<size_t>(p.BH) * p.T), -val);
+      }
+      mbar_arrive(&yz_free[c & 1]);
+      asm volatile("bar.sync 4, 128;" ::: "memory");  // ypre, zpre read before the next chunk's scans
+    }
   } else {
-    // --------------------------------------------------------- epilogue --
+    // ------------------------------------------------ epilogue (2-5) --
     const int g4 = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * g4) << 16;
     // M = 64 accumulators fill lanes 0-15 of each quadrant; the whole warp
@@ -853,60 +921,16 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&empty[s]);  // done with this stage's V and dO rows
-      const float g0_next = (c + 1 < nch) ? take_states(c + 1) : 0.f;
-      // (g) rf_i = sum_{s<=i} beta^(i-s) F_is
-      if (!dead) dead = !mbar_wait(f_full, c & 1, lim);
-      tc_fence_after();
-      float rf = 0.f;
-      {
-        uint32_t r[32];
-        tmem_ld_half32(t_f + lane_off, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int sc = 32 * half + jj;
-          rf += (sc <= row64h) ? bpow[max(row64h - sc, 0)] * __uint_as_float(r[jj]) : 0.f;
-        }
-        rf += __shfl_xor_sync(0xffffffffu, rf, 16);
-      }
-      tc_fence_before();
-      mbar_arrive(f_free);
-      // (h) the chunk's prefix sums, ypre_i = sum_{j<i} y_j and
-      // zpre_i = sum_{s<=i} beta^(i-s) z_s, by two warps (two tokens a lane,
-      // shuffle scans), then this block's part of deta.  (No barrier after:
-      // the scans of the next chunk write only after its first barrier.)
-      float* ypre = zs + C;
-      float* zpre = zs + 2 * C;
+      // hand y, z and <G, M> of chunk c to warps 7-10 (slot c & 1, free once
+      // they are done with chunk c - 2), then take chunk c+1's states
+      if (c >= 2 && !dead) dead = !mbar_wait(&yz_free[c & 1], ((c >> 1) - 1) & 1, lim);
       if (half == 0) {
-        ys[row64h] = y;
-        zs[row64h] = z;
+        ybuf[(c & 1) * C + row64h] = y;
+        zbuf[(c & 1) * C + row64h] = z;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (g4 < 2) {
-        const float a0 = (g4 == 0 ? ys : zs)[2 * lane], a1 = (g4 == 0 ? ys : zs)[2 * lane + 1];
-        // pair sum (y) or pair value beta a0 + a1 (z), then an inclusive scan over the lanes
-        float pr = (g4 == 0) ? a0 + a1 : fmaf(p.beta, a0, a1);
-#pragma unroll
-        for (int k = 1; k < 32; k <<= 1) {
-          const float u = __shfl_up_sync(0xffffffffu, pr, k);
-          if (lane >= k) pr = fmaf(g4 == 0 ? 1.f : bpow[2 * k], u, pr);
-        }
-        const float prev = __shfl_up_sync(0xffffffffu, pr, 1);  // through token 2 lane - 1
-        const float pv = lane > 0 ? prev : 0.f;
-        if (g4 == 0) {
-          ypre[2 * lane] = pv;
-          ypre[2 * lane + 1] = pv + a0;
-        } else {
-          zpre[2 * lane] = fmaf(p.beta, pv, a0);
-          zpre[2 * lane + 1] = pr;
-        }
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (half == 0 && row64h < n) {
-        const int i = row64h;
-        const float val = bpow[i + 1] * (g0 - ypre[i]) - p.sigma * zpre[i] + p.sigma * rf;
-        atomicAdd(TTT_AT(p.deta, static_cast<size_t>(bh) * p.T + c * C + i, 1, static_cast<size_t>(p.BH) * p.T), -val);
-      }
+      if (threadIdx.x == 64) g0buf[c & 1] = g0;
+      mbar_arrive(&yz_ready[c & 1]);
+      const float g0_next = (c + 1 < nch) ? take_states(c + 1) : 0.f;
       g0 = g0_next;
     }
   }
