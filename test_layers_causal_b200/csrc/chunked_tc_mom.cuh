@@ -28,6 +28,7 @@
 //   (1) Sc  = Q K^T                       [unscaled K]
 //   (2) O   = Q Wbf^T + Q~ Mbf^T
 //   (3) W  += V^T K1,  M += V^T K2        K1 = diag(sigma c_{n-1,.}) K, K2 = diag(-sigma beta^(n-1-.)) K
+//                                         (one N = 2D MMA: W, M and K1, K2 are adjacent)
 //   (4) O  += P V                         P = bf16(sigma c * Sc), masked
 // after the epilogue has replaced W by W - g_{n-1} M and M by beta^n M in TMEM.
 #pragma once
@@ -267,6 +268,10 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       constexpr uint32_t ID_SC = idesc_bf16_f32(C, C, false, false);
       constexpr uint32_t ID_O_K = idesc_bf16_f32(C, D, false, false);
       constexpr uint32_t ID_W = idesc_bf16_f32(D, D, true, true);
+      // W and M adjacent in TMEM, K1 and K2 adjacent 64-column blocks in shared
+      // memory: phase B's state update is one N = 2D MMA per step
+      constexpr uint32_t ID_WM = idesc_bf16_f32(D, 2 * D, true, true);
+      static_assert(Cfg::OFF_K2 == Cfg::OFF_K1 + TILE, "K1, K2 adjacent");
       constexpr uint32_t ID_O_PV = idesc_bf16_f32(C, D, false, true);
       const uint64_t d_wbf = sdesc_sw128(sbase + Cfg::OFF_WBF, 16, 1024);
       const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
@@ -311,10 +316,7 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         tc_fence_after();
         // (3) first: it needs only this tile's K1/K2 and the rewritten W, M
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16_ss(t_w, dvm + mn_step(kk), d_k1 + mn_step(kk), ID_W, 1);
-          mma_bf16_ss(t_m, dvm + mn_step(kk), d_k2 + mn_step(kk), ID_W, 1);
-        }
+        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_w, dvm + mn_step(kk), d_k1 + mn_step(kk), ID_WM, 1);
         tc_commit(kt_free);
         // (2) overwrites O: the previous tile's O must have been read out
         if (it > 0 && !dead) dead = !mbar_wait(o_free, (it - 1) & 1, lim);
