@@ -102,7 +102,7 @@ struct TcCfg {
   // 64 x 64 tiles fuse (1) and (2) into one N = C + D MMA, [Sc | O] = Q [K~; Wbf]^T:
   // the K region of a stage then holds K~ and that chunk's Wbf as adjacent rows
   // of one operand (order alternating with the chunk's parity, see below).
-  static constexpr bool MRG = (C == 64 && D == 64);
+  static constexpr bool MRG = (C == 64 && D == 64 && !BWD);
   static constexpr int KWR = MRG ? C + D : C;                // rows per 64-column block of the K region
   static constexpr int KREG = KWR * D * 2;
   static constexpr int OK = TILE, OV = TILE + KREG;          // Q at 0, K region, V
@@ -132,8 +132,7 @@ struct TcCfg {
   static_assert(C <= 2 * D, "P must fit in the Q and K slots");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(TCOLS_USED <= 512, "tensor memory");
-  static_assert(!BWD || (C == 128 && D == 64) || (C == 64 && D == 128),
-                "the reverse passes' epilogue handles 64 values of a row per thread");
+  static_assert(!BWD || D == 64 || C == 64, "the reverse passes' tiles");
 };
 
 // K-major operand (rows x 64-element k-blocks, SW128): descriptor of the
@@ -1074,15 +1073,17 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
         // O[b]: TMEM -> bf16 -> V slot, then the store warp takes it
         {
           const uint32_t sv = sbase + s * STAGE + Cfg::OV;
-          // BWD: this thread's token (row crow of the chunk, 64 columns from
-          // c0), its sigma * eta and its 64 values of vdot, fetched before
-          // the wait (rows past T give zeros, which the TMA store drops)
+          // BWD: this thread's token (row crow of the chunk, NV columns from
+          // c0: a whole row of 128-token tiles, half a row of 64-token ones),
+          // its sigma * eta and its NV values of vdot, fetched before the wait
+          // (rows past T give zeros, which the TMA store drops)
+          constexpr int NV = (C == 128) ? D : D / 2, NU = NV / 8;
           [[maybe_unused]] const int crow = (C == 128) ? qrow : row64h;
-          [[maybe_unused]] const int c0 = (C == 128) ? 0 : 64 * half;
+          [[maybe_unused]] const int c0 = (C == 128) ? 0 : NV * half;
           [[maybe_unused]] size_t rowi = 0;
           [[maybe_unused]] bool live = false;
           [[maybe_unused]] float es_t = 0.f;
-          [[maybe_unused]] uint4 vv[8];
+          [[maybe_unused]] uint4 vv[NU];
           if constexpr (BWD) {
             const int tok = phys(Bs.c0 + j) * C + crow;
             const size_t ntok = static_cast<size_t>(p.BH) * p.T;
@@ -1090,27 +1091,29 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
             rowi = static_cast<size_t>(bh) * p.T + tok;
             es_t = live ? p.sigma * (p.eta ? __ldg(TTT_AT(p.eta, rowi, 1, ntok)) : p.eta_const) : 0.f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) vv[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < NU; ++i) vv[i] = make_uint4(0u, 0u, 0u, 0u);
             if (p.deta && live) {
-              const uint4* src = TTT_AT(static_cast<const uint4*>(p.vdot), (rowi * D + c0) / 8, 8, ntok * D / 8);
+              const uint4* src = TTT_AT(static_cast<const uint4*>(p.vdot), (rowi * D + c0) / 8, NU, ntok * D / 8);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) vv[i] = __ldg(src + i);
+              for (int i = 0; i < NU; ++i) vv[i] = __ldg(src + i);
             }
           }
           if (!dead) dead = !mbar_wait(&o_full[b], (itb >> 1) & 1, lim);
           tc_fence_after();
           const uint32_t t_o = t_o_of(b);
           if constexpr (BWD) {
-            uint32_t r[64];
-            if constexpr (C == 64)
+            uint32_t r[NV];
+            if constexpr (C == 128)
+              tmem_ld64(t_o + lane_off, r);
+            else if constexpr (NV == 64)
               tmem_ld_half64(t_o + lane_off, r);
             else
-              tmem_ld64(t_o + lane_off, r);
+              tmem_ld_half32(t_o + lane_off, r);
             tmem_ld_wait();
             if (p.deta) {
               float dot = 0.f;
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
+              for (int i = 0; i < NU; ++i) {
                 const uint32_t w[4] = {vv[i].x, vv[i].y, vv[i].z, vv[i].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -1122,8 +1125,11 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
               if (live && (C == 128 || half == 0)) *TTT_AT(p.deta, rowi, 1, static_cast<size_t>(p.BH) * p.T) = p.sigma * dot;
             }
 #pragma unroll
-            for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(es_t * __uint_as_float(r[i]));
-            store_row64_bf16(sv, C * 128, crow, c0, r);
+            for (int i = 0; i < NV; ++i) r[i] = __float_as_uint(es_t * __uint_as_float(r[i]));
+            if constexpr (NV == 64)
+              store_row64_bf16(sv, C * 128, crow, c0, r);
+            else
+              store_row32_bf16(sv, C * 128, crow, c0, r);
           } else if constexpr (C == 64 && D == 64) {
             uint32_t r[32];
             tmem_ld_half32(t_o + lane_off, r);

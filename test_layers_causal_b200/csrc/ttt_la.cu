@@ -413,23 +413,23 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
 // K unscaled, the state read out as bf16(W) + bf16(W - bf16(W)), and the
 // epilogue writing o_t := sigma eta_t O_t in bf16 (dv or dk; a->eta,
 // a->eta_const and a->ascent are the layer's) plus, when deta is given,
-// deta_t = sigma vdot_t . O_t from O in fp32.  Tiles: d = 64 with 128
-// tokens, d = 128 with 64 (the two whose shared memory holds the second bf16
-// copy of W).
+// deta_t = sigma vdot_t . O_t from O in fp32.  Tiles of 64 tokens: 64 x 64
+// (not merged: the second bf16 copy of W needs its own buffer; two blocks per
+// SM) at d = 64, 64 x 128 at d = 128.
 size_t workspace_for(const ttt_la_args* a);
 ttt_la_status backward_pass_tc(const ttt_la_args* a, const void* vdot, float* deta, cudaStream_t st) {
   if (!a || (deta && (!vdot || !aligned16(vdot)))) return TTT_LA_ERR_INVALID_ARG;
   const ttt_la_status s = check_seq(a);
   if (s != TTT_LA_OK) return s;
   if (a->dtype != TTT_LA_BF16 || a->beta != 0.f || a->d_k != a->d_v ||
-      !((a->d_k == 64 && a->chunk == 128) || (a->d_k == 128 && a->chunk == 64)))
+      !((a->d_k == 64 && a->chunk == 64) || (a->d_k == 128 && a->chunk == 64)))
     return TTT_LA_ERR_UNSUPPORTED;
   const SegPlan sp = plan_segments(a);
   if (sp.nseg > 1) {
     const size_t need = workspace_for(a);
     if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace)) return TTT_LA_ERR_INVALID_ARG;
   }
-  return a->d_k == 64 ? launch_tc<128, 64, true>(a, sp, st, vdot, deta)
+  return a->d_k == 64 ? launch_tc<64, 64, true>(a, sp, st, vdot, deta)
                       : launch_tc<64, 128, true>(a, sp, st, vdot, deta);
 }
 
@@ -1133,12 +1133,9 @@ ttt_la_args bwdc_mom_dq(const ttt_la_grad_args* a, const float* w0t, const float
   return f;
 }
 
-// bf16: the tiles of the reverse passes (d = 64: 128 tokens, d = 128: 64);
-// fp32: the fp32 chunked path's 64.
-int bwdc_chunk(const ttt_la_grad_args* a) {
-  if (a->dtype != TTT_LA_BF16) return 64;
-  return a->d_k == 128 ? 64 : 128;
-}
+// The reverse passes' tiles: 64 tokens (bf16: 64 x 64, two blocks per SM, at
+// d = 64; 64 x 128 at d = 128); fp32: the fp32 chunked path's 64.
+int bwdc_chunk(const ttt_la_grad_args*) { return 64; }
 
 // Arguments of forward pass p: 0 gives dq, 1 gives u = G k (bf16: dv) and
 // dL/dW_0, 2 gives r = G^T v (bf16: dk).  fp32: rev[] are q, k, v, dO
