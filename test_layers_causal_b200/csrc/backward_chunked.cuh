@@ -53,6 +53,8 @@ struct TransposeParams {
   int n, BH, R, C;
   const float* src[4];
   float* dst[4];
+  float* zero;       // zeroed here as well (zero_n floats), or nullptr
+  long long zero_n;
 };
 
 __global__ void __launch_bounds__(256) transpose_states_kernel(const TransposeParams p) {
@@ -67,6 +69,9 @@ __global__ void __launch_bounds__(256) transpose_states_kernel(const TransposePa
     for (int j = 0; j < 4; ++j)
       if (j < p.n) p.dst[j][o] = p.src[j][i];
   }
+  if (p.zero)
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < p.zero_n; i += stride)
+      p.zero[i] = 0.f;
 }
 
 // dv_t = sigma eta_t u_t, dk_t = sigma eta_t r_t, deta_t = sigma v_t . u_t,

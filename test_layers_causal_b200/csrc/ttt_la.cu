@@ -217,6 +217,18 @@ ttt::SeqParams seq_params(const ttt_la_args* a) {
 
 ttt_la_status launched() { return cudaGetLastError() == cudaSuccess ? TTT_LA_OK : TTT_LA_ERR_CUDA; }
 
+// Zeroes the n words of one call's segment flags and counters.  A kernel
+// rather than cudaMemsetAsync: between two kernels of a CUDA graph a memset
+// node costs about 3 us more, a small kernel node about 1 us (B200).
+__global__ void zero_words_kernel(unsigned* w, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) w[i] = 0u;
+}
+ttt_la_status zero_words(unsigned* w, size_t n, cudaStream_t st) {
+  const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 64));
+  zero_words_kernel<<<blocks, 256, 0, st>>>(w, static_cast<int>(n));
+  return launched();
+}
+
 // ------------------------------------------------------------ recurrent ----
 template <int DK, typename T, bool MOM>
 ttt_la_status launch_recurrent(const ttt_la_args* a, cudaStream_t st) {
@@ -401,8 +413,8 @@ ttt_la_status launch_tc(const ttt_la_args* a, const SegPlan& sp, cudaStream_t st
   if (sp.nseg > 1) {
     p.ws = static_cast<float*>(a->workspace);
     p.flags = reinterpret_cast<unsigned*>(p.ws + tc_ws_floats(bh, sp.nseg, D, sp.coop));
-    if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
-      return TTT_LA_ERR_CUDA;
+    const ttt_la_status s = zero_words(p.flags, tc_flag_words(bh, sp.nseg), st);
+    if (s != TTT_LA_OK) return s;
   }
   return launch_kernel(ttt::chunked_tc_kernel<C, D, BWD>, bh * sp.nseg, 256, Cfg::SMEM, st, sp.coop, mq, mk, mv, mo,
                        p);
@@ -505,8 +517,8 @@ ttt_la_status launch_mom_deta(int BH, int T, const void* q, const void* k, const
   p.X_in = X_in;
   p.deta = deta;
   p.limit_ns = g_limit_ns;
-  // the blocks of a head add their rows' parts
-  if (cudaMemsetAsync(deta, 0, static_cast<size_t>(BH) * T * sizeof(float), st) != cudaSuccess) return TTT_LA_ERR_CUDA;
+  // the blocks of a head add their rows' parts onto deta, which the caller
+  // has zeroed (the state transposes at the start of the call do it)
   return launch_kernel(ttt::mom_bwd_deta_kernel<D>, BH * (D / Cfg::RS), Cfg::THREADS, Cfg::SMEM, st, false, mq, mk, mv,
                        md, p);
 }
@@ -552,8 +564,8 @@ ttt_la_status launch_tc_mom(const ttt_la_args* a, const SegPlan& sp, cudaStream_
     p.ws = static_cast<float*>(a->workspace);
     p.wsc = p.ws + static_cast<size_t>(bh) * sp.nseg * 4 * D * D;
     p.flags = reinterpret_cast<unsigned*>(p.ws + tcm_ws_floats(bh, sp.nseg, D));
-    if (cudaMemsetAsync(p.flags, 0, tc_flag_words(bh, sp.nseg) * sizeof(unsigned), st) != cudaSuccess)
-      return TTT_LA_ERR_CUDA;
+    const ttt_la_status s = zero_words(p.flags, tc_flag_words(bh, sp.nseg), st);
+    if (s != TTT_LA_OK) return s;
   }
   return launch_kernel(ttt::chunked_tc_mom_kernel<D>, bh * sp.nseg, Cfg::THREADS, Cfg::SMEM, st, sp.coop, mq, mk, mv,
                        mo, p);
@@ -1278,7 +1290,11 @@ ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLa
       tp.src[tp.n] = src[i];
       tp.dst[tp.n++] = dst[i];
     }
-  if (tp.n > 0) {
+  // deta is accumulated by the deta kernel's row blocks: zeroed here, which
+  // saves a memset node ahead of that kernel
+  tp.zero = a->grad_eta;
+  tp.zero_n = static_cast<long long>(BH) * a->T;
+  if (tp.n > 0 || tp.zero) {
     ttt::transpose_states_kernel<<<sm_count() * 4, 256, 0, st>>>(tp);
     if ((s = launched()) != TTT_LA_OK) return s;
   }
