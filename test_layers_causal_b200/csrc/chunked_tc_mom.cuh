@@ -31,6 +31,15 @@
 //                                         (one N = 2D MMA: W, M and K1, K2 are adjacent)
 //   (4) O  += P V                         P = bf16(sigma c * Sc), masked
 // after the epilogue has replaced W by W - g_{n-1} M and M by beta^n M in TMEM.
+// At d = 128, (2) and (4) run transposed with M = d = 128:
+//   (2) O^T  = Wbf Q^T + Mbf Q~^T          Wbf, Mbf: A operands in TMEM
+//   (4) O^T += V^T P^T
+// The bf16 copies of W and M then go from the state step into TMEM, not
+// through shared memory, and the MMAs read only Q, Q~, V and P from shared
+// memory (the 64-row form streams all of Wbf and Mbf, 64 KB, per tile for
+// 64 output rows; the tensor core and the epilogue share that bandwidth).
+// The epilogue reads O^T one output column per thread and writes it
+// transposed into the staging tile.
 #pragma once
 #include "common.cuh"
 #include "chunked_tc.cuh"
@@ -59,6 +68,29 @@ struct TcMomParams {
   __device__ __forceinline__ size_t flag_words_of() const { return static_cast<size_t>(BH) * nseg + 1 + BH; }
 };
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16: A (M x K bf16) in tensor memory,
+// row m at lane m, k pairs packed in 32-bit columns (K = 16: 8 columns).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 lanes x 16 consecutive 32-bit columns (thread i: lane base + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 template <int D>
 struct TcMomCfg {
   static constexpr int C = 64;
@@ -83,7 +115,10 @@ struct TcMomCfg {
   static constexpr int NBAR = 5 * NST + 16 + 2 * NSA + 4;
   static constexpr int SMALL = NBAR * 8 + (NST * (C + 1) + (C + 1) + 8 + 4 * C) * 4 + 32;
   static constexpr int SMEM = BIG + SMALL + 1024;
-  static constexpr int TCOLS_USED = C + 3 * D;   // scores, O, W, M
+  // d = 128: O^T (M = d, C columns), bf16 copies of W and M as TMEM A
+  // operands (D / 2 columns each); otherwise O with M = C (D columns)
+  static constexpr bool TR = (D == 128);
+  static constexpr int TCOLS_USED = TR ? 2 * D + 2 * C + D : C + 3 * D;  // W, M, O, scores (, Wbf, Mbf)
   static constexpr int TCOLS = TCOLS_USED <= 256 ? 256 : 512;
   static constexpr int MINB = 1;
   static constexpr int NSCW = 4;                 // K-scaling warps (7 and 8-10), 16 rows each
@@ -208,8 +243,10 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
   auto tile_of = [&](int g) { return chunk0 + (g < nA ? nA - 1 - g : g - nA); };
   const uint32_t t_w = tmem;            // W: D columns, M = D
   const uint32_t t_m = tmem + D;        // M: D columns, M = D
-  const uint32_t t_o = tmem + 2 * D;    // O: D columns, M = C
-  const uint32_t t_sc = tmem + 3 * D;   // scores: C columns, M = C
+  const uint32_t t_o = tmem + 2 * D;    // O: D columns, M = C (d = 128: O^T, C columns, M = D)
+  const uint32_t t_sc = tmem + (Cfg::TR ? 2 * D + C : 3 * D);  // scores: C columns, M = C
+  const uint32_t t_wbf = tmem + 2 * D + 2 * C;  // d = 128: bf16 W (A operand), D / 2 columns
+  const uint32_t t_mbf = t_wbf + D / 2;         // d = 128: bf16 M
   uint8_t* wbf = smem + Cfg::OFF_WBF;
   uint8_t* mbf = smem + Cfg::OFF_MBF;
   uint8_t* k1s = smem + Cfg::OFF_K1;
@@ -273,6 +310,8 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
       constexpr uint32_t ID_WM = idesc_bf16_f32(D, 2 * D, true, true);
       static_assert(Cfg::OFF_K2 == Cfg::OFF_K1 + TILE, "K1, K2 adjacent");
       constexpr uint32_t ID_O_PV = idesc_bf16_f32(C, D, false, true);
+      constexpr uint32_t ID_OT = idesc_bf16_f32(D, C, false, false);     // O^T += Wbf Q^T (A in TMEM)
+      constexpr uint32_t ID_OT_PV = idesc_bf16_f32(D, C, true, false);   // O^T += V^T P^T
       const uint64_t d_wbf = sdesc_sw128(sbase + Cfg::OFF_WBF, 16, 1024);
       const uint64_t d_mbf = sdesc_sw128(sbase + Cfg::OFF_MBF, 16, 1024);
       const uint64_t d_k1 = sdesc_sw128(sbase + Cfg::OFF_K1, C * 128, 1024);
@@ -321,17 +360,30 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         // (2) overwrites O: the previous tile's O must have been read out
         if (it > 0 && !dead) dead = !mbar_wait(o_free, (it - 1) & 1, lim);
         tc_fence_after();
+        if constexpr (Cfg::TR) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_K, kk > 0);
-          mma_bf16_ss(t_o, d_qt + k_step(C, kk), d_mbf + k_step(D, kk), ID_O_K, 1);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            mma_bf16_ts(t_o, t_wbf + 8 * kk, dq + k_step(C, kk), ID_OT, kk > 0);
+            mma_bf16_ts(t_o, t_mbf + 8 * kk, d_qt + k_step(C, kk), ID_OT, 1);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            mma_bf16_ss(t_o, dq + k_step(C, kk), d_wbf + k_step(D, kk), ID_O_K, kk > 0);
+            mma_bf16_ss(t_o, d_qt + k_step(C, kk), d_mbf + k_step(D, kk), ID_O_K, 1);
+          }
         }
         tc_commit(sdone);
         tc_commit(&empty[s]);  // Q and K of this tile are read
         if (!dead) dead = !mbar_wait(p_ready, it & 1, lim);
         tc_fence_after();
+        if constexpr (Cfg::TR) {
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, d_p + k_step(C, kk), dvm + mn_step(kk), ID_O_PV, 1);
+          for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, dvm + mn_step(kk), d_p + k_step(C, kk), ID_OT_PV, 1);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) mma_bf16_ss(t_o, d_p + k_step(C, kk), dvm + mn_step(kk), ID_O_PV, 1);
+        }
         tc_commit(o_full);
       }
       tc_commit(drain);
@@ -766,7 +818,17 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         tmem_ld32(t_w + lane_off + cb * 32, r);
         tmem_ld32(t_m + lane_off + cb * 32, r2);
         tmem_ld_wait();
-        if (wrow_ok) {
+        if constexpr (Cfg::TR) {
+          // bf16 pairs along k: the A-operand layout of an M = 128 MMA (row = lane)
+          uint32_t pw[16], pm[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            pw[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            pm[j] = pack_bf16x2(__uint_as_float(r2[2 * j]), __uint_as_float(r2[2 * j + 1]));
+          }
+          tmem_st16(t_wbf + lane_off + cb * 16, pw);
+          tmem_st16(t_mbf + lane_off + cb * 16, pm);
+        } else if (wrow_ok) {
           store_row32_bf16(wbf, D * 128, wrow, cb * 32, r);
           store_row32_bf16(mbf, D * 128, wrow, cb * 32, r2);
         }
@@ -834,20 +896,37 @@ __global__ void __launch_bounds__(TcMomCfg<D>::THREADS, TcMomCfg<D>::MINB)
         const uint32_t sv = sbase + (it % NST) * STAGE + 2 * TILE;
         if (!dead) dead = !mbar_wait(o_full, it & 1, lim);
         tc_fence_after();
-        if constexpr (D == 64) {
+        if constexpr (Cfg::TR) {
+          // O^T: this thread holds output column d = row128 for the C tokens.
+          // Lane pairs (d even, d + 1) swap halves so that each writes two
+          // adjacent columns of one token: the even lane tokens 2m, the odd
+          // lane tokens 2m + 1.
+          uint32_t r[32], r2[32];
+          tmem_ld32(t_o + lane_off, r);
+          tmem_ld32(t_o + lane_off + 32, r2);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(o_free);
+          const bool odd = lane & 1;
+          const int de = row128 & ~1;
+          const uint32_t cbase = sv + (de >> 6) * C * 128 + (de & 7) * 2;
+          const uint32_t c16 = (de & 63) >> 3;
+          auto put = [&](int m, uint32_t x0, uint32_t x1) {  // tokens 2m, 2m + 1 of column d
+            const float a = __uint_as_float(x0), b = __uint_as_float(x1);
+            const float got = __shfl_xor_sync(0xffffffffu, odd ? a : b, 1);
+            st_shared_b32(cbase + sw128_off(2 * m + (odd ? 1 : 0), c16), odd ? pack_bf16x2(got, b) : pack_bf16x2(a, got));
+          };
+#pragma unroll
+          for (int m = 0; m < 16; ++m) put(m, r[2 * m], r[2 * m + 1]);
+#pragma unroll
+          for (int m = 0; m < 16; ++m) put(16 + m, r2[2 * m], r2[2 * m + 1]);
+        } else {
           uint32_t r[32];
           tmem_ld_half32(t_o + lane_off, r);
           tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(o_free);
           store_row32_bf16(sv, C * 128, row64h, 32 * half, r);
-        } else {
-          uint32_t r[64];
-          tmem_ld_half64(t_o + lane_off, r);
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(o_free);
-          store_row64_bf16(sv, C * 128, row64h, 64 * half, r);
         }
         fence_async_smem();
         mbar_arrive(&staged[it % NST]);
