@@ -334,7 +334,13 @@ def forward_measure(ttt, dev, c, chunk, peaks, sets=4, segments=0):
             "algorithmic_bytes": nbytes, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
             "executed_tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"],
             "traffic": read_traffic(c.name, chunk), "plan": plan, "clocks": clocks,
-            "gpu_launches_per_call": 1}
+            "gpu_launches_per_call": launches_per_forward(plan)}
+
+
+def launches_per_forward(plan):
+    """Kernels one ttt_la_forward_chunked call launches: the chunked kernel,
+    preceded by the flag-zeroing kernel when the plan has several segments."""
+    return 2 if plan["segments"] > 1 else 1
 
 
 def decode_measure(ttt, dev, peaks):
@@ -433,7 +439,8 @@ def phi_measure(ttt, dev, peaks, reps=100):
     return {"workload": "llm_d64 with the frozen gated-MLP feature map (d_in 64 -> d_out 64)",
             "phi_us": phi_us, "phi_bytes": phi_bytes, "phi_hbm_gbs": gbs, "phi_frac": gbs / peaks["hbm_gbs"],
             "layer_us_per_step": layer_us, "tokens_per_s": B * T / (layer_us * 1e-6),
-            "gpu_launches_per_step": 2}
+            "gpu_launches_per_step": 1 + launches_per_forward(ttt.chunked_plan(B, H, T, d, d, chunk=c.chunk, beta=0.0,
+                                                                                eta=True))}
 
 
 def backward_measure(ttt, dev, peaks, name="llm_d64", reps=5):
@@ -490,7 +497,10 @@ def backward_measure(ttt, dev, peaks, name="llm_d64", reps=5):
         gbs = nbytes / (us * 1e-6) / 1e9
         out[form] = {"us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6), "hbm_gbs": gbs,
                      "hbm_frac": gbs / peaks["hbm_gbs"],
-                     "gpu_launches_per_call": 1 if form == "recurrent" else (5 if c.beta else 4)}
+                     # chunked: the state transposes, then (flag zeroing + forward) for dq and, without
+                     # momentum, for each of the two reverse passes; with momentum the two reverse
+                     # launches and the deta launch
+                     "gpu_launches_per_call": 1 if form == "recurrent" else (6 if c.beta else 7)}
     out["chunked_speedup_over_recurrent"] = out["recurrent"]["us_per_call"] / out["chunked"]["us_per_call"]
     del ws
     torch.cuda.empty_cache()
@@ -632,13 +642,14 @@ def run_ours(args, c, ws, rank, local, info):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": kname,
                      "algorithmic_bytes": nbytes, "peak_source": f"{src} copy bandwidth (of {src})",
-                     "timed_unit": "one forward call per step: the flag memset and one kernel launch"},
+                     "timed_unit": "one forward call per step: the flag-zeroing kernel (segmented plans) and "
+                                   "the chunked kernel"},
         "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                    "frac": tflops / peaks["bf16_tflops"], "executed_flops": flops,
                    "peak_source": f"{src} cuBLAS bf16 burst (of {src})"},
         "plan": plan,
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,  # one kernel per step (plus a flag memset when segmented)
+        "gpu_launches": args.steps * launches_per_forward(plan),
         "clocks": clocks,
     }
     del sets, work
