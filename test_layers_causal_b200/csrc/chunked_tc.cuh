@@ -319,6 +319,17 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.limit_ns;
+  // Constant learning rate: K~ = c K with one scalar c = sigma * eta, so the
+  // kernel uses K itself and folds c in where fp32 values become bf16 operands
+  // (P = bf16(c Sc), Wbf = bf16(c W')) and where states cross the boundary.
+  // The W accumulator, the phase-A totals and every published or scanned
+  // state then hold W' = W / c; W_0 is divided by c as it is read, W_T
+  // multiplied by c as it is written.  This removes the K scaler's pass over
+  // every K tile (a 32 KB read and write of shared memory per 128 x 128 tile).
+  bool fold = false;
+  if constexpr (!BWD) fold = p.eta == nullptr && fabsf(p.sigma * p.eta_const) >= 1e-30f;
+  const float fc = fold ? p.sigma * p.eta_const : 1.f;  // c, or 1 without the fold
+  const float finv = fold ? 1.f / fc : 1.f;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -623,7 +634,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
         if (!dead) dead = !mbar_wait(fb, u & 1, lim);
         uint8_t* sk = slotA ? smem + a_koff(x) : smem + s * STAGE + Cfg::OK + krow_of(pb, itb) * 128;
 #pragma unroll 1
-        for (int b0 = 0; b0 < PER_LANE; b0 += BATCH) {
+        for (int b0 = 0; b0 < (fold ? 0 : PER_LANE); b0 += BATCH) {
           uint4 u[BATCH];
           uint32_t off[BATCH];
           float e[BATCH];
@@ -670,6 +681,11 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
     const int row64h = 16 * g4 + (lane & 15), half = lane >> 4;
     bool dead = false;
     constexpr size_t DD = static_cast<size_t>(D) * D;
+    // a row of W' as the bf16 operand Wbf = bf16(c W') (no-op without the fold)
+    auto wscale = [&](auto& r) {
+#pragma unroll
+      for (auto& x : r) x = __float_as_uint(fc * __uint_as_float(x));
+    };
     // The merged 64 x 64 tile (two blocks per SM, 128 registers a thread)
     // runs the decoupled look-back only.
     bool waves = false;
@@ -725,6 +741,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(row[cb * 32 + j]);
           tmem_st32(t_w + lane_off + (cb0 + cb) * 32, r);  // W accumulator := start
+          if (fold) wscale(r);
           if (wrow_ok) {
             if (Cfg::MRG)
               store_row32_bf16(sbase + (gb % NST) * STAGE + Cfg::OK + wrow_of(itb) * 128, Cfg::KWR * 128, wrow,
@@ -786,10 +803,10 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
           for (int v0 = seg * SL + et; v0 < v1; v0 += 256) {
             const bool ok1 = v0 + 128 < v1;
             // the scratch is quad-major, the caller's W_0 and W_T row-major
-            float4 run0 = (it > 1) ? __ldcg(send + v0) : (s4 ? __ldcg(s4 + qm4_to_rm4<D>(v0)) : zero);
+            float4 run0 = (it > 1) ? __ldcg(send + v0) : (s4 ? f4_scale(finv, __ldcg(s4 + qm4_to_rm4<D>(v0))) : zero);
             float4 run1 = !ok1 ? zero
                                : (it > 1) ? __ldcg(send + v0 + 128)
-                                          : (s4 ? __ldcg(s4 + qm4_to_rm4<D>(v0 + 128)) : zero);
+                                          : (s4 ? f4_scale(finv, __ldcg(s4 + qm4_to_rm4<D>(v0 + 128))) : zero);
             for (int j0 = 0; j0 < P; j0 += NB) {
               float4 a0[NB], a1[NB];
 #pragma unroll
@@ -816,8 +833,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
             __stcg(send + v0, run0);
             if (ok1) __stcg(send + v0 + 128, run1);
             if (it == p.nwave && o4) {
-              o4[qm4_to_rm4<D>(v0)] = run0;
-              if (ok1) o4[qm4_to_rm4<D>(v0 + 128)] = run1;
+              o4[qm4_to_rm4<D>(v0)] = f4_scale(fc, run0);
+              if (ok1) o4[qm4_to_rm4<D>(v0 + 128)] = f4_scale(fc, run1);
             }
           }
           __threadfence();
@@ -897,8 +914,9 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
               for (int j = 0; j < 4; ++j) {
                 const float8 x = base_qm ? ld_cg_f8_qm<D>(base, wrow, cb * 8 + 2 * j)
                                          : ld_cg_f8(base + static_cast<size_t>(wrow) * D + cb * 32 + 8 * j);
+                const float sc = base_qm ? 1.f : finv;  // the caller's W_0 enters as W_0 / c
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[8 * j + e] = x.v[e];
+                for (int e = 0; e < 8; ++e) acc[8 * j + e] = sc * x.v[e];
               }
             }
             // NR totals per round (4 x NR x 2 independent 16-byte loads in
@@ -948,6 +966,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(acc[j]);
           tmem_st32(t_w + lane_off + cb * 32, r);  // W accumulator := W_start
+          if (fold) wscale(r);
           if (wrow_ok) {
             if (Cfg::MRG)
               store_row32_bf16(sbase + (gb0 % NST) * STAGE + Cfg::OK + wrow_of(itb) * 128, Cfg::KWR * 128, wrow,
@@ -998,8 +1017,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int jj = 8 * i + 2 * e;
-                w[e] = pack_bf16x2(keep(jj) ? __uint_as_float(r[jj]) : 0.f,
-                                   keep(jj + 1) ? __uint_as_float(r[jj + 1]) : 0.f);
+                w[e] = pack_bf16x2(keep(jj) ? fc * __uint_as_float(r[jj]) : 0.f,
+                                   keep(jj + 1) ? fc * __uint_as_float(r[jj + 1]) : 0.f);
               }
               st_shared_v4(pdst + sw128_off(row64h, 4 * half + i), w[0], w[1], w[2], w[3]);
             }
@@ -1014,8 +1033,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
               for (int jj = 0; jj < 64; jj += 2) {
                 const int col = cb * 64 + jj;
                 const bool k0 = BWD ? col >= qrow : col <= qrow, k1 = BWD ? col + 1 >= qrow : col + 1 <= qrow;
-                const float a0 = k0 ? __uint_as_float(r[jj]) : 0.f;
-                const float a1 = k1 ? __uint_as_float(r[jj + 1]) : 0.f;
+                const float a0 = k0 ? fc * __uint_as_float(r[jj]) : 0.f;
+                const float a1 = k1 ? fc * __uint_as_float(r[jj + 1]) : 0.f;
                 pk[col >> 1] = pack_bf16x2(a0, a1);
               }
             }
@@ -1048,6 +1067,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
             uint32_t r[32];
             tmem_ld_half32(t_w + lane_off, r);
             tmem_ld_wait();
+            if (fold) wscale(r);
             store_row32_bf16(wdst, wblk, row64h, 32 * half, r);
             if constexpr (BWD) {
               to_residual(r);
@@ -1059,6 +1079,7 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
               uint32_t r[64];
               tmem_ld64(t_w + lane_off + cb * 64, r);
               tmem_ld_wait();
+              if (fold) wscale(r);
               store_row64_bf16(wdst, wblk, wrow, cb * 64, r);
               if constexpr (BWD) {
                 to_residual(r);
@@ -1178,8 +1199,8 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
           float4* d4 = reinterpret_cast<float4*>(dst + static_cast<size_t>(wrow) * D + cb * 32);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+            d4[j] = make_float4(fc * __uint_as_float(r[4 * j]), fc * __uint_as_float(r[4 * j + 1]),
+                                fc * __uint_as_float(r[4 * j + 2]), fc * __uint_as_float(r[4 * j + 3]));
         }
       }
     }

@@ -403,6 +403,9 @@ __device__ __forceinline__ float8 ld_cg_f8_qm(const float* m, int r, int q) {
 __device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
+__device__ __forceinline__ float4 f4_scale(float c, float4 a) {
+  return make_float4(c * a.x, c * a.y, c * a.z, c * a.w);
+}
 
 // Loads 4 consecutive elements as fp32 (16 B for fp32, 8 B for bf16).
 __device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
