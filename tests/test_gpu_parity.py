@@ -219,6 +219,46 @@ def test_chunked_tc_ascent_zero_state_and_exact_multiple(d, chunk):
     assert_bf16(S, S_ref, "state")
 
 
+@pytest.mark.parametrize("d,chunk,segments,waves", [(64, 64, 3, False), (128, 128, 3, False), (128, 128, 6, True),
+                                                    (128, 64, 6, True)])
+@pytest.mark.parametrize("ascent", [False, True])
+def test_chunked_tc_const_eta_fold(d, chunk, segments, waves, ascent, monkeypatch):
+    """A constant learning rate runs with sigma * eta folded into P and the bf16
+    copy of W (the state carried as W / (sigma * eta)): W_0 divided on entry,
+    W_T multiplied on exit, in place, in the look-back and the wave schedule,
+    descent and ascent."""
+    monkeypatch.setenv("TTT_LA_WAVE_TOKENS", str(chunk))
+    B, H, T = 1, 2, segments * 4 * chunk - 19
+    plan = ttt.chunked_plan(B, H, T, d, d, chunk=chunk, segments=segments, eta=False)
+    assert plan["cooperative"] == int(waves), plan
+    q, k, v, _, _ = _case(B, H, T, d, d, "bf16", 180 + d + chunk + segments, token_eta=False)
+    ec = 0.37 / math.sqrt(d)
+    S0 = _state(B, H, d, d, 19, scale=0.2)
+    Sx = S0.clone()
+    o, S, _ = ttt.forward_chunked(q, k, v, None, eta_const=ec, chunk=chunk, segments=segments, ascent=ascent,
+                                  state_in=Sx, state_out=Sx)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0 and S.data_ptr() == Sx.data_ptr()
+    o_ref, S_ref, _ = oracle_forward(q, k, v, None, ec, 0.0, ascent, S0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(Sx, S_ref, "state")
+
+
+@pytest.mark.parametrize("ec", [0.0, 1e-35])
+def test_chunked_tc_const_eta_without_fold(ec):
+    """eta = 0 and a scale below the fold's range run the K scaler as for a
+    per-token rate: no update, o = W_0 q, W_T = W_0."""
+    B, H, T, d = 1, 2, 3 * 128 + 5, 128
+    q, k, v, _, _ = _case(B, H, T, d, d, "bf16", 190, token_eta=False)
+    S0 = _state(B, H, d, d, 20, scale=0.2)
+    o, S, _ = ttt.forward_chunked(q, k, v, None, eta_const=ec, chunk=128, segments=2, state_in=S0)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    o_ref, S_ref, _ = oracle_forward(q, k, v, None, ec, 0.0, False, S0)
+    assert_bf16(o, o_ref, "o")
+    assert_bf16(S, S_ref, "state")
+
+
 def test_chunked_tc_short_sequences():
     """T shorter than a chunk, T = 1, and T one past a chunk boundary."""
     for T in (1, 17, 65):
