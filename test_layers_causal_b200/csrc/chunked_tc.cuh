@@ -39,7 +39,8 @@
 // MMAs (one thread, descriptors precomputed), warps 2-5 (128 threads, one
 // TMEM lane each) mask scores, convert fp32 accumulators into bf16 operands,
 // stage O and exchange states, warp 6 stores O with TMA, warp 7 scales every
-// K tile by the learning rate as it lands (fetching eta two tiles ahead).
+// K tile by a per-token learning rate as it lands (fetching eta two tiles
+// ahead; a constant rate is folded into P and the bf16 copy of W instead).
 // Per phase-A chunk the MMA thread issues T += V^T K~ into the score region
 // of TMEM (free outside phase B), so the next run's start state can be loaded
 // into W while phase A runs; per phase-B chunk

@@ -217,6 +217,48 @@ ttt::SeqParams seq_params(const ttt_la_args* a) {
 
 ttt_la_status launched() { return cudaGetLastError() == cudaSuccess ? TTT_LA_OK : TTT_LA_ERR_CUDA; }
 
+// A second stream per device, with a fork and a join event, for launches of
+// one call that do not depend on each other and together fit the SMs (the
+// momentum backward's two reverse launches: 64 blocks of one per SM each).
+// The caller issues fork -> launches -> join under side_mutex(), so calls from
+// several host threads never interleave on the shared events.  Created on
+// first use outside stream capture; a call that finds none while its stream
+// is capturing runs its launches on its own stream, one after the other.
+struct SideStream {
+  int dev;
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+};
+std::mutex& side_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+bool side_stream(cudaStream_t st, SideStream* out) {  // side_mutex() held
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::vector<SideStream> made;
+  for (const SideStream& x : made)
+    if (x.dev == dev) {
+      *out = x;
+      return true;
+    }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return false;
+  }
+  SideStream x{dev, nullptr, nullptr, nullptr};
+  if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  made.push_back(x);
+  *out = x;
+  return true;
+}
+
 // Zeroes the n words of one call's segment flags and counters.  A kernel
 // rather than cudaMemsetAsync: between two kernels of a CUDA graph a memset
 // node costs about 3 us more, a small kernel node about 1 us (B200).
@@ -1303,15 +1345,27 @@ ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLa
   f.workspace_bytes = L.fwd_bytes;
   if ((s = ttt_la_forward_chunked(&f, st)) != TTT_LA_OK) return s;
   const float sigma = a->ascent ? -1.f : 1.f;
-  if ((s = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma, a->beta,
-                             a->grad_state, a->grad_mom, dw0, a->grad_mom_in, st)) != TTT_LA_OK)
+  {
+    // The two reverse launches are independent (64 blocks each, one per SM):
+    // the dk one runs on the side stream, beside the dv one and the deta
+    // launch that follows it; the call's stream waits for it at the end.
+    std::lock_guard<std::mutex> lock(side_mutex());
+    SideStream side;
+    const bool two = side_stream(st, &side);
+    const cudaStream_t sk = two ? side.s : st;
+    if (two && (cudaEventRecord(side.fork, st) != cudaSuccess || cudaStreamWaitEvent(sk, side.fork, 0) != cudaSuccess))
+      return TTT_LA_ERR_CUDA;
+    ttt_la_status sdk = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma,
+                                          a->beta, dwt, dmt, nullptr, nullptr, sk);
+    if (two && (cudaEventRecord(side.join, sk) != cudaSuccess)) sdk = TTT_LA_ERR_CUDA;
+    if (sdk != TTT_LA_OK) return sdk;
+    s = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma, a->beta,
+                          a->grad_state, a->grad_mom, dw0, a->grad_mom_in, st);
+    if (s == TTT_LA_OK && a->grad_eta)
+      s = launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, st);
+    if (two && cudaStreamWaitEvent(st, side.join, 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
     return s;
-  if ((s = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma, a->beta, dwt,
-                             dmt, nullptr, nullptr, st)) != TTT_LA_OK)
-    return s;
-  if (a->grad_eta)
-    return launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, st);
-  return TTT_LA_OK;
+  }
 }
 }  // namespace
 
