@@ -343,6 +343,12 @@ int tc_resident_per_sm(const ttt_la_args* a) {
   return a->chunk == 64 ? tc_per_sm<64, 128>() : tc_per_sm<128, 128>();
 }
 
+// Set (on this host thread) while the momentum backward launches its dq pass
+// beside other kernels: the start states then come from the decoupled
+// look-back, which needs no co-residency of the grid (its blocks wait only
+// for blocks that took their tiles earlier), instead of the cooperative prefix.
+thread_local bool t_lookback_only = false;
+
 SegPlan plan_segments(const ttt_la_args* a) {
   SegPlan s;
   const int C = tc_tile(a);
@@ -367,7 +373,7 @@ SegPlan plan_segments(const ttt_la_args* a) {
   const size_t lookback_bytes = static_cast<size_t>(s.nseg - 1) * a->d_k * a->d_v * sizeof(float);
   // (the 64 x 64 tile without momentum runs the look-back only: see chunked_tc.cuh)
   const bool tile64 = a->beta == 0.f && C == 64 && a->d_k == 64;
-  s.coop = one_wave && (a->beta != 0.f || (lookback_bytes > 192 * 1024 && !tile64));
+  s.coop = !t_lookback_only && one_wave && (a->beta != 0.f || (lookback_bytes > 192 * 1024 && !tile64));
   if (s.coop && a->beta == 0.f) {
     // every run of every wave holds at least one chunk: nwave <= nchunks / nseg
     const int per_run = std::max(1, wave_tokens() / C);
@@ -1343,12 +1349,13 @@ ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLa
   ttt_la_args f = bwdc_mom_dq(a, w0t, m0t);
   f.workspace = L.fwd_bytes ? ws + L.fwd : nullptr;
   f.workspace_bytes = L.fwd_bytes;
-  if ((s = ttt_la_forward_chunked(&f, st)) != TTT_LA_OK) return s;
   const float sigma = a->ascent ? -1.f : 1.f;
   {
-    // The two reverse launches are independent (64 blocks each, one per SM):
-    // the dk one runs on the side stream, beside the dv one and the deta
-    // launch that follows it; the call's stream waits for it at the end.
+    // After the transposes the launches form two independent chains: dk's
+    // reverse launch then dq on the side stream, dv's reverse launch then
+    // deta on the call's stream, which waits for the side stream at the end.
+    // The reverse launches (64 blocks each, one per SM) run side by side; dq
+    // fills the SMs deta leaves, so it runs with the look-back start states.
     std::lock_guard<std::mutex> lock(side_mutex());
     SideStream side;
     const bool two = side_stream(st, &side);
@@ -1357,6 +1364,11 @@ ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLa
       return TTT_LA_ERR_CUDA;
     ttt_la_status sdk = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma,
                                           a->beta, dwt, dmt, nullptr, nullptr, sk);
+    if (sdk == TTT_LA_OK) {
+      t_lookback_only = two;
+      sdk = ttt_la_forward_chunked(&f, sk);
+      t_lookback_only = false;
+    }
     if (two && (cudaEventRecord(side.join, sk) != cudaSuccess)) sdk = TTT_LA_ERR_CUDA;
     if (sdk != TTT_LA_OK) return sdk;
     s = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma, a->beta,
