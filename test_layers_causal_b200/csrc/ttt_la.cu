@@ -239,6 +239,13 @@ bool side_stream(cudaStream_t st, SideStream* out) {  // side_mutex() held
   static std::vector<SideStream> made;
   for (const SideStream& x : made)
     if (x.dev == dev) {
+      // a side stream that another host thread's capture has taken in (it
+      // stays captured until that capture ends) is not used
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(x.s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+        cudaGetLastError();
+        return false;
+      }
       *out = x;
       return true;
     }

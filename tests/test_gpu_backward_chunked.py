@@ -133,3 +133,27 @@ def test_backward_chunked_momentum_agrees_with_recurrent(d):
     torch.cuda.synchronize()
     for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
         assert_bf16(a[n], f64(b[n]), n)
+
+
+def test_backward_chunked_momentum_two_streams_and_graph_capture():
+    """With momentum the call runs its two independent launch chains on two
+    streams. The outputs are the same bits on the default stream, on another
+    stream, and replayed from a captured CUDA graph, which the second stream
+    joins through the call's fork and join events."""
+    x = _mom_case(2, 3, 64 * 9 + 5, 128, 280)
+    kw = dict(eta_const=x["ec"], state_in=x["S0"], grad_state=x["dW"], beta=0.9, mom_in=x["M0"], grad_mom=x["dM"])
+    a = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], **kw)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], **kw)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        c = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], **kw)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
+        assert torch.equal(a[n], b[n]), n
+        assert torch.equal(a[n], c[n]), n
