@@ -217,9 +217,10 @@ ttt::SeqParams seq_params(const ttt_la_args* a) {
 
 ttt_la_status launched() { return cudaGetLastError() == cudaSuccess ? TTT_LA_OK : TTT_LA_ERR_CUDA; }
 
-// A second stream per device, with a fork and a join event, for launches of
-// one call that do not depend on each other and together fit the SMs (the
-// momentum backward's two reverse launches: 64 blocks of one per SM each).
+// A second stream per device, at the device's greatest priority, with a fork
+// and a join event, for a chain of launches that runs beside the call's own
+// stream (the momentum backward's dv reverse launch and deta, its critical
+// path, whose blocks the priority puts on the SMs ahead of the other chain's).
 // The caller issues fork -> launches -> join under side_mutex(), so calls from
 // several host threads never interleave on the shared events.  Created on
 // first use outside stream capture; a call that finds none while its stream
@@ -255,7 +256,9 @@ bool side_stream(cudaStream_t st, SideStream* out) {  // side_mutex() held
     return false;
   }
   SideStream x{dev, nullptr, nullptr, nullptr};
-  if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+  int least = 0, greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+      cudaStreamCreateWithPriority(&x.s, cudaStreamNonBlocking, greatest) != cudaSuccess ||
       cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
@@ -1358,30 +1361,32 @@ ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLa
   f.workspace_bytes = L.fwd_bytes;
   const float sigma = a->ascent ? -1.f : 1.f;
   {
-    // After the transposes the launches form two independent chains: dk's
-    // reverse launch then dq on the side stream, dv's reverse launch then
-    // deta on the call's stream, which waits for the side stream at the end.
-    // The reverse launches (64 blocks each, one per SM) run side by side; dq
-    // fills the SMs deta leaves, so it runs with the look-back start states.
+    // After the transposes the launches form two independent chains: dv's
+    // reverse launch then deta (the longer one) on the side stream, at the
+    // device's greatest priority, and dk's reverse launch then dq on the
+    // call's stream, which waits for the side stream at the end.  The
+    // reverse launches (64 blocks each, one per SM) run side by side; dq fills
+    // the SMs deta leaves (deta's blocks go first), so it runs with the
+    // look-back start states.
     std::lock_guard<std::mutex> lock(side_mutex());
     SideStream side;
     const bool two = side_stream(st, &side);
-    const cudaStream_t sk = two ? side.s : st;
-    if (two && (cudaEventRecord(side.fork, st) != cudaSuccess || cudaStreamWaitEvent(sk, side.fork, 0) != cudaSuccess))
+    const cudaStream_t sv = two ? side.s : st;
+    if (two && (cudaEventRecord(side.fork, st) != cudaSuccess || cudaStreamWaitEvent(sv, side.fork, 0) != cudaSuccess))
       return TTT_LA_ERR_CUDA;
-    ttt_la_status sdk = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma,
-                                          a->beta, dwt, dmt, nullptr, nullptr, sk);
-    if (sdk == TTT_LA_OK) {
+    ttt_la_status sdv = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma,
+                                          a->beta, a->grad_state, a->grad_mom, dw0, a->grad_mom_in, sv);
+    if (sdv == TTT_LA_OK && a->grad_eta)
+      sdv = launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, sv);
+    if (two && cudaEventRecord(side.join, sv) != cudaSuccess) sdv = TTT_LA_ERR_CUDA;
+    if (sdv != TTT_LA_OK) return sdv;
+    s = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma, a->beta, dwt, dmt,
+                          nullptr, nullptr, st);
+    if (s == TTT_LA_OK) {
       t_lookback_only = two;
-      sdk = ttt_la_forward_chunked(&f, sk);
+      s = ttt_la_forward_chunked(&f, st);
       t_lookback_only = false;
     }
-    if (two && (cudaEventRecord(side.join, sk) != cudaSuccess)) sdk = TTT_LA_ERR_CUDA;
-    if (sdk != TTT_LA_OK) return sdk;
-    s = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma, a->beta,
-                          a->grad_state, a->grad_mom, dw0, a->grad_mom_in, st);
-    if (s == TTT_LA_OK && a->grad_eta)
-      s = launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, st);
     if (two && cudaStreamWaitEvent(st, side.join, 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
     return s;
   }
