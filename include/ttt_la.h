@@ -351,8 +351,9 @@ TTT_LA_API ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args *args,
  * q, k, v, grad_o and the reverse runs' outputs; momentum also: dL/dW_0 when
  * grad_state_in is NULL).  Errors as ttt_la_backward_recurrent.
  * Streams: with momentum the call runs two independent chains of launches,
- * one on `stream` and one on a second stream the library keeps per device,
- * joined back into `stream` by an event before the call returns: work queued
+ * one on `stream` and one on a second stream the library keeps per device (at
+ * the device's greatest stream priority), joined back into `stream` by an
+ * event before the call returns: work queued
  * on `stream` afterwards sees every output, as with a single stream.  Under
  * stream capture the second stream joins the capture (created beforehand by
  * an earlier call outside capture; otherwise both chains run on `stream`). */
