@@ -940,4 +940,145 @@ __global__ void __launch_bounds__(MomDetaCfg<D>::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, Cfg::TCOLS);
 }
 
+// ------------------------------------------------------------ dL/dW_0 ----
+// dL/dW_0 = dL/dW_T + sum_t do_t q_t^T: the recurrence of dL/dW does not
+// involve the momentum.  Computed on its own, the deta kernel, which starts
+// from it, need not wait for the reverse kernel that also carries it.
+// Block (b, h, split) sums its share of the 64-token tiles into a TMEM
+// accumulator, acc += do_tile^T q_tile (both operands MN-major, M = N = d),
+// and writes the fp32 partial; mom_g0_sum_kernel adds the partials to
+// dL/dW_T in a fixed order, so the result is the same bits on every run.
+struct MomG0Params {
+  int BH, T, nsplit, tiles_per_split;
+  float* part;  // [nsplit][BH][d][d]
+  uint64_t limit_ns;
+};
+
+template <int D>
+struct MomG0Cfg {
+  static constexpr int C = 64;
+  static constexpr int TILE = C * D * 2;  // one bf16 64-token tile
+  static constexpr int NST = 4;
+  static constexpr int STAGE = 2 * TILE;  // do, then q
+  static constexpr int SMEM = NST * STAGE + 256 + 1024;  // + barriers, alignment slack
+  static constexpr int THREADS = 192;     // TMA, MMA, four readout warps
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) mom_g0_kernel(const __grid_constant__ CUtensorMap tmD,
+                                                        const __grid_constant__ CUtensorMap tmQ,
+                                                        const MomG0Params p) {
+  using Cfg = MomG0Cfg<D>;
+  constexpr int C = Cfg::C, TILE = Cfg::TILE, NST = Cfg::NST, STAGE = Cfg::STAGE;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NST * STAGE);  // [NST] tiles landed
+  uint64_t* empty = full + NST;                                       // [NST] tiles consumed
+  uint64_t* done = empty + NST;                                       // every MMA complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.limit_ns;
+  const int bh = blockIdx.x / p.nsplit, split = blockIdx.x % p.nsplit;
+  const int t_begin = split * p.tiles_per_split;
+  const int n = max(0, min(p.tiles_per_split, (p.T + C - 1) / C - t_begin));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, D);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmD);
+    prefetch_tmap(&tmQ);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tacc = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool dead = false;
+      for (int i = 0; i < n; ++i) {
+        const int s = i % NST;
+        if (i >= NST && !dead) dead = !mbar_wait(&empty[s], ((i / NST) - 1) & 1, lim);
+        mbar_arrive_expect_tx(&full[s], 2 * TILE);
+        uint8_t* st = smem + s * STAGE;
+        const int t0 = (t_begin + i) * C;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_load_3d(&tmD, &full[s], st + kb * C * 128, kb * 64, t0, bh);
+          tma_load_3d(&tmQ, &full[s], st + TILE + kb * C * 128, kb * 64, t0, bh);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool dead = false;
+      constexpr uint32_t ID = idesc_bf16_f32(D, D, true, true);
+      for (int i = 0; i < n; ++i) {
+        const int s = i % NST;
+        if (!dead) dead = !mbar_wait(&full[s], (i / NST) & 1, lim);
+        tc_fence_after();
+        const uint32_t st = sbase + s * STAGE;
+        const uint64_t da = sdesc_sw128(st, C * 128, 1024), db = sdesc_sw128(st + TILE, C * 128, 1024);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          mma_bf16_ss(tacc, da + mn_step(kk), db + mn_step(kk), ID, (i > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      tc_commit(done);  // with no tile, arrives at once
+    }
+  } else {
+    // readout: row d of the accumulator (an M = 64 accumulator fills lanes
+    // 0-15 of each quadrant), written as this split's fp32 partial
+    const int g4 = warp & 3;
+    const bool ok = (D == 128) || lane < 16;
+    const int row = (D == 128) ? 32 * g4 + lane : ok ? 16 * g4 + lane : 0;  // (lanes 16-31 idle at d = 64)
+    bool dead = false;
+    if (!dead) dead = !mbar_wait(done, 0, lim);
+    tc_fence_after();
+    const size_t DD = static_cast<size_t>(D) * D;
+    float* dst = TTT_AT(p.part, (static_cast<size_t>(split) * p.BH + bh) * DD + static_cast<size_t>(row) * D, D,
+                        static_cast<size_t>(p.nsplit) * p.BH * DD);
+#pragma unroll
+    for (int cb = 0; cb < D / 32; ++cb) {
+      uint32_t r[32];
+      tmem_ld32(tacc + (static_cast<uint32_t>(32 * g4) << 16) + cb * 32, r);
+      tmem_ld_wait();
+      if (ok) {
+        float4* d4 = reinterpret_cast<float4*>(dst + cb * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          d4[j] = (n > 0) ? make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tacc, D);
+}
+
+// g0 = dL/dW_T (or zero) + the nsplit partials, in split order.
+__global__ void mom_g0_sum_kernel(const float* GT, const float* part, int nsplit, long long n, float* g0) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float acc = GT ? GT[i] : 0.f;
+    for (int s = 0; s < nsplit; ++s) acc += part[static_cast<long long>(s) * n + i];
+    g0[i] = acc;
+  }
+}
+
 }  // namespace ttt

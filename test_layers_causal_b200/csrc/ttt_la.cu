@@ -217,18 +217,18 @@ ttt::SeqParams seq_params(const ttt_la_args* a) {
 
 ttt_la_status launched() { return cudaGetLastError() == cudaSuccess ? TTT_LA_OK : TTT_LA_ERR_CUDA; }
 
-// A second stream per device, at the device's greatest priority, with a fork
-// and a join event, for a chain of launches that runs beside the call's own
-// stream (the momentum backward's dv reverse launch and deta, its critical
-// path, whose blocks the priority puts on the SMs ahead of the other chain's).
+// Two more streams per device, one at the device's greatest priority, with a
+// fork and two join events, for chains of launches that run beside the call's
+// own stream (the momentum backward: dL/dW_0 then deta, its critical path,
+// whose blocks the priority puts on the SMs first; dv's reverse launch).
 // The caller issues fork -> launches -> join under side_mutex(), so calls from
 // several host threads never interleave on the shared events.  Created on
 // first use outside stream capture; a call that finds none while its stream
 // is capturing runs its launches on its own stream, one after the other.
 struct SideStream {
   int dev;
-  cudaStream_t s;
-  cudaEvent_t fork, join;
+  cudaStream_t s, s2;       // greatest priority; default priority
+  cudaEvent_t fork, join, join2;
 };
 std::mutex& side_mutex() {
   static std::mutex mu;
@@ -242,8 +242,9 @@ bool side_stream(cudaStream_t st, SideStream* out) {  // side_mutex() held
     if (x.dev == dev) {
       // a side stream that another host thread's capture has taken in (it
       // stays captured until that capture ends) is not used
-      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-      if (cudaStreamIsCapturing(x.s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone, cap2 = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(x.s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone ||
+          cudaStreamIsCapturing(x.s2, &cap2) != cudaSuccess || cap2 != cudaStreamCaptureStatusNone) {
         cudaGetLastError();
         return false;
       }
@@ -255,12 +256,14 @@ bool side_stream(cudaStream_t st, SideStream* out) {  // side_mutex() held
     cudaGetLastError();
     return false;
   }
-  SideStream x{dev, nullptr, nullptr, nullptr};
+  SideStream x{dev, nullptr, nullptr, nullptr, nullptr, nullptr};
   int least = 0, greatest = 0;
   if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
       cudaStreamCreateWithPriority(&x.s, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&x.s2, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&x.join2, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
@@ -579,6 +582,33 @@ ttt_la_status launch_mom_deta(int BH, int T, const void* q, const void* k, const
   // has zeroed (the state transposes at the start of the call do it)
   return launch_kernel(ttt::mom_bwd_deta_kernel<D>, BH * (D / Cfg::RS), Cfg::THREADS, Cfg::SMEM, st, false, mq, mk, mv,
                        md, p);
+}
+
+// dL/dW_0 = G_T + sum_t do_t q_t^T into g0 (fp32 [BH][d][d]; G_T may be
+// nullptr): the tensor-core partials over `nsplit` token ranges into `part`,
+// then their sum in a fixed order.
+template <int D>
+ttt_la_status launch_mom_g0(int BH, int T, int nsplit, const void* dO, const void* q, const float* G_T, float* part,
+                            float* g0, cudaStream_t st) {
+  using Cfg = ttt::MomG0Cfg<D>;
+  if (!grant_smem(reinterpret_cast<const void*>(ttt::mom_g0_kernel<D>), Cfg::SMEM)) return TTT_LA_ERR_CUDA;
+  CUtensorMap md, mq;
+  if (!make_map(&md, dO, BH, T, D, Cfg::C) || !make_map(&mq, q, BH, T, D, Cfg::C)) return TTT_LA_ERR_CUDA;
+  ttt::MomG0Params p;
+  std::memset(&p, 0, sizeof p);
+  p.BH = BH;
+  p.T = T;
+  p.nsplit = nsplit;
+  const int tiles = (T + Cfg::C - 1) / Cfg::C;
+  p.tiles_per_split = (tiles + nsplit - 1) / nsplit;
+  p.part = part;
+  p.limit_ns = g_limit_ns;
+  ttt_la_status s = launch_kernel(ttt::mom_g0_kernel<D>, BH * nsplit, Cfg::THREADS, Cfg::SMEM, st, false, md, mq, p);
+  if (s != TTT_LA_OK) return s;
+  const long long n = static_cast<long long>(BH) * D * D;
+  const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, static_cast<long long>(sm_count()) * 4));
+  ttt::mom_g0_sum_kernel<<<blocks, 256, 0, st>>>(G_T, part, nsplit, n, g0);
+  return launched();
 }
 
 size_t workspace_for(const ttt_la_args* a) {
@@ -1172,8 +1202,11 @@ ttt_la_status ttt_la_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 // of the inputs reversed along T and a finishing kernel forms dv, dk, deta.
 namespace {
 struct BwdChunkedLayout {
-  size_t rev[4], u, r, w0t, dwt, m0t, dmt, dw0, fwd, total, fwd_bytes;
+  size_t rev[4], u, r, w0t, dwt, m0t, dmt, dw0, g0part, g0, fwd, total, fwd_bytes;
 };
+
+// Token splits of the momentum backward's dL/dW_0 kernel (64-token tiles).
+int mom_g0_splits(int T) { return std::max(1, std::min(4, (T + 63) / 64)); }
 
 bool bwdc_fused(const ttt_la_grad_args* a) { return a->dtype == TTT_LA_BF16; }
 bool bwdc_mom(const ttt_la_grad_args* a) { return a->beta != 0.f; }
@@ -1292,6 +1325,10 @@ BwdChunkedLayout bwdc_layout(const ttt_la_grad_args* a) {
   off += (mom && a->grad_mom) ? ns : 0;
   L.dw0 = off;
   off += (mom && !a->grad_state_in) ? ns : 0;
+  L.g0part = off;  // momentum: the dL/dW_0 kernel's partials, then their sum
+  off += mom ? static_cast<size_t>(mom_g0_splits(a->T)) * ns : 0;
+  L.g0 = off;
+  off += mom ? ns : 0;
   L.fwd = off;
   L.fwd_bytes = 0;
   if (mom) {
@@ -1361,33 +1398,55 @@ ttt_la_status backward_chunked_mom(const ttt_la_grad_args* a, const BwdChunkedLa
   f.workspace_bytes = L.fwd_bytes;
   const float sigma = a->ascent ? -1.f : 1.f;
   {
-    // After the transposes the launches form two independent chains: dv's
-    // reverse launch then deta (the longer one) on the side stream, at the
-    // device's greatest priority, and dk's reverse launch then dq on the
-    // call's stream, which waits for the side stream at the end.  The
-    // reverse launches (64 blocks each, one per SM) run side by side; dq fills
-    // the SMs deta leaves (deta's blocks go first), so it runs with the
-    // look-back start states.
+    // After the transposes the launches form three independent chains:
+    // dL/dW_0 then deta (the longest, the call's critical path) on a side
+    // stream at the device's greatest priority, dv's reverse launch on a
+    // second side stream, and dk's reverse launch then dq on the call's
+    // stream, which waits for both side streams at the end.  deta starts
+    // from its own dL/dW_0 (a short tensor-core reduction), not from the
+    // reverse launch that also carries it.  dq fills the SMs the others
+    // leave, so it runs with the look-back start states.  Without the side
+    // streams the launches run one after the other on the call's stream, and
+    // deta takes dL/dW_0 from the reverse launch.
     std::lock_guard<std::mutex> lock(side_mutex());
     SideStream side;
     const bool two = side_stream(st, &side);
-    const cudaStream_t sv = two ? side.s : st;
-    if (two && (cudaEventRecord(side.fork, st) != cudaSuccess || cudaStreamWaitEvent(sv, side.fork, 0) != cudaSuccess))
-      return TTT_LA_ERR_CUDA;
-    ttt_la_status sdv = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma,
-                                          a->beta, a->grad_state, a->grad_mom, dw0, a->grad_mom_in, sv);
-    if (sdv == TTT_LA_OK && a->grad_eta)
-      sdv = launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, sv);
-    if (two && cudaEventRecord(side.join, sv) != cudaSuccess) sdv = TTT_LA_ERR_CUDA;
-    if (sdv != TTT_LA_OK) return sdv;
-    s = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma, a->beta, dwt, dmt,
-                          nullptr, nullptr, st);
-    if (s == TTT_LA_OK) {
-      t_lookback_only = two;
-      s = ttt_la_forward_chunked(&f, st);
-      t_lookback_only = false;
+    if (two) {
+      float* part = reinterpret_cast<float*>(ws + L.g0part);
+      float* g0 = reinterpret_cast<float*>(ws + L.g0);
+      if (cudaEventRecord(side.fork, st) != cudaSuccess || cudaStreamWaitEvent(side.s, side.fork, 0) != cudaSuccess ||
+          cudaStreamWaitEvent(side.s2, side.fork, 0) != cudaSuccess)
+        return TTT_LA_ERR_CUDA;
+      ttt_la_status s1 = TTT_LA_OK;
+      if (a->grad_eta) {
+        s1 = launch_mom_g0<D>(BH, a->T, mom_g0_splits(a->T), a->grad_o, a->q, a->grad_state, part, g0, side.s);
+        if (s1 == TTT_LA_OK)
+          s1 = launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, g0, a->mom_in, a->grad_eta,
+                                  side.s);
+      }
+      if (cudaEventRecord(side.join, side.s) != cudaSuccess) s1 = TTT_LA_ERR_CUDA;
+      ttt_la_status s2 = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma,
+                                           a->beta, a->grad_state, a->grad_mom, dw0, a->grad_mom_in, side.s2);
+      if (cudaEventRecord(side.join2, side.s2) != cudaSuccess) s2 = TTT_LA_ERR_CUDA;
+      s = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma, a->beta, dwt,
+                            dmt, nullptr, nullptr, st);
+      if (s == TTT_LA_OK) {
+        t_lookback_only = true;
+        s = ttt_la_forward_chunked(&f, st);
+        t_lookback_only = false;
+      }
+      if (cudaStreamWaitEvent(st, side.join, 0) != cudaSuccess || cudaStreamWaitEvent(st, side.join2, 0) != cudaSuccess)
+        return TTT_LA_ERR_CUDA;
+      return s1 != TTT_LA_OK ? s1 : s2 != TTT_LA_OK ? s2 : s;
     }
-    if (two && cudaStreamWaitEvent(st, side.join, 0) != cudaSuccess) return TTT_LA_ERR_CUDA;
+    s = launch_mom_rev<D>(BH, a->T, a->k, a->q, a->grad_o, a->grad_v, a->eta, a->eta_const, sigma, a->beta,
+                          a->grad_state, a->grad_mom, dw0, a->grad_mom_in, st);
+    if (s == TTT_LA_OK && a->grad_eta)
+      s = launch_mom_deta<D>(BH, a->T, a->q, a->k, a->v, a->grad_o, sigma, a->beta, dw0, a->mom_in, a->grad_eta, st);
+    if (s == TTT_LA_OK)
+      s = launch_mom_rev<D>(BH, a->T, a->v, a->grad_o, a->q, a->grad_k, a->eta, a->eta_const, sigma, a->beta, dwt,
+                            dmt, nullptr, nullptr, st);
+    if (s == TTT_LA_OK) s = ttt_la_forward_chunked(&f, st);
     return s;
   }
 }
