@@ -498,9 +498,9 @@ def backward_measure(ttt, dev, peaks, name="llm_d64", reps=5):
         out[form] = {"us_per_call": us, "tokens_per_s": c.B * c.T / (us * 1e-6), "hbm_gbs": gbs,
                      "hbm_frac": gbs / peaks["hbm_gbs"],
                      # chunked: the state transposes, then (flag zeroing + forward) for dq and, without
-                     # momentum, for each of the two reverse passes; with momentum the two reverse
-                     # launches and the deta launch
-                     "gpu_launches_per_call": 1 if form == "recurrent" else (6 if c.beta else 7)}
+                     # momentum, for each of the two reverse passes; with momentum also the two reverse
+                     # launches, the dL/dW_0 reduction and its sum, and the deta launch
+                     "gpu_launches_per_call": 1 if form == "recurrent" else (8 if c.beta else 7)}
     out["chunked_speedup_over_recurrent"] = out["recurrent"]["us_per_call"] / out["chunked"]["us_per_call"]
     del ws
     torch.cuda.empty_cache()

@@ -350,13 +350,13 @@ TTT_LA_API ttt_la_status ttt_la_backward_recurrent(const ttt_la_grad_args *args,
  * transposed states and one forward workspace (fp32 also: reversed copies of
  * q, k, v, grad_o and the reverse runs' outputs; momentum also: dL/dW_0 when
  * grad_state_in is NULL).  Errors as ttt_la_backward_recurrent.
- * Streams: with momentum the call runs two independent chains of launches,
- * one on `stream` and one on a second stream the library keeps per device (at
- * the device's greatest stream priority), joined back into `stream` by an
- * event before the call returns: work queued
- * on `stream` afterwards sees every output, as with a single stream.  Under
- * stream capture the second stream joins the capture (created beforehand by
- * an earlier call outside capture; otherwise both chains run on `stream`). */
+ * Streams: with momentum the call runs independent chains of launches, one
+ * on `stream` and two on streams the library keeps per device (one at the
+ * device's greatest stream priority), joined back into `stream` by events
+ * before the call returns: work queued on `stream` afterwards sees every
+ * output, as with a single stream.  Under stream capture the library's
+ * streams join the capture (created beforehand by an earlier call outside
+ * capture; otherwise every chain runs on `stream`). */
 TTT_LA_API size_t ttt_la_backward_chunked_workspace_size(const ttt_la_grad_args *args);
 TTT_LA_API ttt_la_status ttt_la_backward_chunked(const ttt_la_grad_args *args, void *stream);
 
