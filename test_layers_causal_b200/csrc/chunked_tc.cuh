@@ -791,14 +791,11 @@ __global__ void __launch_bounds__(256, TcCfg<C, D, BWD>::MINB)
           const float4* s4 = p.S_in ? TTT_AT(reinterpret_cast<const float4*>(p.S_in), bh * DD4, DD4, nst4) : nullptr;
           float4* o4 = p.S_out ? TTT_AT(reinterpret_cast<float4*>(p.S_out), bh * DD4, DD4, nst4) : nullptr;
           TTT_EXPECT(v1 <= static_cast<int>(DD4));
-          // Two positions per thread and up to NB totals per round, every
-          // load of a round issued before its stores: the scan costs a few L2
-          // round trips (its adds are cheap; its latency sits between phase A
-          // and phase B of every wave).
           // Two positions per thread (v0 and v0 + 128), up to NB totals per
           // round with every load of the round issued before its stores: the
-          // scan costs a few L2 round trips (its latency sits between phase A
-          // and phase B of every wave; more totals per round spill registers).
+          // scan costs a few L2 round trips (its adds are cheap; its latency
+          // sits between phase A and phase B of every wave; more totals per
+          // round spill registers).
           constexpr int NB = 4;
           const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int v0 = seg * SL + et; v0 < v1; v0 += 256) {

@@ -21,8 +21,8 @@
 // Phase A walks the segment's tiles backwards so the suffix coefficients carry
 // from tile to tile; the look-back composes the published maps.  Tiles are 64
 // tokens (a 128-token request runs as two 64-token tiles: the same layer),
-// which keeps Q, K, V stages, bf16 copies of W and M, the two scaled K tiles,
-// Q~ = diag(-g) Q and P within shared memory.
+// which keeps the Q, K, V stages, the two scaled K tiles, Q~ = diag(-g) Q, P
+// and (at d = 64) the bf16 copies of W and M within shared memory.
 //
 // Per phase-B tile the MMA thread issues
 //   (1) Sc  = Q K^T                       [unscaled K]
