@@ -407,6 +407,41 @@ def test_long_context_schedules_agree(chunk):
     assert (S - S_ref).norm() / S_ref.norm() < 1e-2
 
 
+def test_chunked_tc_past_2_31_elements():
+    """Maximum sizes: q, k, v and o of 257 heads x 65536 tokens x d = 128
+    (2^31 + 2^24 elements each, 4.3 GB in bf16), so the element offsets of the
+    last heads pass 2^31.  Heads are independent: the first and the last head
+    carry seeded inputs from the generator and are compared with the oracle
+    over the whole sequence, the others hold seeded device noise of the same
+    scale.  Both the automatic plan (one segment per head) and four segments
+    per head (1028 blocks, decoupled look-back) are checked."""
+    H, T, d = 257, 65536, 128
+    assert H * T * d > 2 ** 31
+    qs, ks, vs, zs = make_qkv((1, 2), T, d, d, 31)
+    eta_s = (torch.sigmoid(zs) / math.sqrt(d)).float()
+    g = torch.Generator(device="cuda").manual_seed(5)
+    bf = torch.bfloat16
+
+    def noise():
+        return (torch.randn(1, H, T, d, generator=g, device="cuda", dtype=bf) * (1.0 / math.sqrt(d))).to(bf)
+    q, k, v = noise(), noise(), noise()
+    eta = torch.full((1, H, T), 0.5 / math.sqrt(d), device="cuda")
+    for j, h in enumerate((0, H - 1)):
+        q[0, h], k[0, h], v[0, h] = qs[0, j].to(bf).cuda(), ks[0, j].to(bf).cuda(), vs[0, j].to(bf).cuda()
+        eta[0, h] = eta_s[0, j].cuda()
+    refs = {h: oracle_forward(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], eta[:, h:h + 1], 0.0) for h in (0, H - 1)}
+    for segments in (0, 4):
+        o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=128, segments=segments)
+        torch.cuda.synchronize()
+        assert ttt.device_status() == 0
+        for h, (o_ref, S_ref, _) in refs.items():
+            assert_bf16(o[:, h:h + 1], o_ref, f"o head {h} segments {segments}")
+            assert_bf16(S[:, h:h + 1], S_ref, f"state head {h} segments {segments}")
+        del o, S
+    del q, k, v, eta
+    torch.cuda.empty_cache()
+
+
 # ------------------------------------------------ decode workload ----
 def test_decode_workload_prefill_then_steps():
     """256 sequences x 16 heads, d = 128: chunked prefill of 2048 tokens, then
