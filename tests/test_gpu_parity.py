@@ -407,14 +407,16 @@ def test_long_context_schedules_agree(chunk):
     assert (S - S_ref).norm() / S_ref.norm() < 1e-2
 
 
-def test_chunked_tc_past_2_31_elements():
+@pytest.mark.parametrize("beta", [0.0, 0.9])
+def test_chunked_tc_past_2_31_elements(beta):
     """Maximum sizes: q, k, v and o of 257 heads x 65536 tokens x d = 128
     (2^31 + 2^24 elements each, 4.3 GB in bf16), so the element offsets of the
     last heads pass 2^31.  Heads are independent: the first and the last head
     carry seeded inputs from the generator and are compared with the oracle
     over the whole sequence, the others hold seeded device noise of the same
     scale.  Both the automatic plan (one segment per head) and four segments
-    per head (1028 blocks, decoupled look-back) are checked."""
+    per head (1028 blocks, decoupled look-back) are checked, without and
+    with momentum."""
     H, T, d = 257, 65536, 128
     assert H * T * d > 2 ** 31
     qs, ks, vs, zs = make_qkv((1, 2), T, d, d, 31)
@@ -429,15 +431,18 @@ def test_chunked_tc_past_2_31_elements():
     for j, h in enumerate((0, H - 1)):
         q[0, h], k[0, h], v[0, h] = qs[0, j].to(bf).cuda(), ks[0, j].to(bf).cuda(), vs[0, j].to(bf).cuda()
         eta[0, h] = eta_s[0, j].cuda()
-    refs = {h: oracle_forward(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], eta[:, h:h + 1], 0.0) for h in (0, H - 1)}
+    refs = {h: oracle_forward(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], eta[:, h:h + 1], 0.0, beta)
+            for h in (0, H - 1)}
     for segments in (0, 4):
-        o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=128, segments=segments)
+        o, S, M = ttt.forward_chunked(q, k, v, eta, beta=beta, chunk=128, segments=segments)
         torch.cuda.synchronize()
         assert ttt.device_status() == 0
-        for h, (o_ref, S_ref, _) in refs.items():
+        for h, (o_ref, S_ref, M_ref) in refs.items():
             assert_bf16(o[:, h:h + 1], o_ref, f"o head {h} segments {segments}")
             assert_bf16(S[:, h:h + 1], S_ref, f"state head {h} segments {segments}")
-        del o, S
+            if beta:
+                assert_bf16(M[:, h:h + 1], M_ref, f"momentum head {h} segments {segments}")
+        del o, S, M
     del q, k, v, eta
     torch.cuda.empty_cache()
 
