@@ -136,10 +136,10 @@ def test_backward_chunked_momentum_agrees_with_recurrent(d):
 
 
 def test_backward_chunked_momentum_two_streams_and_graph_capture():
-    """With momentum the call runs its two independent launch chains on two
-    streams. The outputs are the same bits on the default stream, on another
-    stream, and replayed from a captured CUDA graph, which the second stream
-    joins through the call's fork and join events."""
+    """With momentum the call runs its three independent launch chains on
+    three streams. The outputs are the same bits on the default stream, on
+    another stream, and replayed from a captured CUDA graph, which the side
+    streams join through the call's fork and join events."""
     x = _mom_case(2, 3, 64 * 9 + 5, 128, 280)
     kw = dict(eta_const=x["ec"], state_in=x["S0"], grad_state=x["dW"], beta=0.9, mom_in=x["M0"], grad_mom=x["dM"])
     a = _abi.backward_chunked(x["q"], x["k"], x["v"], x["dO"], x["eta"], **kw)
@@ -157,3 +157,36 @@ def test_backward_chunked_momentum_two_streams_and_graph_capture():
     for n in ("dq", "dk", "dv", "deta", "dW0", "dM0"):
         assert torch.equal(a[n], b[n]), n
         assert torch.equal(a[n], c[n]), n
+
+
+@pytest.mark.parametrize("beta", [0.0, 0.9])
+def test_backward_chunked_past_2_31_elements(beta):
+    """Maximum sizes: q, k, v, dO and the gradients of 513 heads x 32768
+    tokens x d = 128 (2^31 + 2^22 elements each, 4.3 GB in bf16).  Heads are
+    independent: the last head, whose element offsets pass 2^31, carries
+    seeded inputs from the generator and is compared with the gradient
+    oracle; the others hold seeded device noise of the same scale."""
+    H, T, d = 513, 32768, 128
+    assert (H - 1) * T * d >= 2 ** 31
+    qs, ks, vs, zs = make_qkv((1, 1), T, d, d, 41)
+    dOs = torch.randn(1, 1, T, d, generator=torch.Generator().manual_seed(42))
+    eta_s = (torch.sigmoid(zs) / math.sqrt(d)).float()
+    g = torch.Generator(device="cuda").manual_seed(6)
+    bf = torch.bfloat16
+
+    def noise(scale):
+        return (torch.randn(1, H, T, d, generator=g, device="cuda", dtype=bf) * scale).to(bf)
+    q, k, v, dO = noise(1.0 / math.sqrt(d)), noise(1.0 / math.sqrt(d)), noise(1.0), noise(1.0)
+    eta = torch.full((1, H, T), 0.5 / math.sqrt(d), device="cuda")
+    h = H - 1
+    q[0, h], k[0, h], v[0, h], dO[0, h] = (t[0, 0].to(bf).cuda() for t in (qs, ks, vs, dOs))
+    eta[0, h] = eta_s[0, 0].cuda()
+    gr = _abi.backward_chunked(q, k, v, dO, eta, beta=beta)
+    torch.cuda.synchronize()
+    sl = slice(h, h + 1)
+    ref = oracle.ttt_backward_f64(f64(q[:, sl]), f64(k[:, sl]), f64(v[:, sl]), f64(eta[:, sl]), f64(dO[:, sl]), None,
+                                  beta=beta)
+    for n in ("dq", "dk", "dv", "deta", "dW0") + (("dM0",) if beta else ()):
+        assert_bf16(gr[n][:, sl], ref[n], f"{n} head {h}")
+    del q, k, v, dO, eta, gr
+    torch.cuda.empty_cache()
