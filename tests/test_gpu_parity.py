@@ -49,6 +49,40 @@ def test_decode_step_parity(dtype, d, beta, ascent):
         assert_f32(M, M_ref, "momentum")
 
 
+@pytest.mark.parametrize("beta", [0.0, 0.9])
+def test_decode_step_past_2_31_state_elements(beta):
+    """Maximum sizes for decode: the fp32 state of 4097 sequences x 32 heads x
+    128 x 128 (2^31 + 2^19 elements, 8.6 GB; with momentum its buffer as
+    large), updated in place by one bf16 step.  The first and the last
+    (sequence, head), whose state offsets pass 2^31, are compared with the
+    oracle's one-token recurrence from the same state."""
+    N, H, d = 4097, 32, 128
+    assert (N * H - 1) * d * d >= 2 ** 31
+    g = torch.Generator(device="cuda").manual_seed(8)
+    bf = torch.bfloat16
+    q = (torch.randn(N, H, d, generator=g, device="cuda") / math.sqrt(d)).to(bf)
+    k = (torch.randn(N, H, d, generator=g, device="cuda") / math.sqrt(d)).to(bf)
+    v = torch.randn(N, H, d, generator=g, device="cuda").to(bf)
+    eta = 0.1 * torch.rand(N, H, generator=g, device="cuda")
+    S = torch.randn(N, H, d, d, generator=g, device="cuda").mul_(0.3)
+    M = torch.randn(N, H, d, d, generator=g, device="cuda").mul_(0.3) if beta else None
+    picks = [(0, 0), (N - 1, H - 1)]
+    sls = {pk: (slice(pk[0], pk[0] + 1), slice(pk[1], pk[1] + 1)) for pk in picks}
+    S0 = {pk: S[sl].clone() for pk, sl in sls.items()}
+    M0 = {pk: (M[sl].clone() if beta else None) for pk, sl in sls.items()}
+    o = ttt.decode_step(q, k, v, S, M, eta=eta, beta=beta)
+    torch.cuda.synchronize()
+    for pk, sl in sls.items():
+        o_ref, S_ref, M_ref = oracle_forward(q[sl][:, :, None], k[sl][:, :, None], v[sl][:, :, None],
+                                             eta[sl][:, :, None], 0.0, beta, False, S0[pk], M0[pk])
+        assert_bf16(o[sl], o_ref[:, :, 0], f"o {pk}")
+        assert_f32(S[sl], S_ref, f"state {pk}")
+        if beta:
+            assert_f32(M[sl], M_ref, f"momentum {pk}")
+    del q, k, v, eta, S, M, o
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------- recurrent ----
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("d", [32, 64, 128])
