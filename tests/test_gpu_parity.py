@@ -481,6 +481,45 @@ def test_chunked_tc_past_2_31_elements(beta):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("path", ["recurrent_bf16", "chunked_f32"])
+def test_other_paths_past_2_31_elements(path):
+    """Maximum sizes on the recurrent kernel (bf16) and the fp32 chunked
+    kernel: 513 heads x 32768 tokens x d = 128 (2^31 + 2^22 elements per
+    tensor).  The last head, whose element offsets pass 2^31, carries seeded
+    inputs from the generator and is compared with the oracle over the whole
+    sequence; the others hold seeded device noise of the same scale."""
+    H, T, d = 513, 32768, 128
+    assert (H - 1) * T * d >= 2 ** 31
+    dt = torch.bfloat16 if path == "recurrent_bf16" else torch.float32
+    qs, ks, vs, zs = make_qkv((1, 1), T, d, d, 51)
+    eta_s = (torch.sigmoid(zs) / math.sqrt(d)).float()
+    g = torch.Generator(device="cuda").manual_seed(7)
+
+    def noise(scale):
+        return (torch.randn(1, H, T, d, generator=g, device="cuda", dtype=dt) * scale).to(dt)
+    q, k, v = noise(1.0 / math.sqrt(d)), noise(1.0 / math.sqrt(d)), noise(1.0)
+    eta = torch.full((1, H, T), 0.5 / math.sqrt(d), device="cuda")
+    h = H - 1
+    q[0, h], k[0, h], v[0, h] = (t[0, 0].to(dt).cuda() for t in (qs, ks, vs))
+    eta[0, h] = eta_s[0, 0].cuda()
+    if path == "recurrent_bf16":
+        o, S, _ = ttt.forward_recurrent(q, k, v, eta)
+    else:
+        o, S, _ = ttt.forward_chunked(q, k, v, eta, chunk=64)
+    torch.cuda.synchronize()
+    assert ttt.device_status() == 0
+    sl = slice(h, h + 1)
+    o_ref, S_ref, _ = oracle_forward(q[:, sl], k[:, sl], v[:, sl], eta[:, sl], 0.0)
+    if dt == torch.float32:
+        assert_f32(o[:, sl], o_ref, "o")
+        assert_f32(S[:, sl], S_ref, "state")
+    else:
+        assert_bf16(o[:, sl], o_ref, "o")
+        assert_bf16(S[:, sl], S_ref, "state")
+    del q, k, v, eta, o, S
+    torch.cuda.empty_cache()
+
+
 # ------------------------------------------------ decode workload ----
 def test_decode_workload_prefill_then_steps():
     """256 sequences x 16 heads, d = 128: chunked prefill of 2048 tokens, then
